@@ -1,0 +1,266 @@
+"""fp64 CPU oracle for the hybrid compressed-sparse attention (CSA/HCA) path.
+
+TEST INFRASTRUCTURE ONLY. This module is the independent, slow, obviously
+correct statement of what the path computes. Only the test suite, the smoke
+check in ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import
+or run it. It shares no code with the CUDA library or its Python binding and
+imports neither; the two sides meet only in the seeded input generator.
+
+Every function takes plain arrays, converts them exactly to float64, and does
+all arithmetic in float64 with numpy. There is no blocking, fusion or
+reordering beyond what each definition states.
+
+Sources (the pages describe the method only in prose):
+
+* "DeepSeek-V4 Architecture Analysis" (architecture_analysis.py),
+  INNOVATIONS section 1, "COMPRESSED SPARSE ATTENTION (CSA)": sliding window of
+  the nearest 128 tokens; learned gated pooling 4 tokens -> 1 with overlapping
+  windows, using absolute position embeddings within the window and an RMSNorm
+  on the compressed output; HCA 128 tokens -> 1; an indexer that scores
+  compressed positions by dot products with per-head importance weights and
+  keeps the top-k; a learnable per-head scalar attention sink.
+* same page, INNOVATIONS section 2, "UNIFIED HEAD DIMENSION": keys and values
+  share one head_dim = 512 representation (K = V); the RoPE dimensions are
+  rotated separately (pre-applied to the inputs here).
+* "DeepSeek-V4-Flash" (llm-atlas model card), table "Champs bruts du
+  config.json": head_dim 512, index_n_heads 64, index_head_dim 128,
+  index_topk 512, sliding_window 128, rms_norm_eps 1e-6,
+  num_attention_heads 64, num_key_value_heads 1.
+
+Readings taken where the pages are silent (each is listed with its reason in
+the design notes):
+
+* R1 CSA windows are 8 tokens long with stride 4: entry j covers tokens
+  [4j, 4j + 7]; a trailing partial window makes no entry. HCA uses window =
+  stride = 128.
+* R2 the pool is a per-dimension softmax over the window positions of
+  (gate + ape[i]), ape indexed by position i inside the window.
+* R4 RMSNorm: y = c / sqrt(mean(c^2) + eps) * norm_w, eps = 1e-6.
+* R6 entry j is visible at position p iff its last token j*stride + win - 1
+  is <= p.
+* R8 the window is tokens max(0, p - W + 1) .. p, not de-duplicated against
+  compressed entries.
+* R9 indexer score s_j = sum_h w_h * max(0, qi_h . ki_j), unscaled.
+* R10 top-k orders by (score descending, index ascending); fewer than k
+  visible entries are all kept and the rest padded with -1.
+* R11 the sink is a per-head logit (not multiplied by the softmax scale) in
+  the denominator, carrying a zero value vector.
+* R12 K = V: one row serves as key and value.
+
+Pins (tests/test_oracle_pins.py) tie every function to something other than
+itself: closed forms, textbook/library special cases (torch rms_norm,
+avg_pool1d, scaled_dot_product_attention), invariants and brute force.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+RMS_EPS = 1e-6
+
+
+def _f64(x) -> np.ndarray:
+    """Exact conversion to float64 (bf16 and fp32 values are representable)."""
+    try:  # torch tensors (bf16 has no numpy dtype): widen in torch first
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# A1: gated-pooling compressor + RMSNorm
+# ---------------------------------------------------------------------------
+
+def n_entries(T: int, win: int, stride: int) -> int:
+    """Number of complete windows of length ``win`` at stride ``stride`` that
+    fit in T tokens (reading R1: a trailing partial window makes no entry)."""
+    if T < win:
+        return 0
+    return (T - win) // stride + 1
+
+
+def rms_norm(c: np.ndarray, norm_w: np.ndarray, eps: float = RMS_EPS) -> np.ndarray:
+    """RMSNorm over the last axis (model card: rms_norm_eps = 1e-6; the
+    architecture analysis, INNOVATIONS section 1: "RMSNorm on compressed
+    output")."""
+    c = _f64(c)
+    rms = np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + eps)
+    return c / rms * _f64(norm_w)
+
+
+def compress(kv, gate, ape, norm_w, win: int, stride: int, eps: float = RMS_EPS,
+             pre_norm: bool = False) -> np.ndarray:
+    """Compress one sequence of raw per-token KV into one entry per window.
+
+    kv, gate: [T, D] (the wkv / wgate projections, RoPE already applied);
+    ape: [win, D] absolute position embedding indexed by the position inside
+    the window; norm_w: [D]. Returns [n_entries(T), D] in float64.
+
+    Follows the architecture analysis, INNOVATIONS section 1: learned gated
+    pooling over (overlapping, for CSA) windows, position embeddings within
+    the window, RMSNorm on the compressed output. For entry j over tokens
+    t = j*stride + i, i = 0..win-1, and every dimension d:
+        a[i, d] = softmax over i of (gate[t, d] + ape[i, d])
+        c[d]    = sum_i a[i, d] * kv[t, d]
+        out     = RMSNorm(c) * norm_w
+    With ``pre_norm`` the pooled c is returned without the norm.
+    """
+    kv = _f64(kv)
+    gate = _f64(gate)
+    ape = _f64(ape)
+    T, D = kv.shape
+    assert gate.shape == (T, D) and ape.shape == (win, D)
+    N = n_entries(T, win, stride)
+    out = np.empty((N, D), dtype=np.float64)
+    block = max(1, (1 << 22) // max(1, win * D))  # bounds the temporaries
+    for j0 in range(0, N, block):
+        j1 = min(N, j0 + block)
+        tok = (np.arange(j0, j1)[:, None] * stride + np.arange(win)[None, :])  # [n, win]
+        logits = gate[tok] + ape[None, :, :]                # [n, win, D]
+        m = logits.max(axis=1, keepdims=True)
+        e = np.exp(logits - m)
+        a = e / e.sum(axis=1, keepdims=True)                # softmax over the window axis
+        out[j0:j1] = (a * kv[tok]).sum(axis=1)
+    if pre_norm:
+        return out
+    return rms_norm(out, norm_w, eps)
+
+
+# ---------------------------------------------------------------------------
+# Causal visibility of compressed entries
+# ---------------------------------------------------------------------------
+
+def n_visible(p: int, win: int, stride: int) -> int:
+    """Entries whose every token is at or before position p (reading R6):
+    entry j is visible iff j*stride + win - 1 <= p, i.e. the number of complete
+    windows in the prefix of p + 1 tokens."""
+    return n_entries(p + 1, win, stride)
+
+
+# ---------------------------------------------------------------------------
+# A2 + A3: indexer scores and top-k selection
+# ---------------------------------------------------------------------------
+
+def index_scores(qi, wi, ki, n_vis: int) -> np.ndarray:
+    """Indexer score of every visible compressed entry for one query.
+
+    qi: [Hi, Di] indexer query heads; wi: [Hi] per-head importance weights;
+    ki: [>= n_vis, Di] indexer keys of the query's sequence.
+    Architecture analysis, INNOVATIONS section 1 (indexer: "dot-product
+    attention + per-head importance weights"); reading R9:
+        s_j = sum_h wi[h] * max(0, qi[h] . ki[j]),  j < n_vis.
+    """
+    qi = _f64(qi)
+    wi = _f64(wi)
+    ki = _f64(ki)[:n_vis]
+    dots = ki @ qi.T                     # [n_vis, Hi]
+    return np.maximum(dots, 0.0) @ wi    # [n_vis]
+
+
+def topk(scores, k: int) -> np.ndarray:
+    """Indices of the min(k, n) best scores, best first, padded with -1 to k.
+
+    Order (reading R10): score descending, ties by index ascending. A full
+    stable sort is the definition (model card: index_topk = 512).
+    """
+    s = _f64(scores)
+    n = s.shape[0]
+    order = np.lexsort((np.arange(n), -s))   # last key is primary
+    out = np.full(k, -1, dtype=np.int64)
+    m = min(k, n)
+    out[:m] = order[:m]
+    return out
+
+
+def index_topk(qi, wi, ki, p: int, k: int, win: int, stride: int):
+    """Scores and the selected index list for one query at position p."""
+    nv = n_visible(p, win, stride)
+    s = index_scores(qi, wi, ki, nv)
+    return topk(s, k), s
+
+
+# ---------------------------------------------------------------------------
+# A4 / A5: MQA over selected rows + sliding window + sink
+# ---------------------------------------------------------------------------
+
+def attend(q, rows, sink, scale: float):
+    """Softmax attention of H query heads over R shared rows plus a sink.
+
+    q: [H, D]; rows: [R, D] used as both key and value (architecture analysis,
+    INNOVATIONS section 2: keys and values share one representation);
+    sink: [H] per-head logit with a zero value (INNOVATIONS section 1,
+    "Attention sink"; reading R11); scale multiplies q . row only.
+    For head h: logits_r = scale * q_h . row_r, plus sink_h;
+        p_r = exp(logit_r - m) / Z,  p_sink = exp(sink_h - m) / Z,
+        out_h = sum_r p_r * row_r.
+    Returns (out [H, D], p [H, R], p_sink [H]).
+    """
+    q = _f64(q)
+    rows = _f64(rows)
+    sink = _f64(sink)
+    H = q.shape[0]
+    R = rows.shape[0]
+    logits = scale * (q @ rows.T) if R else np.zeros((H, 0))
+    m = np.maximum(logits.max(axis=1) if R else -np.inf, sink)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.exp(logits - m[:, None])
+    e_sink = np.exp(sink - m)
+    Z = e.sum(axis=1) + e_sink
+    p = e / Z[:, None]
+    out = p @ rows if R else np.zeros_like(q)
+    return out, p, e_sink / Z
+
+
+def window_rows(kv_win, win_end: int, W: int) -> np.ndarray:
+    """Raw rows max(0, e - W + 1) .. e of one sequence's raw-KV buffer, where e
+    is the buffer row of the query's own token (architecture analysis,
+    INNOVATIONS section 1: each token attends to its nearest 128 tokens;
+    reading R8: the query's own token is included)."""
+    kv_win = _f64(kv_win)
+    lo = max(0, win_end - W + 1)
+    return kv_win[lo:win_end + 1]
+
+
+def sparse_mqa(q, kv_cmp, idx, kv_win, win_end: int, W: int, sink, scale: float):
+    """CSA attention for one query: the selected compressed rows (entries
+    idx >= 0 of this sequence's compressed cache), the sliding window and
+    the sink. Returns out [H, D] (float64)."""
+    kv_cmp = _f64(kv_cmp)
+    idx = np.asarray(idx)
+    sel = kv_cmp[idx[idx >= 0]]
+    rows = np.concatenate([sel, window_rows(kv_win, win_end, W)], axis=0)
+    return attend(q, rows, sink, scale)[0]
+
+
+def hca_mqa(q, kv_cmp, n_cmp: int, kv_win, win_end: int, W: int, sink, scale: float):
+    """HCA attention for one query: every visible compressed entry
+    (architecture analysis, INNOVATIONS section 1: HCA, 128 tokens -> 1, for
+    global context, with no indexer), the sliding window and the sink."""
+    kv_cmp = _f64(kv_cmp)[:n_cmp]
+    rows = np.concatenate([kv_cmp, window_rows(kv_win, win_end, W)], axis=0)
+    return attend(q, rows, sink, scale)[0]
+
+
+# ---------------------------------------------------------------------------
+# Storage rounding (the compressed cache is stored in the input dtype)
+# ---------------------------------------------------------------------------
+
+def round_to(x, dtype: str) -> np.ndarray:
+    """Round float64 values once to 'fp32' or 'bf16' (round to nearest even)
+    and return them as float64. bf16 is a single rounding from fp64 to 8
+    significant bits (normal range only)."""
+    x = _f64(x)
+    if dtype == "fp64":
+        return x.copy()
+    if dtype == "fp32":
+        return x.astype(np.float32).astype(np.float64)
+    if dtype == "bf16":
+        # Round fp64 -> bf16 directly: keep 8 significant bits, ties to even.
+        m, e = np.frexp(x)                  # x = m * 2**e, 0.5 <= |m| < 1
+        scaled = np.ldexp(m, 8)             # 8 significant bits in the integer part
+        r = np.round(scaled)                # numpy rounds half to even
+        return np.ldexp(r, e - 8)
+    raise ValueError(dtype)
