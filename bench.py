@@ -1,0 +1,496 @@
+"""Benchmark of the CSA/HCA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload csa_decode_64k] [--no-secondary] [--no-cpu-baseline]
+
+One step = one pass of the whole path over one batch of the workload: for
+the CSA decode workloads, fold the newest raw window into the compressed
+cache (csa_compress), score + select (csa_index_topk) and attend
+(csa_sparse_mqa); for the HCA workload, append + hca_mqa. Inputs are seeded
+synthetic tensors of the DeepSeek-V4-Flash shapes, resident in HBM. The step
+is captured once in a CUDA graph and replayed; L2 is flushed (a 256 MB
+write) before every timed step, outside the step's events.
+
+Multi-GPU (torchrun): one process per GPU, each serving its own batch of
+independent sequences (weak scaling, no collective on the data path); the
+step time is the max over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores on the same
+workload (rank 0 only) and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from compressed_sparse_attention_15_b200 import _lib, ops, workloads as WL  # noqa: E402
+
+METRIC = "CSA/HCA decode queries/s at 64K–1M ctx; HBM GB/s and % of roofline"
+UNIT = "queries/s"
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# Algorithmic bytes / FLOPs (what the method must move; scratch excluded)
+# --------------------------------------------------------------------------
+
+def algo_bytes(w: WL.Workload):
+    """Per-step algorithmic bytes of each kernel family (dtype sizes: bf16 2,
+    fp32 4, int32 4)."""
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    n_vis = w.N  # decode: every entry is visible
+    b = {}
+    b["compress"] = w.B * (2 * w.T_c * w.D * e + w.win * w.D * 4 + w.D * 4
+                           + ((w.T_c - w.win) // w.stride + 1) * w.D * e)
+    if w.mode == "csa":
+        b["index_scores"] = w.Q * (n_vis * w.Di * e + w.Hi * w.Di * e + w.Hi * 4)
+        b["topk"] = w.Q * w.k * 4
+        rows = w.k + w.W
+        b["mqa"] = w.Q * (rows * w.D * e + 2 * w.H * w.D * e + w.k * 4 + w.H * 4)
+    else:
+        rows = n_vis + w.W
+        b["mqa"] = w.Q * (rows * w.D * e + 2 * w.H * w.D * e + w.H * 4)
+    return b
+
+
+def algo_flops(w: WL.Workload):
+    f = {}
+    if w.mode == "csa":
+        f["index_scores"] = w.Q * w.N * w.Hi * w.Di * 2
+        rows = w.k + w.W
+    else:
+        rows = w.N + w.W
+    f["mqa"] = w.Q * rows * w.H * w.D * 4
+    return f
+
+
+# --------------------------------------------------------------------------
+# The step
+# --------------------------------------------------------------------------
+
+class Step:
+    """Device-resident inputs of one workload and its decode step."""
+
+    def __init__(self, w: WL.Workload, device):
+        self.w = w
+        self.dev = device
+        self.t = {n: WL.make(w, n, device) for n in ("q", "kv_cmp", "kv_win", "sink", "ape", "gate")}
+        if w.mode == "csa":
+            for n in ("qi", "wi", "ki"):
+                self.t[n] = WL.make(w, n, device)
+        self.norm_w = WL.norm_w(w, device)
+        self.n_cmp = ops.visible_entries(w.positions(), w.win, w.stride).to(device)
+        self.win_end = w.win_end().to(device)
+        self.out = torch.empty_like(self.t["q"])
+        self.idx = torch.empty((w.Q, max(1, w.k)), dtype=torch.int32, device=device)
+        self.ws_index = ops.Workspace(device)
+        self.ws_mqa = ops.Workspace(device)
+
+    def compress(self):
+        w, t = self.w, self.t
+        ops.compress(t["kv_win"][:, w.c_src0:w.c_src0 + w.T_c], t["gate"], t["ape"], self.norm_w, w.win, w.stride,
+                     out=t["kv_cmp"][:, w.c_dst0:w.c_dst0 + (w.T_c - w.win) // w.stride + 1])
+
+    def select(self):
+        t = self.t
+        ops.index_topk(t["qi"], t["wi"], t["ki"], self.n_cmp, self.w.k, out=self.idx, ws=self.ws_index)
+
+    def attend(self):
+        w, t = self.w, self.t
+        if w.mode == "csa":
+            ops.sparse_mqa(t["q"], t["kv_cmp"], self.idx, t["kv_win"], self.win_end, t["sink"], w.scale, w.W,
+                           out=self.out, ws=self.ws_mqa)
+        else:
+            ops.hca_mqa(t["q"], t["kv_cmp"], self.n_cmp, t["kv_win"], self.win_end, t["sink"], w.scale, w.W,
+                        out=self.out, ws=self.ws_mqa)
+
+    def parts(self):
+        p = [("compress", self.compress)]
+        if self.w.mode == "csa":
+            p.append(("index_topk", self.select))
+        p.append(("mqa", self.attend))
+        return p
+
+    def run(self):
+        for _, f in self.parts():
+            f()
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        try:
+            self.idx = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.idx = str(torch.cuda.current_device())
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 8:
+                    try:
+                        rows.append((float(p[0]), float(p[1]), p[3:8]))
+                    except ValueError:
+                        pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for _, _, r in rows:
+            for n, v in zip(names, r[1:5]):
+                if v.lower() == "active":
+                    seen.add(n)
+        loaded = sorted(r[0] for r in rows)
+        top = loaded[len(loaded) // 2:]  # samples under load sit in the upper half
+        return {"sm_mhz": statistics.median(top), "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(seen),
+                "samples": len(rows)}
+
+
+def _sync_barrier(dist_on):
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+
+def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=False):
+    step = Step(w, device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(3, args.warmup)):
+        step.run()
+    torch.cuda.synchronize()
+    # Capture one step in a CUDA graph (the library never allocates or
+    # synchronises, so its launches are capturable).
+    n0 = _lib.lib().csa_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device)
+    s.wait_stream(stream)
+    with torch.cuda.stream(s):
+        step.run()
+    stream.wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        step.run()
+    launches_per_step = _lib.lib().csa_launch_count() - n0
+    launches_per_step //= 2  # the warm-up on `s` plus the capture
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    K = args.steps if not secondary else max(10, args.steps // 4)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = Clocks(device)
+    _sync_barrier(dist_on)
+    wall0 = time.perf_counter()
+    with clocks:
+        time.sleep(0.2)
+        for i in range(K):
+            flush.zero_()
+            evs[i][0].record(stream)
+            graph.replay()
+            evs[i][1].record(stream)
+        _sync_barrier(dist_on)
+    wall = time.perf_counter() - wall0
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = sum(step_ms) / K
+    t = torch.tensor([ms], device=device)
+    if dist_on:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # Per-kernel durations: the same kernels launched one by one with events
+    # between them (a host-side head start keeps the launches queued).
+    names = [n for n, _ in step.parts()]
+    per = {n: 0.0 for n in names}
+    Kp = max(5, K // 2)
+    for _ in range(Kp):
+        flush.zero_()
+        torch.cuda._sleep(2_000_000)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        ev[0].record(stream)
+        for i, (_, f) in enumerate(step.parts()):
+            f()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        for i, n in enumerate(names):
+            per[n] += ev[i].elapsed_time(ev[i + 1]) / Kp
+    status = step.ws_mqa.status() | step.ws_index.status()
+    del graph
+    return {"ms": ms_max, "ms_local": ms, "per_kernel_ms": per, "launches_per_step": int(launches_per_step),
+            "wall_s": wall, "clocks": clocks.summary(), "status": status, "K": K, "step": step}
+
+
+def roofline_of(w, per_kernel_ms, hbm_gbs, traffic=None):
+    """Roofline of the kernel with the most algorithmic bytes in the step."""
+    ab = algo_bytes(w)
+    fam = {"index_topk": "index_scores", "mqa": "mqa", "compress": "compress"}
+    best = max(((k, ab[fam[k]]) for k in per_kernel_ms if fam[k] in ab), key=lambda x: x[1])
+    name, nbytes = best
+    ms = per_kernel_ms[name]
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
+            "frac": round(achieved / hbm_gbs, 4), "traffic": traffic, "bytes_per_launch": int(nbytes)}
+
+
+def e2e_ours(args, w: WL.Workload, step: Step, device):
+    """Same metric through the public API with host buffers: every step copies
+    its per-step inputs (q, qi, wi, the newest raw token and the window's
+    gates) from pinned host memory and reads the output back."""
+    t = step.t
+    host = {n: t[n].cpu().pin_memory() for n in ("q", "gate")}
+    if w.mode == "csa":
+        host.update({n: t[n].cpu().pin_memory() for n in ("qi", "wi")})
+    host["kv_new"] = t["kv_win"][:, -1].cpu().pin_memory()
+    out_h = torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    stream = torch.cuda.current_stream(device)
+    K = max(10, args.steps // 2)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    ms = 0.0
+    for i in range(K + 2):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for n in ("q", "gate", "qi", "wi"):
+            if n in host:
+                t[n].copy_(host[n], non_blocking=True)
+        t["kv_win"][:, -1].copy_(host["kv_new"], non_blocking=True)
+        step.run()
+        out_h.copy_(step.out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            ms += a.elapsed_time(b) / K
+    return {"value": round(w.Q / (ms * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4)}
+
+
+# --------------------------------------------------------------------------
+# The oracle on the host (CPU baseline and --impl reference)
+# --------------------------------------------------------------------------
+
+def oracle_step_inputs(w: WL.Workload):
+    import numpy as np
+
+    host = {n: WL.make(w, n) for n in ("q", "sink", "ape", "qi", "wi") if n != "qi" or w.mode == "csa"}
+    if w.mode == "csa":
+        host["ki"] = WL.make(w, "ki")
+    host["np"] = np
+    return host
+
+
+def time_oracle(w: WL.Workload, steps: int, budget_s: float):
+    """Time the fp64 oracle on the host over up to `steps` full batches, stopping
+    once `budget_s` of oracle time has been spent. Input regeneration and row
+    gathering happen outside the timed sections."""
+    import numpy as np
+
+    import oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    host = oracle_step_inputs(w)
+    ape = host["ape"]
+    total, done = 0.0, 0
+    for _ in range(max(1, steps)):
+        for q in range(w.Q):
+            b = q // w.q_per_seq
+            raw = WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.c_src0, w.c_src0 + w.T_c))
+            gate = WL.rows(w, "gate", b * w.T_c + torch.arange(w.T_c))
+            t0 = time.perf_counter()
+            new = O.round_to(O.compress(raw, gate, ape, np.ones(w.D), w.win, w.stride), "bf16")
+            if w.mode == "csa":
+                idx, _ = O.index_topk(host["qi"][q], host["wi"][q], host["ki"][b], int(w.positions()[q]), w.k,
+                                      w.win, w.stride)
+                sel = idx[idx >= 0]
+            else:
+                sel = np.arange(w.N)
+            total += time.perf_counter() - t0
+            rows_c = O.round_to(WL.rows(w, "kv_cmp", b * w.N + torch.as_tensor(sel)), "bf16")
+            rows_c[sel == w.c_dst0] = new[0]
+            e = int(w.win_end()[q])
+            rows_w = O._f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(max(0, e - w.W + 1), e + 1)))
+            t0 = time.perf_counter()
+            O.attend(host["q"][q], np.concatenate([rows_c, rows_w]), host["sink"], w.scale)
+            total += time.perf_counter() - t0
+            done += 1
+        if total >= budget_s:
+            break
+    return {"value": done / total, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"{done} queries ({done // w.Q} full batches of {w.Q}) of {w.name}, fp64 numpy; "
+                      f"input regeneration untimed", "seconds": round(total, 2)}
+
+
+# --------------------------------------------------------------------------
+
+def workload_config(w: WL.Workload):
+    return {"workload": w.name, "batch": w.Q, "context": w.pos0 + 1, "heads": f"{w.H}q:1kv", "head_dim": w.D,
+            "indexer": f"{w.Hi}x{w.Di}" if w.mode == "csa" else None, "topk": w.k or None, "window": w.W,
+            "compress": f"win {w.win} stride {w.stride}", "l2": "flushed: 256 MB write before every timed step",
+            "inputs": "seeded synthetic (counter-based generator), resident in HBM"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="csa_decode_64k", choices=[n for n in WL.WORKLOADS if n != "tiny_csa_prefill_fp32"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WL.WORKLOADS[args.workload]
+    hbm, tflops, peak_kind = _peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        base = time_oracle(w, max(1, args.steps), budget_s=60.0)
+        line = {"metric": METRIC, "value": round(base["value"], 3), "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(w.Q / base["value"] * 1e3, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": workload_config(w), "impl": "reference",
+                "cpu_baseline": base, "e2e": {"value": round(base["value"], 3), "unit": UNIT,
+                                              "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", torch.cuda.current_device())
+
+    r = time_ours(args, w, device, dist_on, rank, world)
+    traffic = None
+    try:
+        with open(args.traffic_json) as f:
+            tj = json.load(f).get(w.name)
+            if tj:
+                traffic = tj.get("bytes_per_launch")
+    except Exception:
+        pass
+    roof = roofline_of(w, r["per_kernel_ms"], hbm, traffic)
+    roof["peak_kind"] = f"{peak_kind} HBM copy bandwidth"
+    e2e = e2e_ours(args, w, r["step"], device)
+    del r["step"]
+    torch.cuda.empty_cache()
+
+    secondary = {}
+    if not args.no_secondary and rank == 0 and not dist_on:
+        for name in ("hca_decode_1m", "csa_decode_1m"):
+            if name == w.name:
+                continue
+            sw = WL.WORKLOADS[name]
+            try:
+                s = time_ours(args, sw, device, False, 0, 1, secondary=True)
+                del s["step"]
+                rf = roofline_of(sw, s["per_kernel_ms"], hbm)
+                step_bytes = sum(algo_bytes(sw).values())
+                secondary[name] = {"queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1), "ms_per_step": round(s["ms"], 4),
+                                   "per_kernel_ms": {k: round(v, 4) for k, v in s["per_kernel_ms"].items()},
+                                   "step_GBps": round(step_bytes / (s["ms"] * 1e-3) / 1e9, 1),
+                                   "step_frac": round(step_bytes / (s["ms"] * 1e-3) / 1e9 / hbm, 4),
+                                   "roofline": rf, "status": s["status"]}
+            except Exception as ex:  # report, do not hide
+                secondary[name] = {"error": repr(ex)}
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline and not dist_on:
+        cpu = time_oracle(w, 1000, budget_s=12.0)
+
+    if rank == 0:
+        step_bytes = sum(algo_bytes(w).values())
+        value = world * w.Q / (r["ms"] * 1e-3)
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": r["K"],
+            "warmup": args.warmup, "ms_per_step": round(r["ms"], 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+            "parallelism": f"replicas x{world} (independent sequences per GPU, no collective)",
+            "step_GBps": round(step_bytes / (r["ms"] * 1e-3) / 1e9, 1),
+            "step_roofline_frac": round(step_bytes / (r["ms"] * 1e-3) / 1e9 / hbm, 4),
+            "per_kernel_ms": {k: round(v, 4) for k, v in r["per_kernel_ms"].items()},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": r["launches_per_step"] * r["K"], "launches_per_step": r["launches_per_step"],
+            "clocks": r["clocks"], "device_status": r["status"], "wall_s_timed_region": round(r["wall_s"], 3),
+            "secondary": secondary or None,
+        }
+        print(json.dumps(line))
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,72 @@
+"""ctypes binding of libcsa.so (the C ABI declared in include/csa.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. Loading fails loudly if the library has not been built; there is no
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
+
+CSA_OK = 0
+CSA_DTYPE_F32 = 0
+CSA_DTYPE_BF16 = 1
+CSA_MAX_TOPK = 2048
+
+# Every function the header declares, with (restype, argtypes).
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_LL = ctypes.c_longlong
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "csa_strerror": (ctypes.c_char_p, [_I]),
+    "csa_compress": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _LL, _LL, _LL, _I, _P]),
+    "csa_index_topk_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "csa_index_topk": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "csa_index_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "csa_topk_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "csa_topk": (_I, [_P, _P, _I, _P, _I, _I, _P, _SZ, _P]),
+    "csa_mqa_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "csa_sparse_mqa": (_I, [_P, _P, _P, _P, _P, _F, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _P, _SZ, _P]),
+    "hca_mqa": (_I, [_P, _P, _P, _P, _F, _P, _I, _I, _I, _I, _I, _P, _I, _P, _I, _I, _I, _P, _SZ, _P]),
+    "csa_workspace_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
+    "csa_launch_count": (ctypes.c_ulonglong, []),
+}
+
+_lib = None
+
+
+class CsaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {strerror(code)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if libcsa.so is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is not built; run `python -m compressed_sparse_attention_15_b200.build` "
+                "(the CUDA kernels are the only implementation of this path)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().csa_strerror(code).decode()
+
+
+def check(fn: str, code: int) -> None:
+    if code != CSA_OK:
+        raise CsaError(fn, code)

@@ -1,0 +1,60 @@
+// Host-side launchers of the kernels, one translation unit per step. Every
+// launcher enqueues on `stream`, returns cudaGetLastError() of its launch,
+// and assumes its arguments were validated by the C-ABI layer (csa_api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa {
+
+// Process-wide count of kernel launches made by the library.
+void note_launches(unsigned n);
+
+struct CompressArgs {
+  const void *kv, *gate;
+  const float *ape, *norm_w;
+  void *out;
+  int B, T, D, win, stride, N;
+  long long kv_ss, gate_ss, out_ss;  // sequence strides in elements
+  int dtype;
+};
+cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream);
+
+struct ScoreArgs {
+  const void *qi;
+  const float *wi;
+  const void *ki;
+  const int32_t *n_cmp;
+  float *scores;
+  int Q, B, Hi, Di, N_max, q_per_seq, dtype;
+  uint32_t *status;
+};
+cudaError_t launch_index_scores(const ScoreArgs &a, cudaStream_t stream);
+
+struct TopkArgs {
+  const float *scores;
+  const int32_t *n_cmp;
+  int32_t *out_idx;
+  int Q, N_max, k;
+  uint32_t *status;
+};
+cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
+
+struct MqaArgs {
+  const void *q, *kv_cmp, *kv_win;
+  const int32_t *idx;      // null for the dense (HCA) variant
+  const int32_t *n_cmp;    // dense variant: visible entries per query
+  const int32_t *win_end;
+  const float *sink;
+  float scale;
+  void *out;
+  int Q, B, H, D, N_max, k, win_len, T_raw, q_per_seq, dtype;
+  void *partials;          // split-K scratch inside the workspace
+  size_t partial_bytes;
+  uint32_t *status;
+};
+cudaError_t launch_mqa(const MqaArgs &a, cudaStream_t stream);
+size_t mqa_partial_bytes(int Q, int H, int D, int rows_max);
+
+}  // namespace csa

@@ -1,0 +1,238 @@
+"""Torch-facing wrappers of the C ABI (include/csa.h).
+
+These functions only check tensor metadata, allocate outputs / workspaces
+with torch (PyTorch is the device-memory allocator and stream provider) and
+pass raw pointers, sizes and the current CUDA stream to libcsa.so. They do no
+arithmetic of the method. Names follow the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float32: _lib.CSA_DTYPE_F32, torch.bfloat16: _lib.CSA_DTYPE_BF16}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}; use torch.float32 or torch.bfloat16") from None
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, device=None, contiguous=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class Workspace:
+    """A reusable device workspace (first 256 bytes: the status word)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        nbytes = max(256, int(nbytes))
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            self.buf[:256].zero_()
+        return self.buf
+
+    def status(self) -> int:
+        """Synchronise, return and clear the status word (0 = clean)."""
+        if self.buf is None:
+            return 0
+        return workspace_status(self.buf)
+
+
+def workspace_status(ws: torch.Tensor) -> int:
+    v = ctypes.c_uint32(0)
+    rc = _lib.lib().csa_workspace_status(_ptr(ws), _stream(ws.device), ctypes.byref(v))
+    if rc not in (_lib.CSA_OK, 5):
+        _lib.check("csa_workspace_status", rc)
+    return int(v.value)
+
+
+def visible_entries(p: torch.Tensor, win: int, stride: int) -> torch.Tensor:
+    """int32 count of compressed entries whose window ends at or before each
+    position p (entry j covers tokens j*stride .. j*stride + win - 1)."""
+    p = torch.as_tensor(p, dtype=torch.int64)
+    n = torch.div(p + 1 - win, stride, rounding_mode="floor") + 1
+    return n.clamp_min(0).to(torch.int32)
+
+
+# ------------------------------------------------------------------ A1
+
+def compress(kv, gate, ape, norm_w, win: int, stride: int, out=None, ratio=None):
+    """Gated-pooling compressor + RMSNorm (csa_compress).
+
+    kv, gate: [B, T, D] (or [T, D]) with contiguous rows and any sequence
+    stride; ape [win, D] fp32; norm_w [D] fp32. Returns / fills out
+    [B, N, D] (rows contiguous, any sequence stride), N = (T - win)//stride + 1.
+    """
+    squeeze = kv.dim() == 2
+    if squeeze:
+        kv, gate = kv.unsqueeze(0), gate.unsqueeze(0)
+    _need(kv, "kv", contiguous=False)
+    _need(gate, "gate", dtype=kv.dtype, device=kv.device, contiguous=False)
+    _need(ape, "ape", dtype=torch.float32, device=kv.device)
+    _need(norm_w, "norm_w", dtype=torch.float32, device=kv.device)
+    B, T, D = kv.shape
+    for t, nm in ((kv, "kv"), (gate, "gate")):
+        if t.shape != (B, T, D) or t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{nm} must be [B, T, D] with contiguous [T, D] rows")
+    N = (T - win) // stride + 1 if T >= win else 0
+    if out is None:
+        out = torch.empty((B, N, D), dtype=kv.dtype, device=kv.device)
+    else:
+        if out.dim() == 2:
+            out = out.unsqueeze(0)
+        _need(out, "out", dtype=kv.dtype, device=kv.device, contiguous=False)
+        if out.shape != (B, N, D) or out.stride(2) != 1 or out.stride(1) != D:
+            raise ValueError("out must be [B, N, D] with contiguous [N, D] rows")
+    rc = _lib.lib().csa_compress(
+        _ptr(kv), _ptr(gate), _ptr(ape), _ptr(norm_w), int(stride if ratio is None else ratio), int(win),
+        int(stride), _ptr(out), B, T, D, kv.stride(0), gate.stride(0), out.stride(0), _dtype_code(kv),
+        _stream(kv.device))
+    _lib.check("csa_compress", rc)
+    return out[0] if squeeze else out
+
+
+# ------------------------------------------------------------- A2 + A3
+
+def _index_common(qi, wi, ki, n_cmp, q_per_seq):
+    _need(qi, "qi")
+    _need(wi, "wi", dtype=torch.float32, device=qi.device)
+    _need(ki, "ki", dtype=qi.dtype, device=qi.device)
+    _need(n_cmp, "n_cmp", dtype=torch.int32, device=qi.device)
+    Q, Hi, Di = qi.shape
+    B, N_max, Di2 = ki.shape
+    if Di2 != Di or wi.shape != (Q, Hi) or n_cmp.shape != (Q,):
+        raise ValueError("shape mismatch among qi [Q,Hi,Di], wi [Q,Hi], ki [B,N,Di], n_cmp [Q]")
+    if q_per_seq is None:
+        if Q % B:
+            raise ValueError("q_per_seq is required when B does not divide Q")
+        q_per_seq = Q // B
+    return Q, Hi, Di, B, N_max, q_per_seq
+
+
+def index_topk(qi, wi, ki, n_cmp, k: int, q_per_seq=None, out=None, ws: Workspace | None = None):
+    """Indexer scores + top-k (csa_index_topk). Returns int32 [Q, k]."""
+    Q, Hi, Di, B, N_max, qps = _index_common(qi, wi, ki, n_cmp, q_per_seq)
+    if out is None:
+        out = torch.empty((Q, k), dtype=torch.int32, device=qi.device)
+    _need(out, "out", dtype=torch.int32, device=qi.device)
+    L = _lib.lib()
+    nbytes = L.csa_index_topk_workspace_bytes(Q, N_max, k)
+    w = (ws or Workspace(qi.device)).get(nbytes)
+    rc = L.csa_index_topk(_ptr(qi), _ptr(wi), _ptr(ki), _ptr(n_cmp), int(k), _ptr(out), Q, B, Hi, Di, N_max, qps,
+                          _dtype_code(qi), _ptr(w), w.numel(), _stream(qi.device))
+    _lib.check("csa_index_topk", rc)
+    return out
+
+
+def index_scores(qi, wi, ki, n_cmp, q_per_seq=None, out=None, ws: Workspace | None = None):
+    """Indexer scores only (csa_index_scores): fp32 [Q, N_max]; entries
+    j >= n_cmp[q] are left as they were in ``out`` (NaN when allocated here)."""
+    Q, Hi, Di, B, N_max, qps = _index_common(qi, wi, ki, n_cmp, q_per_seq)
+    if out is None:
+        out = torch.full((Q, N_max), float("nan"), dtype=torch.float32, device=qi.device)
+    _need(out, "out", dtype=torch.float32, device=qi.device)
+    w = (ws or Workspace(qi.device)).get(256)
+    rc = _lib.lib().csa_index_scores(_ptr(qi), _ptr(wi), _ptr(ki), _ptr(n_cmp), _ptr(out), Q, B, Hi, Di, N_max,
+                                     qps, _dtype_code(qi), _ptr(w), w.numel(), _stream(qi.device))
+    _lib.check("csa_index_scores", rc)
+    return out
+
+
+def topk(scores, n_cmp, k: int, out=None, ws: Workspace | None = None):
+    """Top-k of given fp32 scores [Q, N_max] (csa_topk). Returns int32 [Q, k]."""
+    _need(scores, "scores", dtype=torch.float32)
+    _need(n_cmp, "n_cmp", dtype=torch.int32, device=scores.device)
+    Q, N_max = scores.shape
+    if out is None:
+        out = torch.empty((Q, k), dtype=torch.int32, device=scores.device)
+    _need(out, "out", dtype=torch.int32, device=scores.device)
+    L = _lib.lib()
+    w = (ws or Workspace(scores.device)).get(L.csa_topk_workspace_bytes(Q, N_max, k))
+    rc = L.csa_topk(_ptr(scores), _ptr(n_cmp), int(k), _ptr(out), Q, N_max, _ptr(w), w.numel(),
+                    _stream(scores.device))
+    _lib.check("csa_topk", rc)
+    return out
+
+
+# ------------------------------------------------------------- A4 / A5
+
+def _mqa_common(q, kv_cmp, kv_win, win_end, sink, q_per_seq):
+    _need(q, "q")
+    _need(kv_cmp, "kv_cmp", dtype=q.dtype, device=q.device)
+    _need(kv_win, "kv_win", dtype=q.dtype, device=q.device)
+    _need(win_end, "win_end", dtype=torch.int32, device=q.device)
+    _need(sink, "sink", dtype=torch.float32, device=q.device)
+    Q, H, D = q.shape
+    B, N_max, D2 = kv_cmp.shape
+    B2, T_raw, D3 = kv_win.shape
+    if D2 != D or D3 != D or B2 != B or win_end.shape != (Q,) or sink.shape != (H,):
+        raise ValueError("shape mismatch among q [Q,H,D], kv_cmp [B,N,D], kv_win [B,T,D], win_end [Q], sink [H]")
+    if q_per_seq is None:
+        if Q % B:
+            raise ValueError("q_per_seq is required when B does not divide Q")
+        q_per_seq = Q // B
+    return Q, H, D, B, N_max, T_raw, q_per_seq
+
+
+def sparse_mqa(q, kv_cmp, idx, kv_win, win_end, sink, scale: float, win_len: int, q_per_seq=None, out=None,
+               ws: Workspace | None = None):
+    """CSA attention over the selected entries + window + sink (csa_sparse_mqa)."""
+    Q, H, D, B, N_max, T_raw, qps = _mqa_common(q, kv_cmp, kv_win, win_end, sink, q_per_seq)
+    _need(idx, "idx", dtype=torch.int32, device=q.device)
+    if idx.dim() != 2 or idx.shape[0] != Q:
+        raise ValueError("idx must be [Q, k]")
+    k = idx.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", dtype=q.dtype, device=q.device)
+    L = _lib.lib()
+    w = (ws or Workspace(q.device)).get(L.csa_mqa_workspace_bytes(Q, H, D, k + win_len))
+    rc = L.csa_sparse_mqa(_ptr(q), _ptr(kv_cmp), _ptr(idx), _ptr(kv_win), _ptr(sink), float(scale), _ptr(out), Q, B,
+                          H, D, N_max, k, int(win_len), _ptr(win_end), T_raw, qps, _dtype_code(q), _ptr(w),
+                          w.numel(), _stream(q.device))
+    _lib.check("csa_sparse_mqa", rc)
+    return out
+
+
+def hca_mqa(q, kv_cmp, n_cmp, kv_win, win_end, sink, scale: float, win_len: int, q_per_seq=None, out=None,
+            ws: Workspace | None = None):
+    """HCA attention over every visible entry + window + sink (hca_mqa)."""
+    Q, H, D, B, N_max, T_raw, qps = _mqa_common(q, kv_cmp, kv_win, win_end, sink, q_per_seq)
+    _need(n_cmp, "n_cmp", dtype=torch.int32, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", dtype=q.dtype, device=q.device)
+    L = _lib.lib()
+    w = (ws or Workspace(q.device)).get(L.csa_mqa_workspace_bytes(Q, H, D, N_max + win_len))
+    rc = L.hca_mqa(_ptr(q), _ptr(kv_cmp), _ptr(kv_win), _ptr(sink), float(scale), _ptr(out), Q, B, H, D, N_max,
+                   _ptr(n_cmp), int(win_len), _ptr(win_end), T_raw, qps, _dtype_code(q), _ptr(w), w.numel(),
+                   _stream(q.device))
+    _lib.check("hca_mqa", rc)
+    return out

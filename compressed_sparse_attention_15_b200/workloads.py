@@ -1,0 +1,147 @@
+"""The synthetic workloads of the CSA/HCA path: shapes, positions, buffer
+layout and the seeded recipe of every input tensor.
+
+Pure data: nothing here computes any step of the method. Every tensor is
+drawn by ``synth`` from (seed, tensor id, element index), so the host can
+regenerate any slice the fp64 oracle needs.
+
+Recipe (tensor id: distribution):
+  1 q      [Q, H, D]      N(0,1)      query heads (RoPE already applied)
+  2 kv_cmp [B, N, D]      N(0,1)      compressed KV cache
+  3 kv_win [B, T_raw, D]  N(0,1)      raw-KV buffer holding the window tokens
+  4 qi     [Q, Hi, Di]    N(0,1)      indexer query heads
+  5 wi     [Q, Hi]        U(0,1)      indexer per-head weights (fp32)
+  6 ki     [B, N, Di]     N(0,1)      indexer key cache
+  7 sink   [H]            N(0,1)      per-head sink logit (fp32)
+  8 kv_raw [1, T_c, D]    N(0,1)      raw KV fed to the compressor (1 M-token case)
+  9 gate   [Bc, T_c, D]   N(0,1)      compressor gate logits
+ 10 ape    [win, D]       N(0,0.1)    in-window position embedding (fp32)
+    norm_w [D]            1.0         RMSNorm weight (fp32)
+bf16 tensors are drawn in fp32 and rounded once to bf16 (RNE).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+from . import synth
+
+TID = {"q": 1, "kv_cmp": 2, "kv_win": 3, "qi": 4, "wi": 5, "ki": 6, "sink": 7, "kv_raw": 8, "gate": 9, "ape": 10}
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    mode: str            # "csa" (indexer + top-k + sparse MQA) or "hca" (dense MQA)
+    dtype: torch.dtype
+    B: int               # independent sequences
+    Q: int               # queries
+    H: int               # query heads (one shared KV head)
+    D: int               # head dim (K = V)
+    Hi: int              # indexer heads
+    Di: int              # indexer head dim
+    k: int               # top-k
+    W: int               # sliding window
+    win: int             # compressor window
+    stride: int          # compressor stride (= ratio)
+    N: int               # compressed entries per sequence (cache rows)
+    T_raw: int           # rows of the raw-KV window buffer per sequence
+    pos0: int            # absolute position of query 0 (queries of one sequence are consecutive)
+    raw0: int            # absolute position of kv_win row 0
+    # compressor run inside the workload: raw tokens [c_src0, c_src0 + T_c) of
+    # kv_win (or of kv_raw when c_from_raw) -> cache rows [c_dst0, c_dst0 + n)
+    T_c: int = 0
+    c_src0: int = 0
+    c_dst0: int = 0
+    c_from_raw: bool = False
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def q_per_seq(self) -> int:
+        return self.Q // self.B
+
+    def positions(self) -> torch.Tensor:
+        """Absolute token position p of every query (int64 [Q])."""
+        i = torch.arange(self.Q, dtype=torch.int64)
+        return self.pos0 + i % self.q_per_seq
+
+    def win_end(self) -> torch.Tensor:
+        """Row of kv_win holding each query's own token (int32 [Q])."""
+        return (self.positions() - self.raw0).to(torch.int32)
+
+
+def _csa(**kw):
+    return Workload(mode="csa", win=8, stride=4, **kw)
+
+
+WORKLOADS = {
+    # Tiny CSA prefill, fp32: every token of a 256-token sequence is a query.
+    "tiny_csa_prefill_fp32": _csa(
+        name="tiny_csa_prefill_fp32", dtype=torch.float32, B=1, Q=256, H=4, D=16, Hi=4, Di=16, k=16, W=16,
+        N=63, T_raw=256, pos0=0, raw0=0, T_c=256, c_src0=0, c_dst0=0),
+    # CSA decode at 64 K context, 32 sequences; the decode step also folds the
+    # newest window (tokens L-8 .. L-1) into the last cache row.
+    "csa_decode_64k": _csa(
+        name="csa_decode_64k", dtype=torch.bfloat16, B=32, Q=32, H=64, D=512, Hi=64, Di=128, k=512, W=128,
+        N=16383, T_raw=128, pos0=65535, raw0=65408, T_c=8, c_src0=120, c_dst0=16382),
+    # HCA decode at 1 M context, 16 sequences, dense over all 8,192 entries.
+    "hca_decode_1m": Workload(
+        name="hca_decode_1m", mode="hca", dtype=torch.bfloat16, B=16, Q=16, H=64, D=512, Hi=64, Di=128, k=0,
+        W=128, win=128, stride=128, N=8192, T_raw=128, pos0=1048575, raw0=1048448, T_c=128, c_src0=0,
+        c_dst0=8191),
+    # CSA prefill chunk: 4,096 new tokens after a 131,072-token context.
+    "csa_prefill_chunk_4k": _csa(
+        name="csa_prefill_chunk_4k", dtype=torch.bfloat16, B=1, Q=4096, H=64, D=512, Hi=64, Di=128, k=512,
+        W=128, N=33791, T_raw=4223, pos0=131072, raw0=130945, T_c=4100, c_src0=123, c_dst0=32767),
+    # CSA decode at 1 M context, 8 sequences, top-1024; sequence 0's cache is
+    # produced by compressing its 1,048,576 raw tokens.
+    "csa_decode_1m": _csa(
+        name="csa_decode_1m", dtype=torch.bfloat16, B=8, Q=8, H=64, D=512, Hi=64, Di=128, k=1024, W=128,
+        N=262143, T_raw=128, pos0=1048575, raw0=1048448, T_c=1048576, c_src0=0, c_dst0=0, c_from_raw=True),
+}
+
+
+def tensor_shape(w: Workload, name: str):
+    return {
+        "q": (w.Q, w.H, w.D), "kv_cmp": (w.B, w.N, w.D), "kv_win": (w.B, w.T_raw, w.D),
+        "qi": (w.Q, w.Hi, w.Di), "wi": (w.Q, w.Hi), "ki": (w.B, w.N, w.Di), "sink": (w.H,),
+        "kv_raw": (1, w.T_c, w.D), "ape": (w.win, w.D),
+        "gate": ((1 if w.c_from_raw else w.B), w.T_c, w.D),
+    }[name]
+
+
+def _dtype_of(w: Workload, name: str):
+    return torch.float32 if name in ("wi", "sink", "ape", "norm_w") else w.dtype
+
+
+def make(w: Workload, name: str, device="cpu") -> torch.Tensor:
+    """Materialise one input tensor of workload ``w`` on ``device``."""
+    shape = tensor_shape(w, name)
+    dt = _dtype_of(w, name)
+    if name == "wi":
+        return synth.uniform(w.seed, TID[name], shape, dtype=dt, device=device)
+    std = 0.1 if name == "ape" else 1.0
+    return synth.normal(w.seed, TID[name], shape, std=std, dtype=dt, device=device)
+
+
+def rows(w: Workload, name: str, flat_rows) -> torch.Tensor:
+    """Rows of a tensor (index into its flattened leading dims), regenerated
+    on the host in the workload dtype."""
+    shape = tensor_shape(w, name)
+    std = 0.1 if name == "ape" else 1.0
+    return synth.normal_rows(w.seed, TID[name], shape, flat_rows, std=std, dtype=_dtype_of(w, name))
+
+
+def norm_w(w: Workload, device="cpu") -> torch.Tensor:
+    return torch.ones(w.D, dtype=torch.float32, device=device)
+
+
+def small(w: Workload, **changes) -> Workload:
+    """A copy of ``w`` with some fields changed (test-size variants)."""
+    return dataclasses.replace(w, **changes)

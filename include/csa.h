@@ -1,0 +1,205 @@
+/*
+ * csa.h -- C ABI of libcsa.so: the hybrid compressed-sparse attention
+ * (CSA / HCA) hot path for DeepSeek-V4-Flash shapes on NVIDIA B200 (sm_100a).
+ *
+ * The method is described in prose in "DeepSeek-V4 Architecture Analysis"
+ * (architecture_analysis.py), INNOVATIONS section 1 "COMPRESSED SPARSE
+ * ATTENTION (CSA)" and section 2 "UNIFIED HEAD DIMENSION"; the shapes come
+ * from the "DeepSeek-V4-Flash" model card, table "Champs bruts du config.json"
+ * (head_dim 512, 64 query heads : 1 KV head, index_n_heads 64,
+ * index_head_dim 128, index_topk 512, sliding_window 128, rms_norm_eps 1e-6).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates or frees memory, never synchronises the stream, keeps no
+ *    state between calls and may be called from several host threads.
+ *  - Tensors are dense, row-major, in the element type `dtype`
+ *    (CSA_DTYPE_BF16 or CSA_DTYPE_F32) unless the argument says float / int32.
+ *    bf16 tensors whose row length is a multiple of 8 elements and whose base
+ *    is 16-byte aligned take the tensor-core / vectorised kernels; everything
+ *    else takes the generic kernels (same results within rounding).
+ *  - All arithmetic is fp32 (inputs widened from bf16, products accumulated in
+ *    fp32); outputs are rounded once to `dtype` (round to nearest even).
+ *  - Every argument is checked on the host before any launch. A failed check
+ *    returns a non-zero code and launches nothing.
+ *  - Values that live in device memory (visible counts, indices, window ends)
+ *    cannot be checked on the host: kernels clamp them to the valid range and
+ *    raise a bit in the workspace status word (read with
+ *    csa_workspace_status) instead of reading out of bounds.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Launches
+ *    are asynchronous; a returned CSA_OK means the work was enqueued.
+ *  - Workspaces: the caller passes `ws` (device memory, 256-byte aligned) of at
+ *    least the size the matching *_workspace_bytes() returns. Its first 256
+ *    bytes hold the status word; the library writes the rest freely. The
+ *    status word must be zero before the first call (cudaMemset once); calls
+ *    only ever OR bits into it.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *csa_stream_t; /* identical to cudaStream_t */
+
+/* Return codes. */
+enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID = 1,     /* null pointer, bad size, bad alignment, ratio != stride, k too large */
+  CSA_ERR_UNSUPPORTED = 2, /* no sm_100 device current, or an uncompiled size/dtype combination */
+  CSA_ERR_WORKSPACE = 3,   /* workspace smaller than *_workspace_bytes() */
+  CSA_ERR_CUDA = 4,        /* a CUDA launch or attribute call failed */
+  CSA_ERR_DEVICE = 5       /* (csa_workspace_status only) the status word is non-zero */
+};
+
+/* Element types of the dtype-typed tensors. */
+enum { CSA_DTYPE_F32 = 0, CSA_DTYPE_BF16 = 1 };
+
+/* Bits of the workspace status word. */
+enum {
+  CSA_STATUS_BAD_COUNT = 1u,   /* an n_cmp value was < 0 or > N_max; it was clamped */
+  CSA_STATUS_BAD_INDEX = 2u,   /* an idx value was < -1 or >= N_max; the row was skipped */
+  CSA_STATUS_BAD_WINDOW = 4u,  /* a win_end value was < 0 or >= T_raw; it was clamped */
+  CSA_STATUS_WAIT_TIMEOUT = 8u /* a bounded pipeline wait gave up; that output is invalid */
+};
+
+/* Largest supported top-k. */
+#define CSA_MAX_TOPK 2048
+
+/* Human-readable name of a return code (static string, never NULL). */
+const char *csa_strerror(int code);
+
+/* ------------------------------------------------------------------------
+ * csa_compress -- gated-pooling KV compressor followed by RMSNorm.
+ *
+ * Defined by "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: a
+ * learned gated pooling folds the raw per-token KV of each window into one
+ * entry ("4 tokens -> 1, with overlapping windows" for CSA, "128 tokens -> 1"
+ * for HCA), using absolute position embeddings within the window and an
+ * RMSNorm on the compressed output. For every sequence b, entry j over tokens
+ * t = j*stride + i (i = 0..win-1) and dimension d:
+ *     a[i,d]   = softmax over i of (gate[b,t,d] + ape[i,d])
+ *     c[d]     = sum_i a[i,d] * kv[b,t,d]
+ *     out[b,j] = c / sqrt(mean_d c[d]^2 + 1e-6) * norm_w
+ * Entries j = 0 .. N-1 with N = (T - win) / stride + 1 (a trailing partial
+ * window makes no entry; T < win is an error). CSA uses win 8 / stride 4,
+ * HCA win 128 / stride 128.
+ *
+ *   kv, gate : [B, T, D] dtype; sequence b starts at b * kv_seq_stride
+ *              (resp. gate_seq_stride) elements; 0 means T * D.
+ *   ape      : [win, D] float32.        norm_w : [D] float32.
+ *   ratio    : the compression ratio; must equal `stride`.
+ *   out      : [B, N, D] dtype; sequence b starts at b * out_seq_stride
+ *              elements (0 means N * D), so entries may be written straight
+ *              into a larger cache.
+ * Limits: 1 <= win <= 128, 1 <= stride, 1 <= D <= 4096, B >= 1.
+ * ---------------------------------------------------------------------- */
+int csa_compress(const void *kv, const void *gate, const float *ape, const float *norm_w,
+                 int ratio, int win, int stride, void *out,
+                 int B, int T, int D,
+                 long long kv_seq_stride, long long gate_seq_stride, long long out_seq_stride,
+                 int dtype, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa_index_topk -- indexer scores and top-k selection of compressed entries.
+ *
+ * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1, Indexer: a
+ * learned scorer "selects top-k compressed positions" using "dot-product
+ * attention + per-head importance weights". For query q of sequence
+ * b = q / q_per_seq and every visible entry j < n_cmp[q]:
+ *     s[q,j] = sum_h wi[q,h] * max(0, qi[q,h,:] . ki[b,j,:])     (no scale)
+ * and out_idx[q] holds the min(k, n_cmp[q]) entries of largest score, ties
+ * resolved towards the smaller j, written in ascending j, followed by -1
+ * padding up to k. Scores are fp32 (bf16 products, fp32 accumulation).
+ *
+ *   qi      : [Q, Hi, Di] dtype.        wi : [Q, Hi] float32.
+ *   ki      : [B, N_max, Di] dtype (indexer keys, one cache per sequence).
+ *   n_cmp   : [Q] int32 device array, number of entries visible to query q
+ *             (0 .. N_max); covers decode (all N) and causal prefill alike.
+ *   out_idx : [Q, k] int32.
+ * Limits: 1 <= k <= CSA_MAX_TOPK, Hi <= 128, Di <= 256, Q, B >= 1, 1 <= N_max <= 2^22,
+ * B * q_per_seq >= Q.
+ * Workspace: csa_index_topk_workspace_bytes(Q, N_max, k).
+ * ---------------------------------------------------------------------- */
+size_t csa_index_topk_workspace_bytes(int Q, int N_max, int k);
+int csa_index_topk(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp,
+                   int k, int32_t *out_idx,
+                   int Q, int B, int Hi, int Di, int N_max, int q_per_seq, int dtype,
+                   void *ws, size_t ws_bytes, csa_stream_t stream);
+
+/* The two halves of csa_index_topk, exposed so each can be driven alone.
+ * csa_index_scores writes scores[q, j] (float32, row stride N_max) for
+ * j < n_cmp[q] and leaves the rest of the row untouched.
+ * csa_topk selects from given float32 scores with the same rule as above
+ * (-0.0 and +0.0 compare equal); it reads scores[q, j] for j < n_cmp[q] only. */
+int csa_index_scores(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp,
+                     float *scores, int Q, int B, int Hi, int Di, int N_max, int q_per_seq,
+                     int dtype, void *ws, size_t ws_bytes, csa_stream_t stream);
+size_t csa_topk_workspace_bytes(int Q, int N_max, int k);
+int csa_topk(const float *scores, const int32_t *n_cmp, int k, int32_t *out_idx,
+             int Q, int N_max, void *ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa_sparse_mqa -- MQA over the selected compressed entries, the sliding
+ * window of raw tokens and a per-head attention sink.
+ *
+ * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1 (sliding window:
+ * each token attends to its nearest 128 tokens; attention sink: a learnable
+ * per-head scalar) and section 2 (key and value share one head_dim = 512
+ * representation: K = V). For query q of sequence b = q / q_per_seq, head h:
+ *     rows    = { kv_cmp[b, idx[q,r]] : idx[q,r] >= 0 }
+ *             U { kv_win[b, t] : max(0, e - win_len + 1) <= t <= e },  e = win_end[q]
+ *     logit_r = scale * q[q,h,:] . row_r ;  the sink adds sink[h] (unscaled)
+ *               to the softmax denominator with a zero value
+ *     out[q,h] = sum_r softmax_r * row_r
+ * The window is not de-duplicated against compressed rows.
+ *
+ *   q       : [Q, H, D] dtype (RoPE already applied).
+ *   kv_cmp  : [B, N_max, D] dtype compressed cache.
+ *   idx     : [Q, k] int32 (-1 = unused slot).
+ *   kv_win  : [B, T_raw, D] dtype raw-KV buffer holding the window tokens.
+ *   win_end : [Q] int32 device array, row of kv_win holding query q's token.
+ *   sink    : [H] float32.      out : [Q, H, D] dtype.
+ * Limits: H <= 128, D <= 1024, k + win_len <= 65536, win_len >= 1.
+ * Workspace: csa_mqa_workspace_bytes(Q, H, D, k + win_len).
+ * ---------------------------------------------------------------------- */
+size_t csa_mqa_workspace_bytes(int Q, int H, int D, int rows_max);
+int csa_sparse_mqa(const void *q, const void *kv_cmp, const int32_t *idx, const void *kv_win,
+                   const float *sink, float scale, void *out,
+                   int Q, int B, int H, int D, int N_max, int k, int win_len,
+                   const int32_t *win_end, int T_raw, int q_per_seq, int dtype,
+                   void *ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * hca_mqa -- the dense (heavily compressed, 128 tokens -> 1) variant: as
+ * csa_sparse_mqa but over every visible compressed entry j < n_cmp[q]
+ * instead of an index list ("DeepSeek-V4 Architecture Analysis",
+ * INNOVATIONS section 1, "HCA (128:1): heavy compression for global
+ * context").
+ *   n_cmp : [Q] int32 device array (0 .. N_max).
+ * Workspace: csa_mqa_workspace_bytes(Q, H, D, N_max + win_len).
+ * ---------------------------------------------------------------------- */
+int hca_mqa(const void *q, const void *kv_cmp, const void *kv_win, const float *sink,
+            float scale, void *out,
+            int Q, int B, int H, int D, int N_max, const int32_t *n_cmp, int win_len,
+            const int32_t *win_end, int T_raw, int q_per_seq, int dtype,
+            void *ws, size_t ws_bytes, csa_stream_t stream);
+
+/* Number of kernels this library has launched in this process so far
+ * (a monotonically increasing counter, for profiling and tests). */
+unsigned long long csa_launch_count(void);
+
+/* Synchronises `stream`, copies the workspace status word into *status and
+ * clears it. Returns CSA_OK if it was zero, CSA_ERR_DEVICE if not,
+ * CSA_ERR_CUDA if the copy failed. Test/debug use. */
+int csa_workspace_status(void *ws, csa_stream_t stream, uint32_t *status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H_ */

@@ -1,0 +1,112 @@
+"""A2 indexer scores and A3 top-k: CUDA vs the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from compressed_sparse_attention_15_b200 import ops, synth, workloads as WL
+from helpers import check_topk_set, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _score_inputs(seed, Q, B, N, Hi, Di, dtype):
+    qi = synth.normal(seed, 4, (Q, Hi, Di), dtype=dtype)
+    wi = synth.uniform(seed, 5, (Q, Hi))
+    ki = synth.normal(seed, 6, (B, N, Di), dtype=dtype)
+    return qi, wi, ki
+
+
+@pytest.mark.parametrize("Q,B,N,Hi,Di,dtype", [
+    (256, 1, 63, 4, 16, torch.float32),      # the tiny configuration
+    (6, 3, 1000, 64, 128, torch.bfloat16),   # Flash indexer shape, ragged tail
+    (5, 5, 300, 8, 32, torch.bfloat16),
+    (4, 2, 129, 64, 128, torch.float32),
+])
+def test_index_scores_match_oracle(cuda_device, Q, B, N, Hi, Di, dtype):
+    qi, wi, ki = _score_inputs(1, Q, B, N, Hi, Di, dtype)
+    qps = Q // B
+    # ragged visible counts, including 0, 1 and N
+    n = torch.tensor([[N, 0, 1, N - 1, N // 2, 17][q % 6] for q in range(Q)], dtype=torch.int32)
+    s = ops.index_scores(qi.to(cuda_device), wi.to(cuda_device), ki.to(cuda_device), n.to(cuda_device),
+                         q_per_seq=qps).cpu()
+    for q in range(Q):
+        nv = int(n[q])
+        ref = O.index_scores(qi[q], wi[q], ki[q // qps], nv)
+        got = f64(s[q, :nv])
+        scale = max(np.abs(ref).max(initial=0.0), 1.0)
+        assert np.max(np.abs(got - ref), initial=0.0) <= 2e-5 * scale * (1 if dtype == torch.float32 else 5)
+        assert torch.isnan(s[q, nv:]).all()  # untouched beyond the visible count
+
+
+@pytest.mark.parametrize("N,k", [(1, 1), (100, 100), (101, 100), (1000, 16), (5000, 512), (20000, 2048),
+                                 (262143, 1024)])
+def test_topk_exact_on_given_scores(cuda_device, N, k):
+    # Both sides select from the same fp32 scores: bit-exact index sets.
+    # Scores are quantised so that ties (including +0 / -0) are frequent.
+    Q = 3
+    u = synth.uniform(4, 12, (Q, N))
+    s = torch.floor(u * 50) - 25.0
+    s[s == 0] = -0.0
+    s[1] = u[1]                          # a row without ties
+    n = torch.tensor([N, max(0, N - 7), N // 2], dtype=torch.int32)
+    got = ops.topk(s.to(cuda_device), n.to(cuda_device), k).cpu().numpy()
+    for q in range(Q):
+        nv = int(n[q])
+        want = O.topk(f64(s[q, :nv]), k)
+        m = min(k, nv)
+        assert np.array_equal(np.sort(want[:m]), got[q, :m]), f"query {q}"
+        assert np.all(got[q, m:] == -1)
+
+
+def test_topk_all_equal_scores_take_smallest_indices(cuda_device):
+    s = torch.zeros((2, 5000))
+    s[1, ::2] = -0.0
+    n = torch.tensor([5000, 4000], dtype=torch.int32)
+    got = ops.topk(s.to(cuda_device), n.to(cuda_device), 300).cpu().numpy()
+    assert np.array_equal(got[0], np.arange(300)) and np.array_equal(got[1], np.arange(300))
+
+
+@pytest.mark.parametrize("Q,B,N,Hi,Di,k,dtype", [
+    (256, 1, 63, 4, 16, 16, torch.float32),    # tiny: causal, many exact-zero ties
+    (4, 4, 3000, 64, 128, 512, torch.bfloat16),
+    (3, 1, 700, 64, 128, 2048, torch.bfloat16),  # k > n: everything kept, padded
+])
+def test_index_topk_matches_oracle(cuda_device, Q, B, N, Hi, Di, k, dtype):
+    qi, wi, ki = _score_inputs(2, Q, B, N, Hi, Di, dtype)
+    qps = Q // B
+    if Q == 256:
+        n = ops.visible_entries(torch.arange(Q), 8, 4)   # causal prefill positions 0..255
+    else:
+        n = torch.full((Q,), N, dtype=torch.int32)
+    idx = ops.index_topk(qi.to(cuda_device), wi.to(cuda_device), ki.to(cuda_device), n.to(cuda_device), k,
+                         q_per_seq=qps).cpu().numpy()
+    swaps = 0
+    for q in range(Q):
+        nv = int(n[q])
+        ref_idx, ref_s = O.index_topk(qi[q], wi[q], ki[q // qps], q if Q == 256 else 4 * (N - 1) + 7, k, 8, 4)
+        assert O.n_visible(q if Q == 256 else 4 * (N - 1) + 7, 8, 4) == nv
+        swaps += check_topk_set(idx[q], ref_idx, ref_s, k, nv)
+    assert swaps <= max(2, Q // 8)
+
+
+@pytest.mark.parametrize("name,nq", [("csa_decode_64k", 32), ("csa_decode_1m", 8), ("csa_prefill_chunk_4k", 24)])
+def test_index_topk_full_size(cuda_device, name, nq):
+    # Full-size workloads in the benchmark's launch configuration; the
+    # oracle checks nq queries (all of them for the decode batches).
+    w = WL.WORKLOADS[name]
+    qi, wi, ki = (WL.make(w, t, cuda_device) for t in ("qi", "wi", "ki"))
+    p = w.positions()
+    n = ops.visible_entries(p, w.win, w.stride)
+    idx = ops.index_topk(qi, wi, ki, n.to(cuda_device), w.k, q_per_seq=w.q_per_seq).cpu().numpy()
+    del ki
+    qs = np.unique(np.linspace(0, w.Q - 1, nq).round().astype(int))
+    seqs = sorted({int(q) // w.q_per_seq for q in qs})
+    ki_h = {b: WL.rows(w, "ki", torch.arange(b * w.N, (b + 1) * w.N)) for b in seqs}
+    qi_h, wi_h = WL.make(w, "qi"), WL.make(w, "wi")
+    swaps = 0
+    for q in qs:
+        b = int(q) // w.q_per_seq
+        ref_idx, ref_s = O.index_topk(qi_h[q], wi_h[q], ki_h[b], int(p[q]), w.k, w.win, w.stride)
+        swaps += check_topk_set(idx[q], ref_idx, ref_s, w.k, int(n[q]))
+    assert swaps <= max(2, len(qs) // 4)
