@@ -366,7 +366,7 @@ def time_oracle(w: WL.Workload, steps: int, budget_s: float):
             rows_c = O.round_to(WL.rows(w, "kv_cmp", b * w.N + torch.as_tensor(sel)), "bf16")
             rows_c[sel == w.c_dst0] = new[0]
             e = int(w.win_end()[q])
-            rows_w = O._f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(max(0, e - w.W + 1), e + 1)))
+            rows_w = O.as_f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(max(0, e - w.W + 1), e + 1)))
             t0 = time.perf_counter()
             O.attend(host["q"][q], np.concatenate([rows_c, rows_w]), host["sink"], w.scale)
             total += time.perf_counter() - t0

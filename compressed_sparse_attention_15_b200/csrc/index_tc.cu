@@ -1,14 +1,266 @@
-// A2 on the tensor cores (tcgen05 + TMA) for the Flash indexer shape.
+// A2 on the tensor cores for the Flash indexer shape (64 heads x 128 dims,
+// bf16): s[q,j] = sum_h wi[q,h] * max(0, qi[q,h] . ki[b,j])
+// ("DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1, Indexer;
+// index_n_heads = 64, index_head_dim = 128 in the model card's config.json).
+//
+// Layout of the contraction: the compressed keys are the MMA's M dimension
+// (128 entries per tile), the 64 heads its N, the 128 dims its K. One tile is
+// 8 tcgen05.mma (M128 N64 K16) into a 128-lane x 64-column fp32 TMEM
+// accumulator, so each epilogue thread owns one entry's 64 head products and
+// the weighted ReLU sum over heads is thread-local.
+//
+// Pipeline (persistent, one CTA per SM, 192 threads):
+//   warp 0      TMA producer: 32 KB key tiles into a 5-stage ring, and the
+//               query's 16 KB head block into one of two query slots;
+//   warp 1      MMA issuer (one thread) and TMEM owner (2 accumulators);
+//   warps 2..5  epilogue: tcgen05.ld, ReLU, weighted sum, coalesced store.
+// Each CTA walks a contiguous range of the flat (query, tile) space. Every
+// wait is bounded; a timeout raises CSA_STATUS_WAIT_TIMEOUT, all roles stop,
+// in-flight copies and MMAs are drained (bounded) and TMEM is freed.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
+#include "tmap.h"
 
 namespace csa {
 
+namespace {
+
+constexpr int kHi = 64, kDi = 128;
+constexpr int kTileM = 128;
+constexpr int kStages = 5;
+constexpr uint32_t kTileBytes = kTileM * kDi * 2;  // 32 KB
+constexpr uint32_t kHalfTile = kTileBytes / 2;     // one 64-dim box
+constexpr uint32_t kQBytes = kHi * kDi * 2;        // 16 KB
+constexpr uint32_t kQHalf = kQBytes / 2;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 128;
+
+struct Bars {
+  uint64_t full[kStages], empty[kStages], qfull[2], qempty[2], accfull[2], accempty[2], mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + 2 * kQBytes + sizeof(Bars);
+
+struct Tile {
+  int q, j0, n;
+};
+
+__device__ __forceinline__ Tile tile_of(long long t, int tiles_per_q, const ScoreArgs &a) {
+  Tile r;
+  r.q = (int)(t / tiles_per_q);
+  r.j0 = (int)(t - (long long)r.q * tiles_per_q) * kTileM;
+  int n = a.n_cmp[r.q];
+  r.n = n < 0 ? 0 : (n > a.N_max ? a.N_max : n);
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
+                           ScoreArgs a, int tiles_per_q, long long total, long long per_cta) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *stage_buf = smem;
+  uint8_t *q_buf = smem + kStages * kTileBytes;
+  Bars *bars = reinterpret_cast<Bars *>(q_buf + 2 * kQBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long t_begin = (long long)blockIdx.x * per_cta;
+  const long long t_end = min(total, t_begin + per_cta);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&bars->full[s], 1);
+      tc::mbar_init(&bars->empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->qfull[s], 1);
+      tc::mbar_init(&bars->qempty[s], 1);
+      tc::mbar_init(&bars->accfull[s], 1);
+      tc::mbar_init(&bars->accempty[s], 4 * 32);
+    }
+    tc::mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int *abort = &bars->abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_ki);
+      tc::prefetch_tmap(&tm_qi);
+      int stage = 0, nq = 0, cur_q = -1;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;  // per stage: a load was issued, with this parity
+      for (long long t = t_begin; t < t_end && !*abort; ++t) {
+        const Tile tl = tile_of(t, tiles_per_q, a);
+        if (tl.j0 >= tl.n) continue;
+        if (tl.q != cur_q) {
+          const int slot = nq & 1;
+          const uint32_t qph = (nq >> 1) & 1;
+          if (!tc::mbar_wait(&bars->qempty[slot], qph ^ 1, abort, a.status)) break;
+          tc::mbar_arrive_expect_tx(&bars->qfull[slot], kQBytes);
+          tc::tma_load_2d(q_buf + slot * kQBytes, &tm_qi, 0, tl.q * kHi, &bars->qfull[slot]);
+          tc::tma_load_2d(q_buf + slot * kQBytes + kQHalf, &tm_qi, 64, tl.q * kHi, &bars->qfull[slot]);
+          ++nq;
+          cur_q = tl.q;
+        }
+        if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort, a.status)) break;
+        tc::mbar_arrive_expect_tx(&bars->full[stage], kTileBytes);
+        const int row = (tl.q / a.q_per_seq) * a.N_max + tl.j0;
+        tc::tma_load_2d(stage_buf + stage * kTileBytes, &tm_ki, 0, row, &bars->full[stage]);
+        tc::tma_load_2d(stage_buf + stage * kTileBytes + kHalfTile, &tm_ki, 64, row, &bars->full[stage]);
+        issued_mask |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      // Drain: every load issued must have landed before the CTA may exit.
+      // A phase that was already consumed completes the wait at once.
+      for (int s = 0; s < kStages; ++s)
+        if (issued_mask & (1u << s)) tc::mbar_drain(&bars->full[s], (issued_phase >> s) & 1);
+      for (int i = nq - 1; i >= 0 && i >= nq - 2; --i) tc::mbar_drain(&bars->qfull[i & 1], (i >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
+      int stage = 0, acc = 0, nq = 0, cur_q = -1, slot = 0;
+      uint32_t phase = 0, accph = 0;
+      for (long long t = t_begin; t < t_end && !*abort; ++t) {
+        const Tile tl = tile_of(t, tiles_per_q, a);
+        if (tl.j0 >= tl.n) continue;
+        if (tl.q != cur_q) {
+          if (cur_q >= 0) tc::commit(&bars->qempty[slot]);  // old head block free once its MMAs finish
+          slot = nq & 1;
+          if (!tc::mbar_wait(&bars->qfull[slot], (nq >> 1) & 1, abort, a.status)) break;
+          ++nq;
+          cur_q = tl.q;
+        }
+        if (!tc::mbar_wait(&bars->accempty[acc], accph ^ 1, abort, a.status)) break;
+        if (!tc::mbar_wait(&bars->full[stage], phase, abort, a.status)) break;
+        tc::fence_after_sync();
+        const uint32_t a_base = tc::smem_u32(stage_buf + stage * kTileBytes);
+        const uint32_t b_base = tc::smem_u32(q_buf + slot * kQBytes);
+#pragma unroll
+        for (int kk = 0; kk < kDi / 16; ++kk) {
+          const uint64_t ad = tc::sw128_desc(a_base + (kk >> 2) * kHalfTile + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(b_base + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024);
+          tc::mma_bf16(tmem + acc * 64, ad, bd, idesc, kk > 0);
+        }
+        tc::commit(&bars->empty[stage]);
+        tc::commit(&bars->accfull[acc]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++acc == 2) {
+          acc = 0;
+          accph ^= 1;
+        }
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      tc::commit(&bars->mma_done);
+      tc::mbar_drain(&bars->mma_done, 0);
+    }
+  } else {
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;
+    int acc = 0, cur_q = -1;
+    uint32_t accph = 0;
+    float w[kHi];
+    for (long long t = t_begin; t < t_end && !*abort; ++t) {
+      const Tile tl = tile_of(t, tiles_per_q, a);
+      if (tl.j0 >= tl.n) continue;
+      if (tl.q != cur_q) {
+        const int raw = a.n_cmp[tl.q];
+        if ((raw < 0 || raw > a.N_max) && row == 0) raise_status(a.status, CSA_STATUS_BAD_COUNT);
+#pragma unroll
+        for (int h = 0; h < kHi; h += 4) {
+          const float4 v = __ldg(reinterpret_cast<const float4 *>(a.wi + (size_t)tl.q * kHi + h));
+          w[h] = v.x;
+          w[h + 1] = v.y;
+          w[h + 2] = v.z;
+          w[h + 3] = v.w;
+        }
+        cur_q = tl.q;
+      }
+      const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
+      tc::fence_after_sync();
+      uint32_t v0[32], v1[32];
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * 64;
+      tc::tmem_ld32(taddr, v0);
+      tc::tmem_ld32(taddr + 32, v1);
+      tc::tmem_ld_wait();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars->accempty[acc]);
+      float s = 0.f;
+#pragma unroll
+      for (int h = 0; h < 32; ++h) s = fmaf(w[h], fmaxf(__uint_as_float(v0[h]), 0.f), s);
+#pragma unroll
+      for (int h = 0; h < 32; ++h) s = fmaf(w[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s);
+      const int j = tl.j0 + row;
+      if (j < tl.n) a.scores[(size_t)tl.q * a.N_max + j] = s;
+      if (++acc == 2) {
+        acc = 0;
+        accph ^= 1;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+int num_sms_cached() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
 cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool *taken) {
-  (void)a;
-  (void)stream;
   *taken = false;
-  return cudaSuccess;
+  if (a.dtype != CSA_DTYPE_BF16 || a.Hi != kHi || a.Di != kDi) return cudaSuccess;
+  if (!aligned16(a.qi) || !aligned16(a.ki) || (reinterpret_cast<uintptr_t>(a.wi) & 15)) return cudaSuccess;
+  CUtensorMap tm_ki, tm_qi;
+  if (!make_tmap_bf16_2d(&tm_ki, a.ki, kDi, (uint64_t)a.B * a.N_max, kDi * 2, 64, kTileM)) return cudaSuccess;
+  if (!make_tmap_bf16_2d(&tm_qi, a.qi, kDi, (uint64_t)a.Q * kHi, kDi * 2, 64, kHi)) return cudaSuccess;
+  const int tiles_per_q = (a.N_max + kTileM - 1) / kTileM;
+  const long long total = (long long)a.Q * tiles_per_q;
+  long long grid = num_sms_cached();
+  if (grid > total) grid = total;
+  const long long per_cta = (total + grid - 1) / grid;
+  grid = (total + per_cta - 1) / per_cta;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    attr_set = true;
+  }
+  index_scores_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(tm_ki, tm_qi, a, tiles_per_q, total,
+                                                                             per_cta);
+  note_launches(1);
+  *taken = true;
+  return cudaGetLastError();
 }
 
 }  // namespace csa

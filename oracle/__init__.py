@@ -5,6 +5,7 @@ Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 """
 from .csa_oracle import (  # noqa: F401
     RMS_EPS,
+    as_f64,
     attend,
     compress,
     hca_mqa,

@@ -58,7 +58,7 @@ import numpy as np
 RMS_EPS = 1e-6
 
 
-def _f64(x) -> np.ndarray:
+def as_f64(x) -> np.ndarray:
     """Exact conversion to float64 (bf16 and fp32 values are representable)."""
     try:  # torch tensors (bf16 has no numpy dtype): widen in torch first
         import torch
@@ -86,9 +86,9 @@ def rms_norm(c: np.ndarray, norm_w: np.ndarray, eps: float = RMS_EPS) -> np.ndar
     """RMSNorm over the last axis (model card: rms_norm_eps = 1e-6; the
     architecture analysis, INNOVATIONS section 1: "RMSNorm on compressed
     output")."""
-    c = _f64(c)
+    c = as_f64(c)
     rms = np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + eps)
-    return c / rms * _f64(norm_w)
+    return c / rms * as_f64(norm_w)
 
 
 def compress(kv, gate, ape, norm_w, win: int, stride: int, eps: float = RMS_EPS,
@@ -108,9 +108,9 @@ def compress(kv, gate, ape, norm_w, win: int, stride: int, eps: float = RMS_EPS,
         out     = RMSNorm(c) * norm_w
     With ``pre_norm`` the pooled c is returned without the norm.
     """
-    kv = _f64(kv)
-    gate = _f64(gate)
-    ape = _f64(ape)
+    kv = as_f64(kv)
+    gate = as_f64(gate)
+    ape = as_f64(ape)
     T, D = kv.shape
     assert gate.shape == (T, D) and ape.shape == (win, D)
     N = n_entries(T, win, stride)
@@ -153,9 +153,9 @@ def index_scores(qi, wi, ki, n_vis: int) -> np.ndarray:
     attention + per-head importance weights"); reading R9:
         s_j = sum_h wi[h] * max(0, qi[h] . ki[j]),  j < n_vis.
     """
-    qi = _f64(qi)
-    wi = _f64(wi)
-    ki = _f64(ki)[:n_vis]
+    qi = as_f64(qi)
+    wi = as_f64(wi)
+    ki = as_f64(ki)[:n_vis]
     dots = ki @ qi.T                     # [n_vis, Hi]
     return np.maximum(dots, 0.0) @ wi    # [n_vis]
 
@@ -166,7 +166,7 @@ def topk(scores, k: int) -> np.ndarray:
     Order (reading R10): score descending, ties by index ascending. A full
     stable sort is the definition (model card: index_topk = 512).
     """
-    s = _f64(scores)
+    s = as_f64(scores)
     n = s.shape[0]
     order = np.lexsort((np.arange(n), -s))   # last key is primary
     out = np.full(k, -1, dtype=np.int64)
@@ -198,9 +198,9 @@ def attend(q, rows, sink, scale: float):
         out_h = sum_r p_r * row_r.
     Returns (out [H, D], p [H, R], p_sink [H]).
     """
-    q = _f64(q)
-    rows = _f64(rows)
-    sink = _f64(sink)
+    q = as_f64(q)
+    rows = as_f64(rows)
+    sink = as_f64(sink)
     H = q.shape[0]
     R = rows.shape[0]
     logits = scale * (q @ rows.T) if R else np.zeros((H, 0))
@@ -219,7 +219,7 @@ def window_rows(kv_win, win_end: int, W: int) -> np.ndarray:
     is the buffer row of the query's own token (architecture analysis,
     INNOVATIONS section 1: each token attends to its nearest 128 tokens;
     reading R8: the query's own token is included)."""
-    kv_win = _f64(kv_win)
+    kv_win = as_f64(kv_win)
     lo = max(0, win_end - W + 1)
     return kv_win[lo:win_end + 1]
 
@@ -228,7 +228,7 @@ def sparse_mqa(q, kv_cmp, idx, kv_win, win_end: int, W: int, sink, scale: float)
     """CSA attention for one query: the selected compressed rows (entries
     idx >= 0 of this sequence's compressed cache), the sliding window and
     the sink. Returns out [H, D] (float64)."""
-    kv_cmp = _f64(kv_cmp)
+    kv_cmp = as_f64(kv_cmp)
     idx = np.asarray(idx)
     sel = kv_cmp[idx[idx >= 0]]
     rows = np.concatenate([sel, window_rows(kv_win, win_end, W)], axis=0)
@@ -239,7 +239,7 @@ def hca_mqa(q, kv_cmp, n_cmp: int, kv_win, win_end: int, W: int, sink, scale: fl
     """HCA attention for one query: every visible compressed entry
     (architecture analysis, INNOVATIONS section 1: HCA, 128 tokens -> 1, for
     global context, with no indexer), the sliding window and the sink."""
-    kv_cmp = _f64(kv_cmp)[:n_cmp]
+    kv_cmp = as_f64(kv_cmp)[:n_cmp]
     rows = np.concatenate([kv_cmp, window_rows(kv_win, win_end, W)], axis=0)
     return attend(q, rows, sink, scale)[0]
 
@@ -252,7 +252,7 @@ def round_to(x, dtype: str) -> np.ndarray:
     """Round float64 values once to 'fp32' or 'bf16' (round to nearest even)
     and return them as float64. bf16 is a single rounding from fp64 to 8
     significant bits (normal range only)."""
-    x = _f64(x)
+    x = as_f64(x)
     if dtype == "fp64":
         return x.copy()
     if dtype == "fp32":

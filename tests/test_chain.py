@@ -68,7 +68,7 @@ def test_csa_decode_step_chain(cuda_device):
         gate = WL.rows(w, "gate", b * w.T_c + torch.arange(w.T_c))
         new = O.round_to(O.compress(raw, gate, ape, np.ones(w.D), w.win, w.stride), "bf16")[0]
         rows_c[sel == w.c_dst0] = new
-        rows_w = O._f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.T_raw)))
+        rows_w = O.as_f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.T_raw)))
         qh = WL.rows(w, "q", q * w.H + torch.arange(w.H))
         ref = O.attend(qh, np.concatenate([rows_c, rows_w]), sink, w.scale)[0]
         assert_close(out[q], ref, torch.bfloat16, f"decode chain q={q}")
