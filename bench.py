@@ -112,6 +112,12 @@ class Step:
         ops.compress(t["kv_win"][:, w.c_src0:w.c_src0 + w.T_c], t["gate"], t["ape"], self.norm_w, w.win, w.stride,
                      out=t["kv_cmp"][:, w.c_dst0:w.c_dst0 + (w.T_c - w.win) // w.stride + 1])
 
+    def bulk_compress(self):
+        """The one-off compression of sequence 0's whole raw history."""
+        w, t = self.w, self.t
+        ops.compress(t["kv_raw"], t["gate_raw"], t["ape"], self.norm_w, w.win, w.stride,
+                     out=t["kv_cmp"][0:1, :(w.bulk_T - w.win) // w.stride + 1])
+
     def select(self):
         t = self.t
         ops.index_topk(t["qi"], t["wi"], t["ki"], self.n_cmp, self.w.k, out=self.idx, ws=self.ws_index)
@@ -271,6 +277,35 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     del graph
     return {"ms": ms_max, "ms_local": ms, "per_kernel_ms": per, "launches_per_step": int(launches_per_step),
             "wall_s": wall, "clocks": clocks.summary(), "status": status, "K": K, "step": step}
+
+
+def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
+    """The one-off compression of a 1 M-token raw sequence (kv_raw, gate_raw
+    [1, bulk_T, 512] bf16 -> [1, (bulk_T - 8)/4 + 1, 512]), timed alone."""
+    kv = WL.make(w, "kv_raw", device)
+    gate = WL.make(w, "gate_raw", device)
+    ape = WL.make(w, "ape", device)
+    nw = WL.norm_w(w, device)
+    n = (w.bulk_T - w.win) // w.stride + 1
+    out = torch.empty((1, n, w.D), dtype=w.dtype, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(3):
+        ops.compress(kv, gate, ape, nw, w.win, w.stride, out=out)
+    K = max(5, args.steps // 4)
+    ms = 0.0
+    for _ in range(K):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ops.compress(kv, gate, ape, nw, w.win, w.stride, out=out)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms += a.elapsed_time(b) / K
+    nbytes = 2 * w.bulk_T * w.D * 2 + n * w.D * 2 + w.win * w.D * 4 + w.D * 4
+    gbps = nbytes / (ms * 1e-3) / 1e9
+    return {"tokens": w.bulk_T, "entries": n, "ms": round(ms, 4), "GBps": round(gbps, 1),
+            "frac": round(gbps / hbm_gbs, 4), "bytes": nbytes, "tokens_per_s": round(w.bulk_T / (ms * 1e-3), 1)}
 
 
 def roofline_of(w, per_kernel_ms, hbm_gbs, traffic=None):
@@ -464,6 +499,11 @@ def main():
             except Exception as ex:  # report, do not hide
                 secondary[name] = {"error": repr(ex)}
             torch.cuda.empty_cache()
+        try:
+            secondary["compress_1m_tokens"] = time_bulk_compress(args, WL.WORKLOADS["csa_decode_1m"], device, hbm)
+        except Exception as ex:
+            secondary["compress_1m_tokens"] = {"error": repr(ex)}
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline and not dist_on:

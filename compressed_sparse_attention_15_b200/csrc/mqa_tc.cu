@@ -1,19 +1,562 @@
-// A4 / A5 on the tensor cores (tcgen05 + TMA) for the Flash attention shape.
+// A4 / A5 on the tensor cores for the Flash attention shape: 64 query heads,
+// one shared KV head, head_dim 512, K = V, bf16 in, fp32 accumulation
+// ("DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: sliding window
+// + compressed rows + per-head attention sink; section 2: keys and values
+// share one 512-dim representation).
+//
+// Transposed formulation, so every MMA has M = 128:
+//   S^T[r, h]  = sum_d KV[r, d] Q[h, d]        A = KV tile (K-major), B = Q (K-major)
+//   O^T[d, h] += sum_r KV[r, d] P^T[r, h]      A = the same KV tile read MN-major,
+//                                              B = P^T (MN-major), O^T as 4 x (128 x 64)
+// The 128-row x 512-dim KV tile is gathered once into shared memory (128-byte
+// swizzled, 64-dim boxes) and feeds both products. S^T lives in 64 TMEM
+// columns, O^T in 256. Each softmax thread owns one KV row and its 64 head
+// logits: the per-head tile maximum is a warp transpose-reduction plus a
+// 4-warp exchange; exponentials and the running per-head sums stay
+// thread-local. The running maximum is only moved (and O^T rescaled in TMEM)
+// when a tile's maximum exceeds it by more than 2^8, so P <= 256 in bf16.
+//
+// Work split: query q's row list (selected compressed rows, or all visible
+// ones for HCA, then the window rows) is cut into `splits` runs of whole
+// 128-row tiles, one CTA each. With one split the CTA folds in the sink and
+// writes the output; otherwise it writes (m, l, O) partials and a combine
+// kernel merges them by log-sum-exp together with the sink.
+//
+// Roles (288 threads): warps 0-3 gather rows with cp.async (zero-filling
+// padding rows) per 128-dim chunk; warp 4 issues the MMAs and owns TMEM;
+// warps 5-8 run the softmax and the epilogue. All waits are bounded.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
+#include "tmap.h"
 
 namespace csa {
 
+namespace {
+
+constexpr int kH = 64, kD = 512;
+constexpr int kRows = 128;
+constexpr int kChunks = 4;                          // 128-dim chunks of a row
+constexpr uint32_t kBoxBytes = kRows * 64 * 2;      // 128 rows x 64 dims: 16 KB
+constexpr uint32_t kChunkBytes = 2 * kBoxBytes;     // 128 rows x 128 dims: 32 KB
+constexpr uint32_t kQBoxBytes = kH * 64 * 2;        // 64 heads x 64 dims: 8 KB
+constexpr uint32_t kQBytes = kH * kD * 2;           // 64 KB
+constexpr uint32_t kPBytes = kRows * kH * 2;        // 16 KB
+constexpr int kThreads = 288;
+constexpr int kLoadThreads = 128;
+constexpr int kMmaWarp = 4;
+constexpr int kSoftWarp0 = 5;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m
+constexpr uint32_t kColS = 256;                     // S^T at columns 256..319
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct Small {
+  uint64_t q_full, kv_full[kChunks], kv_empty[kChunks], s_full, p_full, o_done;
+  float red[4][kH];
+  float mref[kH];
+  float alpha[kH];
+  float lsum[kH];
+  uint32_t tmem_base;
+  int abort;
+  int rescale;
+};
+
+constexpr size_t kSmemBytes = 1024 + kChunks * kChunkBytes + kQBytes + kPBytes + sizeof(Small);
+
+struct RowList {
+  int nsel, wlo, R;
+};
+
+__device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *status) {
+  RowList L;
+  L.nsel = a.idx ? a.k : clamp_count(a.n_cmp[qq], a.N_max, status);
+  int e = a.win_end[qq];
+  if (e < 0 || e >= a.T_raw) {
+    raise_status(status, CSA_STATUS_BAD_WINDOW);
+    e = e < 0 ? 0 : a.T_raw - 1;
+  }
+  L.wlo = max(0, e - a.win_len + 1);
+  L.R = L.nsel + (e - L.wlo + 1);
+  return L;
+}
+
+// Source row of list position r, or nullptr for padding / unused (-1) slots.
+__device__ __forceinline__ const bf16 *row_ptr(const MqaArgs &a, const RowList &L, int qq, int b, int r) {
+  if (r < L.nsel) {
+    int j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
+    if (j < -1 || j >= a.N_max) {
+      raise_status(a.status, CSA_STATUS_BAD_INDEX);
+      j = -1;
+    }
+    return j >= 0 ? static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + j) * kD : nullptr;
+  }
+  if (r < L.R) return static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + L.wlo + (r - L.nsel)) * kD;
+  return nullptr;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Warp transpose-reduction of 64 per-lane values: afterwards lane l holds
+// op-reduction over the 32 lanes of heads 2l and 2l+1 in v[0], v[1].
+template <bool kMax>
+__device__ __forceinline__ void transpose_reduce64(float (&v)[64], int lane) {
+#pragma unroll
+  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+    const bool hi = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float send = hi ? v[i] : v[i + n];
+      const float keep = hi ? v[i + n] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, o);
+      v[i] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, MqaArgs a, int splits, int tiles_per_split,
+                  float scale_log2, float *part_o, float *part_ml) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *kv = smem;                                   // [4 chunks][2 boxes][128 rows][128 B]
+  uint8_t *qs = smem + kChunks * kChunkBytes;           // [8 boxes][64 heads][128 B]
+  uint8_t *ps = qs + kQBytes;                           // [128 rows][128 B]  (P^T, MN-major)
+  Small *sm = reinterpret_cast<Small *>(ps + kPBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, qq = blockIdx.y;
+  const int b = qq / a.q_per_seq;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&sm->q_full, 1);
+    for (int m = 0; m < kChunks; ++m) {
+      tc::mbar_init(&sm->kv_full[m], kLoadThreads);
+      tc::mbar_init(&sm->kv_empty[m], 1);
+    }
+    tc::mbar_init(&sm->s_full, 1);
+    tc::mbar_init(&sm->p_full, 4 * 32);
+    tc::mbar_init(&sm->o_done, 1);
+    sm->abort = 0;
+    sm->rescale = 0;
+    tc::fence_barrier_init();
+  }
+  if (threadIdx.x < kH) {
+    sm->mref[threadIdx.x] = -INFINITY;
+    sm->alpha[threadIdx.x] = 1.f;
+  }
+  if (warp == kMmaWarp) tc::tmem_alloc(&sm->tmem_base, kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sm->tmem_base;
+  volatile int *abort = &sm->abort;
+
+  const RowList L = row_list(a, qq, threadIdx.x == 0 ? a.status : nullptr);
+  const int tiles_all = (L.R + kRows - 1) / kRows;
+  const int t0 = split * tiles_per_split;
+  const int t1 = min(tiles_all, t0 + tiles_per_split);
+  const int ntiles = max(0, t1 - t0);
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ loaders
+    const int L_id = threadIdx.x;             // 0..127
+    const int piece = L_id & 15;              // 16-byte piece of a 256-byte chunk row
+    const int r0 = L_id >> 4;                 // rows r0, r0 + 8, ..., r0 + 120
+    const uint32_t kv_base = tc::smem_u32(kv);
+    for (int li = 0; li < ntiles && !*abort; ++li) {
+      const int base = (t0 + li) * kRows;
+      const bf16 *src[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) src[u] = row_ptr(a, L, qq, b, base + r0 + 8 * u);
+      for (int m = 0; m < kChunks; ++m) {
+        if (!tc::mbar_wait(&sm->kv_empty[m], (li & 1) ^ 1, abort, a.status)) break;
+        const uint32_t cbase = kv_base + m * kChunkBytes + (piece >> 3) * kBoxBytes;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r = r0 + 8 * u;
+          const uint32_t dst = cbase + r * 128 + (((piece & 7) ^ (r & 7)) << 4);
+          const bf16 *s = src[u] ? src[u] + m * 128 + piece * 8 : static_cast<const bf16 *>(a.kv_win);
+          cp_async16(dst, s, src[u] != nullptr);
+        }
+        cp_async_arrive(&sm->kv_full[m]);
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool q_issued = false;
+      if (ntiles > 0) {
+        tc::prefetch_tmap(&tm_q);
+        tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
+        for (int bx = 0; bx < kD / 64; ++bx)
+          tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qq * kH, &sm->q_full);
+        q_issued = true;
+      }
+      constexpr uint32_t idesc_s = tc::idesc_bf16(128, 64, 0, 0);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16(128, 64, 1, 1);
+      const uint32_t kv_base = tc::smem_u32(kv), q_base = tc::smem_u32(qs), p_base = tc::smem_u32(ps);
+      bool ok = ntiles == 0 || tc::mbar_wait(&sm->q_full, 0, abort, a.status);
+      for (int li = 0; ok && li < ntiles; ++li) {
+        const uint32_t ph = li & 1;
+        for (int m = 0; m < kChunks && ok; ++m) {
+          ok = tc::mbar_wait(&sm->kv_full[m], ph, abort, a.status);
+          if (!ok) break;
+          tc::fence_after_sync();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint64_t ad = tc::sw128_desc(kv_base + m * kChunkBytes + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024);
+            const uint64_t bd = tc::sw128_desc(q_base + (2 * m + (j >> 2)) * kQBoxBytes + (j & 3) * 32, 16, 1024);
+            tc::mma_bf16(tmem + kColS, ad, bd, idesc_s, (m | j) != 0);
+          }
+        }
+        if (!ok) break;
+        tc::commit(&sm->s_full);
+        ok = tc::mbar_wait(&sm->p_full, ph, abort, a.status);
+        if (!ok) break;
+        tc::fence_after_sync();
+        for (int m = 0; m < kChunks; ++m) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint64_t ad = tc::sw128_desc(kv_base + m * kChunkBytes + j * 2048, kBoxBytes, 1024);
+            const uint64_t bd = tc::sw128_desc(p_base + j * 2048, kPBytes, 1024);
+            tc::mma_bf16(tmem + kColO + 64 * m, ad, bd, idesc_pv, li > 0 || j > 0);
+          }
+          tc::commit(&sm->kv_empty[m]);
+        }
+      }
+      tc::commit(&sm->o_done);
+      tc::mbar_drain(&sm->o_done, 0);
+      if (q_issued) tc::mbar_drain(&sm->q_full, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const bool leader = warp == kSoftWarp0;  // finalises per-head values
+    float l[kH];
+#pragma unroll
+    for (int h = 0; h < kH; ++h) l[h] = 0.f;
+    bool ok = true;
+    for (int li = 0; li < ntiles; ++li) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full, li & 1, abort, a.status));
+      if (!ok) break;
+      tc::fence_after_sync();
+      const int r = (t0 + li) * kRows + row;
+      bool valid = r < L.R;
+      if (valid && r < L.nsel && a.idx) {
+        const int j = a.idx[(size_t)qq * a.k + r];
+        valid = j >= 0 && j < a.N_max;
+      }
+      {
+        float red[kH];
+        uint32_t v0[32], v1[32];
+        tc::tmem_ld32(tmem + lane_off + kColS, v0);
+        tc::tmem_ld32(tmem + lane_off + kColS + 32, v1);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+          red[h] = valid ? __uint_as_float(v0[h]) * scale_log2 : -INFINITY;
+          red[h + 32] = valid ? __uint_as_float(v1[h]) * scale_log2 : -INFINITY;
+        }
+        transpose_reduce64<true>(red, lane);
+        sm->red[quarter][2 * lane] = red[0];
+        sm->red[quarter][2 * lane + 1] = red[1];
+      }
+      named_sync(1, 128);
+      if (leader) {
+        bool any = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int h = 2 * lane + i;
+          const float tm = fmaxf(fmaxf(sm->red[0][h], sm->red[1][h]), fmaxf(sm->red[2][h], sm->red[3][h]));
+          const float mo = sm->mref[h];
+          float al = 1.f;
+          if (mo == -INFINITY || tm > mo + kRescaleLog2) {
+            const float mn = fmaxf(mo, tm);
+            al = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+            sm->mref[h] = mn;
+            any |= mo != -INFINITY;
+          }
+          sm->alpha[h] = al;
+        }
+        any = __any_sync(0xffffffffu, any);
+        if (lane == 0) sm->rescale = any ? 1 : 0;
+      }
+      named_sync(1, 128);
+      const bool rescale = sm->rescale != 0;
+      if (rescale) {
+#pragma unroll
+        for (int h = 0; h < kH; ++h) l[h] *= sm->alpha[h];
+      }
+      // P = exp2(x - mref), summed per head, packed to bf16 into P^T row `row`.
+      uint32_t pk[32];
+      {
+        uint32_t v[32];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          tc::tmem_ld32(tmem + lane_off + kColS + 32 * half, v);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const int h = 32 * half + c;
+            const float m0 = sm->mref[h], m1 = sm->mref[h + 1];
+            const float p0 = (!valid || m0 == -INFINITY) ? 0.f : exp2f(__uint_as_float(v[c]) * scale_log2 - m0);
+            const float p1 = (!valid || m1 == -INFINITY) ? 0.f : exp2f(__uint_as_float(v[c + 1]) * scale_log2 - m1);
+            l[h] += p0;
+            l[h + 1] += p1;
+            __nv_bfloat162 t = __floats2bfloat162_rn(p0, p1);
+            pk[h >> 1] = *reinterpret_cast<uint32_t *>(&t);
+          }
+        }
+      }
+      const uint32_t prow = tc::smem_u32(ps) + row * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t addr = prow + ((c ^ (row & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
+                     "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                     : "memory");
+      }
+      if (rescale && li > 0) {
+        // O^T columns h *= alpha[h]; every PV of the previous tile has
+        // completed (its KV chunks had to be released before this tile's S).
+#pragma unroll 1
+        for (int m = 0; m < kChunks; ++m) {
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            const uint32_t ta = tmem + lane_off + kColO + 64 * m + 32 * half;
+            tc::tmem_ld32(ta, v);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * sm->alpha[32 * half + c]);
+            tmem_st32(ta, v);
+          }
+        }
+        tmem_st_wait();
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc::fence_before_sync();
+      tc::mbar_arrive(&sm->p_full);
+    }
+    // ---- epilogue: per-head sums, then O (partials, or the final output)
+    ok = __all_sync(0xffffffffu, ok && (ntiles == 0 || tc::mbar_wait(&sm->o_done, 0, abort, a.status)));
+    tc::fence_after_sync();
+    transpose_reduce64<false>(l, lane);
+    sm->red[quarter][2 * lane] = l[0];
+    sm->red[quarter][2 * lane + 1] = l[1];
+    named_sync(1, 128);
+    if (leader) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int h = 2 * lane + i;
+        sm->lsum[h] = (sm->red[0][h] + sm->red[1][h]) + (sm->red[2][h] + sm->red[3][h]);
+      }
+    }
+    named_sync(1, 128);
+    const size_t pidx = (size_t)qq * splits + split;
+    if (ok && splits > 1) {
+      if (leader) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int h = 2 * lane + i;
+          part_ml[(pidx * 2) * kH + h] = sm->mref[h];
+          part_ml[(pidx * 2 + 1) * kH + h] = sm->lsum[h];
+        }
+      }
+      float *po = part_o + pidx * (size_t)kH * kD;
+#pragma unroll 1
+      for (int m = 0; m < kChunks; ++m) {
+        const int d = 128 * m + row;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          if (ntiles > 0) {
+            tc::tmem_ld32(tmem + lane_off + kColO + 64 * m + 32 * half, v);
+            tc::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = 0u;
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c) po[(size_t)(32 * half + c) * kD + d] = __uint_as_float(v[c]);
+        }
+      }
+    } else if (ok) {
+      // One split: fold in the sink (logit sink[h], value 0) and normalise.
+      if (leader) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int h = 2 * lane + i;
+          const float mr = sm->mref[h], sk = a.sink[h] * kLog2e;
+          const float M = fmaxf(mr, sk);
+          const float wm = mr == -INFINITY ? 0.f : exp2f(mr - M);
+          sm->alpha[h] = wm / (sm->lsum[h] * wm + exp2f(sk - M));
+        }
+      }
+      named_sync(1, 128);
+      bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qq * kH * kD;
+#pragma unroll 1
+      for (int m = 0; m < kChunks; ++m) {
+        const int d = 128 * m + row;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          tc::tmem_ld32(tmem + lane_off + kColO + 64 * m + 32 * half, v);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            out[(size_t)(32 * half + c) * kD + d] = __float2bfloat16_rn(__uint_as_float(v[c]) * sm->alpha[32 * half + c]);
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Merge the split partials of each query with the sink:
+//   M = max(max_s m_s, sink), L = sum_s l_s 2^(m_s - M) + 2^(sink - M),
+//   out = sum_s O_s 2^(m_s - M) / L   (m and sink in log2 units).
+// Block (query, 16-head group), 256 threads, 32 outputs per thread.
+__global__ void __launch_bounds__(256) mqa_combine_kernel(const float *part_o, const float *part_ml,
+                                                          const float *sink, bf16 *out, int splits) {
+  extern __shared__ float f[];  // [splits][16]
+  const int qq = blockIdx.x, hg = blockIdx.y;
+  for (int i = threadIdx.x; i < 16; i += blockDim.x) {
+    const int h = hg * 16 + i;
+    float M = sink[h] * kLog2e;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[(((size_t)qq * splits + s) * 2) * kH + h]);
+    float Lsum = exp2f(sink[h] * kLog2e - M);
+    for (int s = 0; s < splits; ++s) {
+      const size_t p = ((size_t)qq * splits + s) * 2;
+      const float ms = part_ml[p * kH + h];
+      const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
+      f[s * 16 + i] = w;
+      Lsum += part_ml[(p + 1) * kH + h] * w;
+    }
+    const float inv = 1.f / Lsum;
+    for (int s = 0; s < splits; ++s) f[s * 16 + i] *= inv;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x * 4; e < 16 * kD; e += blockDim.x * 4) {
+    const int i = e / kD, d = e - i * kD, h = hg * 16 + i;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < splits; ++s) {
+      const float w = f[s * 16 + i];
+      const float4 v = *reinterpret_cast<const float4 *>(part_o + (((size_t)qq * splits + s) * kH + h) * kD + d);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+    *reinterpret_cast<uint2 *>(out + ((size_t)qq * kH + h) * kD + d) = pk;
+  }
+}
+
+int num_sms_cached() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split) {
+  const int tiles = (rows_max + kRows - 1) / kRows;
+  int s = num_sms_cached() / (Q > 0 ? Q : 1);
+  s = s < 1 ? 1 : (s > tiles ? tiles : s);
+  const int tps = (tiles + s - 1) / s;
+  *tiles_per_split = tps;
+  *splits = (tiles + tps - 1) / tps;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bool tc_shape(const MqaArgs &a) {
+  return a.dtype == CSA_DTYPE_BF16 && a.H == kH && a.D == kD && aligned16(a.q) && aligned16(a.kv_cmp) &&
+         aligned16(a.kv_win) && aligned16(a.out);
+}
+
+int rows_max_of(const MqaArgs &a) { return (a.idx ? a.k : a.N_max) + a.win_len; }
+
+}  // namespace
+
 size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
-  (void)Q; (void)H; (void)D; (void)rows_max;
-  return 0;
+  if (H != kH || D != kD) return 0;
+  int splits, tps;
+  plan_splits(Q, rows_max, &splits, &tps);
+  if (splits <= 1) return 0;
+  return (size_t)Q * splits * kH * (kD + 2) * sizeof(float);
 }
 
 cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
-  (void)a;
-  (void)stream;
   *taken = false;
-  return cudaSuccess;
+  if (!tc_shape(a)) return cudaSuccess;
+  const int rows_max = rows_max_of(a);
+  int splits, tps;
+  plan_splits(a.Q, rows_max, &splits, &tps);
+  const size_t need = splits > 1 ? (size_t)a.Q * splits * kH * (kD + 2) * sizeof(float) : 0;
+  if (need > a.partial_bytes) return cudaSuccess;  // cannot happen with the documented workspace size
+  CUtensorMap tm_q;
+  if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * kH, kD * 2, 64, kH)) return cudaSuccess;
+  float *part_o = static_cast<float *>(a.partials);
+  float *part_ml = part_o + (size_t)a.Q * splits * kH * kD;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    attr_set = true;
+  }
+  dim3 grid(splits, a.Q);
+  mqa_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, a, splits, tps, a.scale * kLog2e, part_o, part_ml);
+  note_launches(1);
+  if (splits > 1) {
+    dim3 cg(a.Q, kH / 16);
+    mqa_combine_kernel<<<cg, 256, splits * 16 * sizeof(float), stream>>>(part_o, part_ml, a.sink,
+                                                                         static_cast<bf16 *>(a.out), splits);
+    note_launches(1);
+  }
+  *taken = true;
+  return cudaGetLastError();
 }
 
 }  // namespace csa

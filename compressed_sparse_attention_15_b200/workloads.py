@@ -13,9 +13,10 @@ Recipe (tensor id: distribution):
   5 wi     [Q, Hi]        U(0,1)      indexer per-head weights (fp32)
   6 ki     [B, N, Di]     N(0,1)      indexer key cache
   7 sink   [H]            N(0,1)      per-head sink logit (fp32)
-  8 kv_raw [1, T_c, D]    N(0,1)      raw KV fed to the compressor (1 M-token case)
-  9 gate   [Bc, T_c, D]   N(0,1)      compressor gate logits
+  8 kv_raw [1, bulk_T, D] N(0,1)     raw KV of a whole sequence (1 M-token bulk compression)
+  9 gate   [B, T_c, D]    N(0,1)      gate logits of the tokens compressed in a step
  10 ape    [win, D]       N(0,0.1)    in-window position embedding (fp32)
+ 12 gate_raw [1, bulk_T, D] N(0,1)    gate logits of the bulk-compressed sequence
     norm_w [D]            1.0         RMSNorm weight (fp32)
 bf16 tensors are drawn in fp32 and rounded once to bf16 (RNE).
 """
@@ -28,7 +29,8 @@ import torch
 
 from . import synth
 
-TID = {"q": 1, "kv_cmp": 2, "kv_win": 3, "qi": 4, "wi": 5, "ki": 6, "sink": 7, "kv_raw": 8, "gate": 9, "ape": 10}
+TID = {"q": 1, "kv_cmp": 2, "kv_win": 3, "qi": 4, "wi": 5, "ki": 6, "sink": 7, "kv_raw": 8, "gate": 9, "ape": 10,
+       "gate_raw": 12}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -50,12 +52,14 @@ class Workload:
     T_raw: int           # rows of the raw-KV window buffer per sequence
     pos0: int            # absolute position of query 0 (queries of one sequence are consecutive)
     raw0: int            # absolute position of kv_win row 0
-    # compressor run inside the workload: raw tokens [c_src0, c_src0 + T_c) of
-    # kv_win (or of kv_raw when c_from_raw) -> cache rows [c_dst0, c_dst0 + n)
+    # compressor run inside each step: raw tokens [c_src0, c_src0 + T_c) of
+    # kv_win -> cache rows [c_dst0, c_dst0 + n) of every sequence
     T_c: int = 0
     c_src0: int = 0
     c_dst0: int = 0
-    c_from_raw: bool = False
+    # one-off bulk compression of a whole raw sequence (kv_raw / gate_raw) into
+    # sequence 0's cache, reported apart from the decode step
+    bulk_T: int = 0
     seed: int = 0
 
     @property
@@ -99,11 +103,11 @@ WORKLOADS = {
     "csa_prefill_chunk_4k": _csa(
         name="csa_prefill_chunk_4k", dtype=torch.bfloat16, B=1, Q=4096, H=64, D=512, Hi=64, Di=128, k=512,
         W=128, N=33791, T_raw=4223, pos0=131072, raw0=130945, T_c=4100, c_src0=123, c_dst0=32767),
-    # CSA decode at 1 M context, 8 sequences, top-1024; sequence 0's cache is
-    # produced by compressing its 1,048,576 raw tokens.
+    # CSA decode at 1 M context, 8 sequences, top-1024; sequence 0's cache can
+    # be produced by compressing its 1,048,576 raw tokens (the bulk run).
     "csa_decode_1m": _csa(
         name="csa_decode_1m", dtype=torch.bfloat16, B=8, Q=8, H=64, D=512, Hi=64, Di=128, k=1024, W=128,
-        N=262143, T_raw=128, pos0=1048575, raw0=1048448, T_c=1048576, c_src0=0, c_dst0=0, c_from_raw=True),
+        N=262143, T_raw=128, pos0=1048575, raw0=1048448, T_c=8, c_src0=120, c_dst0=262142, bulk_T=1048576),
 }
 
 
@@ -111,8 +115,8 @@ def tensor_shape(w: Workload, name: str):
     return {
         "q": (w.Q, w.H, w.D), "kv_cmp": (w.B, w.N, w.D), "kv_win": (w.B, w.T_raw, w.D),
         "qi": (w.Q, w.Hi, w.Di), "wi": (w.Q, w.Hi), "ki": (w.B, w.N, w.Di), "sink": (w.H,),
-        "kv_raw": (1, w.T_c, w.D), "ape": (w.win, w.D),
-        "gate": ((1 if w.c_from_raw else w.B), w.T_c, w.D),
+        "kv_raw": (1, w.bulk_T, w.D), "gate_raw": (1, w.bulk_T, w.D), "ape": (w.win, w.D),
+        "gate": (w.B, w.T_c, w.D),
     }[name]
 
 

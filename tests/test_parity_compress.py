@@ -79,7 +79,7 @@ def test_compress_full_1m_tokens_sampled(cuda_device):
     # are checked against the oracle.
     w = WL.WORKLOADS["csa_decode_1m"]
     kv = WL.make(w, "kv_raw", cuda_device)
-    gate = WL.make(w, "gate", cuda_device)
+    gate = WL.make(w, "gate_raw", cuda_device)
     ape = WL.make(w, "ape", cuda_device)
     nw = WL.norm_w(w, cuda_device)
     out = ops.compress(kv, gate, ape, nw, 8, 4)
@@ -92,5 +92,5 @@ def test_compress_full_1m_tokens_sampled(cuda_device):
     ref = []
     for j in ents.tolist():
         toks = torch.arange(4 * j, 4 * j + 8)
-        ref.append(O.compress(WL.rows(w, "kv_raw", toks), WL.rows(w, "gate", toks), ape_h, np.ones(512), 8, 4)[0])
+        ref.append(O.compress(WL.rows(w, "kv_raw", toks), WL.rows(w, "gate_raw", toks), ape_h, np.ones(512), 8, 4)[0])
     assert_close(got, np.stack(ref), torch.bfloat16, "compress 1M sampled")

@@ -83,6 +83,30 @@ def test_sparse_with_all_entries_equals_hca(cuda_device):
     assert_close(b, ref, torch.bfloat16, "hca")
 
 
+@pytest.mark.parametrize("mode", ["sparse", "hca"])
+def test_mqa_growing_logits_force_running_max_updates(cuda_device, mode):
+    # Row norms grow along the row list and the softmax scale is large, so
+    # later 128-row tiles raise the per-head running maximum far past the
+    # first tile's: exercises the deferred rescaling of the accumulator.
+    Q, B, N, T_raw, H, D, k, W = 3, 3, 900, 128, 64, 512, 768, 128
+    q, kv_cmp, kv_win, sink = _mqa_inputs(6, Q, B, N, T_raw, H, D, torch.float32)
+    grow = torch.linspace(0.2, 2.0, N).reshape(1, N, 1)
+    kv_cmp = (kv_cmp * grow).to(torch.bfloat16)
+    q, kv_win = q.to(torch.bfloat16), kv_win.to(torch.bfloat16)
+    scale = 0.15
+    we = torch.full((Q,), T_raw - 1, dtype=torch.int32)
+    if mode == "sparse":
+        idx = torch.arange(k, dtype=torch.int32).repeat(Q, 1)  # ascending: norms grow tile by tile
+        out = ops.sparse_mqa(*_dev(cuda_device, q, kv_cmp, idx, kv_win, we, sink), scale, W)
+        ref = [O.sparse_mqa(q[i], kv_cmp[i], idx[i].numpy(), kv_win[i], T_raw - 1, W, sink, scale) for i in range(Q)]
+    else:
+        n = torch.tensor([N, N // 2, 300], dtype=torch.int32)
+        out = ops.hca_mqa(*_dev(cuda_device, q, kv_cmp, n, kv_win, we, sink), scale, W)
+        ref = [O.hca_mqa(q[i], kv_cmp[i], int(n[i]), kv_win[i], T_raw - 1, W, sink, scale) for i in range(Q)]
+    torch.cuda.synchronize()
+    assert_close(out, np.stack(ref), torch.bfloat16, f"growing logits {mode}")
+
+
 def test_sink_at_minus_inf_without_entries_is_window_attention(cuda_device):
     Q, D, H, W = 40, 16, 4, 16
     q, _, kv_win, _ = _mqa_inputs(4, Q, 1, 1, Q, H, D, torch.float32)
