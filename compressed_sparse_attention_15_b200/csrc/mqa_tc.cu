@@ -513,7 +513,7 @@ void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 bool tc_shape(const MqaArgs &a) {
-  return a.dtype == CSA_DTYPE_BF16 && a.H == kH && a.D == kD && aligned16(a.q) && aligned16(a.kv_cmp) &&
+  return a.dtype == CSA_DTYPE_BF16 && a.H == kH && a.D == kD && a.Q <= 65535 && aligned16(a.q) && aligned16(a.kv_cmp) &&
          aligned16(a.kv_win) && aligned16(a.out);
 }
 
