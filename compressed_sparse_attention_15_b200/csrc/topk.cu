@@ -6,13 +6,16 @@
 // towards the smaller index; it is written in ascending index order and
 // padded with -1.
 //
-// Method: radix select (MSD, 8-bit digits) on an order-preserving 32-bit key
-// of the fp32 score finds the k-th largest key tau and how many entries equal
-// to tau are still needed (kk). A final ordered pass keeps every entry with
-// key > tau and the first kk entries (by index) with key == tau; an
-// exclusive prefix count over the block gives each kept entry its output
-// slot, so the output is in ascending index order and deterministic.
-// One 1024-thread block per query.
+// Method: radix select (MSD; digits of 11, 11 and 10 bits) on an
+// order-preserving 32-bit key of each fp32 score finds the k-th largest key
+// tau and how many entries equal to tau are still needed (kk). A final
+// ordered pass keeps every entry with key > tau and the first kk entries (by
+// index) with key == tau; per-warp ballots and an exclusive prefix over the
+// block give each kept entry its output slot, so the output is ascending and
+// deterministic. One 1024-thread block per query. When the query's keys fit
+// in shared memory (n <= 48K) they are read from global memory once and every
+// pass runs on the shared copy; otherwise each pass re-reads the scores
+// (L2-resident right after the scoring kernel).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -22,63 +25,86 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 2048;
+constexpr int kSmemKeys = 48 * 1024;
 
 struct TopkShared {
-  uint32_t hist[256];
+  uint32_t hist[kBins];
+  uint32_t scan[kWarps];
   uint32_t warp_gt[kWarps], warp_eq[kWarps];
   uint32_t prefix, kk;
 };
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
-  __shared__ TopkShared sh;
-  const int q = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n = clamp_count(a.n_cmp[q], a.N_max, threadIdx.x == 0 ? a.status : nullptr);
-  const float *s = a.scores + (size_t)q * a.N_max;
-  int32_t *out = a.out_idx + (size_t)q * a.k;
-  const int k = a.k;
-  if (n <= k) {
-    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
-    return;
+// Exclusive prefix sum over the block (thread order) of one value per thread.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scan, int lane, int warp) {
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  if (threadIdx.x == 0) { sh.prefix = 0; sh.kk = (uint32_t)k; }
+  if (lane == 31) scan[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t t = scan[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    scan[lane] = t;
+  }
+  __syncthreads();
+  const uint32_t r = x - v + (warp > 0 ? scan[warp - 1] : 0u);
+  __syncthreads();
+  return r;
+}
+
+template <bool kCached>
+__device__ __forceinline__ uint32_t key_at(const uint32_t *keys, const float *s, int j) {
+  return kCached ? keys[j] : score_key(s[j]);
+}
+
+template <bool kCached>
+__device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const float *s, int n, int k, int32_t *out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    sh.prefix = 0;
+    sh.kk = (uint32_t)k;
+  }
   uint32_t mask = 0;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+  const int shifts[3] = {21, 10, 0};
+  const uint32_t widths[3] = {11, 11, 10};
+#pragma unroll 1
+  for (int p = 0; p < 3; ++p) {
+    const int shift = shifts[p];
+    const uint32_t dmask = (1u << widths[p]) - 1u;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh.hist[i] = 0;
     __syncthreads();
     const uint32_t prefix = sh.prefix;
-    for (int j = threadIdx.x; j < n; j += kThreads) {
-      const uint32_t u = score_key(s[j]);
-      if ((u & mask) == prefix) atomicAdd(&sh.hist[(u >> shift) & 255u], 1u);
+    for (int base = 0; base < n; base += kThreads) {
+      const int j = base + threadIdx.x;
+      const uint32_t u = j < n ? key_at<kCached>(keys, s, j) : 0u;
+      const bool in = j < n && (u & mask) == prefix;
+      const uint32_t bin = in ? (u >> shift) & dmask : 0xffffffffu;
+      // warp-aggregated increment: one atomic per distinct bin in the warp
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (warp == 0) {
-      // lane L owns bins 8L .. 8L+7; find the bin holding the kk-th largest.
-      const uint32_t kk = sh.kk;
-      uint32_t t = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) t += sh.hist[lane * 8 + i];
-      uint32_t incl = t;  // inclusive suffix sum over lanes >= lane
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
-        if (lane + o < 32) incl += y;
-      }
-      const uint32_t above = incl - t;
-      if (above < kk && kk <= incl) {
-        uint32_t c = above;
-        for (int bin = lane * 8 + 7; bin >= lane * 8; --bin) {
-          const uint32_t h = sh.hist[bin];
-          if (c + h >= kk) {
-            sh.kk = kk - c;
-            sh.prefix = prefix | ((uint32_t)bin << shift);
-            break;
-          }
-          c += h;
-        }
-      }
+    // Thread t owns bins B-1-2t and B-2-2t (descending), so an exclusive
+    // prefix over threads counts the candidates in higher bins.
+    const int b_hi = kBins - 1 - 2 * threadIdx.x, b_lo = b_hi - 1;
+    const uint32_t c_hi = sh.hist[b_hi], c_lo = sh.hist[b_lo];
+    const uint32_t above = block_excl_scan(c_hi + c_lo, sh.scan, lane, warp);
+    const uint32_t kk = sh.kk;
+    if (above < kk && kk <= above + c_hi + c_lo) {
+      const bool in_hi = kk <= above + c_hi;
+      const uint32_t bin = in_hi ? b_hi : b_lo;
+      sh.kk = kk - (in_hi ? above : above + c_hi);
+      sh.prefix = prefix | (bin << shift);
     }
-    mask |= 255u << shift;
+    mask |= dmask << shift;
     __syncthreads();
   }
   const uint32_t tau = sh.prefix, kk = sh.kk;
@@ -88,18 +114,24 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   uint32_t g = 0, e = 0;
   for (int base = lo; base < hi; base += 32) {
     const int j = base + lane;
-    const uint32_t u = j < hi ? score_key(s[j]) : 0u;
+    const uint32_t u = j < hi ? key_at<kCached>(keys, s, j) : 0u;
     g += __popc(__ballot_sync(0xffffffffu, j < hi && u > tau));
     e += __popc(__ballot_sync(0xffffffffu, j < hi && u == tau));
   }
-  if (lane == 0) { sh.warp_gt[warp] = g; sh.warp_eq[warp] = e; }
+  if (lane == 0) {
+    sh.warp_gt[warp] = g;
+    sh.warp_eq[warp] = e;
+  }
   __syncthreads();
   uint32_t G = 0, E = 0;
-  for (int w = 0; w < warp; ++w) { G += sh.warp_gt[w]; E += sh.warp_eq[w]; }
+  for (int w = 0; w < warp; ++w) {
+    G += sh.warp_gt[w];
+    E += sh.warp_eq[w];
+  }
   const uint32_t lt = (1u << lane) - 1u;
   for (int base = lo; base < hi; base += 32) {
     const int j = base + lane;
-    const uint32_t u = j < hi ? score_key(s[j]) : 0u;
+    const uint32_t u = j < hi ? key_at<kCached>(keys, s, j) : 0u;
     const bool is_gt = j < hi && u > tau, is_eq = j < hi && u == tau;
     const uint32_t mg = __ballot_sync(0xffffffffu, is_gt), me = __ballot_sync(0xffffffffu, is_eq);
     const uint32_t Gl = G + __popc(mg & lt), El = E + __popc(me & lt);
@@ -110,10 +142,39 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   }
 }
 
+__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int cache_keys) {
+  extern __shared__ uint32_t keys[];
+  __shared__ TopkShared sh;
+  const int q = blockIdx.x;
+  const int n = clamp_count(a.n_cmp[q], a.N_max, threadIdx.x == 0 ? a.status : nullptr);
+  const float *s = a.scores + (size_t)q * a.N_max;
+  int32_t *out = a.out_idx + (size_t)q * a.k;
+  const int k = a.k;
+  if (n <= k) {
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  if (cache_keys && n <= kSmemKeys) {
+    for (int j = threadIdx.x; j < n; j += kThreads) keys[j] = score_key(s[j]);
+    __syncthreads();
+    select_and_emit<true>(sh, keys, s, n, k, out);
+  } else {
+    select_and_emit<false>(sh, keys, s, n, k, out);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
-  topk_kernel<<<a.Q, kThreads, 0, stream>>>(a);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
+    attr_set = true;
+  }
+  const int cache = a.N_max > a.k;  // a query can only need the keys when n > k
+  const int keys = a.N_max < kSmemKeys ? a.N_max : kSmemKeys;
+  const size_t smem = cache ? (size_t)keys * 4 : 0;
+  topk_kernel<<<a.Q, kThreads, smem, stream>>>(a, cache && a.N_max <= kSmemKeys);
   note_launches(1);
   return cudaGetLastError();
 }
