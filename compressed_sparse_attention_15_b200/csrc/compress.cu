@@ -7,12 +7,20 @@
 //     a[i,d] = softmax_i(gate[t,d] + ape[i,d]),  c[d] = sum_i a[i,d] kv[t,d],
 //     out = c / sqrt(mean(c^2) + 1e-6) * norm_w.
 //
-// The softmax is evaluated in one streaming pass per dimension with a running
-// maximum (one exponential per window element): for each new logit x,
-//     m' = max(m, x), e = exp(min(m, x) - m'),
-//     (l, acc) <- x > m ? (l*e + 1, acc*e + v) : (l + e, acc + e*v).
-// This is the standard online-softmax recurrence; it equals the two-pass
-// definition up to rounding.
+// Three kernels, all fp32 arithmetic:
+//  * compress_window_kernel (bf16, D % 8 == 0): one CTA per entry; the window
+//    positions are split over G thread groups, each thread owns one 16-byte
+//    vector (8 dims) and keeps a running (max, sum, weighted sum) over its
+//    positions; the G partial states are merged through shared memory. Used
+//    when there are few entries (the per-step append) or long windows (HCA).
+//  * compress_stream_kernel (bf16, CSA geometry win = 2 * stride): streams
+//    many entries; WPR warps own a row (8 dims per lane), each 8-token window
+//    is reduced with an exact two-pass softmax in registers (max, then exp2),
+//    the half-window shared with the next entry is carried in registers, and
+//    the RMSNorm sum is exchanged between the row's warps.
+//  * compress_generic_kernel: any dtype / D / window (the fp32 path).
+// The running-state merge is the usual log-sum-exp rescaling; it equals the
+// two-pass definition up to rounding.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -23,8 +31,8 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRmsEps = 1e-6f;
 
-// Generic kernel: one warp per entry, lanes stride over D. Any dtype, any D,
-// any window. fp32 path and fallback for unaligned bf16 tensors.
+// ------------------------------------------------------------------ generic
+
 template <typename T>
 __global__ void __launch_bounds__(256) compress_generic_kernel(CompressArgs a) {
   extern __shared__ float c_smem[];
@@ -65,182 +73,230 @@ __global__ void __launch_bounds__(256) compress_generic_kernel(CompressArgs a) {
   }
 }
 
-// Vectorised bf16 kernel (D <= 512, D % 8 == 0). One warp owns a whole output
-// row: lane L holds the 16-byte vectors L, L+32, ... (VPL of them, 8 dims
-// each), so the RMSNorm is a warp reduction and all loads/stores are 16-byte
-// and coalesced. Each warp walks a contiguous run of entries of one
-// sequence. When win == 2*stride
-// (the overlapping CSA windows) the second half of a window is kept in
-// registers and reused as the first half of the next window, so every raw
-// token is read from memory once.
-struct alignas(16) V8 {
-  __nv_bfloat162 h[4];
-};
+// ------------------------------------------------------------------ bf16 helpers
 
-__device__ __forceinline__ void unpack(const V8 &v, float f[8]) {
+__device__ __forceinline__ void unpack8(const uint4 &v, float f[8]) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float2 t = __bfloat1622float2(v.h[k]);
+    const float2 t = __bfloat1622float2(h[k]);
     f[2 * k] = t.x;
     f[2 * k + 1] = t.y;
   }
 }
 
-template <int VPL>
-struct RowState {
-  float m[VPL][8], l[VPL][8], acc[VPL][8];
-  __device__ __forceinline__ void reset() {
+__device__ __forceinline__ uint4 pack8(const float f[8]) {
+  uint4 v;
+  uint32_t *w = reinterpret_cast<uint32_t *>(&v);
 #pragma unroll
-    for (int v = 0; v < VPL; ++v)
-#pragma unroll
-      for (int k = 0; k < 8; ++k) { m[v][k] = -INFINITY; l[v][k] = 0.f; acc[v][k] = 0.f; }
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(f[2 * k], f[2 * k + 1]);
+    w[k] = *reinterpret_cast<uint32_t *>(&t);
   }
-  // Fold one token (its 8-dim vectors) seen at window position i.
-  __device__ __forceinline__ void fold(const V8 (&kv)[VPL], const V8 (&g)[VPL], const float *ape_i,
-                                       int lane, int nvec) {
+  return v;
+}
+
+// ------------------------------------------------------------------ window-parallel
+
+// Block = G groups x nvec threads (nvec = D / 8, a multiple of 32); thread
+// (g, v) handles dims [8v, 8v + 8) at window positions i = g, g + G, ... .
+// One block per (sequence, entry).
+__global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, int G) {
+  extern __shared__ float ws[];  // [G][3][8][nvec] partial states, then [32] sums
+  const int nvec = a.D / 8;
+  const int v = threadIdx.x % nvec, g = threadIdx.x / nvec;
+  const long long e = blockIdx.x;
+  const int b = (int)(e / a.N), j = (int)(e - (long long)b * a.N);
+  const bf16 *kvj = static_cast<const bf16 *>(a.kv) + b * a.kv_ss + (long long)j * a.stride * a.D;
+  const bf16 *gj = static_cast<const bf16 *>(a.gate) + b * a.gate_ss + (long long)j * a.stride * a.D;
+  float m[8], l[8], acc[8];
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      const int vec = lane + 32 * v;
-      if (vec < nvec) {
+  for (int k = 0; k < 8; ++k) {
+    m[k] = -INFINITY;
+    l[k] = 0.f;
+    acc[k] = 0.f;
+  }
+  // positions g, g + G, ... with four rows of loads in flight per step
+  for (int i0 = g; i0 < a.win; i0 += 4 * G) {
+    uint4 kvv[4], gv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * G;
+      if (i < a.win) {
+        kvv[u] = __ldg(reinterpret_cast<const uint4 *>(kvj + (long long)i * a.D) + v);
+        gv[u] = __ldg(reinterpret_cast<const uint4 *>(gj + (long long)i * a.D) + v);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * G;
+      if (i < a.win) {
         float kf[8], gf[8];
-        unpack(kv[v], kf);
-        unpack(g[v], gf);
-        const float4 a0 = __ldg(reinterpret_cast<const float4 *>(ape_i + vec * 8));
-        const float4 a1 = __ldg(reinterpret_cast<const float4 *>(ape_i + vec * 8 + 4));
+        unpack8(kvv[u], kf);
+        unpack8(gv[u], gf);
+        const float4 a0 = __ldg(reinterpret_cast<const float4 *>(a.ape + (size_t)i * a.D + 8 * v));
+        const float4 a1 = __ldg(reinterpret_cast<const float4 *>(a.ape + (size_t)i * a.D + 8 * v + 4));
         const float ap[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float x = (gf[k] + ap[k]) * kLog2e;  // base-2 logit
-          const float mx = fmaxf(m[v][k], x);
-          const float ex = exp2f(fminf(m[v][k], x) - mx);
-          const bool up = x > m[v][k];
+          const float x = (gf[k] + ap[k]) * kLog2e;
+          const float mx = fmaxf(m[k], x);
+          const float ex = exp2f(fminf(m[k], x) - mx);
+          const bool up = x > m[k];
           const float s_old = up ? ex : 1.f, s_new = up ? 1.f : ex;
-          l[v][k] = l[v][k] * s_old + s_new;
-          acc[v][k] = acc[v][k] * s_old + kf[k] * s_new;
-          m[v][k] = mx;
+          l[k] = l[k] * s_old + s_new;
+          acc[k] = acc[k] * s_old + kf[k] * s_new;
+          m[k] = mx;
         }
       }
     }
   }
-};
-
-template <int VPL>
-__device__ __forceinline__ void load_tok(V8 (&dst)[VPL], const bf16 *row, int lane, int nvec) {
+  // merge the G partial states
+  float *sm = ws;
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) {
-    const int vec = lane + 32 * v;
-    if (vec < nvec) {
-      const uint4 r = __ldg(reinterpret_cast<const uint4 *>(row) + vec);
-      dst[v] = *reinterpret_cast<const V8 *>(&r);
-    }
+  for (int k = 0; k < 8; ++k) {
+    sm[((g * 3 + 0) * 8 + k) * nvec + v] = m[k];
+    sm[((g * 3 + 1) * 8 + k) * nvec + v] = l[k];
+    sm[((g * 3 + 2) * 8 + k) * nvec + v] = acc[k];
   }
-}
-
-template <int VPL>
-__device__ __forceinline__ void finish_row(RowState<VPL> &st, const float *norm_w, bf16 *orow, int lane,
-                                           int nvec, int D) {
-  float ss = 0.f;
-#pragma unroll
-  for (int v = 0; v < VPL; ++v)
+  __syncthreads();
+  float *red = ws + (size_t)G * 3 * 8 * nvec;  // [32]
+  float c[8];
+  if (g == 0) {
+    float ss = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float c = (lane + 32 * v < nvec) ? st.acc[v][k] / st.l[v][k] : 0.f;
-      st.acc[v][k] = c;
-      ss += c * c;
+      float M = -INFINITY;
+      for (int h = 0; h < G; ++h) M = fmaxf(M, sm[((h * 3 + 0) * 8 + k) * nvec + v]);
+      float L = 0.f, A = 0.f;
+      for (int h = 0; h < G; ++h) {
+        const float mh = sm[((h * 3 + 0) * 8 + k) * nvec + v];
+        const float w = mh == -INFINITY ? 0.f : exp2f(mh - M);
+        L += sm[((h * 3 + 1) * 8 + k) * nvec + v] * w;
+        A += sm[((h * 3 + 2) * 8 + k) * nvec + v] * w;
+      }
+      c[k] = A / L;
+      ss += c[k] * c[k];
     }
-  ss = warp_sum(ss);
-  const float r = 1.0f / sqrtf(ss / (float)D + kRmsEps);
+    ss = warp_sum(ss);  // group 0 is whole warps (nvec is a multiple of 32)
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  }
+  __syncthreads();
+  if (g == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < (nvec + 31) / 32; ++w) tot += red[w];
+    const float r = 1.0f / sqrtf(tot / (float)a.D + kRmsEps);
+    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * v));
+    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * v + 4));
+    const float nw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) {
-    const int vec = lane + 32 * v;
-    if (vec < nvec) {
-      const float4 w0 = __ldg(reinterpret_cast<const float4 *>(norm_w + vec * 8));
-      const float4 w1 = __ldg(reinterpret_cast<const float4 *>(norm_w + vec * 8 + 4));
-      const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      V8 o;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        o.h[k] = __floats2bfloat162_rn(st.acc[v][2 * k] * r * w[2 * k], st.acc[v][2 * k + 1] * r * w[2 * k + 1]);
-      reinterpret_cast<uint4 *>(orow)[vec] = *reinterpret_cast<const uint4 *>(&o);
-    }
+    for (int k = 0; k < 8; ++k) c[k] = c[k] * r * nw[k];
+    bf16 *o = static_cast<bf16 *>(a.out) + b * a.out_ss + (long long)j * a.D;
+    reinterpret_cast<uint4 *>(o)[v] = pack8(c);
   }
 }
 
-// Each warp: entries [e0, e1) of the flattened (sequence, entry) space,
-// restarting the carry at sequence boundaries.
-template <int VPL, int CARRY_S>
-__global__ void __launch_bounds__(256) compress_bf16_kernel(CompressArgs a, long long per_warp) {
-  const int lane = threadIdx.x & 31;
-  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// ------------------------------------------------------------------ streaming (CSA)
+
+// WPR warps own one row (8 dims per lane, D = 256 * WPR); each group of WPR
+// warps walks a contiguous run of the flattened (sequence, entry) space.
+// S = stride, window = 2 S; ape (pre-scaled by log2 e) lives in shared memory.
+template <int WPR, int S>
+__global__ void __launch_bounds__(256) compress_stream_kernel(CompressArgs a, long long per_group) {
+  constexpr int W = 2 * S;
+  extern __shared__ float ape_s[];  // [W][D] * log2 e
+  __shared__ float grp_sum[8];
+  const int D = a.D;
+  for (int i = threadIdx.x; i < W * D; i += blockDim.x) ape_s[i] = a.ape[i] * kLog2e;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = warp / WPR, sub = warp % WPR;
+  const int v = sub * 32 + lane;  // this lane's 16-byte vector of the row
+  const long long gid = (long long)blockIdx.x * (8 / WPR) + grp;
   const long long total = (long long)a.B * a.N;
-  long long e = gw * per_warp;
-  const long long e1 = min(total, e + per_warp);
-  if (e >= e1) return;
-  const int nvec = a.D / 8;
+  long long e = gid * per_group;
+  const long long e1 = min(total, e + per_group);
   const bf16 *kv = static_cast<const bf16 *>(a.kv);
   const bf16 *gate = static_cast<const bf16 *>(a.gate);
   bf16 *out = static_cast<bf16 *>(a.out);
-  RowState<VPL> st;
-  if (CARRY_S > 0) {
-    constexpr int S = CARRY_S > 0 ? CARRY_S : 1;  // win == 2 * S == 2 * stride
-    V8 ck[S][VPL], cg[S][VPL];
-    int cur_b = -1;
-    int j = 0;
-    for (; e < e1; ++e) {
-      const int b = (int)(e / a.N);
-      j = (int)(e - (long long)b * a.N);
-      const bf16 *kvb = kv + b * a.kv_ss;
-      const bf16 *gb = gate + b * a.gate_ss;
-      if (b != cur_b) {  // (re)load the first half of the window
-#pragma unroll
-        for (int i = 0; i < S; ++i) {
-          load_tok<VPL>(ck[i], kvb + ((long long)j * S + i) * a.D, lane, nvec);
-          load_tok<VPL>(cg[i], gb + ((long long)j * S + i) * a.D, lane, nvec);
-        }
-        cur_b = b;
-      }
-      V8 nk[S][VPL], ng[S][VPL];
+  const float4 n0 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * v));
+  const float4 n1 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * v + 4));
+  const float nw[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+  uint4 ck[S], cg[S];  // the carried half window (packed bf16)
+  int cur_b = -1, cur_j = -2;
+  for (; e < e1; ++e) {
+    const int b = (int)(e / a.N);
+    const int j = (int)(e - (long long)b * a.N);
+    const bf16 *kvb = kv + b * a.kv_ss;
+    const bf16 *gb = gate + b * a.gate_ss;
+    if (b != cur_b || j != cur_j + 1) {
 #pragma unroll
       for (int i = 0; i < S; ++i) {
-        load_tok<VPL>(nk[i], kvb + ((long long)j * S + S + i) * a.D, lane, nvec);
-        load_tok<VPL>(ng[i], gb + ((long long)j * S + S + i) * a.D, lane, nvec);
+        ck[i] = __ldg(reinterpret_cast<const uint4 *>(kvb + ((long long)j * S + i) * D) + v);
+        cg[i] = __ldg(reinterpret_cast<const uint4 *>(gb + ((long long)j * S + i) * D) + v);
       }
-      st.reset();
-#pragma unroll
-      for (int i = 0; i < S; ++i) st.fold(ck[i], cg[i], a.ape + (size_t)i * a.D, lane, nvec);
-#pragma unroll
-      for (int i = 0; i < S; ++i) st.fold(nk[i], ng[i], a.ape + (size_t)(S + i) * a.D, lane, nvec);
-      finish_row<VPL>(st, a.norm_w, out + b * a.out_ss + (long long)j * a.D, lane, nvec, a.D);
-#pragma unroll
-      for (int i = 0; i < S; ++i)
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) { ck[i][v] = nk[i][v]; cg[i][v] = ng[i][v]; }
     }
-  } else {
-    for (; e < e1; ++e) {
-      const int b = (int)(e / a.N);
-      const int j = (int)(e - (long long)b * a.N);
-      const bf16 *kvj = kv + b * a.kv_ss + (long long)j * a.stride * a.D;
-      const bf16 *gj = gate + b * a.gate_ss + (long long)j * a.stride * a.D;
-      st.reset();
-      int i = 0;
-      for (; i + 4 <= a.win; i += 4) {  // four tokens in flight per step
-        V8 tk[4][VPL], tg[4][VPL];
+    cur_b = b;
+    cur_j = j;
+    uint4 nk[S], ng[S];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          load_tok<VPL>(tk[u], kvj + (long long)(i + u) * a.D, lane, nvec);
-          load_tok<VPL>(tg[u], gj + (long long)(i + u) * a.D, lane, nvec);
-        }
+    for (int i = 0; i < S; ++i) {
+      nk[i] = __ldg(reinterpret_cast<const uint4 *>(kvb + ((long long)j * S + S + i) * D) + v);
+      ng[i] = __ldg(reinterpret_cast<const uint4 *>(gb + ((long long)j * S + S + i) * D) + v);
+    }
+    // pass 1: base-2 logits and their per-dim maximum over the window
+    float x[W][8];
+    float mx[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) st.fold(tk[u], tg[u], a.ape + (size_t)(i + u) * a.D, lane, nvec);
+    for (int i = 0; i < W; ++i) {
+      float gf[8];
+      unpack8(i < S ? cg[i] : ng[i - S], gf);
+      const float4 a0 = *reinterpret_cast<const float4 *>(ape_s + i * D + 8 * v);
+      const float4 a1 = *reinterpret_cast<const float4 *>(ape_s + i * D + 8 * v + 4);
+      const float ap[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        x[i][k] = fmaf(gf[k], kLog2e, ap[k]);
+        mx[k] = i == 0 ? x[i][k] : fmaxf(mx[k], x[i][k]);
       }
-      for (; i < a.win; ++i) {
-        V8 tk[VPL], tg[VPL];
-        load_tok<VPL>(tk, kvj + (long long)i * a.D, lane, nvec);
-        load_tok<VPL>(tg, gj + (long long)i * a.D, lane, nvec);
-        st.fold(tk, tg, a.ape + (size_t)i * a.D, lane, nvec);
+    }
+    // pass 2: weights, their sum and the weighted sum of kv
+    float l[8], acc[8];
+#pragma unroll
+    for (int i = 0; i < W; ++i) {
+      float kf[8];
+      unpack8(i < S ? ck[i] : nk[i - S], kf);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float p = exp2f(x[i][k] - mx[k]);
+        l[k] = i == 0 ? p : l[k] + p;
+        acc[k] = i == 0 ? p * kf[k] : fmaf(p, kf[k], acc[k]);
       }
-      finish_row<VPL>(st, a.norm_w, out + b * a.out_ss + (long long)j * a.D, lane, nvec, a.D);
+    }
+    float c[8], ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      c[k] = acc[k] / l[k];
+      ss = fmaf(c[k], c[k], ss);
+    }
+    ss = warp_sum(ss);
+    if (WPR > 1) {
+      // exchange the partial sums of the row's warps (one named barrier per group)
+      if (lane == 0) grp_sum[warp] = ss;
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(32 * WPR) : "memory");
+      ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < WPR; ++w) ss += grp_sum[grp * WPR + w];
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(32 * WPR) : "memory");
+    }
+    const float r = 1.0f / sqrtf(ss / (float)D + kRmsEps);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) c[k] = c[k] * r * nw[k];
+    reinterpret_cast<uint4 *>(out + b * a.out_ss + (long long)j * D)[v] = pack8(c);
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+      ck[i] = nk[i];
+      cg[i] = ng[i];
     }
   }
 }
@@ -257,39 +313,53 @@ int num_sms() {
   return g_num_sms;
 }
 
-template <int VPL, int CARRY_S>
-cudaError_t launch_bf16(const CompressArgs &a, cudaStream_t stream) {
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+template <int WPR, int S>
+cudaError_t launch_stream(const CompressArgs &a, cudaStream_t stream) {
   const long long total = (long long)a.B * a.N;
-  // About 16 resident warps per SM, each walking a contiguous run.
-  long long warps = (long long)num_sms() * 16;
-  if (warps > total) warps = total;
-  const long long per_warp = (total + warps - 1) / warps;
-  warps = (total + per_warp - 1) / per_warp;
-  const int threads = 256;
-  const long long blocks = (warps * 32 + threads - 1) / threads;
-  compress_bf16_kernel<VPL, CARRY_S><<<(unsigned)blocks, threads, 0, stream>>>(a, per_warp);
+  const int groups_per_block = 8 / WPR;  // 256 threads
+  long long groups = (long long)num_sms() * groups_per_block * 2;
+  if (groups > total) groups = total;
+  const long long per = (total + groups - 1) / groups;
+  groups = (total + per - 1) / per;
+  const long long blocks = (groups + groups_per_block - 1) / groups_per_block;
+  const size_t smem = (size_t)2 * S * a.D * sizeof(float);
+  compress_stream_kernel<WPR, S><<<(unsigned)blocks, 256, smem, stream>>>(a, per);
   note_launches(1);
   return cudaGetLastError();
 }
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
 
 cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
   if (a.N <= 0) return cudaSuccess;
-  const bool vec_ok = a.dtype == CSA_DTYPE_BF16 && a.D % 8 == 0 && a.D <= 512 && aligned16(a.kv) &&
+  const long long total = (long long)a.B * a.N;
+  const bool vec_ok = a.dtype == CSA_DTYPE_BF16 && a.D % 8 == 0 && a.D >= 64 && a.D <= 1024 && aligned16(a.kv) &&
                       aligned16(a.gate) && aligned16(a.out) && aligned16(a.ape) && aligned16(a.norm_w) &&
                       a.kv_ss % 8 == 0 && a.gate_ss % 8 == 0 && a.out_ss % 8 == 0;
   if (vec_ok) {
-    const int nvec = a.D / 8;
-    const bool carry4 = a.win == 8 && a.stride == 4;  // the CSA geometry
-    if (nvec <= 32) return carry4 ? launch_bf16<1, 4>(a, stream) : launch_bf16<1, 0>(a, stream);
-    return carry4 ? launch_bf16<2, 4>(a, stream) : launch_bf16<2, 0>(a, stream);
+    const bool csa4 = a.win == 8 && a.stride == 4;
+    if (csa4 && total > 4LL * num_sms() && (a.D == 512 || a.D == 256))
+      return a.D == 512 ? launch_stream<2, 4>(a, stream) : launch_stream<1, 4>(a, stream);
+    if ((a.D / 8) % 32 == 0) {
+      const int nvec = a.D / 8;
+      int G = a.win < 16 ? a.win : 16;
+      while (G > 1 && G * nvec > 512) G >>= 1;
+      const size_t smem = ((size_t)G * 3 * 8 * nvec + 32) * sizeof(float);
+      static bool attr_set = false;
+      if (!attr_set) {
+        cudaFuncSetAttribute(compress_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(((size_t)3 * 8 * 512 + 32) * sizeof(float)));
+        attr_set = true;
+      }
+      compress_window_kernel<<<(unsigned)total, G * nvec, smem, stream>>>(a, G);
+      note_launches(1);
+      return cudaGetLastError();
+    }
   }
   const int threads = 256, wpb = threads / 32;
   const size_t smem = (size_t)wpb * a.D * sizeof(float);
-  const long long total = (long long)a.B * a.N;
   long long blocks = (total + wpb - 1) / wpb;
   if (blocks > 65535LL * 16) blocks = 65535LL * 16;
   static bool attr_set = false;  // the attribute is a per-function fact: set it once

@@ -22,9 +22,11 @@
 // writes the output; otherwise it writes (m, l, O) partials and a combine
 // kernel merges them by log-sum-exp together with the sink.
 //
-// Roles (288 threads): warps 0-3 gather rows with cp.async (zero-filling
-// padding rows) per 128-dim chunk; warp 4 issues the MMAs and owns TMEM;
-// warps 5-8 run the softmax and the epilogue. All waits are bounded.
+// Roles (192 threads): warp 0 gathers rows with TMA tile::gather4 (each lane
+// one group of 4 rows, one 64-dim box per instruction; the compressed segment
+// is padded to a multiple of 4 rows so a group never mixes the compressed
+// cache and the raw window buffer); warp 1 issues the MMAs and owns TMEM;
+// warps 2-5 run the softmax and the epilogue. All waits are bounded.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -42,10 +44,9 @@ constexpr uint32_t kChunkBytes = 2 * kBoxBytes;     // 128 rows x 128 dims: 32 K
 constexpr uint32_t kQBoxBytes = kH * 64 * 2;        // 64 heads x 64 dims: 8 KB
 constexpr uint32_t kQBytes = kH * kD * 2;           // 64 KB
 constexpr uint32_t kPBytes = kRows * kH * 2;        // 16 KB
-constexpr int kThreads = 288;
-constexpr int kLoadThreads = 128;
-constexpr int kMmaWarp = 4;
-constexpr int kSoftWarp0 = 5;
+constexpr int kThreads = 192;
+constexpr int kMmaWarp = 1;
+constexpr int kSoftWarp0 = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m
 constexpr uint32_t kColS = 256;                     // S^T at columns 256..319
@@ -65,8 +66,10 @@ struct Small {
 
 constexpr size_t kSmemBytes = 1024 + kChunks * kChunkBytes + kQBytes + kPBytes + sizeof(Small);
 
+// Row list of one query: compressed rows [0, nsel) (padded with unused rows
+// up to nsel4, a multiple of 4), then the window rows [nsel4, R).
 struct RowList {
-  int nsel, wlo, R;
+  int nsel, nsel4, wlo, R;
 };
 
 __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *status) {
@@ -78,34 +81,42 @@ __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *
     e = e < 0 ? 0 : a.T_raw - 1;
   }
   L.wlo = max(0, e - a.win_len + 1);
-  L.R = L.nsel + (e - L.wlo + 1);
+  L.nsel4 = (L.nsel + 3) & ~3;
+  L.R = L.nsel4 + (e - L.wlo + 1);
   return L;
 }
 
-// Source row of list position r, or nullptr for padding / unused (-1) slots.
-__device__ __forceinline__ const bf16 *row_ptr(const MqaArgs &a, const RowList &L, int qq, int b, int r) {
-  if (r < L.nsel) {
-    int j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
-    if (j < -1 || j >= a.N_max) {
-      raise_status(a.status, CSA_STATUS_BAD_INDEX);
-      j = -1;
+// TMA row coordinate of list position r: in the compressed cache viewed as
+// [B * N_max, 512] when r < nsel4, else in the window buffer viewed as
+// [B * T_raw, 512]. Unused, padding and out-of-range positions get a valid
+// row of the same tensor (their logits are masked).
+__device__ __forceinline__ int row_coord(const MqaArgs &a, const RowList &L, int qq, int b, int r, bool *valid) {
+  if (r < L.nsel4) {
+    int j = -1;
+    if (r < L.nsel) {
+      j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
+      if (j < -1 || j >= a.N_max) {
+        raise_status(a.status, CSA_STATUS_BAD_INDEX);
+        j = -1;
+      }
     }
-    return j >= 0 ? static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + j) * kD : nullptr;
+    *valid = j >= 0;
+    return b * a.N_max + (j >= 0 ? j : 0);
   }
-  if (r < L.R) return static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + L.wlo + (r - L.nsel)) * kD;
-  return nullptr;
+  const int t = r - L.nsel4;
+  *valid = r < L.R;
+  return b * a.T_raw + (r < L.R ? L.wlo + t : L.wlo);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int col, int r0, int r1, int r2,
+                                            int r3, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(col), "r"(r0), "r"(r1), "r"(r2),
+        "r"(r3)
+      : "memory");
 }
-
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -143,7 +154,8 @@ __device__ __forceinline__ void transpose_reduce64(float (&v)[64], int lane) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, MqaArgs a, int splits, int tiles_per_split,
+    mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp,
+                  const __grid_constant__ CUtensorMap tm_win, MqaArgs a, int splits, int tiles_per_split,
                   float scale_log2, float *part_o, float *part_ml) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -158,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tc::mbar_init(&sm->q_full, 1);
     for (int m = 0; m < kChunks; ++m) {
-      tc::mbar_init(&sm->kv_full[m], kLoadThreads);
+      tc::mbar_init(&sm->kv_full[m], 1);
       tc::mbar_init(&sm->kv_empty[m], 1);
     }
     tc::mbar_init(&sm->s_full, 1);
@@ -185,31 +197,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t1 = min(tiles_all, t0 + tiles_per_split);
   const int ntiles = max(0, t1 - t0);
 
-  if (warp < 4) {
-    // ------------------------------------------------------------ loaders
-    const int L_id = threadIdx.x;             // 0..127
-    const int piece = L_id & 15;              // 16-byte piece of a 256-byte chunk row
-    const int r0 = L_id >> 4;                 // rows r0, r0 + 8, ..., r0 + 120
+  if (warp == 0) {
+    // ------------------------------------------------------------ loader
+    // Lane g owns rows 4g .. 4g+3 of every tile.
     const uint32_t kv_base = tc::smem_u32(kv);
-    for (int li = 0; li < ntiles && !*abort; ++li) {
-      const int base = (t0 + li) * kRows;
-      const bf16 *src[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) src[u] = row_ptr(a, L, qq, b, base + r0 + 8 * u);
-      for (int m = 0; m < kChunks; ++m) {
-        if (!tc::mbar_wait(&sm->kv_empty[m], (li & 1) ^ 1, abort, a.status)) break;
-        const uint32_t cbase = kv_base + m * kChunkBytes + (piece >> 3) * kBoxBytes;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int r = r0 + 8 * u;
-          const uint32_t dst = cbase + r * 128 + (((piece & 7) ^ (r & 7)) << 4);
-          const bf16 *s = src[u] ? src[u] + m * 128 + piece * 8 : static_cast<const bf16 *>(a.kv_win);
-          cp_async16(dst, s, src[u] != nullptr);
-        }
-        cp_async_arrive(&sm->kv_full[m]);
-      }
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_cmp);
+      tc::prefetch_tmap(&tm_win);
     }
-    cp_async_wait_all();
+    int rc[4];
+    bool cmp = true;
+    auto coords = [&](int li) {
+      const int r = (t0 + li) * kRows + 4 * lane;
+      bool v;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rc[i] = row_coord(a, L, qq, b, r + i, &v);
+      cmp = r < L.nsel4;
+    };
+    if (ntiles > 0) coords(0);
+    for (int li = 0; li < ntiles && !*abort; ++li) {
+      bool ok = true;
+      for (int m = 0; m < kChunks; ++m) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[m], (li & 1) ^ 1, abort, a.status));
+        if (!ok) break;
+        if (lane == 0) tc::mbar_arrive_expect_tx(&sm->kv_full[m], kChunkBytes);
+        __syncwarp();
+        const CUtensorMap *map = cmp ? &tm_cmp : &tm_win;
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx)
+          tma_gather4(kv_base + m * kChunkBytes + bx * kBoxBytes + lane * 512, map, 128 * m + 64 * bx, rc[0], rc[1],
+                      rc[2], rc[3], &sm->kv_full[m]);
+      }
+      if (!ok) break;
+      if (li + 1 < ntiles) coords(li + 1);  // next tile's rows while this one computes
+    }
+    // Drain: the last tile's copies have landed once kv_full of its phase
+    // completed (also true if it was consumed already).
+    if (lane == 0 && ntiles > 0)
+      for (int m = 0; m < kChunks; ++m) tc::mbar_drain(&sm->kv_full[m], (ntiles - 1) & 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -267,15 +292,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int h = 0; h < kH; ++h) l[h] = 0.f;
     bool ok = true;
+    int idx_next = 0;
+    {
+      const int r = t0 * kRows + row;
+      if (ntiles > 0 && a.idx && r < L.nsel) idx_next = a.idx[(size_t)qq * a.k + r];
+    }
     for (int li = 0; li < ntiles; ++li) {
       ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full, li & 1, abort, a.status));
       if (!ok) break;
       tc::fence_after_sync();
       const int r = (t0 + li) * kRows + row;
-      bool valid = r < L.R;
-      if (valid && r < L.nsel && a.idx) {
-        const int j = a.idx[(size_t)qq * a.k + r];
-        valid = j >= 0 && j < a.N_max;
+      bool valid;
+      if (r < L.nsel4) {
+        valid = r < L.nsel && (!a.idx || (idx_next >= 0 && idx_next < a.N_max));
+      } else {
+        valid = r < L.R;
+      }
+      if (li + 1 < ntiles) {  // the next tile's index, loaded while this tile is processed
+        const int rn = r + kRows;
+        idx_next = (a.idx && rn < L.nsel) ? a.idx[(size_t)qq * a.k + rn] : 0;
       }
       {
         float red[kH];
@@ -517,16 +552,19 @@ bool tc_shape(const MqaArgs &a) {
          aligned16(a.kv_win) && aligned16(a.out);
 }
 
-int rows_max_of(const MqaArgs &a) { return (a.idx ? a.k : a.N_max) + a.win_len; }
+int rows_max_of(const MqaArgs &a) { return (((a.idx ? a.k : a.N_max) + 3) & ~3) + a.win_len; }
 
 }  // namespace
 
 size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
-  if (H != kH || D != kD) return 0;
-  int splits, tps;
-  plan_splits(Q, rows_max, &splits, &tps);
-  if (splits <= 1) return 0;
-  return (size_t)Q * splits * kH * (kD + 2) * sizeof(float);
+  if (H != kH || D != kD || Q < 1) return 0;
+  // Upper bound on the split count the launcher can pick for any row list of
+  // at most rows_max rows (+3 rows of padding): min(tiles, SMs / Q).
+  const int tiles = (rows_max + 3 + kRows - 1) / kRows;
+  int s = num_sms_cached() / Q;
+  s = s < 1 ? 1 : (s > tiles ? tiles : s);
+  if (s <= 1) return 0;
+  return (size_t)Q * s * kH * (kD + 2) * sizeof(float);
 }
 
 cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
@@ -537,8 +575,10 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   plan_splits(a.Q, rows_max, &splits, &tps);
   const size_t need = splits > 1 ? (size_t)a.Q * splits * kH * (kD + 2) * sizeof(float) : 0;
   if (need > a.partial_bytes) return cudaSuccess;  // cannot happen with the documented workspace size
-  CUtensorMap tm_q;
+  CUtensorMap tm_q, tm_cmp, tm_win;
   if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * kH, kD * 2, 64, kH)) return cudaSuccess;
+  if (!make_tmap_bf16_2d(&tm_cmp, a.kv_cmp, kD, (uint64_t)a.B * a.N_max, kD * 2, 64, 1)) return cudaSuccess;
+  if (!make_tmap_bf16_2d(&tm_win, a.kv_win, kD, (uint64_t)a.B * a.T_raw, kD * 2, 64, 1)) return cudaSuccess;
   float *part_o = static_cast<float *>(a.partials);
   float *part_ml = part_o + (size_t)a.Q * splits * kH * kD;
   static bool attr_set = false;
@@ -547,7 +587,8 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
     attr_set = true;
   }
   dim3 grid(splits, a.Q);
-  mqa_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, a, splits, tps, a.scale * kLog2e, part_o, part_ml);
+  mqa_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_cmp, tm_win, a, splits, tps, a.scale * kLog2e,
+                                                        part_o, part_ml);
   note_launches(1);
   if (splits > 1) {
     dim3 cg(a.Q, kH / 16);
