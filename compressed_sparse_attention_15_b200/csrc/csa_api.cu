@@ -80,13 +80,13 @@ int csa_compress(const void *kv, const void *gate, const float *ape, const float
 }
 
 size_t csa_topk_workspace_bytes(int Q, int N_max, int k) {
-  (void)Q; (void)N_max; (void)k;
-  return kStatusBytes;
+  if (Q < 1 || N_max < 1 || k < 1) return kStatusBytes;
+  return kStatusBytes + align256(topk_scratch_bytes(Q, N_max, k));
 }
 
 size_t csa_index_topk_workspace_bytes(int Q, int N_max, int k) {
   if (Q < 1 || N_max < 1) return kStatusBytes;
-  return kStatusBytes + align256((size_t)Q * N_max * sizeof(float)) + csa_topk_workspace_bytes(Q, N_max, k);
+  return kStatusBytes + align256((size_t)Q * N_max * sizeof(float)) + align256(topk_scratch_bytes(Q, N_max, k > 0 ? k : 1));
 }
 
 static int check_scores(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int Q, int B, int Hi,
@@ -124,7 +124,8 @@ int csa_topk(const float *scores, const int32_t *n_cmp, int k, int32_t *out_idx,
   if (!ws || !ws_aligned(ws) || ws_bytes < csa_topk_workspace_bytes(Q, N_max, k)) return CSA_ERR_WORKSPACE;
   if (!device_ok()) return CSA_ERR_UNSUPPORTED;
   TopkArgs a{scores, n_cmp, out_idx, Q, N_max, k, status_of(ws)};
-  return cuda_rc(launch_topk(a, (cudaStream_t)stream));
+  return cuda_rc(launch_topk(a, (cudaStream_t)stream, static_cast<char *>(ws) + kStatusBytes,
+                             ws_bytes - kStatusBytes));
 }
 
 int csa_index_topk(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int k, int32_t *out_idx,
@@ -140,7 +141,9 @@ int csa_index_topk(const void *qi, const float *wi, const void *ki, const int32_
   cudaError_t e = launch_index_scores(sa, (cudaStream_t)stream);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   TopkArgs ta{scores, n_cmp, out_idx, Q, N_max, k, status_of(ws)};
-  return cuda_rc(launch_topk(ta, (cudaStream_t)stream));
+  const size_t sbytes = align256((size_t)Q * N_max * sizeof(float));
+  return cuda_rc(launch_topk(ta, (cudaStream_t)stream, static_cast<char *>(ws) + kStatusBytes + sbytes,
+                             ws_bytes - kStatusBytes - sbytes));
 }
 
 size_t csa_mqa_workspace_bytes(int Q, int H, int D, int rows_max) {

@@ -39,7 +39,10 @@ struct TopkArgs {
   int Q, N_max, k;
   uint32_t *status;
 };
-cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
+// scratch (may be null): device memory for the two-stage selection of long
+// lists, at least topk_scratch_bytes() bytes; without it one stage is used.
+cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, size_t scratch_bytes);
+size_t topk_scratch_bytes(int Q, int N_max, int k);
 
 struct MqaArgs {
   const void *q, *kv_cmp, *kv_win;

@@ -14,8 +14,10 @@
 // block give each kept entry its output slot, so the output is ascending and
 // deterministic. One 1024-thread block per query. When the query's keys fit
 // in shared memory (n <= 48K) they are read from global memory once and every
-// pass runs on the shared copy; otherwise each pass re-reads the scores
-// (L2-resident right after the scoring kernel).
+// pass runs on the shared copy. Longer lists (the 1 M-token context: 262,143
+// entries) take two stages: exact top-k of 16K-entry segments in parallel,
+// then the same selection over the concatenated segment winners. Without
+// scratch space a single block re-reads the scores on every pass.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -65,8 +67,10 @@ __device__ __forceinline__ uint32_t key_at(const uint32_t *keys, const float *s,
   return kCached ? keys[j] : score_key(s[j]);
 }
 
-template <bool kCached>
-__device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const float *s, int n, int k, int32_t *out) {
+// Select the k largest of n keys (ties -> smaller position) and call
+// emit(slot, position, key) for each, slots 0..k-1 in ascending position.
+template <bool kCached, class Emit>
+__device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const float *s, int n, int k, Emit emit) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     sh.prefix = 0;
@@ -135,8 +139,8 @@ __device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const floa
     const bool is_gt = j < hi && u > tau, is_eq = j < hi && u == tau;
     const uint32_t mg = __ballot_sync(0xffffffffu, is_gt), me = __ballot_sync(0xffffffffu, is_eq);
     const uint32_t Gl = G + __popc(mg & lt), El = E + __popc(me & lt);
-    if (is_gt) out[Gl + min(El, kk)] = j;
-    else if (is_eq && El < kk) out[Gl + El] = j;
+    if (is_gt) emit(Gl + min(El, kk), j, u);
+    else if (is_eq && El < kk) emit(Gl + El, j, u);
     G += __popc(mg);
     E += __popc(me);
   }
@@ -154,22 +158,114 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int cache_ke
     for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
     return;
   }
+  auto emit = [out](uint32_t slot, int j, uint32_t) { out[slot] = j; };
   if (cache_keys && n <= kSmemKeys) {
     for (int j = threadIdx.x; j < n; j += kThreads) keys[j] = score_key(s[j]);
     __syncthreads();
-    select_and_emit<true>(sh, keys, s, n, k, out);
+    select_and_emit<true>(sh, keys, s, n, k, emit);
   } else {
-    select_and_emit<false>(sh, keys, s, n, k, out);
+    select_and_emit<false>(sh, keys, s, n, k, emit);
   }
+}
+
+// Two-stage selection for long lists. Stage 1: segment g of query q (kSeg
+// entries) keeps its own top-k (an entry of the global top-k set is always in
+// its segment's top-k set under the same order) as (key, index) candidates,
+// ascending. Stage 2: the concatenated candidates of a query are ascending in
+// index, so selecting by position with the same tie rule gives the global set.
+constexpr int kSeg = 16384;
+
+__global__ void __launch_bounds__(kThreads) topk_stage1_kernel(TopkArgs a, uint32_t *cand_key, int32_t *cand_idx,
+                                                               int32_t *cand_cnt, int nseg) {
+  extern __shared__ uint32_t keys[];
+  __shared__ TopkShared sh;
+  const int g = blockIdx.x, q = blockIdx.y;
+  const int n = clamp_count(a.n_cmp[q], a.N_max, (threadIdx.x == 0 && g == 0) ? a.status : nullptr);
+  const int j0 = g * kSeg;
+  const int len = max(0, min(kSeg, n - j0));
+  const float *s = a.scores + (size_t)q * a.N_max + j0;
+  const size_t cbase = ((size_t)q * nseg + g) * a.k;
+  uint32_t *ck = cand_key + cbase;
+  int32_t *ci = cand_idx + cbase;
+  if (threadIdx.x == 0) cand_cnt[(size_t)q * nseg + g] = min(len, a.k);
+  if (len <= a.k) {
+    for (int i = threadIdx.x; i < len; i += kThreads) {
+      ck[i] = score_key(s[i]);
+      ci[i] = j0 + i;
+    }
+    return;
+  }
+  for (int j = threadIdx.x; j < len; j += kThreads) keys[j] = score_key(s[j]);
+  __syncthreads();
+  select_and_emit<true>(sh, keys, s, len, a.k, [ck, ci, j0](uint32_t slot, int j, uint32_t u) {
+    ck[slot] = u;
+    ci[slot] = j0 + j;
+  });
+}
+
+__global__ void __launch_bounds__(kThreads) topk_stage2_kernel(TopkArgs a, const uint32_t *cand_key,
+                                                               const int32_t *cand_idx, const int32_t *cand_cnt,
+                                                               int nseg) {
+  extern __shared__ uint32_t keys[];  // [kSmemKeys / 2] keys then [kSmemKeys / 2] indices
+  __shared__ TopkShared sh;
+  __shared__ int offs[kThreads + 1];
+  int32_t *idxs = reinterpret_cast<int32_t *>(keys + kSmemKeys / 2);
+  const int q = blockIdx.x;
+  const int n = clamp_count(a.n_cmp[q], a.N_max, nullptr);
+  int32_t *out = a.out_idx + (size_t)q * a.k;
+  if (n <= a.k) {
+    for (int i = threadIdx.x; i < a.k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  if (threadIdx.x == 0) {
+    int o = 0;
+    for (int g = 0; g < nseg; ++g) {
+      offs[g] = o;
+      o += cand_cnt[(size_t)q * nseg + g];
+    }
+    offs[nseg] = o;
+  }
+  __syncthreads();
+  const int total = offs[nseg];
+  for (int g = 0; g < nseg; ++g) {
+    const int c = offs[g + 1] - offs[g];
+    const size_t cbase = ((size_t)q * nseg + g) * a.k;
+    for (int i = threadIdx.x; i < c; i += kThreads) {
+      keys[offs[g] + i] = cand_key[cbase + i];
+      idxs[offs[g] + i] = cand_idx[cbase + i];
+    }
+  }
+  __syncthreads();
+  select_and_emit<true>(sh, keys, nullptr, total, a.k,
+                        [out, idxs](uint32_t slot, int j, uint32_t) { out[slot] = idxs[j]; });
 }
 
 }  // namespace
 
-cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
+size_t topk_scratch_bytes(int Q, int N_max, int k) {
+  const int nseg = (N_max + kSeg - 1) / kSeg;
+  if (N_max <= kSmemKeys || (size_t)nseg * k > (size_t)kSmemKeys / 2 || nseg > kThreads) return 0;
+  return (size_t)Q * nseg * (k * 8 + 4) + 256;
+}
+
+cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, size_t scratch_bytes) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
+    cudaFuncSetAttribute(topk_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSeg * 4);
+    cudaFuncSetAttribute(topk_stage2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     attr_set = true;
+  }
+  const size_t need = topk_scratch_bytes(a.Q, a.N_max, a.k);
+  if (need > 0 && scratch && scratch_bytes >= need && a.Q <= 65535) {
+    const int nseg = (a.N_max + kSeg - 1) / kSeg;
+    uint32_t *ck = static_cast<uint32_t *>(scratch);
+    int32_t *ci = reinterpret_cast<int32_t *>(ck + (size_t)a.Q * nseg * a.k);
+    int32_t *cc = ci + (size_t)a.Q * nseg * a.k;
+    topk_stage1_kernel<<<dim3(nseg, a.Q), kThreads, kSeg * 4, stream>>>(a, ck, ci, cc, nseg);
+    topk_stage2_kernel<<<a.Q, kThreads, kSmemKeys * 4, stream>>>(a, ck, ci, cc, nseg);
+    note_launches(2);
+    return cudaGetLastError();
   }
   const int cache = a.N_max > a.k;  // a query can only need the keys when n > k
   const int keys = a.N_max < kSmemKeys ? a.N_max : kSmemKeys;

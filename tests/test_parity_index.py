@@ -40,8 +40,9 @@ def test_index_scores_match_oracle(cuda_device, Q, B, N, Hi, Di, dtype):
 
 
 @pytest.mark.parametrize("N,k", [(1, 1), (100, 100), (101, 100), (1000, 16), (5000, 512), (20000, 2048),
-                                 (262143, 1024)])
+                                 (49153, 512), (100000, 2048), (262143, 1024), (300000, 64)])
 def test_topk_exact_on_given_scores(cuda_device, N, k):
+    # (the largest cases take the two-stage selection: 16K-entry segments)
     # Both sides select from the same fp32 scores: bit-exact index sets.
     # Scores are quantised so that ties (including +0 / -0) are frequent.
     Q = 3
