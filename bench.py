@@ -35,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from compressed_sparse_attention_15_b200 import _lib, ops, workloads as WL  # noqa: E402
+from compressed_sparse_attention_15_b200.step import DecodeStep  # noqa: E402
 
 METRIC = "CSA/HCA decode queries/s at 64K–1M ctx; HBM GB/s and % of roofline"
 UNIT = "queries/s"
@@ -90,57 +91,30 @@ def algo_flops(w: WL.Workload):
 # --------------------------------------------------------------------------
 
 class Step:
-    """Device-resident inputs of one workload and its decode step."""
+    """Device-resident inputs of one workload wrapped in the package's
+    DecodeStep (graph-captured decode step)."""
 
-    def __init__(self, w: WL.Workload, device):
+    def __init__(self, w: WL.Workload, device, graph: bool = True):
         self.w = w
         self.dev = device
         self.t = {n: WL.make(w, n, device) for n in ("q", "kv_cmp", "kv_win", "sink", "ape", "gate")}
         if w.mode == "csa":
             for n in ("qi", "wi", "ki"):
                 self.t[n] = WL.make(w, n, device)
-        self.norm_w = WL.norm_w(w, device)
-        self.n_cmp = ops.visible_entries(w.positions(), w.win, w.stride).to(device)
-        self.win_end = w.win_end().to(device)
-        self.out = torch.empty_like(self.t["q"])
-        self.idx = torch.empty((w.Q, max(1, w.k)), dtype=torch.int32, device=device)
-        self.ws_index = ops.Workspace(device)
-        self.ws_mqa = ops.Workspace(device)
-
-    def compress(self):
-        w, t = self.w, self.t
-        ops.compress(t["kv_win"][:, w.c_src0:w.c_src0 + w.T_c], t["gate"], t["ape"], self.norm_w, w.win, w.stride,
-                     out=t["kv_cmp"][:, w.c_dst0:w.c_dst0 + (w.T_c - w.win) // w.stride + 1])
-
-    def bulk_compress(self):
-        """The one-off compression of sequence 0's whole raw history."""
-        w, t = self.w, self.t
-        ops.compress(t["kv_raw"], t["gate_raw"], t["ape"], self.norm_w, w.win, w.stride,
-                     out=t["kv_cmp"][0:1, :(w.bulk_T - w.win) // w.stride + 1])
-
-    def select(self):
         t = self.t
-        ops.index_topk(t["qi"], t["wi"], t["ki"], self.n_cmp, self.w.k, out=self.idx, ws=self.ws_index)
-
-    def attend(self):
-        w, t = self.w, self.t
-        if w.mode == "csa":
-            ops.sparse_mqa(t["q"], t["kv_cmp"], self.idx, t["kv_win"], self.win_end, t["sink"], w.scale, w.W,
-                           out=self.out, ws=self.ws_mqa)
-        else:
-            ops.hca_mqa(t["q"], t["kv_cmp"], self.n_cmp, t["kv_win"], self.win_end, t["sink"], w.scale, w.W,
-                        out=self.out, ws=self.ws_mqa)
+        self.ds = DecodeStep(
+            q=t["q"], kv_cmp=t["kv_cmp"], kv_win=t["kv_win"], sink=t["sink"], scale=w.scale, win_len=w.W,
+            win_end=w.win_end().to(device), n_cmp=ops.visible_entries(w.positions(), w.win, w.stride).to(device),
+            ape=t["ape"], norm_w=WL.norm_w(w, device), gate=t["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
+            win=w.win, stride=w.stride, qi=t.get("qi"), wi=t.get("wi"), ki=t.get("ki"),
+            k=w.k if w.mode == "csa" else None, graph=graph)
+        self.out = self.ds.out
 
     def parts(self):
-        p = [("compress", self.compress)]
-        if self.w.mode == "csa":
-            p.append(("index_topk", self.select))
-        p.append(("mqa", self.attend))
-        return p
+        return self.ds.parts()
 
     def run(self):
-        for _, f in self.parts():
-            f()
+        return self.ds.run()
 
 
 class Clocks:
@@ -212,28 +186,13 @@ def _sync_barrier(dist_on):
 
 
 def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=False):
-    step = Step(w, device)
+    n0 = _lib.lib().csa_launch_count()
+    step = Step(w, device)  # runs the step once eagerly, then captures it
+    launches_per_step = (_lib.lib().csa_launch_count() - n0) // 2
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     for _ in range(max(3, args.warmup)):
         step.run()
-    torch.cuda.synchronize()
-    # Capture one step in a CUDA graph (the library never allocates or
-    # synchronises, so its launches are capturable).
-    n0 = _lib.lib().csa_launch_count()
-    graph = torch.cuda.CUDAGraph()
-    s = torch.cuda.Stream(device)
-    s.wait_stream(stream)
-    with torch.cuda.stream(s):
-        step.run()
-    stream.wait_stream(s)
-    torch.cuda.synchronize()
-    with torch.cuda.graph(graph):
-        step.run()
-    launches_per_step = _lib.lib().csa_launch_count() - n0
-    launches_per_step //= 2  # the warm-up on `s` plus the capture
-    for _ in range(3):
-        graph.replay()
     torch.cuda.synchronize()
 
     K = args.steps if not secondary else max(10, args.steps // 4)
@@ -246,7 +205,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
         for i in range(K):
             flush.zero_()
             evs[i][0].record(stream)
-            graph.replay()
+            step.run()
             evs[i][1].record(stream)
         _sync_barrier(dist_on)
     wall = time.perf_counter() - wall0
@@ -273,8 +232,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
         torch.cuda.synchronize()
         for i, n in enumerate(names):
             per[n] += ev[i].elapsed_time(ev[i + 1]) / Kp
-    status = step.ws_mqa.status() | step.ws_index.status()
-    del graph
+    status = step.ds.status()
     return {"ms": ms_max, "ms_local": ms, "per_kernel_ms": per, "launches_per_step": int(launches_per_step),
             "wall_s": wall, "clocks": clocks.summary(), "status": status, "K": K, "step": step}
 

@@ -6,7 +6,7 @@ per-head sink -- runs in hand-written sm_100a CUDA kernels behind the C ABI of
 libcsa.so (include/csa.h). ``ops`` holds the torch-facing wrappers; the
 library is loaded on first use and its absence is an error.
 """
-from . import ops, synth, workloads  # noqa: F401
+from . import ops, step, synth, workloads  # noqa: F401
 from .ops import (  # noqa: F401
     Workspace,
     compress,
@@ -25,3 +25,4 @@ def build(force: bool = False) -> str:
     from .build import build as _build
 
     return _build(force=force)
+from .step import DecodeStep  # noqa: F401,E402

@@ -4,28 +4,31 @@
 // + compressed rows + per-head attention sink; section 2: keys and values
 // share one 512-dim representation).
 //
-// Transposed formulation, so every MMA has M = 128:
-//   S^T[r, h]  = sum_d KV[r, d] Q[h, d]        A = KV tile (K-major), B = Q (K-major)
-//   O^T[d, h] += sum_r KV[r, d] P^T[r, h]      A = the same KV tile read MN-major,
-//                                              B = P^T (MN-major), O^T as 4 x (128 x 64)
-// The 128-row x 512-dim KV tile is gathered once into shared memory (128-byte
-// swizzled, 64-dim boxes) and feeds both products. S^T lives in 64 TMEM
-// columns, O^T in 256. Each softmax thread owns one KV row and its 64 head
-// logits: the per-head tile maximum is a warp transpose-reduction plus a
-// 4-warp exchange; exponentials and the running per-head sums stay
-// thread-local. The running maximum is only moved (and O^T rescaled in TMEM)
-// when a tile's maximum exceeds it by more than 2^8, so P <= 256 in bf16.
+// Transposed formulation:
+//   S^T[r, h]  = sum_d KV[r, d] Q[h, d]      M = 64 rows,  N = 64 heads, K-major A and B
+//   O^T[d, h] += sum_r KV[r, d] P^T[r, h]    M = 128 dims, N = 64 heads, A = the same KV
+//                                            tile read MN-major, B = P^T (MN-major)
+// A 64-row x 512-dim KV tile is loaded once into shared memory (128-byte
+// swizzled, 64-dim boxes) and feeds both products. Two tile buffers, two S^T
+// TMEM buffers and two P^T buffers make a software pipeline: while the
+// softmax warps turn S^T(t) into P(t), the tensor core computes S^T(t+1) and
+// TMA loads tile t+2. The MMA thread issues S(t+1) before PV(t).
+// An M = 64 accumulator occupies TMEM lanes 0-15 of each 32-lane quarter, so
+// each softmax warp owns 16 rows; a row's 64 head logits stay in one thread.
+// The per-head tile maximum is a warp transpose-reduction plus a 4-warp
+// exchange; the running per-head maximum only moves (and O^T is rescaled in
+// TMEM, after the previous P.V has completed) when a tile's maximum exceeds
+// it by more than 2^8, so P <= 256 in bf16.
 //
-// Work split: query q's row list (selected compressed rows, or all visible
-// ones for HCA, then the window rows) is cut into `splits` runs of whole
-// 128-row tiles, one CTA each. With one split the CTA folds in the sink and
-// writes the output; otherwise it writes (m, l, O) partials and a combine
-// kernel merges them by log-sum-exp together with the sink.
+// Loads: contiguous runs of 64 rows (HCA entries, window rows) are single TMA
+// boxes of 64 rows; top-k rows use TMA tile::gather4 (4 rows per instruction;
+// the compressed segment is padded to a multiple of 4 rows so no group mixes
+// the compressed cache and the raw window buffer).
 //
-// Roles (192 threads): warp 0 gathers rows with TMA tile::gather4 (each lane
-// one group of 4 rows, one 64-dim box per instruction; the compressed segment
-// is padded to a multiple of 4 rows so a group never mixes the compressed
-// cache and the raw window buffer); warp 1 issues the MMAs and owns TMEM;
+// Work split: query q's row list is cut into `splits` runs of whole tiles, one
+// CTA each. With one split the CTA folds in the sink and writes the output;
+// otherwise it writes (m, l, O) partials merged by mqa_combine_kernel.
+// Roles (192 threads): warp 0 loads, warp 1 issues the MMAs and owns TMEM,
 // warps 2-5 run the softmax and the epilogue. All waits are bounded.
 #include "common.cuh"
 #include "kernels.h"
@@ -37,24 +40,23 @@ namespace csa {
 namespace {
 
 constexpr int kH = 64, kD = 512;
-constexpr int kRows = 128;
-constexpr int kChunks = 4;                          // 128-dim chunks of a row
-constexpr uint32_t kBoxBytes = kRows * 64 * 2;      // 128 rows x 64 dims: 16 KB
-constexpr uint32_t kChunkBytes = 2 * kBoxBytes;     // 128 rows x 128 dims: 32 KB
-constexpr uint32_t kQBoxBytes = kH * 64 * 2;        // 64 heads x 64 dims: 8 KB
-constexpr uint32_t kQBytes = kH * kD * 2;           // 64 KB
-constexpr uint32_t kPBytes = kRows * kH * 2;        // 16 KB
+constexpr int kRows = 64;                           // rows per tile
+constexpr uint32_t kBoxBytes = kRows * 128;         // 64 rows x 64 dims: 8 KB
+constexpr uint32_t kTileBytes = 8 * kBoxBytes;      // 64 rows x 512 dims: 64 KB
+constexpr uint32_t kQBoxBytes = kH * 128;           // 64 heads x 64 dims: 8 KB
+constexpr uint32_t kQBytes = 8 * kQBoxBytes;        // 64 KB
+constexpr uint32_t kPBytes = kRows * kH * 2;        // 8 KB
 constexpr int kThreads = 192;
 constexpr int kMmaWarp = 1;
 constexpr int kSoftWarp0 = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m
-constexpr uint32_t kColS = 256;                     // S^T at columns 256..319
+constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m (M = 128 layout)
+constexpr uint32_t kColS = 256;                     // S^T buffer j at 256 + 64j (M = 64 layout)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
 struct Small {
-  uint64_t q_full, kv_full[kChunks], kv_empty[kChunks], s_full, p_full, o_done;
+  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done, o_done;
   float red[4][kH];
   float mref[kH];
   float alpha[kH];
@@ -64,7 +66,7 @@ struct Small {
   int rescale;
 };
 
-constexpr size_t kSmemBytes = 1024 + kChunks * kChunkBytes + kQBytes + kPBytes + sizeof(Small);
+constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kQBytes + 2 * kPBytes + sizeof(Small);
 
 // Row list of one query: compressed rows [0, nsel) (padded with unused rows
 // up to nsel4, a multiple of 4), then the window rows [nsel4, R).
@@ -88,9 +90,9 @@ __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *
 
 // TMA row coordinate of list position r: in the compressed cache viewed as
 // [B * N_max, 512] when r < nsel4, else in the window buffer viewed as
-// [B * T_raw, 512]. Unused, padding and out-of-range positions get a valid
-// row of the same tensor (their logits are masked).
-__device__ __forceinline__ int row_coord(const MqaArgs &a, const RowList &L, int qq, int b, int r, bool *valid) {
+// [B * T_raw, 512]. Unused and padding positions get a valid row of the same
+// tensor (their logits are masked).
+__device__ __forceinline__ int row_coord(const MqaArgs &a, const RowList &L, int qq, int b, int r) {
   if (r < L.nsel4) {
     int j = -1;
     if (r < L.nsel) {
@@ -100,21 +102,18 @@ __device__ __forceinline__ int row_coord(const MqaArgs &a, const RowList &L, int
         j = -1;
       }
     }
-    *valid = j >= 0;
     return b * a.N_max + (j >= 0 ? j : 0);
   }
-  const int t = r - L.nsel4;
-  *valid = r < L.R;
-  return b * a.T_raw + (r < L.R ? L.wlo + t : L.wlo);
+  return b * a.T_raw + (r < L.R ? L.wlo + (r - L.nsel4) : L.wlo);
 }
 
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int col, int r0, int r1, int r2,
-                                            int r3, uint64_t *bar) {
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int col, const int (&rc)[4],
+                                            uint64_t *bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(col), "r"(r0), "r"(r1), "r"(r2),
-        "r"(r3)
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(col), "r"(rc[0]), "r"(rc[1]),
+        "r"(rc[2]), "r"(rc[3])
       : "memory");
 }
 
@@ -136,8 +135,8 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Warp transpose-reduction of 64 per-lane values: afterwards lane l holds
-// op-reduction over the 32 lanes of heads 2l and 2l+1 in v[0], v[1].
+// Warp transpose-reduction of 64 per-lane values: afterwards lane l holds the
+// reduction over the 32 lanes of heads 2l and 2l+1 in v[0], v[1].
 template <bool kMax>
 __device__ __forceinline__ void transpose_reduce64(float (&v)[64], int lane) {
 #pragma unroll
@@ -154,27 +153,29 @@ __device__ __forceinline__ void transpose_reduce64(float (&v)[64], int lane) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp,
-                  const __grid_constant__ CUtensorMap tm_win, MqaArgs a, int splits, int tiles_per_split,
+    mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp_g,
+                  const __grid_constant__ CUtensorMap tm_win_g, const __grid_constant__ CUtensorMap tm_cmp_t,
+                  const __grid_constant__ CUtensorMap tm_win_t, MqaArgs a, int splits, int tiles_per_split,
                   float scale_log2, float *part_o, float *part_ml) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *kv = smem;                                   // [4 chunks][2 boxes][128 rows][128 B]
-  uint8_t *qs = smem + kChunks * kChunkBytes;           // [8 boxes][64 heads][128 B]
-  uint8_t *ps = qs + kQBytes;                           // [128 rows][128 B]  (P^T, MN-major)
-  Small *sm = reinterpret_cast<Small *>(ps + kPBytes);
+  uint8_t *kv = smem;                              // [2 tiles][8 boxes][64 rows][128 B]
+  uint8_t *qs = smem + 2 * kTileBytes;             // [8 boxes][64 heads][128 B]
+  uint8_t *ps = qs + kQBytes;                      // [2][64 rows][128 B]  (P^T, MN-major)
+  Small *sm = reinterpret_cast<Small *>(ps + 2 * kPBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, qq = blockIdx.y;
   const int b = qq / a.q_per_seq;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&sm->q_full, 1);
-    for (int m = 0; m < kChunks; ++m) {
-      tc::mbar_init(&sm->kv_full[m], 1);
-      tc::mbar_init(&sm->kv_empty[m], 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&sm->kv_full[i], 1);
+      tc::mbar_init(&sm->kv_empty[i], 1);
+      tc::mbar_init(&sm->s_full[i], 1);
+      tc::mbar_init(&sm->p_full[i], 4 * 32);
     }
-    tc::mbar_init(&sm->s_full, 1);
-    tc::mbar_init(&sm->p_full, 4 * 32);
+    tc::mbar_init(&sm->pv_done, 1);
     tc::mbar_init(&sm->o_done, 1);
     sm->abort = 0;
     sm->rescale = 0;
@@ -199,42 +200,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ loader
-    // Lane g owns rows 4g .. 4g+3 of every tile.
     const uint32_t kv_base = tc::smem_u32(kv);
     if (lane == 0) {
-      tc::prefetch_tmap(&tm_cmp);
-      tc::prefetch_tmap(&tm_win);
+      tc::prefetch_tmap(&tm_cmp_g);
+      tc::prefetch_tmap(&tm_win_g);
+      tc::prefetch_tmap(&tm_cmp_t);
+      tc::prefetch_tmap(&tm_win_t);
     }
-    int rc[4];
-    bool cmp = true;
-    auto coords = [&](int li) {
-      const int r = (t0 + li) * kRows + 4 * lane;
-      bool v;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) rc[i] = row_coord(a, L, qq, b, r + i, &v);
-      cmp = r < L.nsel4;
-    };
-    if (ntiles > 0) coords(0);
+    int issued = 0;
     for (int li = 0; li < ntiles && !*abort; ++li) {
-      bool ok = true;
-      for (int m = 0; m < kChunks; ++m) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[m], (li & 1) ^ 1, abort, a.status));
-        if (!ok) break;
-        if (lane == 0) tc::mbar_arrive_expect_tx(&sm->kv_full[m], kChunkBytes);
-        __syncwarp();
-        const CUtensorMap *map = cmp ? &tm_cmp : &tm_win;
+      const int buf = li & 1;
+      const int r0 = (t0 + li) * kRows;
+      // A tile is one contiguous run when it lies in the window part, or in
+      // the compressed part of a dense (HCA) row list.
+      const bool win_run = r0 >= L.nsel4;
+      const bool cmp_run = !a.idx && r0 + kRows <= L.nsel4;
+      int rc[4];
+      const CUtensorMap *gmap = &tm_cmp_g;
+      if (!win_run && !cmp_run && lane < 16) {
+        const int r = r0 + 4 * lane;
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
-          tma_gather4(kv_base + m * kChunkBytes + bx * kBoxBytes + lane * 512, map, 128 * m + 64 * bx, rc[0], rc[1],
-                      rc[2], rc[3], &sm->kv_full[m]);
+        for (int i = 0; i < 4; ++i) rc[i] = row_coord(a, L, qq, b, r + i);
+        gmap = r < L.nsel4 ? &tm_cmp_g : &tm_win_g;
       }
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[buf], ((li >> 1) & 1) ^ 1, abort, a.status));
       if (!ok) break;
-      if (li + 1 < ntiles) coords(li + 1);  // next tile's rows while this one computes
+      const uint32_t dst = kv_base + buf * kTileBytes;
+      if (lane == 0) tc::mbar_arrive_expect_tx(&sm->kv_full[buf], kTileBytes);
+      __syncwarp();
+      if (win_run || cmp_run) {
+        if (lane < 8) {
+          const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
+          tc::tma_load_2d(kv + buf * kTileBytes + lane * kBoxBytes, win_run ? &tm_win_t : &tm_cmp_t, 64 * lane, row,
+                          &sm->kv_full[buf]);
+        }
+      } else if (lane < 16) {
+#pragma unroll
+        for (int bx = 0; bx < 8; ++bx) tma_gather4(dst + bx * kBoxBytes + lane * 512, gmap, 64 * bx, rc, &sm->kv_full[buf]);
+      }
+      issued = li + 1;
     }
-    // Drain: the last tile's copies have landed once kv_full of its phase
-    // completed (also true if it was consumed already).
-    if (lane == 0 && ntiles > 0)
-      for (int m = 0; m < kChunks; ++m) tc::mbar_drain(&sm->kv_full[m], (ntiles - 1) & 1);
+    // Drain: the copies of the last two tiles must have landed before exit.
+    if (lane == 0)
+      for (int li = max(0, issued - 2); li < issued; ++li) tc::mbar_drain(&sm->kv_full[li & 1], (li >> 1) & 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -246,38 +254,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qq * kH, &sm->q_full);
         q_issued = true;
       }
-      constexpr uint32_t idesc_s = tc::idesc_bf16(128, 64, 0, 0);
+      constexpr uint32_t idesc_s = tc::idesc_bf16(64, 64, 0, 0);
       constexpr uint32_t idesc_pv = tc::idesc_bf16(128, 64, 1, 1);
       const uint32_t kv_base = tc::smem_u32(kv), q_base = tc::smem_u32(qs), p_base = tc::smem_u32(ps);
       bool ok = ntiles == 0 || tc::mbar_wait(&sm->q_full, 0, abort, a.status);
-      for (int li = 0; ok && li < ntiles; ++li) {
-        const uint32_t ph = li & 1;
-        for (int m = 0; m < kChunks && ok; ++m) {
-          ok = tc::mbar_wait(&sm->kv_full[m], ph, abort, a.status);
-          if (!ok) break;
-          tc::fence_after_sync();
+      auto pv = [&](int t) {  // O^T += V^T(t) P^T(t)
+        const int pb = t & 1;
+        if (!tc::mbar_wait(&sm->p_full[pb], (t >> 1) & 1, abort, a.status)) return false;
+        tc::fence_after_sync();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint64_t ad = tc::sw128_desc(kv_base + m * kChunkBytes + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024);
-            const uint64_t bd = tc::sw128_desc(q_base + (2 * m + (j >> 2)) * kQBoxBytes + (j & 3) * 32, 16, 1024);
-            tc::mma_bf16(tmem + kColS, ad, bd, idesc_s, (m | j) != 0);
+        for (int m = 0; m < 4; ++m) {
+#pragma unroll
+          for (int j = 0; j < kRows / 16; ++j) {
+            const uint64_t ad = tc::sw128_desc(kv_base + pb * kTileBytes + 2 * m * kBoxBytes + j * 2048, kBoxBytes, 1024);
+            const uint64_t bd = tc::sw128_desc(p_base + pb * kPBytes + j * 2048, kPBytes, 1024);
+            tc::mma_bf16(tmem + kColO + 64 * m, ad, bd, idesc_pv, t > 0 || j > 0);
           }
         }
-        if (!ok) break;
-        tc::commit(&sm->s_full);
-        ok = tc::mbar_wait(&sm->p_full, ph, abort, a.status);
+        tc::commit(&sm->kv_empty[pb]);
+        tc::commit(&sm->pv_done);
+        return true;
+      };
+      for (int li = 0; ok && li < ntiles; ++li) {
+        const int buf = li & 1;
+        ok = tc::mbar_wait(&sm->kv_full[buf], (li >> 1) & 1, abort, a.status);
         if (!ok) break;
         tc::fence_after_sync();
-        for (int m = 0; m < kChunks; ++m) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint64_t ad = tc::sw128_desc(kv_base + m * kChunkBytes + j * 2048, kBoxBytes, 1024);
-            const uint64_t bd = tc::sw128_desc(p_base + j * 2048, kPBytes, 1024);
-            tc::mma_bf16(tmem + kColO + 64 * m, ad, bd, idesc_pv, li > 0 || j > 0);
-          }
-          tc::commit(&sm->kv_empty[m]);
+        const uint32_t kb = kv_base + buf * kTileBytes;
+#pragma unroll 8
+        for (int j = 0; j < kD / 16; ++j) {
+          const uint64_t ad = tc::sw128_desc(kb + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(q_base + (j >> 2) * kQBoxBytes + (j & 3) * 32, 16, 1024);
+          tc::mma_bf16(tmem + kColS + 64 * buf, ad, bd, idesc_s, j > 0);
         }
+        tc::commit(&sm->s_full[buf]);
+        if (li > 0) ok = pv(li - 1);
       }
+      if (ok && ntiles > 0) pv(ntiles - 1);
       tc::commit(&sm->o_done);
       tc::mbar_drain(&sm->o_done, 0);
       if (q_issued) tc::mbar_drain(&sm->q_full, 0);
@@ -285,9 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
+    const int row = quarter * 16 + lane;                 // S^T row (lanes 0-15 of the quarter)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const bool leader = warp == kSoftWarp0;  // finalises per-head values
+    const bool leader = warp == kSoftWarp0;
     float l[kH];
 #pragma unroll
     for (int h = 0; h < kH; ++h) l[h] = 0.f;
@@ -295,28 +308,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     int idx_next = 0;
     {
       const int r = t0 * kRows + row;
-      if (ntiles > 0 && a.idx && r < L.nsel) idx_next = a.idx[(size_t)qq * a.k + r];
+      if (ntiles > 0 && lane < 16 && a.idx && r < L.nsel) idx_next = a.idx[(size_t)qq * a.k + r];
     }
     for (int li = 0; li < ntiles; ++li) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full, li & 1, abort, a.status));
+      const int buf = li & 1;
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full[buf], (li >> 1) & 1, abort, a.status));
       if (!ok) break;
       tc::fence_after_sync();
       const int r = (t0 + li) * kRows + row;
-      bool valid;
-      if (r < L.nsel4) {
-        valid = r < L.nsel && (!a.idx || (idx_next >= 0 && idx_next < a.N_max));
-      } else {
-        valid = r < L.R;
-      }
-      if (li + 1 < ntiles) {  // the next tile's index, loaded while this tile is processed
+      bool valid = lane < 16;
+      if (valid) valid = r < L.nsel4 ? (r < L.nsel && (!a.idx || (idx_next >= 0 && idx_next < a.N_max))) : r < L.R;
+      if (li + 1 < ntiles && lane < 16) {  // the next tile's index, loaded while this tile is processed
         const int rn = r + kRows;
         idx_next = (a.idx && rn < L.nsel) ? a.idx[(size_t)qq * a.k + rn] : 0;
       }
+      const uint32_t sbase = tmem + lane_off + kColS + 64 * buf;
       {
         float red[kH];
         uint32_t v0[32], v1[32];
-        tc::tmem_ld32(tmem + lane_off + kColS, v0);
-        tc::tmem_ld32(tmem + lane_off + kColS + 32, v1);
+        tc::tmem_ld32(sbase, v0);
+        tc::tmem_ld32(sbase + 32, v1);
         tc::tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
@@ -359,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          tc::tmem_ld32(tmem + lane_off + kColS + 32 * half, v);
+          tc::tmem_ld32(sbase + 32 * half, v);
           tc::tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
@@ -374,35 +385,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      const uint32_t prow = tc::smem_u32(ps) + row * 128;
+      if (lane < 16) {
+        const uint32_t prow = tc::smem_u32(ps) + buf * kPBytes + row * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t addr = prow + ((c ^ (row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
-                     "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                     : "memory");
-      }
-      if (rescale && li > 0) {
-        // O^T columns h *= alpha[h]; every PV of the previous tile has
-        // completed (its KV chunks had to be released before this tile's S).
-#pragma unroll 1
-        for (int m = 0; m < kChunks; ++m) {
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            const uint32_t ta = tmem + lane_off + kColO + 64 * m + 32 * half;
-            tc::tmem_ld32(ta, v);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * sm->alpha[32 * half + c]);
-            tmem_st32(ta, v);
-          }
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t addr = prow + ((c ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
+                       "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                       : "memory");
         }
-        tmem_st_wait();
+      }
+      if (li > 0) {
+        // P.V of the previous tile must be complete before O^T may be
+        // touched; consumed every tile so the barrier phases stay in step.
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->pv_done, (li - 1) & 1, abort, a.status));
+        if (!ok) break;
+        tc::fence_after_sync();
+        if (rescale) {
+#pragma unroll 1
+          for (int m = 0; m < 4; ++m) {
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              uint32_t v[32];
+              const uint32_t ta = tmem + lane_off + kColO + 64 * m + 32 * half;
+              tc::tmem_ld32(ta, v);
+              tc::tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * sm->alpha[32 * half + c]);
+              tmem_st32(ta, v);
+            }
+          }
+          tmem_st_wait();
+        }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc::fence_before_sync();
-      tc::mbar_arrive(&sm->p_full);
+      tc::mbar_arrive(&sm->p_full[buf]);
     }
     // ---- epilogue: per-head sums, then O (partials, or the final output)
     ok = __all_sync(0xffffffffu, ok && (ntiles == 0 || tc::mbar_wait(&sm->o_done, 0, abort, a.status)));
@@ -419,6 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     named_sync(1, 128);
+    const int orow = quarter * 32 + lane;  // O^T row (dims) within a 128-dim chunk
     const size_t pidx = (size_t)qq * splits + split;
     if (ok && splits > 1) {
       if (leader) {
@@ -431,8 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float *po = part_o + pidx * (size_t)kH * kD;
 #pragma unroll 1
-      for (int m = 0; m < kChunks; ++m) {
-        const int d = 128 * m + row;
+      for (int m = 0; m < 4; ++m) {
+        const int d = 128 * m + orow;
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           uint32_t v[32];
@@ -462,8 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_sync(1, 128);
       bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qq * kH * kD;
 #pragma unroll 1
-      for (int m = 0; m < kChunks; ++m) {
-        const int d = 128 * m + row;
+      for (int m = 0; m < 4; ++m) {
+        const int d = 128 * m + orow;
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           uint32_t v[32];
@@ -490,19 +509,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Block (query, 16-head group), 256 threads, 32 outputs per thread.
 __global__ void __launch_bounds__(256) mqa_combine_kernel(const float *part_o, const float *part_ml,
                                                           const float *sink, bf16 *out, int splits) {
-  extern __shared__ float f[];  // [splits][16]
+  extern __shared__ float f[];  // [splits][16] weights, then [2][splits][16] (m, l)
   const int qq = blockIdx.x, hg = blockIdx.y;
-  for (int i = threadIdx.x; i < 16; i += blockDim.x) {
-    const int h = hg * 16 + i;
-    float M = sink[h] * kLog2e;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[(((size_t)qq * splits + s) * 2) * kH + h]);
-    float Lsum = exp2f(sink[h] * kLog2e - M);
+  float *ml = f + splits * 16;
+  for (int i = threadIdx.x; i < 2 * splits * 16; i += blockDim.x) {  // all (m, l) loads in flight at once
+    const int which = i / (splits * 16), rem = i - which * splits * 16, s = rem / 16, h = hg * 16 + rem % 16;
+    ml[i] = part_ml[(((size_t)qq * splits + s) * 2 + which) * kH + h];
+  }
+  __syncthreads();
+  if (threadIdx.x < 16) {
+    const int i = threadIdx.x, h = hg * 16 + i;
+    const float sk = sink[h] * kLog2e;
+    float M = sk;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[s * 16 + i]);
+    float Lsum = exp2f(sk - M);
     for (int s = 0; s < splits; ++s) {
-      const size_t p = ((size_t)qq * splits + s) * 2;
-      const float ms = part_ml[p * kH + h];
+      const float ms = ml[s * 16 + i];
       const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
       f[s * 16 + i] = w;
-      Lsum += part_ml[(p + 1) * kH + h] * w;
+      Lsum += ml[(splits + s) * 16 + i] * w;
     }
     const float inv = 1.f / Lsum;
     for (int s = 0; s < splits; ++s) f[s * 16 + i] *= inv;
@@ -548,8 +573,8 @@ void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 bool tc_shape(const MqaArgs &a) {
-  return a.dtype == CSA_DTYPE_BF16 && a.H == kH && a.D == kD && a.Q <= 65535 && aligned16(a.q) && aligned16(a.kv_cmp) &&
-         aligned16(a.kv_win) && aligned16(a.out);
+  return a.dtype == CSA_DTYPE_BF16 && a.H == kH && a.D == kD && a.Q <= 65535 && aligned16(a.q) &&
+         aligned16(a.kv_cmp) && aligned16(a.kv_win) && aligned16(a.out);
 }
 
 int rows_max_of(const MqaArgs &a) { return (((a.idx ? a.k : a.N_max) + 3) & ~3) + a.win_len; }
@@ -570,15 +595,18 @@ size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
 cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   *taken = false;
   if (!tc_shape(a)) return cudaSuccess;
-  const int rows_max = rows_max_of(a);
   int splits, tps;
-  plan_splits(a.Q, rows_max, &splits, &tps);
+  plan_splits(a.Q, rows_max_of(a), &splits, &tps);
   const size_t need = splits > 1 ? (size_t)a.Q * splits * kH * (kD + 2) * sizeof(float) : 0;
   if (need > a.partial_bytes) return cudaSuccess;  // cannot happen with the documented workspace size
-  CUtensorMap tm_q, tm_cmp, tm_win;
-  if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * kH, kD * 2, 64, kH)) return cudaSuccess;
-  if (!make_tmap_bf16_2d(&tm_cmp, a.kv_cmp, kD, (uint64_t)a.B * a.N_max, kD * 2, 64, 1)) return cudaSuccess;
-  if (!make_tmap_bf16_2d(&tm_win, a.kv_win, kD, (uint64_t)a.B * a.T_raw, kD * 2, 64, 1)) return cudaSuccess;
+  CUtensorMap tm_q, tm_cmp_g, tm_win_g, tm_cmp_t, tm_win_t;
+  const uint64_t cmp_rows = (uint64_t)a.B * a.N_max, win_rows = (uint64_t)a.B * a.T_raw;
+  if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * kH, kD * 2, 64, kH) ||
+      !make_tmap_bf16_2d(&tm_cmp_g, a.kv_cmp, kD, cmp_rows, kD * 2, 64, 1) ||
+      !make_tmap_bf16_2d(&tm_win_g, a.kv_win, kD, win_rows, kD * 2, 64, 1) ||
+      !make_tmap_bf16_2d(&tm_cmp_t, a.kv_cmp, kD, cmp_rows, kD * 2, 64, kRows) ||
+      !make_tmap_bf16_2d(&tm_win_t, a.kv_win, kD, win_rows, kD * 2, 64, kRows))
+    return cudaSuccess;
   float *part_o = static_cast<float *>(a.partials);
   float *part_ml = part_o + (size_t)a.Q * splits * kH * kD;
   static bool attr_set = false;
@@ -587,13 +615,13 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
     attr_set = true;
   }
   dim3 grid(splits, a.Q);
-  mqa_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_cmp, tm_win, a, splits, tps, a.scale * kLog2e,
-                                                        part_o, part_ml);
+  mqa_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_cmp_g, tm_win_g, tm_cmp_t, tm_win_t, a, splits, tps,
+                                                        a.scale * kLog2e, part_o, part_ml);
   note_launches(1);
   if (splits > 1) {
     dim3 cg(a.Q, kH / 16);
-    mqa_combine_kernel<<<cg, 256, splits * 16 * sizeof(float), stream>>>(part_o, part_ml, a.sink,
-                                                                         static_cast<bf16 *>(a.out), splits);
+    mqa_combine_kernel<<<cg, 256, splits * 48 * sizeof(float), stream>>>(part_o, part_ml, a.sink,
+                                                                        static_cast<bf16 *>(a.out), splits);
     note_launches(1);
   }
   *taken = true;

@@ -1,0 +1,101 @@
+"""A whole decode step of one CSA or HCA attention layer, replayed from a
+CUDA graph.
+
+The step over device-resident caches is:
+  1. fold the newest raw window of every sequence into its compressed cache
+     (csa_compress; CSA every 4 tokens, HCA every 128) -- on a forked stream,
+     concurrently with 2 when the layer is CSA;
+  2. CSA only: score every visible compressed entry and select the top-k
+     (csa_index_topk);
+  3. attend over the selected (CSA) or all visible (HCA) entries + the
+     sliding window + the per-head sink (csa_sparse_mqa / hca_mqa).
+The library never allocates or synchronises, so the launches are captured
+once into a CUDA graph and each step is one graph launch. Buffers are bound
+at construction; later steps see whatever the caller wrote into them.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import ops
+
+
+class DecodeStep:
+    def __init__(self, *, q, kv_cmp, kv_win, sink, scale: float, win_len: int, win_end, n_cmp,
+                 ape, norm_w, gate, append_src0: int, append_dst0: int, win: int, stride: int,
+                 qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True):
+        self.csa = qi is not None
+        self.q, self.kv_cmp, self.kv_win, self.sink = q, kv_cmp, kv_win, sink
+        self.scale, self.win_len, self.win_end, self.n_cmp = float(scale), int(win_len), win_end, n_cmp
+        self.ape, self.norm_w, self.gate = ape, norm_w, gate
+        self.win, self.stride = int(win), int(stride)
+        T_c = gate.shape[1]
+        n_new = (T_c - self.win) // self.stride + 1
+        self.kv_src = kv_win[:, append_src0:append_src0 + T_c]
+        self.cmp_dst = kv_cmp[:, append_dst0:append_dst0 + n_new]
+        self.qi, self.wi, self.ki, self.k = qi, wi, ki, k
+        dev = q.device
+        self.out = out if out is not None else torch.empty_like(q)
+        self.idx = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev) if self.csa else None
+        self.ws_index = ops.Workspace(dev)
+        self.ws_mqa = ops.Workspace(dev)
+        self.side = torch.cuda.Stream(dev)
+        self.graph = None
+        self.run_eager()  # sizes the workspaces and sets kernel attributes
+        torch.cuda.synchronize(dev)
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._launch()
+            self.graph = g
+
+    # -- the parts, on the current stream --------------------------------
+    def append(self):
+        ops.compress(self.kv_src, self.gate, self.ape, self.norm_w, self.win, self.stride, out=self.cmp_dst)
+
+    def select(self):
+        ops.index_topk(self.qi, self.wi, self.ki, self.n_cmp, self.k, out=self.idx, ws=self.ws_index)
+
+    def attend(self):
+        if self.csa:
+            ops.sparse_mqa(self.q, self.kv_cmp, self.idx, self.kv_win, self.win_end, self.sink, self.scale,
+                           self.win_len, out=self.out, ws=self.ws_mqa)
+        else:
+            ops.hca_mqa(self.q, self.kv_cmp, self.n_cmp, self.kv_win, self.win_end, self.sink, self.scale,
+                        self.win_len, out=self.out, ws=self.ws_mqa)
+
+    def parts(self):
+        p = [("compress", self.append)]
+        if self.csa:
+            p.append(("index_topk", self.select))
+        p.append(("mqa", self.attend))
+        return p
+
+    def _launch(self):
+        main = torch.cuda.current_stream()
+        if self.csa:
+            # the append only feeds the attention: overlap it with the indexer
+            self.side.wait_stream(main)
+            with torch.cuda.stream(self.side):
+                self.append()
+            self.select()
+            main.wait_stream(self.side)
+        else:
+            self.append()
+        self.attend()
+
+    def run_eager(self):
+        """The step as individual launches (no graph)."""
+        self._launch()
+
+    def run(self):
+        """One step: a single graph launch on the current stream."""
+        if self.graph is None:
+            self._launch()
+        else:
+            self.graph.replay()
+        return self.out
+
+    def status(self) -> int:
+        """Synchronise and return (and clear) the device status bits."""
+        return self.ws_index.status() | self.ws_mqa.status()
