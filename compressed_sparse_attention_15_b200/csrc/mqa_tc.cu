@@ -506,48 +506,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Merge the split partials of each query with the sink:
 //   M = max(max_s m_s, sink), L = sum_s l_s 2^(m_s - M) + 2^(sink - M),
 //   out = sum_s O_s 2^(m_s - M) / L   (m and sink in log2 units).
-// Block (query, 16-head group), 256 threads, 32 outputs per thread.
-__global__ void __launch_bounds__(256) mqa_combine_kernel(const float *part_o, const float *part_ml,
+// One block per (query, head); thread t owns dims 4t..4t+3 and issues the
+// loads of all splits at once.
+__global__ void __launch_bounds__(128) mqa_combine_kernel(const float *part_o, const float *part_ml,
                                                           const float *sink, bf16 *out, int splits) {
-  extern __shared__ float f[];  // [splits][16] weights, then [2][splits][16] (m, l)
-  const int qq = blockIdx.x, hg = blockIdx.y;
-  float *ml = f + splits * 16;
-  for (int i = threadIdx.x; i < 2 * splits * 16; i += blockDim.x) {  // all (m, l) loads in flight at once
-    const int which = i / (splits * 16), rem = i - which * splits * 16, s = rem / 16, h = hg * 16 + rem % 16;
+  extern __shared__ float w[];  // [splits] weights, then [2][splits] (m, l)
+  const int qq = blockIdx.x, h = blockIdx.y;
+  float *ml = w + splits;
+  for (int i = threadIdx.x; i < 2 * splits; i += blockDim.x) {
+    const int which = i / splits, s = i - which * splits;
     ml[i] = part_ml[(((size_t)qq * splits + s) * 2 + which) * kH + h];
   }
   __syncthreads();
-  if (threadIdx.x < 16) {
-    const int i = threadIdx.x, h = hg * 16 + i;
+  if (threadIdx.x == 0) {
     const float sk = sink[h] * kLog2e;
     float M = sk;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[s * 16 + i]);
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[s]);
     float Lsum = exp2f(sk - M);
     for (int s = 0; s < splits; ++s) {
-      const float ms = ml[s * 16 + i];
-      const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
-      f[s * 16 + i] = w;
-      Lsum += ml[(splits + s) * 16 + i] * w;
+      const float ww = ml[s] == -INFINITY ? 0.f : exp2f(ml[s] - M);
+      w[s] = ww;
+      Lsum += ml[splits + s] * ww;
     }
     const float inv = 1.f / Lsum;
-    for (int s = 0; s < splits; ++s) f[s * 16 + i] *= inv;
+    for (int s = 0; s < splits; ++s) w[s] *= inv;
   }
   __syncthreads();
-  for (int e = threadIdx.x * 4; e < 16 * kD; e += blockDim.x * 4) {
-    const int i = e / kD, d = e - i * kD, h = hg * 16 + i;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < splits; ++s) {
-      const float w = f[s * 16 + i];
-      const float4 v = *reinterpret_cast<const float4 *>(part_o + (((size_t)qq * splits + s) * kH + h) * kD + d);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-    *reinterpret_cast<uint2 *>(out + ((size_t)qq * kH + h) * kD + d) = pk;
+  const int d = 4 * threadIdx.x;
+  const float *src = part_o + ((size_t)qq * splits * kH + h) * kD + d;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int s = 0; s < splits; ++s) {
+    const float4 v = *reinterpret_cast<const float4 *>(src + (size_t)s * kH * kD);
+    const float ww = w[s];
+    acc.x = fmaf(ww, v.x, acc.x);
+    acc.y = fmaf(ww, v.y, acc.y);
+    acc.z = fmaf(ww, v.z, acc.z);
+    acc.w = fmaf(ww, v.w, acc.w);
   }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+  *reinterpret_cast<uint2 *>(out + ((size_t)qq * kH + h) * kD + d) = pk;
 }
 
 int num_sms_cached() {
@@ -619,9 +618,9 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
                                                         a.scale * kLog2e, part_o, part_ml);
   note_launches(1);
   if (splits > 1) {
-    dim3 cg(a.Q, kH / 16);
-    mqa_combine_kernel<<<cg, 256, splits * 48 * sizeof(float), stream>>>(part_o, part_ml, a.sink,
-                                                                        static_cast<bf16 *>(a.out), splits);
+    dim3 cg(a.Q, kH);
+    mqa_combine_kernel<<<cg, kD / 4, splits * 3 * sizeof(float), stream>>>(part_o, part_ml, a.sink,
+                                                                          static_cast<bf16 *>(a.out), splits);
     note_launches(1);
   }
   *taken = true;

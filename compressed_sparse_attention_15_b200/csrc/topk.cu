@@ -6,9 +6,9 @@
 // towards the smaller index; it is written in ascending index order and
 // padded with -1.
 //
-// Method: radix select (MSD; digits of 11, 11 and 10 bits) on an
-// order-preserving 32-bit key of each fp32 score finds the k-th largest key
-// tau and how many entries equal to tau are still needed (kk). A final
+// Method: radix select (MSD, 11-bit digits over the occupied key range) on
+// an order-preserving 32-bit key of each fp32 score finds the k-th largest
+// key tau and how many entries equal to tau are still needed (kk). A final
 // ordered pass keeps every entry with key > tau and the first kk entries (by
 // index) with key == tau; per-warp ballots and an exclusive prefix over the
 // block give each kept entry its output slot, so the output is ascending and
@@ -34,7 +34,7 @@ struct TopkShared {
   uint32_t hist[kBins];
   uint32_t scan[kWarps];
   uint32_t warp_gt[kWarps], warp_eq[kWarps];
-  uint32_t prefix, kk;
+  uint32_t prefix, kk, kmin, krange;
 };
 
 // Exclusive prefix sum over the block (thread order) of one value per thread.
@@ -69,31 +69,57 @@ __device__ __forceinline__ uint32_t key_at(const uint32_t *keys, const float *s,
 
 // Select the k largest of n keys (ties -> smaller position) and call
 // emit(slot, position, key) for each, slots 0..k-1 in ascending position.
+// The radix digits are taken over (key - min key), from the highest set bit
+// of the key range down, so the first digit already splits the keys that
+// actually occur (scores of one query usually share sign and exponent).
 template <bool kCached, class Emit>
 __device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const float *s, int n, int k, Emit emit) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) {
-    sh.prefix = 0;
-    sh.kk = (uint32_t)k;
+  // key range
+  uint32_t lo_k = 0xffffffffu, hi_k = 0u;
+  for (int j = threadIdx.x; j < n; j += kThreads) {
+    const uint32_t u = key_at<kCached>(keys, s, j);
+    lo_k = min(lo_k, u);
+    hi_k = max(hi_k, u);
   }
-  uint32_t mask = 0;
-  const int shifts[3] = {21, 10, 0};
-  const uint32_t widths[3] = {11, 11, 10};
-#pragma unroll 1
-  for (int p = 0; p < 3; ++p) {
-    const int shift = shifts[p];
-    const uint32_t dmask = (1u << widths[p]) - 1u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo_k = min(lo_k, __shfl_xor_sync(0xffffffffu, lo_k, o));
+    hi_k = max(hi_k, __shfl_xor_sync(0xffffffffu, hi_k, o));
+  }
+  if (lane == 0) {
+    sh.warp_gt[warp] = lo_k;
+    sh.warp_eq[warp] = hi_k;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = sh.warp_gt[lane], b = sh.warp_eq[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+      b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
+    }
+    if (lane == 0) {
+      sh.kmin = a;
+      sh.prefix = 0;
+      sh.kk = (uint32_t)k;
+    }
+    if (lane == 1) sh.krange = b - a;
+  }
+  __syncthreads();
+  const uint32_t kmin = sh.kmin, range = sh.krange;
+  const int nbits = range == 0 ? 0 : 32 - __clz(range);
+  uint32_t mask = 0;  // bits of (key - kmin) fixed so far
+  for (int top = nbits; top > 0;) {
+    const int width = top >= 11 ? 11 : top;
+    const int shift = top - width;
+    const uint32_t dmask = (1u << width) - 1u;
     for (int i = threadIdx.x; i < kBins; i += kThreads) sh.hist[i] = 0;
     __syncthreads();
     const uint32_t prefix = sh.prefix;
-    for (int base = 0; base < n; base += kThreads) {
-      const int j = base + threadIdx.x;
-      const uint32_t u = j < n ? key_at<kCached>(keys, s, j) : 0u;
-      const bool in = j < n && (u & mask) == prefix;
-      const uint32_t bin = in ? (u >> shift) & dmask : 0xffffffffu;
-      // warp-aggregated increment: one atomic per distinct bin in the warp
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (in && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (uint32_t)__popc(peers));
+    for (int j = threadIdx.x; j < n; j += kThreads) {
+      const uint32_t u = key_at<kCached>(keys, s, j) - kmin;
+      if ((u & mask) == prefix) atomicAdd(&sh.hist[(u >> shift) & dmask], 1u);
     }
     __syncthreads();
     // Thread t owns bins B-1-2t and B-2-2t (descending), so an exclusive
@@ -109,9 +135,10 @@ __device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const floa
       sh.prefix = prefix | (bin << shift);
     }
     mask |= dmask << shift;
+    top = shift;
     __syncthreads();
   }
-  const uint32_t tau = sh.prefix, kk = sh.kk;
+  const uint32_t tau = sh.prefix + kmin, kk = sh.kk;
   // Ordered compaction: warp w scans the contiguous range [lo, hi).
   const int per_warp = (((n + kWarps - 1) / kWarps) + 31) & ~31;
   const int lo = min(n, warp * per_warp), hi = min(n, lo + per_warp);
