@@ -56,6 +56,8 @@ const char *csa_strerror(int code) {
     case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE: workspace too small or not 256-byte aligned";
     case CSA_ERR_CUDA: return "CSA_ERR_CUDA: a CUDA call failed";
     case CSA_ERR_DEVICE: return "CSA_ERR_DEVICE: the workspace status word is set";
+    case CSA_ERR_SCRATCH_LIMIT:
+      return "CSA_ERR_SCRATCH_LIMIT: the request needs more than the built-in scratch of csa_index_topk_noalloc";
     default: return "unknown csa status code";
   }
 }

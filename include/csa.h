@@ -54,7 +54,9 @@ enum {
   CSA_ERR_UNSUPPORTED = 2, /* no sm_100 device current, or an uncompiled size/dtype combination */
   CSA_ERR_WORKSPACE = 3,   /* workspace smaller than *_workspace_bytes() */
   CSA_ERR_CUDA = 4,        /* a CUDA launch or attribute call failed */
-  CSA_ERR_DEVICE = 5       /* (csa_workspace_status only) the status word is non-zero */
+  CSA_ERR_DEVICE = 5,      /* (csa_workspace_status only) the status word is non-zero */
+  CSA_ERR_SCRATCH_LIMIT = 6 /* (csa_index_topk_noalloc only) the request needs more scratch than
+                               CSA_NOALLOC_SCRATCH_BYTES */
 };
 
 /* Element types of the dtype-typed tensors. */
@@ -189,6 +191,32 @@ int hca_mqa(const void *q, const void *kv_cmp, const void *kv_win, const float *
             int Q, int B, int H, int D, int N_max, const int32_t *n_cmp, int win_len,
             const int32_t *win_end, int T_raw, int q_per_seq, int dtype,
             void *ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa_index_topk_noalloc -- csa_index_topk for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot provide device memory of their own: a plugin that only receives the
+ * input and output pointers from a host framework whose memory pools it must
+ * not bypass, or a latency-bound decode loop that may not call cudaMalloc
+ * (which can synchronise the device) in the middle of a step. It computes
+ * exactly what csa_index_topk computes, with the same arguments minus the
+ * workspace, and allocates nothing: its scratch is a buffer built into the
+ * library, CSA_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that loads
+ * the library until the process exits.
+ *  - Requests whose csa_index_topk_workspace_bytes(Q, N_max, k) exceeds that
+ *    size return CSA_ERR_SCRATCH_LIMIT and launch nothing.
+ *  - The first call on a device looks the buffer's device address up (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one buffer and it keeps the last call's contents;
+ *    calls whose work overlaps on the GPU (different streams or host
+ *    threads) race on it. Device-side status bits are cleared at the start
+ *    of every call and cannot be read back through this entry point.
+ * ---------------------------------------------------------------------- */
+#define CSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int csa_index_topk_noalloc(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int k,
+                           int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max, int q_per_seq,
+                           int dtype, csa_stream_t stream);
 
 /* Number of kernels this library has launched in this process so far
  * (a monotonically increasing counter, for profiling and tests). */

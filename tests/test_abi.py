@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported_and_bound(L):
 
 
 def test_strerror(L):
-    for c in range(6):
+    for c in range(7):
         assert _lib.strerror(c).startswith("CSA_")
     assert "unknown" in _lib.strerror(99)
 
