@@ -390,6 +390,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    ap.add_argument("--once", action="store_true",
+                    help="profiling aid: build the step without a graph and launch each of its kernels once more")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -415,6 +417,14 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
         return 1
+    if args.once:
+        step = Step(w, torch.device("cuda", 0), graph=False)  # runs the step once while building it
+        torch.cuda.synchronize()
+        for _, f in step.parts():
+            f()
+        torch.cuda.synchronize()
+        print(json.dumps({"once": w.name, "status": step.ds.status()}))
+        return 0
     dist_on = world > 1
     if dist_on:
         import datetime
