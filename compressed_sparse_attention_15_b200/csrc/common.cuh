@@ -53,4 +53,11 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Programmatic dependent launch. Kernels are launched so that they may start
+// while the previous kernel in the stream finishes; pdl_wait() blocks until
+// that kernel has completed and its writes are visible, and must precede the
+// first read of any input. pdl_release() lets the next kernel begin launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace csa

@@ -36,6 +36,8 @@ constexpr float kRmsEps = 1e-6f;
 template <typename T>
 __global__ void __launch_bounds__(256) compress_generic_kernel(CompressArgs a) {
   extern __shared__ float c_smem[];
+  pdl_wait();
+  pdl_release();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, wpb = blockDim.x >> 5;
   float *c = c_smem + (size_t)warp * a.D;
   const long long total = (long long)a.B * a.N;
@@ -103,6 +105,8 @@ __device__ __forceinline__ uint4 pack8(const float f[8]) {
 // One block per (sequence, entry).
 __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, int G) {
   extern __shared__ float ws[];  // [G][3][8][nvec] partial states, then [32] sums
+  pdl_wait();
+  pdl_release();
   const int nvec = a.D / 8;
   const int v = threadIdx.x % nvec, g = threadIdx.x / nvec;
   const long long e = blockIdx.x;
@@ -207,6 +211,8 @@ __global__ void __launch_bounds__(256) compress_stream_kernel(CompressArgs a, lo
   extern __shared__ float ape_s[];  // [W][D] * log2 e
   __shared__ float grp_sum[8];
   const int D = a.D;
+  pdl_wait();
+  pdl_release();
   for (int i = threadIdx.x; i < W * D; i += blockDim.x) ape_s[i] = a.ape[i] * kLog2e;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -325,9 +331,7 @@ cudaError_t launch_stream(const CompressArgs &a, cudaStream_t stream) {
   groups = (total + per - 1) / per;
   const long long blocks = (groups + groups_per_block - 1) / groups_per_block;
   const size_t smem = (size_t)2 * S * a.D * sizeof(float);
-  compress_stream_kernel<WPR, S><<<(unsigned)blocks, 256, smem, stream>>>(a, per);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(compress_stream_kernel<WPR, S>, dim3((unsigned)blocks), dim3(256), smem, stream, a, per);
 }
 
 }  // namespace
@@ -353,9 +357,7 @@ cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
                              (int)(((size_t)3 * 8 * 512 + 32) * sizeof(float)));
         attr_set = true;
       }
-      compress_window_kernel<<<(unsigned)total, G * nvec, smem, stream>>>(a, G);
-      note_launches(1);
-      return cudaGetLastError();
+      return launch_pdl(compress_window_kernel, dim3((unsigned)total), dim3(G * nvec), smem, stream, a, G);
     }
   }
   const int threads = 256, wpb = threads / 32;
@@ -369,11 +371,8 @@ cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
     attr_set = true;
   }
   if (a.dtype == CSA_DTYPE_F32)
-    compress_generic_kernel<float><<<(unsigned)blocks, threads, smem, stream>>>(a);
-  else
-    compress_generic_kernel<bf16><<<(unsigned)blocks, threads, smem, stream>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+    return launch_pdl(compress_generic_kernel<float>, dim3((unsigned)blocks), dim3(threads), smem, stream, a);
+  return launch_pdl(compress_generic_kernel<bf16>, dim3((unsigned)blocks), dim3(threads), smem, stream, a);
 }
 
 }  // namespace csa

@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(256) index_scores_generic_kernel(ScoreArgs a) 
   float *sk = sq + Hi * Di;               // [64][Di + 1] (padded against bank conflicts)
   float *sw = sk + kTileJ * (Di + 1);     // [Hi]
   float *part = sw + Hi;                  // [4][64]
+  pdl_wait();
+  pdl_release();
   const int q = blockIdx.x;
   const int n = clamp_count(a.n_cmp[q], a.N_max, threadIdx.x == 0 ? a.status : nullptr);
   const int j0 = blockIdx.y * kTileJ;
@@ -74,12 +76,8 @@ cudaError_t launch_index_scores(const ScoreArgs &a, cudaStream_t stream) {
     cudaFuncSetAttribute(index_scores_generic_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     attr_set = true;
   }
-  if (a.dtype == CSA_DTYPE_F32)
-    index_scores_generic_kernel<float><<<grid, 256, smem, stream>>>(a);
-  else
-    index_scores_generic_kernel<bf16><<<grid, 256, smem, stream>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+  if (a.dtype == CSA_DTYPE_F32) return launch_pdl(index_scores_generic_kernel<float>, grid, dim3(256), smem, stream, a);
+  return launch_pdl(index_scores_generic_kernel<bf16>, grid, dim3(256), smem, stream, a);
 }
 
 }  // namespace csa

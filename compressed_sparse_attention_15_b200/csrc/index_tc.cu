@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
+  pdl_wait();  // inputs may come from the previous kernel in the stream
+  pdl_release();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -256,11 +258,9 @@ cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool
     cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     attr_set = true;
   }
-  index_scores_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(tm_ki, tm_qi, a, tiles_per_q, total,
-                                                                             per_cta);
-  note_launches(1);
   *taken = true;
-  return cudaGetLastError();
+  return launch_pdl(index_scores_tc_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tm_ki, tm_qi, a,
+                    tiles_per_q, total, per_cta);
 }
 
 }  // namespace csa

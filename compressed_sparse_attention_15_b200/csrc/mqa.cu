@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(kThreads) mqa_generic_kernel(MqaArgs a) {
   __shared__ float m_s[HG], l_s[HG], alpha_s[HG];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int qq = blockIdx.x, h0 = blockIdx.y * HG;
+  pdl_wait();
+  pdl_release();
   const int b = qq / a.q_per_seq;
   uint32_t *st = tid == 0 ? a.status : nullptr;
   const int nsel = a.idx ? a.k : clamp_count(a.n_cmp[qq], a.N_max, st);
@@ -148,9 +150,7 @@ cudaError_t launch_generic(const MqaArgs &a, cudaStream_t stream) {
     attr_set = true;
   }
   dim3 grid(a.Q, a.H / HG);
-  mqa_generic_kernel<T, HG><<<grid, kThreads, smem, stream>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(mqa_generic_kernel<T, HG>, grid, dim3(kThreads), smem, stream, a);
 }
 
 template <typename T>

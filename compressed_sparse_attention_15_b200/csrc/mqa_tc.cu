@@ -58,12 +58,13 @@ constexpr float kRescaleLog2 = 8.0f;
 struct Small {
   uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done, o_done;
   float red[4][kH];
-  float mref[kH];
+  alignas(16) float mref[kH];
   float alpha[kH];
   float lsum[kH];
   uint32_t tmem_base;
   int abort;
   int rescale;
+  int need[4];  // per tile (mod 4): some logit exceeded the running maximum by more than 2^8
 };
 
 constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kQBytes + 2 * kPBytes + sizeof(Small);
@@ -115,6 +116,14 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(col), "r"(rc[0]), "r"(rc[1]),
         "r"(rc[2]), "r"(rc[3])
       : "memory");
+}
+
+// 2^x on the SFU (relative error about 2^-22; flushes subnormal results to
+// zero, which only ever meets weights far below the bf16 resolution of P).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void named_sync(int id, int n) {
@@ -179,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&sm->o_done, 1);
     sm->abort = 0;
     sm->rescale = 0;
+    for (int i = 0; i < 4; ++i) sm->need[i] = 0;
     tc::fence_barrier_init();
   }
   if (threadIdx.x < kH) {
@@ -191,6 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = sm->tmem_base;
   volatile int *abort = &sm->abort;
+  pdl_wait();  // inputs (indices, queries, caches) may come from the previous kernel
+  pdl_release();
 
   const RowList L = row_list(a, qq, threadIdx.x == 0 ? a.status : nullptr);
   const int tiles_all = (L.R + kRows - 1) / kRows;
@@ -262,14 +274,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pb = t & 1;
         if (!tc::mbar_wait(&sm->p_full[pb], (t >> 1) & 1, abort, a.status)) return false;
         tc::fence_after_sync();
+        const uint64_t ad0 = tc::sw128_desc(kv_base + pb * kTileBytes, kBoxBytes, 1024);
+        const uint64_t bd0 = tc::sw128_desc(p_base + pb * kPBytes, kPBytes, 1024);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
 #pragma unroll
-          for (int j = 0; j < kRows / 16; ++j) {
-            const uint64_t ad = tc::sw128_desc(kv_base + pb * kTileBytes + 2 * m * kBoxBytes + j * 2048, kBoxBytes, 1024);
-            const uint64_t bd = tc::sw128_desc(p_base + pb * kPBytes + j * 2048, kPBytes, 1024);
-            tc::mma_bf16(tmem + kColO + 64 * m, ad, bd, idesc_pv, t > 0 || j > 0);
-          }
+          for (int j = 0; j < kRows / 16; ++j)
+            tc::mma_bf16(tmem + kColO + 64 * m, ad0 + (uint64_t)((2 * m * kBoxBytes + j * 2048) >> 4),
+                         bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv, t > 0 || j > 0);
         }
         tc::commit(&sm->kv_empty[pb]);
         tc::commit(&sm->pv_done);
@@ -280,13 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = tc::mbar_wait(&sm->kv_full[buf], (li >> 1) & 1, abort, a.status);
         if (!ok) break;
         tc::fence_after_sync();
-        const uint32_t kb = kv_base + buf * kTileBytes;
-#pragma unroll 8
-        for (int j = 0; j < kD / 16; ++j) {
-          const uint64_t ad = tc::sw128_desc(kb + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sw128_desc(q_base + (j >> 2) * kQBoxBytes + (j & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem + kColS + 64 * buf, ad, bd, idesc_s, j > 0);
-        }
+        // descriptors differ only in the start-address field (16-byte units)
+        const uint64_t ad0 = tc::sw128_desc(kv_base + buf * kTileBytes, 16, 1024);
+        const uint64_t bd0 = tc::sw128_desc(q_base, 16, 1024);
+#pragma unroll
+        for (int j = 0; j < kD / 16; ++j)
+          tc::mma_bf16(tmem + kColS + 64 * buf, ad0 + (uint64_t)(((j >> 2) * kBoxBytes + (j & 3) * 32) >> 4),
+                       bd0 + (uint64_t)(((j >> 2) * kQBoxBytes + (j & 3) * 32) >> 4), idesc_s, j > 0);
         tc::commit(&sm->s_full[buf]);
         if (li > 0) ok = pv(li - 1);
       }
@@ -323,67 +335,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         idx_next = (a.idx && rn < L.nsel) ? a.idx[(size_t)qq * a.k + rn] : 0;
       }
       const uint32_t sbase = tmem + lane_off + kColS + 64 * buf;
-      {
-        float red[kH];
-        uint32_t v0[32], v1[32];
-        tc::tmem_ld32(sbase, v0);
+      uint32_t v0[32], v1[32];
+      tc::tmem_ld32(sbase, v0);
+      tc::tmem_ld32(sbase + 32, v1);
+      tc::tmem_ld_wait();
+      // Fast path: the running per-head maximum moves only when some logit
+      // of the tile exceeds it by more than 2^8 (always on the first tile).
+      bool over = false;
+      if (valid) {
+#pragma unroll
+        for (int h = 0; h < kH; h += 4) {
+          const float4 mr = *reinterpret_cast<const float4 *>(&sm->mref[h]);
+          const float mm[4] = {mr.x, mr.y, mr.z, mr.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float x = __uint_as_float(h + i < 32 ? v0[h + i] : v1[h + i - 32]) * scale_log2;
+            over |= x > mm[i] + kRescaleLog2;
+          }
+        }
+      }
+      if (leader && lane == 0) sm->need[(li + 2) & 3] = 0;  // slot of tile li + 2, last read at tile li - 2
+      if (__any_sync(0xffffffffu, over) && lane == 0) atomicOr(&sm->need[li & 3], 1);
+      named_sync(1, 128);
+      bool rescale = false;
+      if (sm->need[li & 3] != 0) {
+        {
+          float red[kH];
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            red[h] = valid ? __uint_as_float(v0[h]) * scale_log2 : -INFINITY;
+            red[h + 32] = valid ? __uint_as_float(v1[h]) * scale_log2 : -INFINITY;
+          }
+          transpose_reduce64<true>(red, lane);
+          sm->red[quarter][2 * lane] = red[0];
+          sm->red[quarter][2 * lane + 1] = red[1];
+        }
+        named_sync(1, 128);
+        if (leader) {
+          bool any = false;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int h = 2 * lane + i;
+            const float tm = fmaxf(fmaxf(sm->red[0][h], sm->red[1][h]), fmaxf(sm->red[2][h], sm->red[3][h]));
+            const float mo = sm->mref[h];
+            float al = 1.f;
+            if (mo == -INFINITY || tm > mo + kRescaleLog2) {
+              const float mn = fmaxf(mo, tm);
+              al = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+              sm->mref[h] = mn;
+              any |= mo != -INFINITY;
+            }
+            sm->alpha[h] = al;
+          }
+          any = __any_sync(0xffffffffu, any);
+          if (lane == 0) sm->rescale = any ? 1 : 0;
+        }
+        named_sync(1, 128);
+        rescale = sm->rescale != 0;
+        if (rescale) {
+#pragma unroll
+          for (int h = 0; h < kH; ++h) l[h] *= sm->alpha[h];
+        }
+        tc::tmem_ld32(sbase, v0);  // the logits again (registers were released for the reduction)
         tc::tmem_ld32(sbase + 32, v1);
         tc::tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          red[h] = valid ? __uint_as_float(v0[h]) * scale_log2 : -INFINITY;
-          red[h + 32] = valid ? __uint_as_float(v1[h]) * scale_log2 : -INFINITY;
-        }
-        transpose_reduce64<true>(red, lane);
-        sm->red[quarter][2 * lane] = red[0];
-        sm->red[quarter][2 * lane + 1] = red[1];
       }
-      named_sync(1, 128);
-      if (leader) {
-        bool any = false;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int h = 2 * lane + i;
-          const float tm = fmaxf(fmaxf(sm->red[0][h], sm->red[1][h]), fmaxf(sm->red[2][h], sm->red[3][h]));
-          const float mo = sm->mref[h];
-          float al = 1.f;
-          if (mo == -INFINITY || tm > mo + kRescaleLog2) {
-            const float mn = fmaxf(mo, tm);
-            al = mo == -INFINITY ? 0.f : exp2f(mo - mn);
-            sm->mref[h] = mn;
-            any |= mo != -INFINITY;
-          }
-          sm->alpha[h] = al;
-        }
-        any = __any_sync(0xffffffffu, any);
-        if (lane == 0) sm->rescale = any ? 1 : 0;
-      }
-      named_sync(1, 128);
-      const bool rescale = sm->rescale != 0;
-      if (rescale) {
-#pragma unroll
-        for (int h = 0; h < kH; ++h) l[h] *= sm->alpha[h];
-      }
-      // P = exp2(x - mref), summed per head, packed to bf16 into P^T row `row`.
+      // P = 2^(x - mref), summed per head, packed to bf16 into P^T row `row`.
       uint32_t pk[32];
-      {
-        uint32_t v[32];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tc::tmem_ld32(sbase + 32 * half, v);
-          tc::tmem_ld_wait();
+      for (int h = 0; h < kH; h += 4) {
+        const float4 mr = *reinterpret_cast<const float4 *>(&sm->mref[h]);
+        const float mm[4] = {mr.x, mr.y, mr.z, mr.w};
+        float p[4];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const int h = 32 * half + c;
-            const float m0 = sm->mref[h], m1 = sm->mref[h + 1];
-            const float p0 = (!valid || m0 == -INFINITY) ? 0.f : exp2f(__uint_as_float(v[c]) * scale_log2 - m0);
-            const float p1 = (!valid || m1 == -INFINITY) ? 0.f : exp2f(__uint_as_float(v[c + 1]) * scale_log2 - m1);
-            l[h] += p0;
-            l[h + 1] += p1;
-            __nv_bfloat162 t = __floats2bfloat162_rn(p0, p1);
-            pk[h >> 1] = *reinterpret_cast<uint32_t *>(&t);
-          }
+        for (int i = 0; i < 4; ++i) {
+          const float x = fmaf(__uint_as_float(h + i < 32 ? v0[h + i] : v1[h + i - 32]), scale_log2, -mm[i]);
+          p[i] = valid ? ex2_approx(x) : 0.f;
+          l[h + i] += p[i];
         }
+        __nv_bfloat162 t0 = __floats2bfloat162_rn(p[0], p[1]), t1 = __floats2bfloat162_rn(p[2], p[3]);
+        pk[h >> 1] = *reinterpret_cast<uint32_t *>(&t0);
+        pk[(h >> 1) + 1] = *reinterpret_cast<uint32_t *>(&t1);
       }
       if (lane < 16) {
         const uint32_t prow = tc::smem_u32(ps) + buf * kPBytes + row * 128;
@@ -512,6 +544,8 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const float *part_o, c
                                                           const float *sink, bf16 *out, int splits) {
   extern __shared__ float w[];  // [splits] weights, then [2][splits] (m, l)
   const int qq = blockIdx.x, h = blockIdx.y;
+  pdl_wait();
+  pdl_release();
   float *ml = w + splits;
   for (int i = threadIdx.x; i < 2 * splits; i += blockDim.x) {
     const int which = i / splits, s = i - which * splits;
@@ -614,17 +648,12 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
     attr_set = true;
   }
   dim3 grid(splits, a.Q);
-  mqa_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_cmp_g, tm_win_g, tm_cmp_t, tm_win_t, a, splits, tps,
-                                                        a.scale * kLog2e, part_o, part_ml);
-  note_launches(1);
-  if (splits > 1) {
-    dim3 cg(a.Q, kH);
-    mqa_combine_kernel<<<cg, kD / 4, splits * 3 * sizeof(float), stream>>>(part_o, part_ml, a.sink,
-                                                                          static_cast<bf16 *>(a.out), splits);
-    note_launches(1);
-  }
   *taken = true;
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(mqa_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_cmp_g, tm_win_g, tm_cmp_t,
+                             tm_win_t, a, splits, tps, a.scale * kLog2e, part_o, part_ml);
+  if (e != cudaSuccess || splits <= 1) return e;
+  return launch_pdl(mqa_combine_kernel, dim3(a.Q, kH), dim3(kD / 4), splits * 3 * sizeof(float), stream,
+                    (const float *)part_o, (const float *)part_ml, a.sink, static_cast<bf16 *>(a.out), splits);
 }
 
 }  // namespace csa

@@ -12,12 +12,11 @@
 // ordered pass keeps every entry with key > tau and the first kk entries (by
 // index) with key == tau; per-warp ballots and an exclusive prefix over the
 // block give each kept entry its output slot, so the output is ascending and
-// deterministic. One 1024-thread block per query. When the query's keys fit
-// in shared memory (n <= 48K) they are read from global memory once and every
-// pass runs on the shared copy. Longer lists (the 1 M-token context: 262,143
-// entries) take two stages: exact top-k of 16K-entry segments in parallel,
-// then the same selection over the concatenated segment winners. Without
-// scratch space a single block re-reads the scores on every pass.
+// deterministic. Lists of up to 8K entries: one 1024-thread block per query
+// with the keys cached in shared memory. Longer lists take two stages: the
+// exact top-k of 4K-32K-entry segments in parallel, then the same selection
+// over the concatenated segment winners. Without scratch space a single block
+// per query does it all (re-reading the scores per pass beyond 48K entries).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -176,6 +175,8 @@ __device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const floa
 __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int cache_keys) {
   extern __shared__ uint32_t keys[];
   __shared__ TopkShared sh;
+  pdl_wait();
+  pdl_release();
   const int q = blockIdx.x;
   const int n = clamp_count(a.n_cmp[q], a.N_max, threadIdx.x == 0 ? a.status : nullptr);
   const float *s = a.scores + (size_t)q * a.N_max;
@@ -195,17 +196,32 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int cache_ke
   }
 }
 
-// Two-stage selection for long lists. Stage 1: segment g of query q (kSeg
+// Two-stage selection for long lists. Stage 1: segment g of query q (`seg`
 // entries) keeps its own top-k (an entry of the global top-k set is always in
 // its segment's top-k set under the same order) as (key, index) candidates,
 // ascending. Stage 2: the concatenated candidates of a query are ascending in
 // index, so selecting by position with the same tie rule gives the global set.
-constexpr int kSeg = 16384;
+// Segments start at 4K entries and double until the winners of all segments
+// fit the stage-2 shared-memory cache.
+bool plan_two_stage(int N_max, int k, int *seg, int *nseg) {
+  if (N_max <= 8192) return false;
+  for (int s = 4096; s <= 32768; s *= 2) {
+    const int n = (N_max + s - 1) / s;
+    if ((long long)n * k <= kSmemKeys / 2 && n <= kThreads && N_max > 2 * s) {
+      *seg = s;
+      *nseg = n;
+      return true;
+    }
+  }
+  return false;
+}
 
 __global__ void __launch_bounds__(kThreads) topk_stage1_kernel(TopkArgs a, uint32_t *cand_key, int32_t *cand_idx,
-                                                               int32_t *cand_cnt, int nseg) {
+                                                               int32_t *cand_cnt, int nseg, int kSeg) {
   extern __shared__ uint32_t keys[];
   __shared__ TopkShared sh;
+  pdl_wait();
+  pdl_release();
   const int g = blockIdx.x, q = blockIdx.y;
   const int n = clamp_count(a.n_cmp[q], a.N_max, (threadIdx.x == 0 && g == 0) ? a.status : nullptr);
   const int j0 = g * kSeg;
@@ -235,6 +251,8 @@ __global__ void __launch_bounds__(kThreads) topk_stage2_kernel(TopkArgs a, const
                                                                int nseg) {
   extern __shared__ uint32_t keys[];  // [kSmemKeys / 2] keys then [kSmemKeys / 2] indices
   __shared__ TopkShared sh;
+  pdl_wait();
+  pdl_release();
   __shared__ int offs[kThreads + 1];
   int32_t *idxs = reinterpret_cast<int32_t *>(keys + kSmemKeys / 2);
   const int q = blockIdx.x;
@@ -270,8 +288,8 @@ __global__ void __launch_bounds__(kThreads) topk_stage2_kernel(TopkArgs a, const
 }  // namespace
 
 size_t topk_scratch_bytes(int Q, int N_max, int k) {
-  const int nseg = (N_max + kSeg - 1) / kSeg;
-  if (N_max <= kSmemKeys || (size_t)nseg * k > (size_t)kSmemKeys / 2 || nseg > kThreads) return 0;
+  int seg, nseg;
+  if (!plan_two_stage(N_max, k, &seg, &nseg)) return 0;
   return (size_t)Q * nseg * (k * 8 + 4) + 256;
 }
 
@@ -279,27 +297,26 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, s
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
-    cudaFuncSetAttribute(topk_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSeg * 4);
+    cudaFuncSetAttribute(topk_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 * 4);
     cudaFuncSetAttribute(topk_stage2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     attr_set = true;
   }
+  int seg = 0, nseg = 0;
   const size_t need = topk_scratch_bytes(a.Q, a.N_max, a.k);
-  if (need > 0 && scratch && scratch_bytes >= need && a.Q <= 65535) {
-    const int nseg = (a.N_max + kSeg - 1) / kSeg;
+  if (need > 0 && scratch && scratch_bytes >= need && a.Q <= 65535 && plan_two_stage(a.N_max, a.k, &seg, &nseg)) {
     uint32_t *ck = static_cast<uint32_t *>(scratch);
     int32_t *ci = reinterpret_cast<int32_t *>(ck + (size_t)a.Q * nseg * a.k);
     int32_t *cc = ci + (size_t)a.Q * nseg * a.k;
-    topk_stage1_kernel<<<dim3(nseg, a.Q), kThreads, kSeg * 4, stream>>>(a, ck, ci, cc, nseg);
-    topk_stage2_kernel<<<a.Q, kThreads, kSmemKeys * 4, stream>>>(a, ck, ci, cc, nseg);
-    note_launches(2);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(topk_stage1_kernel, dim3(nseg, a.Q), dim3(kThreads), (size_t)seg * 4, stream, a, ck, ci,
+                               cc, nseg, seg);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(topk_stage2_kernel, dim3(a.Q), dim3(kThreads), (size_t)kSmemKeys * 4, stream, a,
+                      (const uint32_t *)ck, (const int32_t *)ci, (const int32_t *)cc, nseg);
   }
   const int cache = a.N_max > a.k;  // a query can only need the keys when n > k
   const int keys = a.N_max < kSmemKeys ? a.N_max : kSmemKeys;
   const size_t smem = cache ? (size_t)keys * 4 : 0;
-  topk_kernel<<<a.Q, kThreads, smem, stream>>>(a, cache && a.N_max <= kSmemKeys);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(a.Q), dim3(kThreads), smem, stream, a, (int)(cache && a.N_max <= kSmemKeys));
 }
 
 }  // namespace csa
