@@ -185,6 +185,19 @@ def _sync_barrier(dist_on):
         torch.cuda.synchronize()
 
 
+def max_over_ranks(ms: float, dist_on: bool, device) -> float:
+    """The job's step time: the slowest rank's mean step time."""
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist_on:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, q_per_rank: int, ms_max: float) -> float:
+    """Whole-job queries/s: every rank serves q_per_rank queries per step."""
+    return world * q_per_rank / (ms_max * 1e-3)
+
+
 def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=False):
     n0 = _lib.lib().csa_launch_count()
     step = Step(w, device)  # runs the step once eagerly, then captures it
@@ -211,10 +224,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     wall = time.perf_counter() - wall0
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = sum(step_ms) / K
-    t = torch.tensor([ms], device=device)
-    if dist_on:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist_on, device)
 
     # Per-kernel durations: the same kernels launched one by one with events
     # between them (a host-side head start keeps the launches queued).
@@ -433,6 +443,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", torch.cuda.current_device())
 
+    w = WL.shard(w, rank)  # this rank's own sequences (same shapes)
     r = time_ours(args, w, device, dist_on, rank, world)
     traffic = None
     try:
@@ -479,7 +490,7 @@ def main():
 
     if rank == 0:
         step_bytes = sum(algo_bytes(w).values())
-        value = world * w.Q / (r["ms"] * 1e-3)
+        value = job_value(world, w.Q, r["ms"])
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": r["K"],
             "warmup": args.warmup, "ms_per_step": round(r["ms"], 4), "higher_is_better": True, "scaling": "weak",

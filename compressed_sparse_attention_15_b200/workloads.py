@@ -146,6 +146,15 @@ def norm_w(w: Workload, device="cpu") -> torch.Tensor:
     return torch.ones(w.D, dtype=torch.float32, device=device)
 
 
+def shard(w: Workload, rank: int) -> Workload:
+    """The batch that process ``rank`` serves when several GPUs each run their
+    own independent sequences: the same shapes, its own draws (rank 0's batch
+    is ``w`` itself)."""
+    if rank < 0:
+        raise ValueError("rank must be >= 0")
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
 def small(w: Workload, **changes) -> Workload:
     """A copy of ``w`` with some fields changed (test-size variants)."""
     return dataclasses.replace(w, **changes)
