@@ -9,7 +9,8 @@ cache (csa_compress), score + select (csa_index_topk) and attend
 (csa_sparse_mqa); for the HCA workload, append + hca_mqa. Inputs are seeded
 synthetic tensors of the DeepSeek-V4-Flash shapes, resident in HBM. The step
 is captured once in a CUDA graph and replayed; L2 is flushed (a 256 MB
-write) before every timed step, outside the step's events.
+write, then a 256 MB read of another buffer so that no dirty line is left to
+write back) before every timed step, outside the step's events.
 
 Multi-GPU (torchrun): one process per GPU, each serving its own batch of
 independent sequences (weak scaling, no collective on the data path); the
@@ -94,13 +95,36 @@ class Step:
     """Device-resident inputs of one workload wrapped in the package's
     DecodeStep (graph-captured decode step)."""
 
-    def __init__(self, w: WL.Workload, device, graph: bool = True):
+    # inputs that change every decode step; they live in one staging buffer so
+    # that the end-to-end run moves them with a single host-to-device copy
+    PER_STEP = ("q", "gate", "qi", "wi")
+
+    def __init__(self, w: WL.Workload, device, graph: bool = True, caches=None):
         self.w = w
         self.dev = device
-        self.t = {n: WL.make(w, n, device) for n in ("q", "kv_cmp", "kv_win", "sink", "ape", "gate")}
-        if w.mode == "csa":
-            for n in ("qi", "wi", "ki"):
-                self.t[n] = WL.make(w, n, device)
+        self.graph = graph
+        names = [n for n in self.PER_STEP if w.mode == "csa" or n not in ("qi", "wi")]
+        shapes = {n: WL.tensor_shape(w, n) for n in names}
+        shapes["kv_new"] = (w.B, w.D)  # the newest raw token of each sequence
+        dts = {n: torch.float32 if n == "wi" else w.dtype for n in shapes}
+        offs, total = {}, 0
+        for n, shp in shapes.items():
+            offs[n] = total
+            total += -(-math.prod(shp) * torch.empty((), dtype=dts[n]).element_size() // 256) * 256
+        self.stage = torch.empty(total, dtype=torch.uint8, device=device)
+        self.t = {}
+        for n, shp in shapes.items():
+            nb = math.prod(shp) * torch.empty((), dtype=dts[n]).element_size()
+            self.t[n] = self.stage[offs[n]:offs[n] + nb].view(dts[n]).view(shp)
+        if caches is None:
+            caches = {n: WL.make(w, n, device) for n in ("kv_cmp", "kv_win", "sink", "ape")}
+            if w.mode == "csa":
+                caches["ki"] = WL.make(w, "ki", device)
+        self.caches = caches
+        self.t.update(caches)
+        for n in names:
+            self.t[n].copy_(WL.make(w, n, device))
+        self.t["kv_new"].copy_(self.t["kv_win"][:, -1])
         t = self.t
         self.ds = DecodeStep(
             q=t["q"], kv_cmp=t["kv_cmp"], kv_win=t["kv_win"], sink=t["sink"], scale=w.scale, win_len=w.W,
@@ -109,9 +133,28 @@ class Step:
             win=w.win, stride=w.stride, qi=t.get("qi"), wi=t.get("wi"), ki=t.get("ki"),
             k=w.k if w.mode == "csa" else None, graph=graph)
         self.out = self.ds.out
+        self._scores = None
+
+    def twin(self):
+        """A second step over the same caches with its own input staging
+        buffer and output (double buffering for the end-to-end pipeline)."""
+        return Step(self.w, self.dev, graph=self.graph, caches=self.caches)
 
     def parts(self):
-        return self.ds.parts()
+        """The step's kernels one call at a time (per-kernel timing and the
+        profiling aid). The CSA select call is split into its two kernels,
+        scores then top-k, through their own entry points."""
+        ds = self.ds
+        if not ds.csa:
+            return ds.parts()
+        if self._scores is None:
+            self._scores = torch.empty((self.w.Q, self.w.N), dtype=torch.float32, device=self.dev)
+            self._ws_s, self._ws_t = ops.Workspace(self.dev), ops.Workspace(self.dev)
+        sc = self._scores
+        return [("compress", ds.append),
+                ("index_scores", lambda: ops.index_scores(ds.qi, ds.wi, ds.ki, ds.n_cmp, out=sc, ws=self._ws_s)),
+                ("topk", lambda: ops.topk(sc, ds.n_cmp, ds.k, out=ds.idx, ws=self._ws_t)),
+                ("mqa", ds.attend)]
 
     def run(self):
         return self.ds.run()
@@ -178,6 +221,20 @@ class Clocks:
                 "samples": len(rows)}
 
 
+class L2Flush:
+    """Evicts L2 between timed steps: a 256 MB write (twice the L2), then a
+    256 MB read of another buffer, so that the write's dirty lines are written
+    back here and not during the next timed step."""
+
+    def __init__(self, device):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+
 def _sync_barrier(dist_on):
     torch.cuda.synchronize()
     if dist_on:
@@ -202,7 +259,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     n0 = _lib.lib().csa_launch_count()
     step = Step(w, device)  # runs the step once eagerly, then captures it
     launches_per_step = (_lib.lib().csa_launch_count() - n0) // 2
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     stream = torch.cuda.current_stream(device)
     for _ in range(max(3, args.warmup)):
         step.run()
@@ -216,7 +273,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     with clocks:
         time.sleep(0.2)
         for i in range(K):
-            flush.zero_()
+            flush()
             evs[i][0].record(stream)
             step.run()
             evs[i][1].record(stream)
@@ -232,7 +289,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     per = {n: 0.0 for n in names}
     Kp = max(5, K // 2)
     for _ in range(Kp):
-        flush.zero_()
+        flush()
         torch.cuda._sleep(2_000_000)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         ev[0].record(stream)
@@ -256,14 +313,14 @@ def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
     nw = WL.norm_w(w, device)
     n = (w.bulk_T - w.win) // w.stride + 1
     out = torch.empty((1, n, w.D), dtype=w.dtype, device=device)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     stream = torch.cuda.current_stream(device)
     for _ in range(3):
         ops.compress(kv, gate, ape, nw, w.win, w.stride, out=out)
     K = max(5, args.steps // 4)
     ms = 0.0
     for _ in range(K):
-        flush.zero_()
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         ops.compress(kv, gate, ape, nw, w.win, w.stride, out=out)
@@ -277,49 +334,87 @@ def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
 
 
 def roofline_of(w, per_kernel_ms, hbm_gbs, traffic=None):
-    """Roofline of the kernel with the most algorithmic bytes in the step."""
+    """Roofline of the kernel with the most algorithmic bytes in the step.
+    ``traffic`` maps a part name to its measured DRAM bytes per launch."""
     ab = algo_bytes(w)
-    fam = {"index_topk": "index_scores", "mqa": "mqa", "compress": "compress"}
-    best = max(((k, ab[fam[k]]) for k in per_kernel_ms if fam[k] in ab), key=lambda x: x[1])
+    best = max(((k, ab[k]) for k in per_kernel_ms if k in ab), key=lambda x: x[1])
     name, nbytes = best
+    traffic = (traffic or {}).get(name)
     ms = per_kernel_ms[name]
     achieved = nbytes / (ms * 1e-3) / 1e9
     return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
             "frac": round(achieved / hbm_gbs, 4), "traffic": traffic, "bytes_per_launch": int(nbytes)}
 
 
+def load_traffic(path, workload):
+    """DRAM bytes per launch of each part, from the committed ncu summary
+    (profiles/traffic.json): {part: bytes}, for the kernels as they stand."""
+    try:
+        with open(path) as f:
+            entry = json.load(f).get(workload) or {}
+    except (OSError, ValueError):
+        return {}
+    return {part: v["dram_bytes_per_launch"] for part, v in entry.items()
+            if isinstance(v, dict) and v.get("dram_bytes_per_launch")}
+
+
 def e2e_ours(args, w: WL.Workload, step: Step, device):
-    """Same metric through the public API with host buffers: every step copies
-    its per-step inputs (q, qi, wi, the newest raw token and the window's
-    gates) from pinned host memory and reads the output back."""
-    t = step.t
-    host = {n: t[n].cpu().pin_memory() for n in ("q", "gate")}
-    if w.mode == "csa":
-        host.update({n: t[n].cpu().pin_memory() for n in ("qi", "wi")})
-    host["kv_new"] = t["kv_win"][:, -1].cpu().pin_memory()
-    out_h = torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * out_h.element_size()
-    stream = torch.cuda.current_stream(device)
-    K = max(10, args.steps // 2)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
-    ms = 0.0
-    for i in range(K + 2):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for n in ("q", "gate", "qi", "wi"):
-            if n in host:
-                t[n].copy_(host[n], non_blocking=True)
-        t["kv_win"][:, -1].copy_(host["kv_new"], non_blocking=True)
-        step.run()
-        out_h.copy_(step.out, non_blocking=True)
-        b.record(stream)
-        torch.cuda.synchronize()
+    """Same metric through the public API with host buffers, as a serving loop
+    runs it: every step copies its per-step inputs (q, qi, wi, the window's
+    gates and the newest raw token of each sequence, packed in one pinned
+    staging buffer) to the device in one copy, places the new token in the
+    raw-KV buffer, runs the step and reads its output back. Two input/output
+    buffer sets alternate, so that step i's copies overlap the compute of its
+    neighbours (copies on their own streams, ordered by events). The step's
+    working set (the caches it reads) exceeds L2, so the steps run back to
+    back; the timed region spans K whole steps, first copy to last read."""
+    pair = [step, step.twin()]
+    host = step.stage.cpu().pin_memory()
+    outs = [torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True) for st in pair]
+    h2d = host.numel()
+    d2h = outs[0].numel() * outs[0].element_size()
+    comp = torch.cuda.current_stream(device)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in pair]
+    ev_done = [torch.cuda.Event() for _ in pair]
+    ev_out = [torch.cuda.Event() for _ in pair]
+    kv_win = step.t["kv_win"]
+
+    def one(i):
+        b = i % 2
+        st = pair[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[b])  # step i - 2 has consumed this staging buffer
+            st.stage.copy_(host, non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
         if i >= 2:
-            ms += a.elapsed_time(b) / K
+            comp.wait_event(ev_out[b])  # step i - 2's output has been read back
+        kv_win[:, -1].copy_(st.t["kv_new"])
+        st.run()
+        ev_done[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            outs[b].copy_(st.out, non_blocking=True)
+            ev_out[b].record(s_out)
+
+    K = max(20, args.steps)
+    for i in range(4):  # warm-up
+        one(i)
+    torch.cuda.synchronize()
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    s_in.wait_stream(comp)
+    for i in range(K):
+        one(i)
+    comp.wait_stream(s_out)
+    e.record(comp)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(e) / K
     return {"value": round(w.Q / (ms * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4)}
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
+            "pipelined": "two buffer sets; copies on their own streams overlap neighbouring steps"}
 
 
 # --------------------------------------------------------------------------
@@ -386,7 +481,7 @@ def time_oracle(w: WL.Workload, steps: int, budget_s: float):
 def workload_config(w: WL.Workload):
     return {"workload": w.name, "batch": w.Q, "context": w.pos0 + 1, "heads": f"{w.H}q:1kv", "head_dim": w.D,
             "indexer": f"{w.Hi}x{w.Di}" if w.mode == "csa" else None, "topk": w.k or None, "window": w.W,
-            "compress": f"win {w.win} stride {w.stride}", "l2": "flushed: 256 MB write before every timed step",
+            "compress": f"win {w.win} stride {w.stride}", "l2": "flushed before every timed step: 256 MB write, then 256 MB read (clean eviction)",
             "inputs": "seeded synthetic (counter-based generator), resident in HBM"}
 
 
@@ -445,14 +540,7 @@ def main():
 
     w = WL.shard(w, rank)  # this rank's own sequences (same shapes)
     r = time_ours(args, w, device, dist_on, rank, world)
-    traffic = None
-    try:
-        with open(args.traffic_json) as f:
-            tj = json.load(f).get(w.name)
-            if tj:
-                traffic = tj.get("bytes_per_launch")
-    except Exception:
-        pass
+    traffic = load_traffic(args.traffic_json, w.name)
     roof = roofline_of(w, r["per_kernel_ms"], hbm, traffic)
     roof["peak_kind"] = f"{peak_kind} HBM copy bandwidth"
     e2e = e2e_ours(args, w, r["step"], device)
@@ -468,7 +556,7 @@ def main():
             try:
                 s = time_ours(args, sw, device, False, 0, 1, secondary=True)
                 del s["step"]
-                rf = roofline_of(sw, s["per_kernel_ms"], hbm)
+                rf = roofline_of(sw, s["per_kernel_ms"], hbm, load_traffic(args.traffic_json, name))
                 step_bytes = sum(algo_bytes(sw).values())
                 secondary[name] = {"queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1), "ms_per_step": round(s["ms"], 4),
                                    "per_kernel_ms": {k: round(v, 4) for k, v in s["per_kernel_ms"].items()},

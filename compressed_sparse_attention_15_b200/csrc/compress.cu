@@ -8,11 +8,14 @@
 //     out = c / sqrt(mean(c^2) + 1e-6) * norm_w.
 //
 // Three kernels, all fp32 arithmetic:
-//  * compress_window_kernel (bf16, D % 8 == 0): one CTA per entry; the window
-//    positions are split over G thread groups, each thread owns one 16-byte
-//    vector (8 dims) and keeps a running (max, sum, weighted sum) over its
-//    positions; the G partial states are merged through shared memory. Used
-//    when there are few entries (the per-step append) or long windows (HCA).
+//  * compress_window_kernel (bf16, D % 8 == 0): one CTA (or, for windows of
+//    32+ tokens, a cluster of up to 8 CTAs splitting the positions) per
+//    entry; the positions are split over G thread groups, each thread owns
+//    one 16-byte vector (8 dims) and keeps a running (max, sum, weighted sum)
+//    over its positions; the G partial states are merged through shared
+//    memory; a cluster's blocks then each finish D / C of the dims from all
+//    blocks' states through distributed shared memory. Used when there
+//    are few entries (the per-step append) or long windows (HCA).
 //  * compress_stream_kernel (bf16, CSA geometry win = 2 * stride): streams
 //    many entries; WPR warps own a row (8 dims per lane), each 8-token window
 //    is reduced with an exact two-pass softmax in registers (max, then exp2),
@@ -101,15 +104,20 @@ __device__ __forceinline__ uint4 pack8(const float f[8]) {
 // ------------------------------------------------------------------ window-parallel
 
 // Block = G groups x nvec threads (nvec = D / 8, a multiple of 32); thread
-// (g, v) handles dims [8v, 8v + 8) at window positions i = g, g + G, ... .
-// One block per (sequence, entry).
+// (g, v) handles dims [8v, 8v + 8) at window positions i = i0 + g, i0 + g + G,
+// ... < i1. One cluster of C blocks per (sequence, entry): block c of the
+// cluster takes positions [c P, c P + P), P = ceil(win / C); the C partial
+// states are merged by block 0 through distributed shared memory.
 __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, int G) {
-  extern __shared__ float ws[];  // [G][3][8][nvec] partial states, then [32] sums
+  extern __shared__ float ws[];  // [G][3][8][nvec] partial states, then [32] sums, then [3][8][nvec] block state
   pdl_wait();
   pdl_release();
   const int nvec = a.D / 8;
   const int v = threadIdx.x % nvec, g = threadIdx.x / nvec;
-  const long long e = blockIdx.x;
+  const uint32_t C = cluster_size(), crank = cluster_rank();
+  const int P = (a.win + (int)C - 1) / (int)C;
+  const int pos0 = (int)crank * P, pos1 = min(a.win, pos0 + P);
+  const long long e = blockIdx.x / C;
   const int b = (int)(e / a.N), j = (int)(e - (long long)b * a.N);
   const bf16 *kvj = static_cast<const bf16 *>(a.kv) + b * a.kv_ss + (long long)j * a.stride * a.D;
   const bf16 *gj = static_cast<const bf16 *>(a.gate) + b * a.gate_ss + (long long)j * a.stride * a.D;
@@ -120,13 +128,13 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
     l[k] = 0.f;
     acc[k] = 0.f;
   }
-  // positions g, g + G, ... with four rows of loads in flight per step
-  for (int i0 = g; i0 < a.win; i0 += 4 * G) {
+  // positions pos0 + g, pos0 + g + G, ... with four rows of loads in flight per step
+  for (int i0 = pos0 + g; i0 < pos1; i0 += 4 * G) {
     uint4 kvv[4], gv[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int i = i0 + u * G;
-      if (i < a.win) {
+      if (i < pos1) {
         kvv[u] = __ldg(reinterpret_cast<const uint4 *>(kvj + (long long)i * a.D) + v);
         gv[u] = __ldg(reinterpret_cast<const uint4 *>(gj + (long long)i * a.D) + v);
       }
@@ -134,7 +142,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int i = i0 + u * G;
-      if (i < a.win) {
+      if (i < pos1) {
         float kf[8], gf[8];
         unpack8(kvv[u], kf);
         unpack8(gv[u], gf);
@@ -165,9 +173,10 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
   }
   __syncthreads();
   float *red = ws + (size_t)G * 3 * 8 * nvec;  // [32]
+  float *blk = red + 32;                        // [3][8][nvec]: this block's merged state
   float c[8];
+  float M8[8], L8[8], A8[8];
   if (g == 0) {
-    float ss = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       float M = -INFINITY;
@@ -179,7 +188,78 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
         L += sm[((h * 3 + 1) * 8 + k) * nvec + v] * w;
         A += sm[((h * 3 + 2) * 8 + k) * nvec + v] * w;
       }
-      c[k] = A / L;
+      M8[k] = M;
+      L8[k] = L;
+      A8[k] = A;
+      if (C > 1) {
+        blk[(0 * 8 + k) * nvec + v] = M;
+        blk[(1 * 8 + k) * nvec + v] = L;
+        blk[(2 * 8 + k) * nvec + v] = A;
+      }
+    }
+  }
+  if (C > 1) {
+    // Block c of the cluster finishes dims [c D / C, (c + 1) D / C): merge
+    // the C block states of each, then the RMSNorm with the cluster's total
+    // sum of squares (every remote load of a thread issued before use).
+    cluster_sync();  // every block's state is published
+    const int per = a.D / (int)C, t = threadIdx.x;
+    const bool mine = t < per;
+    const int d = (int)crank * per + t;
+    const int di = (d & 7) * nvec + (d >> 3);  // dim 8v + k lives at [.][k][v]
+    float cd = 0.f;
+    if (mine) {
+      float mr[8], lr[8], ar[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < (int)C) {
+          mr[r] = ld_peer_f(&blk[di], r);
+          lr[r] = ld_peer_f(&blk[8 * nvec + di], r);
+          ar[r] = ld_peer_f(&blk[16 * nvec + di], r);
+        }
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < (int)C) M = fmaxf(M, mr[r]);
+      float L = 0.f, A = 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < (int)C) {
+          const float w = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - M);
+          L += lr[r] * w;
+          A += ar[r] * w;
+        }
+      cd = A / L;
+    }
+    const float ss = warp_sum(mine ? cd * cd : 0.f);
+    if ((t & 31) == 0) red[t >> 5] = ss;  // at most 16 warps
+    __syncthreads();
+    if (t == 0) {
+      float tot = 0.f;
+      for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) tot += red[w];
+      red[16] = tot;  // this block's share, read by the peers
+    }
+    cluster_sync();  // every block's share is published
+    if (mine) {
+      float sr[8], tot = 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < (int)C) sr[r] = ld_peer_f(&red[16], r);
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < (int)C) tot += sr[r];
+      const float rn = 1.0f / sqrtf(tot / (float)a.D + kRmsEps);
+      bf16 *o = static_cast<bf16 *>(a.out) + b * a.out_ss + (long long)j * a.D;
+      o[d] = __float2bfloat16_rn(cd * rn * a.norm_w[d]);
+    }
+    cluster_sync();  // no block leaves while a peer may still read its share
+    return;
+  }
+  if (g == 0) {
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      c[k] = A8[k] / L8[k];
       ss += c[k] * c[k];
     }
     ss = warp_sum(ss);  // group 0 is whole warps (nvec is a multiple of 32)
@@ -348,16 +428,26 @@ cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
       return a.D == 512 ? launch_stream<2, 4>(a, stream) : launch_stream<1, 4>(a, stream);
     if ((a.D / 8) % 32 == 0) {
       const int nvec = a.D / 8;
-      int G = a.win < 16 ? a.win : 16;
+      // Long windows and few entries: a cluster of C blocks per entry, at
+      // least 16 positions each, about two blocks per SM in all.
+      // (C a power of two, so that it divides D)
+      int C = 1;
+      if (a.win >= 32) {
+        const long long fill = (2LL * num_sms() + total - 1) / total;
+        while (2 * C <= 8 && 2 * C <= a.win / 16 && 2 * C <= fill) C *= 2;
+      }
+      const int P = (a.win + C - 1) / C;
+      int G = P < 16 ? P : 16;
       while (G > 1 && G * nvec > 512) G >>= 1;
-      const size_t smem = ((size_t)G * 3 * 8 * nvec + 32) * sizeof(float);
+      const size_t smem = ((size_t)(G + 1) * 3 * 8 * nvec + 32) * sizeof(float);
       static bool attr_set = false;
       if (!attr_set) {
         cudaFuncSetAttribute(compress_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(((size_t)3 * 8 * 512 + 32) * sizeof(float)));
+                             (int)(((size_t)4 * 8 * 512 + 32) * sizeof(float)));
         attr_set = true;
       }
-      return launch_pdl(compress_window_kernel, dim3((unsigned)total), dim3(G * nvec), smem, stream, a, G);
+      return launch_pdl_cluster(compress_window_kernel, dim3((unsigned)(total * C)), dim3(G * nvec), smem, stream,
+                                (unsigned)C, a, G);
     }
   }
   const int threads = 256, wpb = threads / 32;

@@ -12,24 +12,30 @@
 // swizzled, 64-dim boxes) and feeds both products. Two tile buffers, two S^T
 // TMEM buffers and two P^T buffers make a software pipeline: while the
 // softmax warps turn S^T(t) into P(t), the tensor core computes S^T(t+1) and
-// TMA loads tile t+2. The MMA thread issues S(t+1) before PV(t).
+// the loaders fill the other buffer. The MMA thread issues S^T and P.V each
+// as soon as its inputs are ready.
 // An M = 64 accumulator occupies TMEM lanes 0-15 of each 32-lane quarter, so
-// each softmax warp owns 16 rows; a row's 64 head logits stay in one thread.
-// The per-head tile maximum is a warp transpose-reduction plus a 4-warp
-// exchange; the running per-head maximum only moves (and O^T is rescaled in
-// TMEM, after the previous P.V has completed) when a tile's maximum exceeds
-// it by more than 2^8, so P <= 256 in bf16.
+// each softmax warp owns 16 rows; read with the 16x256b shape, every thread
+// holds 2 rows x 16 heads. The per-head tile maximum is a 3-step shuffle
+// reduction plus a 4-warp exchange; the running per-head maximum only moves
+// (and O^T is rescaled in TMEM, after the previous P.V has completed) when a
+// tile's maximum exceeds it by more than 2^8, so P <= 256 in bf16.
 //
 // Loads: contiguous runs of 64 rows (HCA entries, window rows) are single TMA
-// boxes of 64 rows; top-k rows use TMA tile::gather4 (4 rows per instruction;
-// the compressed segment is padded to a multiple of 4 rows so no group mixes
-// the compressed cache and the raw window buffer).
+// boxes of 64 rows; top-k rows are gathered with 16-byte cp.async copies by
+// the two loader warps (TMA gathers issue too slowly for 1 KB rows). The
+// compressed segment is padded to a multiple of 4 rows (unused, masked).
 //
-// Work split: query q's row list is cut into `splits` runs of whole tiles, one
-// CTA each. With one split the CTA folds in the sink and writes the output;
-// otherwise it writes (m, l, O) partials merged by mqa_combine_kernel.
-// Roles (192 threads): warp 0 loads, warp 1 issues the MMAs and owns TMEM,
-// warps 2-5 run the softmax and the epilogue. All waits are bounded.
+// Work split: query q's row list is cut into `splits` (<= 8) runs of whole
+// tiles, one CTA each, the CTAs of a query forming one thread-block cluster.
+// With one split the CTA folds in the sink and writes the output; otherwise
+// every CTA stages its unnormalised (m, l, O) in shared memory and, after a
+// cluster barrier, merges 1/splits of the output from all of them through
+// distributed shared memory.
+// Roles (224 threads): warps 0-1 load (one per tile buffer), warp 2 issues
+// the MMAs and owns TMEM, warps 3-6 run the softmax and the epilogue. All
+// mbarrier waits are bounded; the softmax warps take every decision to stop
+// together (a barrier reduction), so no named barrier is left half-joined.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -46,10 +52,12 @@ constexpr uint32_t kTileBytes = 8 * kBoxBytes;      // 64 rows x 512 dims: 64 KB
 constexpr uint32_t kQBoxBytes = kH * 128;           // 64 heads x 64 dims: 8 KB
 constexpr uint32_t kQBytes = 8 * kQBoxBytes;        // 64 KB
 constexpr uint32_t kPBytes = kRows * kH * 2;        // 8 KB
-constexpr int kThreads = 192;
-constexpr int kMmaWarp = 1;
-constexpr int kSoftWarp0 = 2;
+constexpr int kLoadWarps = 2;
+constexpr int kThreads = 224;
+constexpr int kMmaWarp = 2;
+constexpr int kSoftWarp0 = 3;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxSplits = 8;                       // splits of one query form one (portable-size) cluster
 constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m (M = 128 layout)
 constexpr uint32_t kColS = 256;                     // S^T buffer j at 256 + 64j (M = 64 layout)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -65,6 +73,7 @@ struct Small {
   int abort;
   int rescale;
   int need[4];  // per tile (mod 4): some logit exceeded the running maximum by more than 2^8
+  const bf16 *rowp[2][kRows];  // gathered tiles: source row of each tile row (null: zero-fill)
 };
 
 constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kQBytes + 2 * kPBytes + sizeof(Small);
@@ -89,34 +98,12 @@ __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *
   return L;
 }
 
-// TMA row coordinate of list position r: in the compressed cache viewed as
-// [B * N_max, 512] when r < nsel4, else in the window buffer viewed as
-// [B * T_raw, 512]. Unused and padding positions get a valid row of the same
-// tensor (their logits are masked).
-__device__ __forceinline__ int row_coord(const MqaArgs &a, const RowList &L, int qq, int b, int r) {
-  if (r < L.nsel4) {
-    int j = -1;
-    if (r < L.nsel) {
-      j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
-      if (j < -1 || j >= a.N_max) {
-        raise_status(a.status, CSA_STATUS_BAD_INDEX);
-        j = -1;
-      }
-    }
-    return b * a.N_max + (j >= 0 ? j : 0);
-  }
-  return b * a.T_raw + (r < L.R ? L.wlo + (r - L.nsel4) : L.wlo);
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
 }
 
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int col, const int (&rc)[4],
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(col), "r"(rc[0]), "r"(rc[1]),
-        "r"(rc[2]), "r"(rc[3])
-      : "memory");
-}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // 2^x on the SFU (relative error about 2^-22; flushes subnormal results to
 // zero, which only ever meets weights far below the bf16 resolution of P).
@@ -124,6 +111,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Named barrier over n threads that also ORs `pred` across them: every
+// participant gets the same answer.
+__device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, %2, %3, p; selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void named_sync(int id, int n) {
@@ -144,28 +143,25 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Warp transpose-reduction of 64 per-lane values: afterwards lane l holds the
-// reduction over the 32 lanes of heads 2l and 2l+1 in v[0], v[1].
-template <bool kMax>
-__device__ __forceinline__ void transpose_reduce64(float (&v)[64], int lane) {
-#pragma unroll
-  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
-    const bool hi = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < n; ++i) {
-      const float send = hi ? v[i] : v[i + n];
-      const float keep = hi ? v[i + n] : v[i];
-      const float got = __shfl_xor_sync(0xffffffffu, send, o);
-      v[i] = kMax ? fmaxf(keep, got) : keep + got;
-    }
-  }
+// tcgen05.ld of 16 TMEM lanes x 64 columns (16x256b shape, 8 repeats): for
+// column group c, thread t gets r[4c + e] = (lane t/4, column 8c + 2(t%4) + e)
+// and r[4c + 2 + e] = (lane t/4 + 8, same column), e = 0, 1.
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp_g,
-                  const __grid_constant__ CUtensorMap tm_win_g, const __grid_constant__ CUtensorMap tm_cmp_t,
+    mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp_t,
                   const __grid_constant__ CUtensorMap tm_win_t, MqaArgs a, int splits, int tiles_per_split,
-                  float scale_log2, float *part_o, float *part_ml) {
+                  float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *kv = smem;                              // [2 tiles][8 boxes][64 rows][128 B]
@@ -179,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tc::mbar_init(&sm->q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&sm->kv_full[i], 1);
+      tc::mbar_init(&sm->kv_full[i], 32);
       tc::mbar_init(&sm->kv_empty[i], 1);
       tc::mbar_init(&sm->s_full[i], 1);
       tc::mbar_init(&sm->p_full[i], 4 * 32);
@@ -210,51 +206,73 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t1 = min(tiles_all, t0 + tiles_per_split);
   const int ntiles = max(0, t1 - t0);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ loader
-    const uint32_t kv_base = tc::smem_u32(kv);
+  if (warp < kLoadWarps) {
+    // ------------------------------------------------------------ loaders
+    // Warp g fills tile buffer g (tiles g, g + 2, ...). A contiguous run is 8
+    // TMA boxes issued by lane 0. A gathered tile is 4096 16-byte cp.async
+    // copies, 128 per lane, each warp instruction moving 512 contiguous bytes
+    // of one row; every lane waits for its own copies, fences them for the
+    // tensor core and arrives, so kv_full expects 32 arrivals either way.
+    const int g = warp;
+    const uint32_t buf_base = tc::smem_u32(kv) + g * kTileBytes;
     if (lane == 0) {
-      tc::prefetch_tmap(&tm_cmp_g);
-      tc::prefetch_tmap(&tm_win_g);
       tc::prefetch_tmap(&tm_cmp_t);
       tc::prefetch_tmap(&tm_win_t);
     }
-    int issued = 0;
-    for (int li = 0; li < ntiles && !*abort; ++li) {
-      const int buf = li & 1;
+    int last = -1;
+    for (int li = g; li < ntiles; li += 2) {
       const int r0 = (t0 + li) * kRows;
       // A tile is one contiguous run when it lies in the window part, or in
       // the compressed part of a dense (HCA) row list.
       const bool win_run = r0 >= L.nsel4;
       const bool cmp_run = !a.idx && r0 + kRows <= L.nsel4;
-      int rc[4];
-      const CUtensorMap *gmap = &tm_cmp_g;
-      if (!win_run && !cmp_run && lane < 16) {
-        const int r = r0 + 4 * lane;
+      __syncwarp();  // the previous tile's copies have read rowp[g]
+      if (!win_run && !cmp_run) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) rc[i] = row_coord(a, L, qq, b, r + i);
-        gmap = r < L.nsel4 ? &tm_cmp_g : &tm_win_g;
-      }
-      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[buf], ((li >> 1) & 1) ^ 1, abort, a.status));
-      if (!ok) break;
-      const uint32_t dst = kv_base + buf * kTileBytes;
-      if (lane == 0) tc::mbar_arrive_expect_tx(&sm->kv_full[buf], kTileBytes);
-      __syncwarp();
-      if (win_run || cmp_run) {
-        if (lane < 8) {
-          const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
-          tc::tma_load_2d(kv + buf * kTileBytes + lane * kBoxBytes, win_run ? &tm_win_t : &tm_cmp_t, 64 * lane, row,
-                          &sm->kv_full[buf]);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int r = r0 + lane + 32 * hh;
+          const bf16 *p = nullptr;
+          if (r < L.nsel) {
+            int j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
+            if (j < -1 || j >= a.N_max) {
+              raise_status(a.status, CSA_STATUS_BAD_INDEX);
+              j = -1;
+            }
+            if (j >= 0) p = static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + j) * kD;
+          } else if (r >= L.nsel4 && r < L.R) {
+            p = static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + L.wlo + (r - L.nsel4)) * kD;
+          }
+          sm->rowp[g][lane + 32 * hh] = p;
         }
-      } else if (lane < 16) {
-#pragma unroll
-        for (int bx = 0; bx < 8; ++bx) tma_gather4(dst + bx * kBoxBytes + lane * 512, gmap, 64 * bx, rc, &sm->kv_full[buf]);
       }
-      issued = li + 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status))) break;
+      if (win_run || cmp_run) {
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(&sm->kv_full[g], kTileBytes);
+          const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
+          for (int bx = 0; bx < 8; ++bx)
+            tc::tma_load_2d(kv + g * kTileBytes + bx * kBoxBytes, win_run ? &tm_win_t : &tm_cmp_t, 64 * bx, row,
+                            &sm->kv_full[g]);
+        } else {
+          tc::mbar_arrive(&sm->kv_full[g]);
+        }
+      } else {
+        __syncwarp();  // rowp[g] written by every lane
+#pragma unroll 8
+        for (int i = 0; i < 2 * kRows; ++i) {
+          const int row = i >> 1, c16 = lane + 32 * (i & 1);  // 16-byte piece c16 of the 1 KB row
+          const bf16 *src = sm->rowp[g][row];
+          const uint32_t dst = buf_base + (c16 >> 3) * kBoxBytes + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
+          cp_async16(dst, src ? src + c16 * 8 : static_cast<const bf16 *>(a.kv_win), src != nullptr);
+        }
+        cp_async_wait_all();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc::mbar_arrive(&sm->kv_full[g]);
+      }
+      last = li;
     }
-    // Drain: the copies of the last two tiles must have landed before exit.
-    if (lane == 0)
-      for (int li = max(0, issued - 2); li < issued; ++li) tc::mbar_drain(&sm->kv_full[li & 1], (li >> 1) & 1);
+    // Drain: a TMA tile still in flight must land before the CTA exits.
+    if (lane == 0 && last >= 0) tc::mbar_drain(&sm->kv_full[g], (last >> 1) & 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -270,39 +288,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_pv = tc::idesc_bf16(128, 64, 1, 1);
       const uint32_t kv_base = tc::smem_u32(kv), q_base = tc::smem_u32(qs), p_base = tc::smem_u32(ps);
       bool ok = ntiles == 0 || tc::mbar_wait(&sm->q_full, 0, abort, a.status);
-      auto pv = [&](int t) {  // O^T += V^T(t) P^T(t)
-        const int pb = t & 1;
-        if (!tc::mbar_wait(&sm->p_full[pb], (t >> 1) & 1, abort, a.status)) return false;
-        tc::fence_after_sync();
-        const uint64_t ad0 = tc::sw128_desc(kv_base + pb * kTileBytes, kBoxBytes, 1024);
-        const uint64_t bd0 = tc::sw128_desc(p_base + pb * kPBytes, kPBytes, 1024);
+      const uint64_t ad_kv = tc::sw128_desc(kv_base, 16, 1024), bd_q = tc::sw128_desc(q_base, 16, 1024);
+      const uint64_t ad_v = tc::sw128_desc(kv_base, kBoxBytes, 1024), bd_p = tc::sw128_desc(p_base, kPBytes, 1024);
+      // Two streams of work, issued as soon as each is ready: S^T(ns) once
+      // tile ns has landed (and the softmax is done with S^T(ns - 2)), and
+      // P.V(np) once P(np) is written. Neither waits behind the other, so the
+      // P.V that frees a tile buffer is never held up by the next tile's load.
+      int ns = 0, np = 0;
+      uint32_t idle = 0;
+      uint64_t t_idle = 0;
+      while (ok && np < ntiles) {
+        bool progressed = false;
+        if (np < ns && tc::mbar_test_wait(&sm->p_full[np & 1], (np >> 1) & 1)) {
+          // O^T += V^T(np) P^T(np)
+          const int pb = np & 1;
+          tc::fence_after_sync();
+          const uint64_t ad0 = ad_v + (uint64_t)((pb * kTileBytes) >> 4), bd0 = bd_p + (uint64_t)((pb * kPBytes) >> 4);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+          for (int m = 0; m < 4; ++m) {
 #pragma unroll
-          for (int j = 0; j < kRows / 16; ++j)
-            tc::mma_bf16(tmem + kColO + 64 * m, ad0 + (uint64_t)((2 * m * kBoxBytes + j * 2048) >> 4),
-                         bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv, t > 0 || j > 0);
+            for (int j = 0; j < kRows / 16; ++j)
+              tc::mma_bf16(tmem + kColO + 64 * m, ad0 + (uint64_t)((2 * m * kBoxBytes + j * 2048) >> 4),
+                           bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv, np > 0 || j > 0);
+          }
+          tc::commit(&sm->kv_empty[pb]);
+          tc::commit(&sm->pv_done);
+          ++np;
+          progressed = true;
         }
-        tc::commit(&sm->kv_empty[pb]);
-        tc::commit(&sm->pv_done);
-        return true;
-      };
-      for (int li = 0; ok && li < ntiles; ++li) {
-        const int buf = li & 1;
-        ok = tc::mbar_wait(&sm->kv_full[buf], (li >> 1) & 1, abort, a.status);
-        if (!ok) break;
-        tc::fence_after_sync();
-        // descriptors differ only in the start-address field (16-byte units)
-        const uint64_t ad0 = tc::sw128_desc(kv_base + buf * kTileBytes, 16, 1024);
-        const uint64_t bd0 = tc::sw128_desc(q_base, 16, 1024);
+        // S^T(ns) overwrites the S^T buffer of tile ns - 2: P.V(ns - 2) must
+        // have been issued, i.e. its softmax has finished reading it.
+        if (ns < ntiles && ns <= np + 1 && tc::mbar_test_wait(&sm->kv_full[ns & 1], (ns >> 1) & 1)) {
+          const int buf = ns & 1;
+          tc::fence_after_sync();
+          const uint64_t ad0 = ad_kv + (uint64_t)((buf * kTileBytes) >> 4);
 #pragma unroll
-        for (int j = 0; j < kD / 16; ++j)
-          tc::mma_bf16(tmem + kColS + 64 * buf, ad0 + (uint64_t)(((j >> 2) * kBoxBytes + (j & 3) * 32) >> 4),
-                       bd0 + (uint64_t)(((j >> 2) * kQBoxBytes + (j & 3) * 32) >> 4), idesc_s, j > 0);
-        tc::commit(&sm->s_full[buf]);
-        if (li > 0) ok = pv(li - 1);
+          for (int j = 0; j < kD / 16; ++j)
+            tc::mma_bf16(tmem + kColS + 64 * buf, ad0 + (uint64_t)(((j >> 2) * kBoxBytes + (j & 3) * 32) >> 4),
+                         bd_q + (uint64_t)(((j >> 2) * kQBoxBytes + (j & 3) * 32) >> 4), idesc_s, j > 0);
+          tc::commit(&sm->s_full[buf]);
+          ++ns;
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+          t_idle = 0;
+          continue;
+        }
+        if (*abort) {
+          ok = false;
+        } else if ((++idle & 63) == 0) {
+          const uint64_t now = tc::globaltimer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > tc::kWaitLimitNs) {
+            raise_status(a.status, CSA_STATUS_WAIT_TIMEOUT);
+            *abort = 1;
+            ok = false;
+          }
+        }
       }
-      if (ok && ntiles > 0) pv(ntiles - 1);
       tc::commit(&sm->o_done);
       tc::mbar_drain(&sm->o_done, 0);
       if (q_issued) tc::mbar_drain(&sm->q_full, 0);
@@ -310,65 +355,78 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;
-    const int row = quarter * 16 + lane;                 // S^T row (lanes 0-15 of the quarter)
+    // A warp owns the 16 S^T rows of its TMEM quarter (M = 64 layout) and
+    // reads them with the 16x256b shape: lane t holds rows rq = t/4 and
+    // rq + 8 for heads 8c + 2cq + {0, 1} (c = 0..7, cq = t%4).
+    const int rq = lane >> 2, cq = lane & 3;
+    const int rowA = quarter * 16 + rq, rowB = rowA + 8;  // tile rows of this thread
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const bool leader = warp == kSoftWarp0;
-    float l[kH];
+    float l[16];  // running sums of heads 8c + 2cq + e at l[2c + e]
 #pragma unroll
-    for (int h = 0; h < kH; ++h) l[h] = 0.f;
+    for (int i = 0; i < 16; ++i) l[i] = 0.f;
     bool ok = true;
-    int idx_next = 0;
-    {
-      const int r = t0 * kRows + row;
-      if (ntiles > 0 && lane < 16 && a.idx && r < L.nsel) idx_next = a.idx[(size_t)qq * a.k + r];
+    int idxA = 0, idxB = 0;
+    if (ntiles > 0 && a.idx) {
+      const int r = t0 * kRows + rowA;
+      if (r < L.nsel) idxA = a.idx[(size_t)qq * a.k + r];
+      if (r + 8 < L.nsel) idxB = a.idx[(size_t)qq * a.k + r + 8];
     }
     for (int li = 0; li < ntiles; ++li) {
       const int buf = li & 1;
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full[buf], (li >> 1) & 1, abort, a.status));
-      if (!ok) break;
+      const bool got = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full[buf], (li >> 1) & 1, abort, a.status));
       tc::fence_after_sync();
-      const int r = (t0 + li) * kRows + row;
-      bool valid = lane < 16;
-      if (valid) valid = r < L.nsel4 ? (r < L.nsel && (!a.idx || (idx_next >= 0 && idx_next < a.N_max))) : r < L.R;
-      if (li + 1 < ntiles && lane < 16) {  // the next tile's index, loaded while this tile is processed
-        const int rn = r + kRows;
-        idx_next = (a.idx && rn < L.nsel) ? a.idx[(size_t)qq * a.k + rn] : 0;
+      const int rA = (t0 + li) * kRows + rowA, rB = rA + 8;
+      const bool validA = rA < L.nsel4 ? (rA < L.nsel && (!a.idx || (idxA >= 0 && idxA < a.N_max))) : rA < L.R;
+      const bool validB = rB < L.nsel4 ? (rB < L.nsel && (!a.idx || (idxB >= 0 && idxB < a.N_max))) : rB < L.R;
+      if (li + 1 < ntiles && a.idx) {  // the next tile's indices, loaded while this tile is processed
+        idxA = rA + kRows < L.nsel ? a.idx[(size_t)qq * a.k + rA + kRows] : 0;
+        idxB = rB + kRows < L.nsel ? a.idx[(size_t)qq * a.k + rB + kRows] : 0;
       }
-      const uint32_t sbase = tmem + lane_off + kColS + 64 * buf;
-      uint32_t v0[32], v1[32];
-      tc::tmem_ld32(sbase, v0);
-      tc::tmem_ld32(sbase + 32, v1);
+      uint32_t v[32];
+      tmem_ld_16x256b_x8(tmem + lane_off + kColS + 64 * buf, v);
       tc::tmem_ld_wait();
+      // logits in log2 units; invalid rows are -inf
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          v[4 * c + e] = __float_as_uint(validA ? __uint_as_float(v[4 * c + e]) * scale_log2 : -INFINITY);
+          v[4 * c + 2 + e] = __float_as_uint(validB ? __uint_as_float(v[4 * c + 2 + e]) * scale_log2 : -INFINITY);
+        }
       // Fast path: the running per-head maximum moves only when some logit
       // of the tile exceeds it by more than 2^8 (always on the first tile).
       bool over = false;
-      if (valid) {
 #pragma unroll
-        for (int h = 0; h < kH; h += 4) {
-          const float4 mr = *reinterpret_cast<const float4 *>(&sm->mref[h]);
-          const float mm[4] = {mr.x, mr.y, mr.z, mr.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float x = __uint_as_float(h + i < 32 ? v0[h + i] : v1[h + i - 32]) * scale_log2;
-            over |= x > mm[i] + kRescaleLog2;
-          }
-        }
+      for (int c = 0; c < 8; ++c) {
+        const float2 mr = *reinterpret_cast<const float2 *>(&sm->mref[8 * c + 2 * cq]);
+        over |= __uint_as_float(v[4 * c]) > mr.x + kRescaleLog2 || __uint_as_float(v[4 * c + 1]) > mr.y + kRescaleLog2 ||
+                __uint_as_float(v[4 * c + 2]) > mr.x + kRescaleLog2 || __uint_as_float(v[4 * c + 3]) > mr.y + kRescaleLog2;
       }
       if (leader && lane == 0) sm->need[(li + 2) & 3] = 0;  // slot of tile li + 2, last read at tile li - 2
       if (__any_sync(0xffffffffu, over) && lane == 0) atomicOr(&sm->need[li & 3], 1);
-      named_sync(1, 128);
+      if (bar_any(1, 128, !(got && ok))) {  // S^T(li) missing, or the previous P.V never completed
+        ok = false;
+        break;
+      }
       bool rescale = false;
       if (sm->need[li & 3] != 0) {
-        {
-          float red[kH];
+        // per-head tile maximum: over the thread's two rows, then over the 8
+        // lanes of the same cq, then over the 4 warps
+        float mx[16];
 #pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            red[h] = valid ? __uint_as_float(v0[h]) * scale_log2 : -INFINITY;
-            red[h + 32] = valid ? __uint_as_float(v1[h]) * scale_log2 : -INFINITY;
-          }
-          transpose_reduce64<true>(red, lane);
-          sm->red[quarter][2 * lane] = red[0];
-          sm->red[quarter][2 * lane + 1] = red[1];
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) mx[2 * c + e] = fmaxf(__uint_as_float(v[4 * c + e]), __uint_as_float(v[4 * c + 2 + e]));
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
+        if (rq == 0) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) sm->red[quarter][8 * c + 2 * cq + e] = mx[2 * c + e];
         }
         named_sync(1, 128);
         if (leader) {
@@ -394,36 +452,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = sm->rescale != 0;
         if (rescale) {
 #pragma unroll
-          for (int h = 0; h < kH; ++h) l[h] *= sm->alpha[h];
+          for (int c = 0; c < 8; ++c) {
+            const float2 al = *reinterpret_cast<const float2 *>(&sm->alpha[8 * c + 2 * cq]);
+            l[2 * c] *= al.x;
+            l[2 * c + 1] *= al.y;
+          }
         }
-        tc::tmem_ld32(sbase, v0);  // the logits again (registers were released for the reduction)
-        tc::tmem_ld32(sbase + 32, v1);
-        tc::tmem_ld_wait();
       }
-      // P = 2^(x - mref), summed per head, packed to bf16 into P^T row `row`.
-      uint32_t pk[32];
-#pragma unroll
-      for (int h = 0; h < kH; h += 4) {
-        const float4 mr = *reinterpret_cast<const float4 *>(&sm->mref[h]);
-        const float mm[4] = {mr.x, mr.y, mr.z, mr.w};
-        float p[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float x = fmaf(__uint_as_float(h + i < 32 ? v0[h + i] : v1[h + i - 32]), scale_log2, -mm[i]);
-          p[i] = valid ? ex2_approx(x) : 0.f;
-          l[h + i] += p[i];
-        }
-        __nv_bfloat162 t0 = __floats2bfloat162_rn(p[0], p[1]), t1 = __floats2bfloat162_rn(p[2], p[3]);
-        pk[h >> 1] = *reinterpret_cast<uint32_t *>(&t0);
-        pk[(h >> 1) + 1] = *reinterpret_cast<uint32_t *>(&t1);
-      }
-      if (lane < 16) {
-        const uint32_t prow = tc::smem_u32(ps) + buf * kPBytes + row * 128;
+      // P = 2^(x - mref), rounded to bf16, summed per head, packed in pairs of heads and
+      // stored into rows rowA / rowB of P^T (128-byte rows, 16-byte chunks
+      // swizzled by row & 7; rowA and rowB share row & 7).
+      {
+        const uint32_t pbase = tc::smem_u32(ps) + buf * kPBytes + 4 * cq;
+        const uint32_t swz = rowA & 7;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const uint32_t addr = prow + ((c ^ (row & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
-                       "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+          const float2 mr = *reinterpret_cast<const float2 *>(&sm->mref[8 * c + 2 * cq]);
+          // (an invalid row is -inf, and so may mref be while no valid row has been seen)
+          const float pa0 = validA ? ex2_approx(__uint_as_float(v[4 * c]) - mr.x) : 0.f;
+          const float pa1 = validA ? ex2_approx(__uint_as_float(v[4 * c + 1]) - mr.y) : 0.f;
+          const float pb0 = validB ? ex2_approx(__uint_as_float(v[4 * c + 2]) - mr.x) : 0.f;
+          const float pb1 = validB ? ex2_approx(__uint_as_float(v[4 * c + 3]) - mr.y) : 0.f;
+          __nv_bfloat162 ta = __floats2bfloat162_rn(pa0, pa1), tb = __floats2bfloat162_rn(pb0, pb1);
+          // the sums take the same bf16 weights as P.V, so that a dominant
+          // row's weight (up to 2^8 between rescales) cancels exactly
+          const float2 fa = __bfloat1622float2(ta), fb = __bfloat1622float2(tb);
+          l[2 * c] += fa.x + fb.x;
+          l[2 * c + 1] += fa.y + fb.y;
+          const uint32_t off = (uint32_t)((c ^ swz) << 4);
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(pbase + rowA * 128 + off), "r"(*reinterpret_cast<uint32_t *>(&ta))
+                       : "memory");
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(pbase + rowB * 128 + off), "r"(*reinterpret_cast<uint32_t *>(&tb))
                        : "memory");
         }
       }
@@ -431,9 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P.V of the previous tile must be complete before O^T may be
         // touched; consumed every tile so the barrier phases stay in step.
         ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->pv_done, (li - 1) & 1, abort, a.status));
-        if (!ok) break;
         tc::fence_after_sync();
-        if (rescale) {
+        if (ok && rescale) {
 #pragma unroll 1
           for (int m = 0; m < 4; ++m) {
 #pragma unroll 1
@@ -457,10 +515,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue: per-head sums, then O (partials, or the final output)
     ok = __all_sync(0xffffffffu, ok && (ntiles == 0 || tc::mbar_wait(&sm->o_done, 0, abort, a.status)));
     tc::fence_after_sync();
-    transpose_reduce64<false>(l, lane);
-    sm->red[quarter][2 * lane] = l[0];
-    sm->red[quarter][2 * lane + 1] = l[1];
-    named_sync(1, 128);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) l[i] += __shfl_xor_sync(0xffffffffu, l[i], o);
+    if (rq == 0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) sm->red[quarter][8 * c + 2 * cq + e] = l[2 * c + e];
+    }
+    ok = !bar_any(1, 128, !ok);  // every softmax warp takes the same branch below
     if (leader) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -470,24 +535,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_sync(1, 128);
     const int orow = quarter * 32 + lane;  // O^T row (dims) within a 128-dim chunk
-    const size_t pidx = (size_t)qq * splits + split;
-    if (ok && splits > 1) {
-      if (leader) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int h = 2 * lane + i;
-          part_ml[(pidx * 2) * kH + h] = sm->mref[h];
-          part_ml[(pidx * 2 + 1) * kH + h] = sm->lsum[h];
-        }
-      }
-      float *po = part_o + pidx * (size_t)kH * kD;
+    if (splits > 1) {
+      // Stage this split's unnormalised O (fp32, [64 heads][512 dims]) in
+      // the tile buffers, which no copy or MMA touches any more, for the
+      // cluster merge below; its (mref, lsum) stay in shared memory.
+      float *ostage = reinterpret_cast<float *>(kv);
 #pragma unroll 1
       for (int m = 0; m < 4; ++m) {
         const int d = 128 * m + orow;
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           uint32_t v[32];
-          if (ntiles > 0) {
+          if (ok && ntiles > 0) {
             tc::tmem_ld32(tmem + lane_off + kColO + 64 * m + 32 * half, v);
             tc::tmem_ld_wait();
           } else {
@@ -495,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 32; ++c) v[c] = 0u;
           }
 #pragma unroll
-          for (int c = 0; c < 32; ++c) po[(size_t)(32 * half + c) * kD + d] = __uint_as_float(v[c]);
+          for (int c = 0; c < 32; ++c) ostage[(32 * half + c) * kD + d] = __uint_as_float(v[c]);
         }
       }
     } else if (ok) {
@@ -533,54 +592,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
-}
-
-// Merge the split partials of each query with the sink:
-//   M = max(max_s m_s, sink), L = sum_s l_s 2^(m_s - M) + 2^(sink - M),
-//   out = sum_s O_s 2^(m_s - M) / L   (m and sink in log2 units).
-// One block per (query, head); thread t owns dims 4t..4t+3 and issues the
-// loads of all splits at once.
-__global__ void __launch_bounds__(128) mqa_combine_kernel(const float *part_o, const float *part_ml,
-                                                          const float *sink, bf16 *out, int splits) {
-  extern __shared__ float w[];  // [splits] weights, then [2][splits] (m, l)
-  const int qq = blockIdx.x, h = blockIdx.y;
-  pdl_wait();
-  pdl_release();
-  float *ml = w + splits;
-  for (int i = threadIdx.x; i < 2 * splits; i += blockDim.x) {
-    const int which = i / splits, s = i - which * splits;
-    ml[i] = part_ml[(((size_t)qq * splits + s) * 2 + which) * kH + h];
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const float sk = sink[h] * kLog2e;
-    float M = sk;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[s]);
-    float Lsum = exp2f(sk - M);
-    for (int s = 0; s < splits; ++s) {
-      const float ww = ml[s] == -INFINITY ? 0.f : exp2f(ml[s] - M);
-      w[s] = ww;
-      Lsum += ml[splits + s] * ww;
+  if (splits > 1) {
+    // The splits of query qq are the blocks of one cluster (rank = split).
+    // Merge with the sink, every block taking 1/splits of the outputs:
+    //   M = max(max_s m_s, sink), L = sum_s l_s 2^(m_s - M) + 2^(sink - M),
+    //   out = sum_s O_s 2^(m_s - M) / L   (m and sink in log2 units).
+    cluster_sync();  // every split's O, mref and lsum are staged
+    float *coef = reinterpret_cast<float *>(ps);  // [splits][64]: 2^(m_s - M) / L
+    if (threadIdx.x < kH) {
+      const int h = threadIdx.x;
+      float mr[kMaxSplits], lr[kMaxSplits];
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (r < splits) {
+          mr[r] = ld_peer_f(&sm->mref[h], r);
+          lr[r] = ld_peer_f(&sm->lsum[h], r);
+        }
+      const float sk = a.sink[h] * kLog2e;
+      float M = sk;
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (r < splits) M = fmaxf(M, mr[r]);
+      float Lsum = exp2f(sk - M), w[kMaxSplits];
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (r < splits) {
+          w[r] = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - M);
+          Lsum += lr[r] * w[r];
+        }
+      const float inv = 1.f / Lsum;
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (r < splits) coef[r * kH + h] = w[r] * inv;
     }
-    const float inv = 1.f / Lsum;
-    for (int s = 0; s < splits; ++s) w[s] *= inv;
+    __syncthreads();
+    const float *ostage = reinterpret_cast<const float *>(kv);
+    bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qq * kH * kD;
+    constexpr int kGroups = kH * kD / 4;  // 4-dim groups of the output
+    const int g1 = (split + 1) * kGroups / splits;
+    for (int gi = split * kGroups / splits + threadIdx.x; gi < g1; gi += kThreads) {
+      const int h = gi / (kD / 4), d = 4 * (gi % (kD / 4));
+      float4 v[kMaxSplits];
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (r < splits) v[r] = ld_peer_f4(ostage + h * kD + d, r);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (r < splits) {
+          const float c = coef[r * kH + h];
+          acc.x = fmaf(c, v[r].x, acc.x);
+          acc.y = fmaf(c, v[r].y, acc.y);
+          acc.z = fmaf(c, v[r].z, acc.z);
+          acc.w = fmaf(c, v[r].w, acc.w);
+        }
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+      *reinterpret_cast<uint2 *>(out + h * kD + d) =
+          make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+    }
+    cluster_sync();  // no block leaves while a peer may still read its staging buffer
   }
-  __syncthreads();
-  const int d = 4 * threadIdx.x;
-  const float *src = part_o + ((size_t)qq * splits * kH + h) * kD + d;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-  for (int s = 0; s < splits; ++s) {
-    const float4 v = *reinterpret_cast<const float4 *>(src + (size_t)s * kH * kD);
-    const float ww = w[s];
-    acc.x = fmaf(ww, v.x, acc.x);
-    acc.y = fmaf(ww, v.y, acc.y);
-    acc.z = fmaf(ww, v.z, acc.z);
-    acc.w = fmaf(ww, v.w, acc.w);
-  }
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-  uint2 pk = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-  *reinterpret_cast<uint2 *>(out + ((size_t)qq * kH + h) * kD + d) = pk;
 }
 
 int num_sms_cached() {
@@ -597,6 +668,7 @@ int num_sms_cached() {
 void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split) {
   const int tiles = (rows_max + kRows - 1) / kRows;
   int s = num_sms_cached() / (Q > 0 ? Q : 1);
+  s = s > kMaxSplits ? kMaxSplits : s;
   s = s < 1 ? 1 : (s > tiles ? tiles : s);
   const int tps = (tiles + s - 1) / s;
   *tiles_per_split = tps;
@@ -614,46 +686,29 @@ int rows_max_of(const MqaArgs &a) { return (((a.idx ? a.k : a.N_max) + 3) & ~3) 
 
 }  // namespace
 
-size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
-  if (H != kH || D != kD || Q < 1) return 0;
-  // Upper bound on the split count the launcher can pick for any row list of
-  // at most rows_max rows (+3 rows of padding): min(tiles, SMs / Q).
-  const int tiles = (rows_max + 3 + kRows - 1) / kRows;
-  int s = num_sms_cached() / Q;
-  s = s < 1 ? 1 : (s > tiles ? tiles : s);
-  if (s <= 1) return 0;
-  return (size_t)Q * s * kH * (kD + 2) * sizeof(float);
-}
+// The splits of a query merge through distributed shared memory: no
+// workspace beyond the status word.
+size_t mqa_tc_partial_bytes(int, int, int, int) { return 0; }
 
 cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   *taken = false;
   if (!tc_shape(a)) return cudaSuccess;
   int splits, tps;
   plan_splits(a.Q, rows_max_of(a), &splits, &tps);
-  const size_t need = splits > 1 ? (size_t)a.Q * splits * kH * (kD + 2) * sizeof(float) : 0;
-  if (need > a.partial_bytes) return cudaSuccess;  // cannot happen with the documented workspace size
-  CUtensorMap tm_q, tm_cmp_g, tm_win_g, tm_cmp_t, tm_win_t;
+  CUtensorMap tm_q, tm_cmp_t, tm_win_t;
   const uint64_t cmp_rows = (uint64_t)a.B * a.N_max, win_rows = (uint64_t)a.B * a.T_raw;
   if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * kH, kD * 2, 64, kH) ||
-      !make_tmap_bf16_2d(&tm_cmp_g, a.kv_cmp, kD, cmp_rows, kD * 2, 64, 1) ||
-      !make_tmap_bf16_2d(&tm_win_g, a.kv_win, kD, win_rows, kD * 2, 64, 1) ||
       !make_tmap_bf16_2d(&tm_cmp_t, a.kv_cmp, kD, cmp_rows, kD * 2, 64, kRows) ||
       !make_tmap_bf16_2d(&tm_win_t, a.kv_win, kD, win_rows, kD * 2, 64, kRows))
     return cudaSuccess;
-  float *part_o = static_cast<float *>(a.partials);
-  float *part_ml = part_o + (size_t)a.Q * splits * kH * kD;
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     attr_set = true;
   }
-  dim3 grid(splits, a.Q);
   *taken = true;
-  cudaError_t e = launch_pdl(mqa_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tm_q, tm_cmp_g, tm_win_g, tm_cmp_t,
-                             tm_win_t, a, splits, tps, a.scale * kLog2e, part_o, part_ml);
-  if (e != cudaSuccess || splits <= 1) return e;
-  return launch_pdl(mqa_combine_kernel, dim3(a.Q, kH), dim3(kD / 4), splits * 3 * sizeof(float), stream,
-                    (const float *)part_o, (const float *)part_ml, a.sink, static_cast<bf16 *>(a.out), splits);
+  return launch_pdl_cluster(mqa_tc_kernel, dim3(splits, a.Q), dim3(kThreads), kSmemBytes, stream, (unsigned)splits,
+                            tm_q, tm_cmp_t, tm_win_t, a, splits, tps, a.scale * kLog2e);
 }
 
 }  // namespace csa

@@ -12,11 +12,18 @@
 // ordered pass keeps every entry with key > tau and the first kk entries (by
 // index) with key == tau; per-warp ballots and an exclusive prefix over the
 // block give each kept entry its output slot, so the output is ascending and
-// deterministic. Lists of up to 8K entries: one 1024-thread block per query
-// with the keys cached in shared memory. Longer lists take two stages: the
-// exact top-k of 4K-32K-entry segments in parallel, then the same selection
-// over the concatenated segment winners. Without scratch space a single block
-// per query does it all (re-reading the scores per pass beyond 48K entries).
+// deterministic.
+//
+// Launch shapes. Few queries (a decode batch): the list of one query is cut
+// into C contiguous slices, one CTA of a thread-block cluster each (C <= 8,
+// about SMs / Q); the slices' histograms are summed through distributed
+// shared memory at every radix pass, and each CTA emits its own slice at the
+// offset given by the counts of the slices before it. Many queries: one
+// 1024-thread CTA per query with the keys cached in shared memory (up to
+// 48K entries). Longer lists with many queries take two stages: the exact
+// top-k of 4K-32K-entry segments in parallel, then the same selection over
+// the concatenated segment winners. Without scratch space a single CTA per
+// query does it all (re-reading the scores per pass beyond 48K entries).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -59,6 +66,31 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scan, 
   const uint32_t r = x - v + (warp > 0 ? scan[warp - 1] : 0u);
   __syncthreads();
   return r;
+}
+
+// keys[j] = score_key(s[j]) for j < len, with 8 loads per thread in flight
+// (a plain strided loop waits out one load latency per iteration). Returns
+// this thread's min and max key in lo / hi.
+__device__ __forceinline__ void cache_keys(uint32_t *keys, const float *s, int len, uint32_t &lo, uint32_t &hi) {
+  constexpr int U = 8;
+  for (int j0 = threadIdx.x; j0 < len; j0 += kThreads * U) {
+    float x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * kThreads;
+      x[u] = j < len ? s[j] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * kThreads;
+      if (j < len) {
+        const uint32_t k = score_key(x[u]);
+        keys[j] = k;
+        lo = min(lo, k);
+        hi = max(hi, k);
+      }
+    }
+  }
 }
 
 template <bool kCached>
@@ -172,7 +204,7 @@ __device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const floa
   }
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int cache_keys) {
+__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int use_cache) {
   extern __shared__ uint32_t keys[];
   __shared__ TopkShared sh;
   pdl_wait();
@@ -187,13 +219,202 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int cache_ke
     return;
   }
   auto emit = [out](uint32_t slot, int j, uint32_t) { out[slot] = j; };
-  if (cache_keys && n <= kSmemKeys) {
-    for (int j = threadIdx.x; j < n; j += kThreads) keys[j] = score_key(s[j]);
+  if (use_cache && n <= kSmemKeys) {
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    cache_keys(keys, s, n, lo, hi);
     __syncthreads();
     select_and_emit<true>(sh, keys, s, n, k, emit);
   } else {
     select_and_emit<false>(sh, keys, s, n, k, emit);
   }
+}
+
+struct ClusterShared {
+  uint32_t hist[2][kBins];  // pass p uses hist[p & 1]; peers read it after the pass's cluster barrier
+  uint32_t scan[kWarps];
+  uint32_t warp_gt[kWarps], warp_eq[kWarps];
+  uint32_t lmin, lmax, cnt_gt, cnt_eq;  // this slice's key range and kept counts (read by peers)
+  uint32_t prefix, kk, kmin, krange, base_gt, base_eq;
+};
+
+// One query per cluster; CTA c of C selects over the slice
+// [c * S, c * S + S) of the list, S = ceil(n / C) rounded up to 32.
+__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkArgs a) {
+  extern __shared__ uint32_t keys[];
+  __shared__ ClusterShared cs;
+  pdl_wait();
+  pdl_release();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t C = cluster_size(), c = cluster_rank();
+  const int q = blockIdx.y;
+  const int n = clamp_count(a.n_cmp[q], a.N_max, (threadIdx.x == 0 && c == 0) ? a.status : nullptr);
+  const int k = a.k;
+  int32_t *out = a.out_idx + (size_t)q * k;
+  if (n <= k) {  // the same for every CTA of the cluster: no CTA touches a peer
+    if (c == 0)
+      for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const int S = ((n + (int)C - 1) / (int)C + 31) & ~31;
+  const int j0 = (int)c * S;
+  const int len = max(0, min(S, n - j0));
+  const float *s = a.scores + (size_t)q * a.N_max + j0;
+
+  // Keys of the slice into shared memory, with the slice's key range.
+  uint32_t lo_k = 0xffffffffu, hi_k = 0u;
+  cache_keys(keys, s, len, lo_k, hi_k);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo_k = min(lo_k, __shfl_xor_sync(0xffffffffu, lo_k, o));
+    hi_k = max(hi_k, __shfl_xor_sync(0xffffffffu, hi_k, o));
+  }
+  if (lane == 0) {
+    cs.warp_gt[warp] = lo_k;
+    cs.warp_eq[warp] = hi_k;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t x = cs.warp_gt[lane], y = cs.warp_eq[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
+      y = max(y, __shfl_xor_sync(0xffffffffu, y, o));
+    }
+    if (lane == 0) {
+      cs.lmin = x;
+      cs.lmax = y;
+    }
+  }
+  cluster_sync();  // every slice's range is published
+  if (warp == 0) {
+    uint32_t x = 0xffffffffu, y = 0u;
+    if ((uint32_t)lane < C) {
+      x = ld_peer(&cs.lmin, lane);
+      y = ld_peer(&cs.lmax, lane);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
+      y = max(y, __shfl_xor_sync(0xffffffffu, y, o));
+    }
+    if (lane == 0) {
+      cs.kmin = x;
+      cs.krange = y - x;
+      cs.prefix = 0;
+      cs.kk = (uint32_t)k;
+    }
+  }
+  __syncthreads();
+  const uint32_t kmin = cs.kmin, range = cs.krange;
+  const int nbits = range == 0 ? 0 : 32 - __clz(range);
+  uint32_t mask = 0;
+  int pass = 0;
+  for (int top = nbits; top > 0; ++pass) {
+    const int width = top >= 11 ? 11 : top;
+    const int shift = top - width;
+    const uint32_t dmask = (1u << width) - 1u;
+    uint32_t *hist = cs.hist[pass & 1];
+    for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = cs.prefix;
+    for (int j = threadIdx.x; j < len; j += kThreads) {
+      const uint32_t u = keys[j] - kmin;
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+    }
+    cluster_sync();  // every slice's histogram of this pass is complete
+    const int b_hi = kBins - 1 - 2 * threadIdx.x, b_lo = b_hi - 1;
+    uint32_t ph[8], pl[8];  // all remote loads in flight before the sums
+#pragma unroll
+    for (uint32_t r = 0; r < 8; ++r)
+      if (r < C) {
+        ph[r] = ld_peer(&hist[b_hi], r);
+        pl[r] = ld_peer(&hist[b_lo], r);
+      }
+    uint32_t c_hi = 0, c_lo = 0;
+#pragma unroll
+    for (uint32_t r = 0; r < 8; ++r)
+      if (r < C) {
+        c_hi += ph[r];
+        c_lo += pl[r];
+      }
+    const uint32_t above = block_excl_scan(c_hi + c_lo, cs.scan, lane, warp);
+    const uint32_t kk = cs.kk;
+    if (above < kk && kk <= above + c_hi + c_lo) {
+      const bool in_hi = kk <= above + c_hi;
+      const uint32_t bin = in_hi ? b_hi : b_lo;
+      cs.kk = kk - (in_hi ? above : above + c_hi);
+      cs.prefix = prefix | (bin << shift);
+    }
+    mask |= dmask << shift;
+    top = shift;
+    __syncthreads();
+  }
+  const uint32_t tau = cs.prefix + kmin, kk = cs.kk;
+
+  // Ordered compaction: count, exchange the slice totals, then emit.
+  const int per_warp = (((len + kWarps - 1) / kWarps) + 31) & ~31;
+  const int lo = min(len, warp * per_warp), hi = min(len, lo + per_warp);
+  uint32_t g = 0, e = 0;
+  for (int base = lo; base < hi; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = j < hi ? keys[j] : 0u;
+    g += __popc(__ballot_sync(0xffffffffu, j < hi && u > tau));
+    e += __popc(__ballot_sync(0xffffffffu, j < hi && u == tau));
+  }
+  if (lane == 0) {
+    cs.warp_gt[warp] = g;
+    cs.warp_eq[warp] = e;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t x = cs.warp_gt[lane], y = cs.warp_eq[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x += __shfl_xor_sync(0xffffffffu, x, o);
+      y += __shfl_xor_sync(0xffffffffu, y, o);
+    }
+    if (lane == 0) {
+      cs.cnt_gt = x;
+      cs.cnt_eq = y;
+    }
+  }
+  cluster_sync();  // every slice's counts are published
+  if (warp == 0) {
+    uint32_t x = 0, y = 0;
+    if ((uint32_t)lane < c) {
+      x = ld_peer(&cs.cnt_gt, lane);
+      y = ld_peer(&cs.cnt_eq, lane);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x += __shfl_xor_sync(0xffffffffu, x, o);
+      y += __shfl_xor_sync(0xffffffffu, y, o);
+    }
+    if (lane == 0) {
+      cs.base_gt = x;
+      cs.base_eq = y;
+    }
+  }
+  cluster_arrive();  // this CTA reads no peer after this point
+  __syncthreads();
+  uint32_t G = cs.base_gt, E = cs.base_eq;
+  for (int w = 0; w < warp; ++w) {
+    G += cs.warp_gt[w];
+    E += cs.warp_eq[w];
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = j < hi ? keys[j] : 0u;
+    const bool is_gt = j < hi && u > tau, is_eq = j < hi && u == tau;
+    const uint32_t mg = __ballot_sync(0xffffffffu, is_gt), me = __ballot_sync(0xffffffffu, is_eq);
+    const uint32_t Gl = G + __popc(mg & lt), El = E + __popc(me & lt);
+    if (is_gt) out[Gl + min(El, kk)] = j0 + j;
+    else if (is_eq && El < kk) out[Gl + El] = j0 + j;
+    G += __popc(mg);
+    E += __popc(me);
+  }
+  cluster_wait();  // no peer reads this CTA's shared memory any more
 }
 
 // Two-stage selection for long lists. Stage 1: segment g of query q (`seg`
@@ -204,7 +425,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int cache_ke
 // Segments start at 4K entries and double until the winners of all segments
 // fit the stage-2 shared-memory cache.
 bool plan_two_stage(int N_max, int k, int *seg, int *nseg) {
-  if (N_max <= 8192) return false;
+  // While a row's keys fit in shared memory the single-pass kernel reads the
+  // scores once and is faster than two launches.
+  if (N_max <= kSmemKeys) return false;
   for (int s = 4096; s <= 32768; s *= 2) {
     const int n = (N_max + s - 1) / s;
     if ((long long)n * k <= kSmemKeys / 2 && n <= kThreads && N_max > 2 * s) {
@@ -238,7 +461,8 @@ __global__ void __launch_bounds__(kThreads) topk_stage1_kernel(TopkArgs a, uint3
     }
     return;
   }
-  for (int j = threadIdx.x; j < len; j += kThreads) keys[j] = score_key(s[j]);
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  cache_keys(keys, s, len, lo, hi);
   __syncthreads();
   select_and_emit<true>(sh, keys, s, len, a.k, [ck, ci, j0](uint32_t slot, int j, uint32_t u) {
     ck[slot] = u;
@@ -287,6 +511,21 @@ __global__ void __launch_bounds__(kThreads) topk_stage2_kernel(TopkArgs a, const
 
 }  // namespace
 
+// Cluster size for one query's list: about SMs / Q CTAs, at most 8, at
+// least 2K entries per CTA, the slice's keys within the shared-memory cache.
+int plan_cluster(int Q, int N_max, int k) {
+  if (Q < 1 || N_max <= k || N_max < 4096) return 0;
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int C = sms / Q;
+  C = C > 8 ? 8 : C;
+  const int by_len = (N_max + 2047) / 2048;
+  C = C > by_len ? by_len : C;
+  if (C < 2 || (N_max + C - 1) / C > kSmemKeys - 32 || Q > 65535) return 0;
+  return C;
+}
+
 size_t topk_scratch_bytes(int Q, int N_max, int k) {
   int seg, nseg;
   if (!plan_two_stage(N_max, k, &seg, &nseg)) return 0;
@@ -299,7 +538,13 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, s
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     cudaFuncSetAttribute(topk_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 * 4);
     cudaFuncSetAttribute(topk_stage2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
+    cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     attr_set = true;
+  }
+  if (const int C = plan_cluster(a.Q, a.N_max, a.k)) {
+    const int S = ((a.N_max + C - 1) / C + 31) & ~31;
+    return launch_pdl_cluster(topk_cluster_kernel, dim3(C, a.Q), dim3(kThreads), (size_t)S * 4, stream, (unsigned)C,
+                              a);
   }
   int seg = 0, nseg = 0;
   const size_t need = topk_scratch_bytes(a.Q, a.N_max, a.k);

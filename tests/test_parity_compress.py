@@ -30,6 +30,9 @@ def _oracle(kv, gate, ape, w, win, stride):
     (2, 300, 64, 5, 3, torch.float32),       # other window geometry
     (1, 8, 512, 8, 4, torch.bfloat16),       # exactly one window
     (4, 130, 256, 128, 128, torch.bfloat16),  # one HCA window per sequence, D = 256
+    (3, 200, 512, 48, 16, torch.bfloat16),   # cluster of 3 blocks per entry, 16 positions each
+    (2, 150, 512, 40, 8, torch.bfloat16),    # cluster of 2, 20 positions each (ragged over 8 groups)
+    (2, 300, 512, 64, 32, torch.bfloat16),   # cluster of 4
 ])
 def test_compress_matches_oracle(cuda_device, B, T, D, win, stride, dtype):
     kv, gate, ape, w, dev = _inputs(1, B, T, D, win, dtype, cuda_device, gate_scale=2.0)

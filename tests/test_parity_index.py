@@ -42,7 +42,7 @@ def test_index_scores_match_oracle(cuda_device, Q, B, N, Hi, Di, dtype):
 @pytest.mark.parametrize("N,k", [(1, 1), (100, 100), (101, 100), (1000, 16), (5000, 512), (20000, 2048),
                                  (49153, 512), (100000, 2048), (262143, 1024), (300000, 64)])
 def test_topk_exact_on_given_scores(cuda_device, N, k):
-    # (the largest cases take the two-stage selection: 16K-entry segments)
+    # (from 49153 entries up the selection is two-stage: segments, then a merge)
     # Both sides select from the same fp32 scores: bit-exact index sets.
     # Scores are quantised so that ties (including +0 / -0) are frequent.
     Q = 3
@@ -57,6 +57,32 @@ def test_topk_exact_on_given_scores(cuda_device, N, k):
         want = O.topk(f64(s[q, :nv]), k)
         m = min(k, nv)
         assert np.array_equal(np.sort(want[:m]), got[q, :m]), f"query {q}"
+        assert np.all(got[q, m:] == -1)
+
+
+@pytest.mark.parametrize("Q,N,k,shape", [
+    (32, 16383, 512, "cluster of 4 CTAs per query (64K-context decode batch)"),
+    (8, 262143, 1024, "cluster of 8 CTAs per query, 32K entries each (1M-context decode batch)"),
+    (5, 4500, 512, "cluster of 3, a short last slice"),
+    (100, 5000, 512, "one CTA per query, keys cached"),
+    (100, 60000, 64, "two stages: segment winners, then a merge"),
+    (76, 1 << 20, 2048, "one CTA per query re-reading the scores (winners too many to merge)"),
+])
+def test_topk_every_launch_shape(cuda_device, Q, N, k, shape):
+    # The launch shape follows from (Q, N, k) and the GPU's 148 SMs. Scores
+    # are drawn on the device; the checked rows are drawn again on the host.
+    u = synth.uniform(5, 13, (Q, N), device=cuda_device)
+    s = torch.floor(u * 4096) - 2048.0              # ties at every threshold
+    n = torch.tensor([N - (q % 5) * 3 for q in range(Q)], dtype=torch.int32)
+    n[1] = min(N, k + 1)                             # just above k: one entry dropped
+    got = ops.topk(s, n.to(cuda_device), k).cpu().numpy()
+    del u, s
+    for q in sorted({0, 1, Q // 2, Q - 1}):
+        nv = int(n[q])
+        row = synth.uniform_at(5, 13, q * N + torch.arange(nv, dtype=torch.int64))
+        want = O.topk(f64(torch.floor(row * 4096) - 2048.0), k)
+        m = min(k, nv)
+        assert np.array_equal(np.sort(want[:m]), got[q, :m]), f"{shape}: query {q}"
         assert np.all(got[q, m:] == -1)
 
 
