@@ -26,8 +26,9 @@
 // the two loader warps (TMA gathers issue too slowly for 1 KB rows). The
 // compressed segment is padded to a multiple of 4 rows (unused, masked).
 //
-// Work split: query q's row list is cut into `splits` (<= 8) runs of whole
-// tiles, one CTA each, the CTAs of a query forming one thread-block cluster.
+// Work split: query q's row list is cut into `splits` (<= 16) runs of whole
+// tiles, one CTA each, the CTAs of a query forming one thread-block cluster
+// (the largest size for which every query's cluster is resident at once).
 // With one split the CTA folds in the sink and writes the output; otherwise
 // every CTA stages its unnormalised (m, l, O) in shared memory and, after a
 // cluster barrier, merges 1/splits of the output from all of them through
@@ -57,7 +58,7 @@ constexpr int kThreads = 224;
 constexpr int kMmaWarp = 2;
 constexpr int kSoftWarp0 = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxSplits = 8;                       // splits of one query form one (portable-size) cluster
+constexpr int kMaxSplits = 16;                      // splits of one query form one cluster (<= 16 CTAs)
 constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m (M = 128 layout)
 constexpr uint32_t kColS = 256;                     // S^T buffer j at 256 + 64j (M = 64 layout)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -665,14 +666,62 @@ int num_sms_cached() {
   return n;
 }
 
+void set_kernel_attributes() {
+  static bool done = false;
+  if (!done) {
+    cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    done = true;
+  }
+}
+
+// How many clusters of `size` CTAs of this kernel the GPU holds at once
+// (one CTA per SM, and a cluster must fit in one GPC).
+int max_active_clusters(int size) {
+  static int cache[kMaxSplits + 1] = {0};
+  if (size < 1 || size > kMaxSplits) return 0;
+  if (cache[size] == 0) {
+    set_kernel_attributes();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(size, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = size;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cache[size] = n > 0 ? n : -1;
+  }
+  return cache[size] > 0 ? cache[size] : 0;
+}
+
+// Split query rows into runs of whole tiles: the largest cluster size (up to
+// SMs / Q and 16) for which all Q clusters are resident at once; one split
+// when no cluster size fits.
 void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split) {
   const int tiles = (rows_max + kRows - 1) / kRows;
-  int s = num_sms_cached() / (Q > 0 ? Q : 1);
-  s = s > kMaxSplits ? kMaxSplits : s;
-  s = s < 1 ? 1 : (s > tiles ? tiles : s);
-  const int tps = (tiles + s - 1) / s;
-  *tiles_per_split = tps;
-  *splits = (tiles + tps - 1) / tps;
+  int hi = num_sms_cached() / (Q > 0 ? Q : 1);
+  hi = hi > kMaxSplits ? kMaxSplits : hi;
+  hi = hi > tiles ? tiles : hi;
+  for (int s = hi; s >= 2; --s) {
+    const int tps = (tiles + s - 1) / s;
+    const int sp = (tiles + tps - 1) / tps;
+    if (sp >= 2 && max_active_clusters(sp) >= Q) {
+      *splits = sp;
+      *tiles_per_split = tps;
+      return;
+    }
+  }
+  *splits = 1;
+  *tiles_per_split = tiles > 0 ? tiles : 1;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -701,11 +750,7 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
       !make_tmap_bf16_2d(&tm_cmp_t, a.kv_cmp, kD, cmp_rows, kD * 2, 64, kRows) ||
       !make_tmap_bf16_2d(&tm_win_t, a.kv_win, kD, win_rows, kD * 2, 64, kRows))
     return cudaSuccess;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    attr_set = true;
-  }
+  set_kernel_attributes();
   *taken = true;
   return launch_pdl_cluster(mqa_tc_kernel, dim3(splits, a.Q), dim3(kThreads), kSmemBytes, stream, (unsigned)splits,
                             tm_q, tm_cmp_t, tm_win_t, a, splits, tps, a.scale * kLog2e);

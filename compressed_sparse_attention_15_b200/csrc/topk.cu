@@ -36,12 +36,35 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kSmemKeys = 48 * 1024;
 
+constexpr int kFew = 32;  // a boundary bin this small is finished by one warp
+
 struct TopkShared {
   uint32_t hist[kBins];
   uint32_t scan[kWarps];
   uint32_t warp_gt[kWarps], warp_eq[kWarps];
-  uint32_t prefix, kk, kmin, krange;
+  uint32_t prefix, kk, kmin, krange, bcnt, ncand;
+  uint32_t cand[kFew];
 };
+
+// The kk-th largest (1 <= kk <= n) of n <= 32 keys held one per lane (lanes
+// >= n hold nothing), and how many of the keys exceed it. Every lane of the
+// warp gets both.
+__device__ __forceinline__ void warp_select(uint32_t c, int n, uint32_t kk, uint32_t &tau, uint32_t &n_gt) {
+  const int lane = threadIdx.x & 31;
+  uint32_t gt = 0, ge = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t cj = __shfl_sync(0xffffffffu, c, j);
+    if (j < n) {
+      gt += cj > c;
+      ge += cj >= c;
+    }
+  }
+  const uint32_t hit = __ballot_sync(0xffffffffu, lane < n && gt < kk && kk <= ge);
+  const int src = __ffs(hit) - 1;
+  tau = __shfl_sync(0xffffffffu, c, src);
+  n_gt = __shfl_sync(0xffffffffu, gt, src);
+}
 
 // Exclusive prefix sum over the block (thread order) of one value per thread.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scan, int lane, int warp) {
@@ -164,10 +187,33 @@ __device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const floa
       const uint32_t bin = in_hi ? b_hi : b_lo;
       sh.kk = kk - (in_hi ? above : above + c_hi);
       sh.prefix = prefix | (bin << shift);
+      sh.bcnt = in_hi ? c_hi : c_lo;
+      sh.ncand = 0;
     }
     mask |= dmask << shift;
     top = shift;
     __syncthreads();
+    if (top > 0 && sh.bcnt <= kFew) {
+      // Few keys share the boundary bin: collect them and let one warp find
+      // the exact kk-th largest instead of further passes over every key.
+      const uint32_t pre = sh.prefix;
+      for (int j = threadIdx.x; j < n; j += kThreads) {
+        const uint32_t u = key_at<kCached>(keys, s, j) - kmin;
+        if ((u & mask) == pre) sh.cand[atomicAdd(&sh.ncand, 1u)] = u;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int nc = (int)sh.ncand;
+        uint32_t t, ngt;
+        warp_select(lane < nc ? sh.cand[lane] : 0u, nc, sh.kk, t, ngt);
+        if (lane == 0) {
+          sh.prefix = t;
+          sh.kk -= ngt;
+        }
+      }
+      __syncthreads();
+      break;
+    }
   }
   const uint32_t tau = sh.prefix + kmin, kk = sh.kk;
   // Ordered compaction: warp w scans the contiguous range [lo, hi).
@@ -230,11 +276,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int use_cach
 }
 
 struct ClusterShared {
-  uint32_t hist[2][kBins];  // pass p uses hist[p & 1]; peers read it after the pass's cluster barrier
+  alignas(16) uint32_t hist[2][kBins];  // pass p uses hist[p & 1]; peers read it after the pass's cluster barrier
   uint32_t scan[kWarps];
   uint32_t warp_gt[kWarps], warp_eq[kWarps];
   uint32_t lmin, lmax, cnt_gt, cnt_eq;  // this slice's key range and kept counts (read by peers)
-  uint32_t prefix, kk, kmin, krange, base_gt, base_eq;
+  uint32_t prefix, kk, kmin, krange, base_gt, base_eq, bcnt, ncand;
+  uint32_t cand[kFew];  // this slice's keys in the boundary bin (when the bin holds <= kFew in all)
 };
 
 // One query per cluster; CTA c of C selects over the slice
@@ -322,32 +369,87 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkArgs a) {
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
     }
     cluster_sync();  // every slice's histogram of this pass is complete
-    const int b_hi = kBins - 1 - 2 * threadIdx.x, b_lo = b_hi - 1;
-    uint32_t ph[8], pl[8];  // all remote loads in flight before the sums
+    // Threads 0..511 sum bins 4t'..4t'+3 (t' = 511 - t, descending order) of
+    // every slice with one 16-byte remote load per slice.
+    uint32_t cb[4] = {0u, 0u, 0u, 0u};
+    if (threadIdx.x < kBins / 4) {
+      const int b0 = kBins - 4 - 4 * threadIdx.x;
+      uint4 pv[8];
 #pragma unroll
-    for (uint32_t r = 0; r < 8; ++r)
-      if (r < C) {
-        ph[r] = ld_peer(&hist[b_hi], r);
-        pl[r] = ld_peer(&hist[b_lo], r);
-      }
-    uint32_t c_hi = 0, c_lo = 0;
+      for (uint32_t r = 0; r < 8; ++r)
+        if (r < C) pv[r] = ld_peer_u4(&hist[b0], r);
 #pragma unroll
-    for (uint32_t r = 0; r < 8; ++r)
-      if (r < C) {
-        c_hi += ph[r];
-        c_lo += pl[r];
-      }
-    const uint32_t above = block_excl_scan(c_hi + c_lo, cs.scan, lane, warp);
+      for (uint32_t r = 0; r < 8; ++r)
+        if (r < C) {
+          cb[0] += pv[r].w;  // bin b0 + 3 (highest first)
+          cb[1] += pv[r].z;
+          cb[2] += pv[r].y;
+          cb[3] += pv[r].x;
+        }
+    }
+    const uint32_t tot = cb[0] + cb[1] + cb[2] + cb[3];
+    const uint32_t above = block_excl_scan(tot, cs.scan, lane, warp);
     const uint32_t kk = cs.kk;
-    if (above < kk && kk <= above + c_hi + c_lo) {
-      const bool in_hi = kk <= above + c_hi;
-      const uint32_t bin = in_hi ? b_hi : b_lo;
-      cs.kk = kk - (in_hi ? above : above + c_hi);
+    if (threadIdx.x < kBins / 4 && above < kk && kk <= above + tot) {
+      uint32_t acc = above, bc = cb[0];
+      int i = 0;
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+        if (i == q && kk > acc + bc) {
+          acc += bc;
+          i = q + 1;
+          bc = cb[q + 1];
+        }
+      const uint32_t bin = (uint32_t)(kBins - 1 - 4 * threadIdx.x - i);
+      cs.kk = kk - acc;
       cs.prefix = prefix | (bin << shift);
+      cs.bcnt = bc;
+      cs.ncand = 0;
     }
     mask |= dmask << shift;
     top = shift;
     __syncthreads();
+    if (top > 0 && cs.bcnt <= kFew) {
+      // Few keys share the boundary bin across the cluster: every slice
+      // publishes its share, every CTA gathers all of them and one warp finds
+      // the exact kk-th largest (the same in every CTA).
+      const uint32_t pre = cs.prefix;
+      for (int j = threadIdx.x; j < len; j += kThreads) {
+        const uint32_t u = keys[j] - kmin;
+        if ((u & mask) == pre) cs.cand[atomicAdd(&cs.ncand, 1u)] = u;
+      }
+      cluster_sync();  // every slice's candidates are published
+      if (warp == 0) {
+        const uint32_t cnt = (uint32_t)lane < C ? ld_peer(&cs.ncand, lane) : 0u;
+        uint32_t inc = cnt;  // inclusive scan of the slices' counts
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const uint32_t excl = inc - cnt;
+        const int nc = (int)__shfl_sync(0xffffffffu, inc, 31);
+        // candidate number `lane` belongs to the last slice starting at or before it
+        uint32_t owner = 0, base = 0;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const uint32_t e_r = __shfl_sync(0xffffffffu, excl, r), c_r = __shfl_sync(0xffffffffu, cnt, r);
+          if ((uint32_t)r < C && c_r > 0 && e_r <= (uint32_t)lane) {
+            owner = (uint32_t)r;
+            base = e_r;
+          }
+        }
+        const uint32_t c = lane < nc ? ld_peer(&cs.cand[lane - base], owner) : 0u;
+        uint32_t t, ngt;
+        warp_select(c, nc, cs.kk, t, ngt);
+        if (lane == 0) {
+          cs.prefix = t;
+          cs.kk -= ngt;
+        }
+      }
+      __syncthreads();
+      break;
+    }
   }
   const uint32_t tau = cs.prefix + kmin, kk = cs.kk;
 
