@@ -8,9 +8,12 @@ from .csa_oracle import (  # noqa: F401
     as_f64,
     attend,
     compress,
+    e4m3_decode,
     hca_mqa,
     index_scores,
+    index_scores_fp8,
     index_topk,
+    index_topk_fp8,
     n_entries,
     n_visible,
     rms_norm,

@@ -46,6 +46,13 @@ the design notes):
 * R11 the sink is a per-head logit (not multiplied by the softmax scale) in
   the denominator, carrying a zero value vector.
 * R12 K = V: one row serves as key and value.
+* R18 FP8 indexer (the next row after the bf16 path): indexer keys and
+  queries are OCP FP8 E4M3 codes ("fmt": "e4m3", "quant_method": "fp8" in the
+  quantization_config of "deepseek-ai/DeepSeek-V4-Flash-0731", table "Config
+  changes"; the indexer is trained with quantization-aware training,
+  Architecture analysis INNOVATIONS section 1) with one positive fp32 scale
+  per row: per compressed entry for the keys, per (query, head) for the
+  queries; value = scale * decoded code. The score is R9 on those values.
 
 Pins (tests/test_oracle_pins.py) tie every function to something other than
 itself: closed forms, textbook/library special cases (torch rms_norm,
@@ -158,6 +165,38 @@ def index_scores(qi, wi, ki, n_vis: int) -> np.ndarray:
     ki = as_f64(ki)[:n_vis]
     dots = ki @ qi.T                     # [n_vis, Hi]
     return np.maximum(dots, 0.0) @ wi    # [n_vis]
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of OCP FP8 E4M3 codes (uint8), written from the format's
+    definition: bit 7 sign, bits 6-3 exponent (bias 7), bits 2-0 mantissa;
+    exponent 0 is subnormal, m/8 * 2^-6; otherwise (1 + m/8) * 2^(e - 7);
+    S.1111.111 is NaN and there are no infinities (the "fn" variant, largest
+    finite value 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    return np.where((c & 0x7F) == 0x7F, np.nan, sign * mag)
+
+
+def index_scores_fp8(qi8, sq, wi, ki8, sk, n_vis: int) -> np.ndarray:
+    """Indexer scores on FP8 inputs (reading R18), for one query:
+        qi[h] = sq[h] * e4m3(qi8[h]),  ki[j] = sk[j] * e4m3(ki8[j]),
+        s_j = sum_h wi[h] * max(0, qi[h] . ki[j]),  j < n_vis.
+    qi8: [Hi, Di] uint8 codes, sq: [Hi]; ki8: [>= n_vis, Di] uint8 codes,
+    sk: [>= n_vis]; wi: [Hi]."""
+    qi = e4m3_decode(qi8) * as_f64(sq)[:, None]
+    ki = e4m3_decode(np.asarray(ki8)[:n_vis]) * as_f64(sk)[:n_vis, None]
+    return index_scores(qi, wi, ki, n_vis)
+
+
+def index_topk_fp8(qi8, sq, wi, ki8, sk, p: int, k: int, win: int, stride: int):
+    """FP8 scores and the selected index list for one query at position p."""
+    nv = n_visible(p, win, stride)
+    s = index_scores_fp8(qi8, sq, wi, ki8, sk, nv)
+    return topk(s, k), s
 
 
 def topk(scores, k: int) -> np.ndarray:

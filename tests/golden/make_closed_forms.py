@@ -52,7 +52,25 @@ topk = {
               {"k": 8, "idx": [1, 2, 4, 0, 3, 5, -1, -1]}],
 }
 
+index_fp8 = {
+    "citation": "deepseek-ai/DeepSeek-V4-Flash-0731, table 'Config changes': quantization_config fmt e4m3, "
+                "quant_method fp8; DeepSeek-V4 Architecture Analysis, INNOVATIONS section 1 (indexer: "
+                "dot products with per-head importance weights, trained with QAT); OCP FP8 E4M3 format "
+                "(sign, 4-bit exponent with bias 7, 3-bit mantissa)",
+    "derivation": "Codes: 0x38 = 2^(7-7) = 1, 0x40 = 2^(8-7) = 2, 0xB8 = -1. Queries (Hi = 2, Di = 2): "
+                  "head 0 codes (0x38, 0x40) scale 2 -> (2, 4); head 1 codes (0x40, 0xB8) scale 1/2 -> "
+                  "(1, -1/2). Keys: entry 0 codes (0x38, 0x38) scale 1/2 -> (1/2, 1/2); entry 1 codes "
+                  "(0x40, 0x38) scale 1 -> (2, 1); entry 2 codes (0xB8, 0xB8) scale 1 -> (-1, -1). "
+                  "Dots: entry 0: head 0 1 + 2 = 3, head 1 1/2 - 1/4 = 1/4; entry 1: head 0 4 + 4 = 8, "
+                  "head 1 2 - 1/2 = 3/2; entry 2: head 0 -6, head 1 -1/2 (both ReLU 0). Weights (1, 1/4): "
+                  "s = (3 + 1/16, 8 + 3/8, 0).",
+    "qi8": [[0x38, 0x40], [0x40, 0xB8]], "sq": [2.0, 0.5], "wi": [1.0, 0.25],
+    "ki8": [[0x38, 0x38], [0x40, 0x38], [0xB8, 0xB8]], "sk": [0.5, 1.0, 1.0],
+    "scores": [3.0625, 8.375, 0.0],
+}
+
 for name, obj in (("compress_two_token.json", compress), ("attend_two_row_sink.json", attend),
+                  ("index_fp8_two_entries.json", index_fp8),
                   ("topk_ties.json", topk)):
     with open(os.path.join(HERE, name), "w") as f:
         json.dump(obj, f, indent=1)

@@ -180,6 +180,62 @@ def test_index_ignores_entries_past_the_visible_count():
     np.testing.assert_array_equal(a, O.index_scores(qi, w, ki2, 9))
 
 
+# ----------------------------------------------------------- FP8 indexer (R18)
+
+def test_e4m3_decode_matches_torch_float8_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))  # -0 is 0x80
+
+
+def test_e4m3_decode_values_from_the_format_definition():
+    cases = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 / 8 * 2.0 ** -6, 0x08: 2.0 ** -6, 0x38: 1.0, 0x3F: 1.875,
+             0x40: 2.0, 0x7E: 448.0, 0xB8: -1.0, 0xFE: -448.0}
+    got = O.e4m3_decode(list(cases))
+    assert np.array_equal(got, np.array(list(cases.values())))
+    assert np.isnan(O.e4m3_decode([0x7F, 0xFF])).all()
+
+
+def test_index_fp8_closed_form_two_entries():
+    g = _golden("index_fp8_two_entries.json")
+    got = O.index_scores_fp8(np.array(g["qi8"], np.uint8), g["sq"], g["wi"], np.array(g["ki8"], np.uint8),
+                             g["sk"], 3)
+    assert np.array_equal(got, np.array(g["scores"]))
+
+
+def test_index_fp8_scales_are_homogeneous():
+    Hi, Di, n = 5, 24, 40
+    qi8 = rng.integers(0, 0x7F, size=(Hi, Di), dtype=np.uint8) | (rng.integers(0, 2, (Hi, Di)) << 7).astype(np.uint8)
+    ki8 = rng.integers(0, 0x7F, size=(n, Di), dtype=np.uint8) | (rng.integers(0, 2, (n, Di)) << 7).astype(np.uint8)
+    sq, sk, wi = rng.uniform(0.1, 2, Hi), rng.uniform(0.1, 2, n), rng.uniform(0, 1, Hi)
+    base = O.index_scores_fp8(qi8, sq, wi, ki8, sk, n)
+    # one positive factor on every key scale scales every score by it
+    assert np.allclose(O.index_scores_fp8(qi8, sq, wi, ki8, 3.0 * sk, n), 3.0 * base, rtol=1e-13)
+    # per-entry key scales scale each entry's score
+    f = rng.uniform(0.5, 4, n)
+    assert np.allclose(O.index_scores_fp8(qi8, sq, wi, ki8, f * sk, n), f * base, rtol=1e-13)
+    # a query scale folds into the head weight (max(0, a x) = a max(0, x) for a > 0)
+    a = rng.uniform(0.5, 4, Hi)
+    assert np.allclose(O.index_scores_fp8(qi8, a * sq, wi, ki8, sk, n), O.index_scores_fp8(qi8, sq, a * wi, ki8, sk, n),
+                       rtol=1e-13)
+
+
+def test_index_fp8_unit_scales_single_head_is_a_plain_dot_of_decoded_codes():
+    # Hi = 1, w = 1, unit scales, codes of positive values only: s_j = qi . ki_j
+    # with qi, ki the values the codes stand for (torch's float8 conversion).
+    Di, n = 16, 12
+    qi8 = rng.integers(0x08, 0x7E, size=(1, Di), dtype=np.uint8)
+    ki8 = rng.integers(0x08, 0x7E, size=(n, Di), dtype=np.uint8)
+    tq = torch.from_numpy(qi8).view(torch.float8_e4m3fn).to(torch.float64)
+    tk = torch.from_numpy(ki8).view(torch.float8_e4m3fn).to(torch.float64)
+    got = O.index_scores_fp8(qi8, [1.0], [1.0], ki8, np.ones(n), n)
+    assert np.allclose(got, (tk @ tq[0]).numpy(), rtol=1e-15)
+
+
 def test_topk_closed_form_ties():
     g = _golden("topk_ties.json")
     for case in g["cases"]:
