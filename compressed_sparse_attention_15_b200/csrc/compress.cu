@@ -131,12 +131,15 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
   // positions pos0 + g, pos0 + g + G, ... with four rows of loads in flight per step
   for (int i0 = pos0 + g; i0 < pos1; i0 += 4 * G) {
     uint4 kvv[4], gv[4];
+    float4 ap0[4], ap1[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int i = i0 + u * G;
       if (i < pos1) {
         kvv[u] = __ldg(reinterpret_cast<const uint4 *>(kvj + (long long)i * a.D) + v);
         gv[u] = __ldg(reinterpret_cast<const uint4 *>(gj + (long long)i * a.D) + v);
+        ap0[u] = __ldg(reinterpret_cast<const float4 *>(a.ape + (size_t)i * a.D + 8 * v));
+        ap1[u] = __ldg(reinterpret_cast<const float4 *>(a.ape + (size_t)i * a.D + 8 * v + 4));
       }
     }
 #pragma unroll
@@ -146,8 +149,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
         float kf[8], gf[8];
         unpack8(kvv[u], kf);
         unpack8(gv[u], gf);
-        const float4 a0 = __ldg(reinterpret_cast<const float4 *>(a.ape + (size_t)i * a.D + 8 * v));
-        const float4 a1 = __ldg(reinterpret_cast<const float4 *>(a.ape + (size_t)i * a.D + 8 * v + 4));
+        const float4 a0 = ap0[u], a1 = ap1[u];
         const float ap[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -163,7 +165,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
       }
     }
   }
-  // merge the G partial states
+  // publish the G partial states
   float *sm = ws;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -173,29 +175,29 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
   }
   __syncthreads();
   float *red = ws + (size_t)G * 3 * 8 * nvec;  // [32]
-  float *blk = red + 32;                        // [3][8][nvec]: this block's merged state
-  float c[8];
-  float M8[8], L8[8], A8[8];
-  if (g == 0) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float M = -INFINITY;
-      for (int h = 0; h < G; ++h) M = fmaxf(M, sm[((h * 3 + 0) * 8 + k) * nvec + v]);
-      float L = 0.f, A = 0.f;
-      for (int h = 0; h < G; ++h) {
-        const float mh = sm[((h * 3 + 0) * 8 + k) * nvec + v];
-        const float w = mh == -INFINITY ? 0.f : exp2f(mh - M);
-        L += sm[((h * 3 + 1) * 8 + k) * nvec + v] * w;
-        A += sm[((h * 3 + 2) * 8 + k) * nvec + v] * w;
-      }
-      M8[k] = M;
-      L8[k] = L;
-      A8[k] = A;
-      if (C > 1) {
-        blk[(0 * 8 + k) * nvec + v] = M;
-        blk[(1 * 8 + k) * nvec + v] = L;
-        blk[(2 * 8 + k) * nvec + v] = A;
-      }
+  float *blk = red + 32;                        // [3][8][nvec]: this block's merged state, or [D] results
+  const int t = threadIdx.x;
+  // Merge the G states, one dimension per thread: dim 8 vv + kk at
+  // i = kk * nvec + vv (consecutive threads read consecutive words).
+  float ssl = 0.f;
+  for (int i = t; i < a.D; i += blockDim.x) {
+    float M = -INFINITY;
+    for (int h = 0; h < G; ++h) M = fmaxf(M, sm[(h * 3 + 0) * 8 * nvec + i]);
+    float L = 0.f, A = 0.f;
+    for (int h = 0; h < G; ++h) {
+      const float mh = sm[(h * 3 + 0) * 8 * nvec + i];
+      const float w = mh == -INFINITY ? 0.f : exp2f(mh - M);
+      L += sm[(h * 3 + 1) * 8 * nvec + i] * w;
+      A += sm[(h * 3 + 2) * 8 * nvec + i] * w;
+    }
+    if (C > 1) {
+      blk[0 * 8 * nvec + i] = M;
+      blk[1 * 8 * nvec + i] = L;
+      blk[2 * 8 * nvec + i] = A;
+    } else {
+      const float cd = A / L;
+      blk[i] = cd;
+      ssl += cd * cd;
     }
   }
   if (C > 1) {
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
     // the C block states of each, then the RMSNorm with the cluster's total
     // sum of squares (every remote load of a thread issued before use).
     cluster_sync();  // every block's state is published
-    const int per = a.D / (int)C, t = threadIdx.x;
+    const int per = a.D / (int)C;
     const bool mine = t < per;
     const int d = (int)crank * per + t;
     const int di = (d & 7) * nvec + (d >> 3);  // dim 8v + k lives at [.][k][v]
@@ -255,28 +257,21 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
     cluster_sync();  // no block leaves while a peer may still read its share
     return;
   }
-  if (g == 0) {
-    float ss = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      c[k] = A8[k] / L8[k];
-      ss += c[k] * c[k];
-    }
-    ss = warp_sum(ss);  // group 0 is whole warps (nvec is a multiple of 32)
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  }
+  const float ss = warp_sum(ssl);
+  if ((t & 31) == 0) red[t >> 5] = ss;  // at most 16 warps
   __syncthreads();
-  if (g == 0) {
+  if (t < nvec) {
     float tot = 0.f;
-    for (int w = 0; w < (nvec + 31) / 32; ++w) tot += red[w];
-    const float r = 1.0f / sqrtf(tot / (float)a.D + kRmsEps);
-    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * v));
-    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * v + 4));
+    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) tot += red[w];
+    const float rn = 1.0f / sqrtf(tot / (float)a.D + kRmsEps);
+    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * t));
+    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(a.norm_w + 8 * t + 4));
     const float nw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float c[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) c[k] = c[k] * r * nw[k];
+    for (int k = 0; k < 8; ++k) c[k] = blk[k * nvec + t] * rn * nw[k];
     bf16 *o = static_cast<bf16 *>(a.out) + b * a.out_ss + (long long)j * a.D;
-    reinterpret_cast<uint4 *>(o)[v] = pack8(c);
+    reinterpret_cast<uint4 *>(o)[t] = pack8(c);
   }
 }
 
