@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
 CSA_OK = 0
 CSA_DTYPE_F32 = 0
 CSA_DTYPE_BF16 = 1
+CSA_DTYPE_E4M3 = 2
 CSA_MAX_TOPK = 2048
 
 # Every function the header declares, with (restype, argtypes).
@@ -28,6 +29,8 @@ SIGNATURES = {
     "csa_index_topk_workspace_bytes": (_SZ, [_I, _I, _I]),
     "csa_index_topk": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "csa_index_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "csa_index_scores_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "csa_index_topk_fp8": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "csa_topk_workspace_bytes": (_SZ, [_I, _I, _I]),
     "csa_topk": (_I, [_P, _P, _I, _P, _I, _I, _P, _SZ, _P]),
     "csa_mqa_workspace_bytes": (_SZ, [_I, _I, _I, _I]),

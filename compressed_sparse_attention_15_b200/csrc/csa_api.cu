@@ -148,6 +148,48 @@ int csa_index_topk(const void *qi, const float *wi, const void *ki, const int32_
                              ws_bytes - kStatusBytes - sbytes));
 }
 
+static int check_scores_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                            const int32_t *n_cmp, int Q, int B, int Hi, int Di, int N_max, int q_per_seq) {
+  if (!qi8 || !sq || !wi || !ki8 || !sk || !n_cmp) return CSA_ERR_INVALID;
+  if (Q < 1 || B < 1 || Hi < 1 || Hi > 128 || Di < 1 || Di > 256 || N_max < 1 || N_max > (1 << 22) || q_per_seq < 1)
+    return CSA_ERR_INVALID;
+  if ((long long)B * q_per_seq < Q) return CSA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(sq) | reinterpret_cast<uintptr_t>(wi) | reinterpret_cast<uintptr_t>(sk) |
+       reinterpret_cast<uintptr_t>(n_cmp)) & 3)
+    return CSA_ERR_INVALID;
+  return CSA_OK;
+}
+
+int csa_index_scores_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                         const int32_t *n_cmp, float *scores, int Q, int B, int Hi, int Di, int N_max, int q_per_seq,
+                         void *ws, size_t ws_bytes, csa_stream_t stream) {
+  int rc = check_scores_fp8(qi8, sq, wi, ki8, sk, n_cmp, Q, B, Hi, Di, N_max, q_per_seq);
+  if (rc) return rc;
+  if (!scores || (reinterpret_cast<uintptr_t>(scores) & 3)) return CSA_ERR_INVALID;
+  if (!ws || !ws_aligned(ws) || ws_bytes < kStatusBytes) return CSA_ERR_WORKSPACE;
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  ScoreArgs a{qi8, wi, ki8, n_cmp, scores, Q, B, Hi, Di, N_max, q_per_seq, CSA_DTYPE_E4M3, status_of(ws), sq, sk};
+  return cuda_rc(launch_index_scores(a, (cudaStream_t)stream));
+}
+
+int csa_index_topk_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                       const int32_t *n_cmp, int k, int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max,
+                       int q_per_seq, void *ws, size_t ws_bytes, csa_stream_t stream) {
+  int rc = check_scores_fp8(qi8, sq, wi, ki8, sk, n_cmp, Q, B, Hi, Di, N_max, q_per_seq);
+  if (rc) return rc;
+  if (!out_idx || (reinterpret_cast<uintptr_t>(out_idx) & 3) || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (!ws || !ws_aligned(ws) || ws_bytes < csa_index_topk_workspace_bytes(Q, N_max, k)) return CSA_ERR_WORKSPACE;
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kStatusBytes);
+  ScoreArgs sa{qi8, wi, ki8, n_cmp, scores, Q, B, Hi, Di, N_max, q_per_seq, CSA_DTYPE_E4M3, status_of(ws), sq, sk};
+  cudaError_t e = launch_index_scores(sa, (cudaStream_t)stream);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  TopkArgs ta{scores, n_cmp, out_idx, Q, N_max, k, status_of(ws)};
+  const size_t sbytes = align256((size_t)Q * N_max * sizeof(float));
+  return cuda_rc(launch_topk(ta, (cudaStream_t)stream, static_cast<char *>(ws) + kStatusBytes + sbytes,
+                             ws_bytes - kStatusBytes - sbytes));
+}
+
 size_t csa_mqa_workspace_bytes(int Q, int H, int D, int rows_max) {
   if (Q < 1 || H < 1 || D < 1 || rows_max < 1) return kStatusBytes;
   return kStatusBytes + align256(mqa_partial_bytes(Q, H, D, rows_max));

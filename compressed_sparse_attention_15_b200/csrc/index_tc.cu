@@ -1,7 +1,12 @@
-// A2 on the tensor cores for the Flash indexer shape (64 heads x 128 dims,
-// bf16): s[q,j] = sum_h wi[q,h] * max(0, qi[q,h] . ki[b,j])
+// A2 on the tensor cores for the Flash indexer shape (64 heads x 128 dims):
+// s[q,j] = sum_h wi[q,h] * max(0, qi[q,h] . ki[b,j])
 // ("DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1, Indexer;
 // index_n_heads = 64, index_head_dim = 128 in the model card's config.json).
+// Two element formats: bf16 (kind::f16 MMAs, K = 16), and FP8 E4M3 codes
+// with per-row scales (kind::f8f6f4 MMAs, K = 32; quantization_config fmt
+// e4m3 of "deepseek-ai/DeepSeek-V4-Flash-0731"): with qi = sq * codes and
+// ki = sk * codes, s[q,j] = sk[j] * sum_h (wi[q,h] sq[q,h]) max(0, acc[h]),
+// acc being the code-by-code product (all scales positive).
 //
 // Layout of the contraction: the compressed keys are the MMA's M dimension
 // (128 entries per tile), the 64 heads its N, the 128 dims its K. One tile is
@@ -10,8 +15,9 @@
 // the weighted ReLU sum over heads is thread-local.
 //
 // Pipeline (persistent, one CTA per SM, 192 threads):
-//   warp 0      TMA producer: 32 KB key tiles into a 5-stage ring, and the
-//               query's 16 KB head block into one of two query slots;
+//   warp 0      TMA producer: key tiles (32 KB bf16 / 16 KB FP8) into a ring
+//               of 5 / 10 stages, and the query's head block (16 / 8 KB) into
+//               one of two query slots;
 //   warp 1      MMA issuer (one thread) and TMEM owner (2 accumulators);
 //   warps 2..5  epilogue: tcgen05.ld, ReLU, weighted sum, coalesced store.
 // Each CTA walks a contiguous range of the flat (query, tile) space. Every
@@ -28,43 +34,63 @@ namespace {
 
 constexpr int kHi = 64, kDi = 128;
 constexpr int kTileM = 128;
-constexpr int kStages = 5;
-constexpr uint32_t kTileBytes = kTileM * kDi * 2;  // 32 KB
-constexpr uint32_t kHalfTile = kTileBytes / 2;     // one 64-dim box
-constexpr uint32_t kQBytes = kHi * kDi * 2;        // 16 KB
-constexpr uint32_t kQHalf = kQBytes / 2;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 128;
 
+// Per element format: a tile is 128 entries x 128 dims; a TMA box carries 64
+// bf16 / 128 FP8 dims (128 bytes, the swizzle span) of 128 rows = 16 KB.
+template <bool kFp8>
+struct Fmt {
+  static constexpr int kElem = kFp8 ? 1 : 2;
+  static constexpr int kStages = kFp8 ? 10 : 5;
+  static constexpr int kBoxes = kFp8 ? 1 : 2;              // boxes per tile / per query block
+  static constexpr int kKSteps = kFp8 ? 4 : 8;             // MMAs per tile (32 bytes of K each)
+  static constexpr uint32_t kTileBytes = kTileM * kDi * kElem;
+  static constexpr uint32_t kBoxBytes = kTileBytes / kBoxes;  // 16 KB
+  static constexpr uint32_t kQBytes = kHi * kDi * kElem;
+  static constexpr uint32_t kQBox = kQBytes / kBoxes;         // 8 KB
+  static constexpr uint32_t kIdesc = kFp8 ? tc::idesc_e4m3(128, 64) : tc::idesc_bf16(128, 64, 0, 0);
+};
+
+template <int kStages>
 struct Bars {
   uint64_t full[kStages], empty[kStages], qfull[2], qempty[2], accfull[2], accempty[2], mma_done;
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + 2 * kQBytes + sizeof(Bars);
+template <bool kFp8>
+constexpr size_t smem_bytes() {
+  return 1024 + Fmt<kFp8>::kStages * Fmt<kFp8>::kTileBytes + 2 * Fmt<kFp8>::kQBytes + sizeof(Bars<Fmt<kFp8>::kStages>);
+}
 
 struct Tile {
-  int q, j0, n;
+  int q, j0;
 };
 
-__device__ __forceinline__ Tile tile_of(long long t, int tiles_per_q, const ScoreArgs &a) {
+// Tile t of the flat (query, 128-entry tile) space. Every tile of a query's
+// row is loaded and multiplied; entries at or past the query's visible count
+// are only masked in the epilogue, so that no role waits on that count
+// before its first copy or MMA.
+__device__ __forceinline__ Tile tile_of(long long t, int tiles_per_q) {
   Tile r;
   r.q = (int)(t / tiles_per_q);
   r.j0 = (int)(t - (long long)r.q * tiles_per_q) * kTileM;
-  int n = a.n_cmp[r.q];
-  r.n = n < 0 ? 0 : (n > a.N_max ? a.N_max : n);
   return r;
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
                            ScoreArgs a, int tiles_per_q, long long total, long long per_cta) {
+  using F = Fmt<kFp8>;
+  constexpr int kStages = F::kStages;
+  constexpr uint32_t kTileBytes = F::kTileBytes, kQBytes = F::kQBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stage_buf = smem;
   uint8_t *q_buf = smem + kStages * kTileBytes;
-  Bars *bars = reinterpret_cast<Bars *>(q_buf + 2 * kQBytes);
+  Bars<kStages> *bars = reinterpret_cast<Bars<kStages> *>(q_buf + 2 * kQBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long t_begin = (long long)blockIdx.x * per_cta;
   const long long t_end = min(total, t_begin + per_cta);
@@ -101,23 +127,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;  // per stage: a load was issued, with this parity
       for (long long t = t_begin; t < t_end && !*abort; ++t) {
-        const Tile tl = tile_of(t, tiles_per_q, a);
-        if (tl.j0 >= tl.n) continue;
+        const Tile tl = tile_of(t, tiles_per_q);
         if (tl.q != cur_q) {
           const int slot = nq & 1;
           const uint32_t qph = (nq >> 1) & 1;
           if (!tc::mbar_wait(&bars->qempty[slot], qph ^ 1, abort, a.status)) break;
           tc::mbar_arrive_expect_tx(&bars->qfull[slot], kQBytes);
-          tc::tma_load_2d(q_buf + slot * kQBytes, &tm_qi, 0, tl.q * kHi, &bars->qfull[slot]);
-          tc::tma_load_2d(q_buf + slot * kQBytes + kQHalf, &tm_qi, 64, tl.q * kHi, &bars->qfull[slot]);
+          for (int bx = 0; bx < F::kBoxes; ++bx)
+            tc::tma_load_2d(q_buf + slot * kQBytes + bx * F::kQBox, &tm_qi, bx * 64, tl.q * kHi, &bars->qfull[slot]);
           ++nq;
           cur_q = tl.q;
         }
         if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort, a.status)) break;
         tc::mbar_arrive_expect_tx(&bars->full[stage], kTileBytes);
         const int row = (tl.q / a.q_per_seq) * a.N_max + tl.j0;
-        tc::tma_load_2d(stage_buf + stage * kTileBytes, &tm_ki, 0, row, &bars->full[stage]);
-        tc::tma_load_2d(stage_buf + stage * kTileBytes + kHalfTile, &tm_ki, 64, row, &bars->full[stage]);
+        for (int bx = 0; bx < F::kBoxes; ++bx)
+          tc::tma_load_2d(stage_buf + stage * kTileBytes + bx * F::kBoxBytes, &tm_ki, bx * 64, row, &bars->full[stage]);
         issued_mask |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages) {
@@ -133,12 +158,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0, 0);
+      constexpr uint32_t idesc = F::kIdesc;
       int stage = 0, acc = 0, nq = 0, cur_q = -1, slot = 0;
       uint32_t phase = 0, accph = 0;
       for (long long t = t_begin; t < t_end && !*abort; ++t) {
-        const Tile tl = tile_of(t, tiles_per_q, a);
-        if (tl.j0 >= tl.n) continue;
+        const Tile tl = tile_of(t, tiles_per_q);
         if (tl.q != cur_q) {
           if (cur_q >= 0) tc::commit(&bars->qempty[slot]);  // old head block free once its MMAs finish
           slot = nq & 1;
@@ -152,10 +176,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_base = tc::smem_u32(stage_buf + stage * kTileBytes);
         const uint32_t b_base = tc::smem_u32(q_buf + slot * kQBytes);
 #pragma unroll
-        for (int kk = 0; kk < kDi / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(a_base + (kk >> 2) * kHalfTile + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sw128_desc(b_base + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem + acc * 64, ad, bd, idesc, kk > 0);
+        for (int kk = 0; kk < F::kKSteps; ++kk) {  // 32 bytes of K per MMA, 4 per 128-byte box
+          const uint64_t ad = tc::sw128_desc(a_base + (kk >> 2) * F::kBoxBytes + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(b_base + (kk >> 2) * F::kQBox + (kk & 3) * 32, 16, 1024);
+          if constexpr (kFp8)
+            tc::mma_f8(tmem + acc * 64, ad, bd, idesc, kk > 0);
+          else
+            tc::mma_bf16(tmem + acc * 64, ad, bd, idesc, kk > 0);
         }
         tc::commit(&bars->empty[stage]);
         tc::commit(&bars->accfull[acc]);
@@ -175,18 +202,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
-    int acc = 0, cur_q = -1;
+    int acc = 0, cur_q = -1, cur_n = 0;
     uint32_t accph = 0;
     float w[kHi];
     for (long long t = t_begin; t < t_end && !*abort; ++t) {
-      const Tile tl = tile_of(t, tiles_per_q, a);
-      if (tl.j0 >= tl.n) continue;
+      const Tile tl = tile_of(t, tiles_per_q);
       if (tl.q != cur_q) {
         const int raw = a.n_cmp[tl.q];
         if ((raw < 0 || raw > a.N_max) && row == 0) raise_status(a.status, CSA_STATUS_BAD_COUNT);
+        cur_n = raw < 0 ? 0 : (raw > a.N_max ? a.N_max : raw);
 #pragma unroll
         for (int h = 0; h < kHi; h += 4) {
-          const float4 v = __ldg(reinterpret_cast<const float4 *>(a.wi + (size_t)tl.q * kHi + h));
+          float4 v = __ldg(reinterpret_cast<const float4 *>(a.wi + (size_t)tl.q * kHi + h));
+          if constexpr (kFp8) {  // the query scales fold into the head weights
+            const float4 sc = __ldg(reinterpret_cast<const float4 *>(a.sq + (size_t)tl.q * kHi + h));
+            v.x *= sc.x;
+            v.y *= sc.y;
+            v.z *= sc.z;
+            v.w *= sc.w;
+          }
           w[h] = v.x;
           w[h + 1] = v.y;
           w[h + 2] = v.z;
@@ -210,7 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int h = 0; h < 32; ++h) s = fmaf(w[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s);
       const int j = tl.j0 + row;
-      if (j < tl.n) a.scores[(size_t)tl.q * a.N_max + j] = s;
+      if (j < cur_n) {
+        if constexpr (kFp8) s *= a.sk[(size_t)(tl.q / a.q_per_seq) * a.N_max + j];
+        a.scores[(size_t)tl.q * a.N_max + j] = s;
+      }
       if (++acc == 2) {
         acc = 0;
         accph ^= 1;
@@ -242,11 +279,15 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool *taken) {
   *taken = false;
-  if (a.dtype != CSA_DTYPE_BF16 || a.Hi != kHi || a.Di != kDi) return cudaSuccess;
+  const bool fp8 = a.dtype == CSA_DTYPE_E4M3;
+  if (!(fp8 || a.dtype == CSA_DTYPE_BF16) || a.Hi != kHi || a.Di != kDi) return cudaSuccess;
   if (!aligned16(a.qi) || !aligned16(a.ki) || (reinterpret_cast<uintptr_t>(a.wi) & 15)) return cudaSuccess;
+  if (fp8 && (reinterpret_cast<uintptr_t>(a.sq) & 15)) return cudaSuccess;
   CUtensorMap tm_ki, tm_qi;
-  if (!make_tmap_bf16_2d(&tm_ki, a.ki, kDi, (uint64_t)a.B * a.N_max, kDi * 2, 64, kTileM)) return cudaSuccess;
-  if (!make_tmap_bf16_2d(&tm_qi, a.qi, kDi, (uint64_t)a.Q * kHi, kDi * 2, 64, kHi)) return cudaSuccess;
+  const int esz = fp8 ? 1 : 2, box = fp8 ? 128 : 64;
+  auto mk = fp8 ? make_tmap_u8_2d : make_tmap_bf16_2d;
+  if (!mk(&tm_ki, a.ki, kDi, (uint64_t)a.B * a.N_max, kDi * esz, box, kTileM)) return cudaSuccess;
+  if (!mk(&tm_qi, a.qi, kDi, (uint64_t)a.Q * kHi, kDi * esz, box, kHi)) return cudaSuccess;
   const int tiles_per_q = (a.N_max + kTileM - 1) / kTileM;
   const long long total = (long long)a.Q * tiles_per_q;
   long long grid = num_sms_cached();
@@ -255,12 +296,18 @@ cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool
   grid = (total + per_cta - 1) / per_cta;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaFuncSetAttribute(index_scores_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes<false>());
+    cudaFuncSetAttribute(index_scores_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes<true>());
     attr_set = true;
   }
   *taken = true;
-  return launch_pdl(index_scores_tc_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tm_ki, tm_qi, a,
-                    tiles_per_q, total, per_cta);
+  if (fp8)
+    return launch_pdl(index_scores_tc_kernel<true>, dim3((unsigned)grid), dim3(kThreads), smem_bytes<true>(), stream,
+                      tm_ki, tm_qi, a, tiles_per_q, total, per_cta);
+  return launch_pdl(index_scores_tc_kernel<false>, dim3((unsigned)grid), dim3(kThreads), smem_bytes<false>(), stream,
+                    tm_ki, tm_qi, a, tiles_per_q, total, per_cta);
 }
 
 }  // namespace csa

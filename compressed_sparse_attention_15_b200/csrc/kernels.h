@@ -65,6 +65,8 @@ struct ScoreArgs {
   float *scores;
   int Q, B, Hi, Di, N_max, q_per_seq, dtype;
   uint32_t *status;
+  const float *sq = nullptr;  // CSA_DTYPE_E4M3: per (query, head) scale [Q, Hi]
+  const float *sk = nullptr;  // CSA_DTYPE_E4M3: per entry scale [B, N_max]
 };
 cudaError_t launch_index_scores(const ScoreArgs &a, cudaStream_t stream);
 

@@ -181,6 +181,54 @@ def topk(scores, n_cmp, k: int, out=None, ws: Workspace | None = None):
     return out
 
 
+# ------------------------------------------------------- A2 / A3 on FP8 inputs
+
+def _index_fp8_common(qi8, sq, wi, ki8, sk, n_cmp, q_per_seq):
+    _need(qi8, "qi8", dtype=torch.uint8)
+    dev = qi8.device
+    for t, nm in ((sq, "sq"), (wi, "wi"), (sk, "sk")):
+        _need(t, nm, dtype=torch.float32, device=dev)
+    _need(ki8, "ki8", dtype=torch.uint8, device=dev)
+    _need(n_cmp, "n_cmp", dtype=torch.int32, device=dev)
+    Q, Hi, Di = qi8.shape
+    B, N_max, Di2 = ki8.shape
+    if Di2 != Di or wi.shape != (Q, Hi) or sq.shape != (Q, Hi) or sk.shape != (B, N_max) or n_cmp.shape != (Q,):
+        raise ValueError("shape mismatch among qi8 [Q,Hi,Di], sq/wi [Q,Hi], ki8 [B,N,Di], sk [B,N], n_cmp [Q]")
+    if q_per_seq is None:
+        if Q % B:
+            raise ValueError("q_per_seq is required when B does not divide Q")
+        q_per_seq = Q // B
+    return Q, Hi, Di, B, N_max, q_per_seq
+
+
+def index_scores_fp8(qi8, sq, wi, ki8, sk, n_cmp, q_per_seq=None, out=None, ws: Workspace | None = None):
+    """Indexer scores on FP8 E4M3 codes with per-row scales
+    (csa_index_scores_fp8): fp32 [Q, N_max], entries past n_cmp untouched."""
+    Q, Hi, Di, B, N_max, qps = _index_fp8_common(qi8, sq, wi, ki8, sk, n_cmp, q_per_seq)
+    if out is None:
+        out = torch.full((Q, N_max), float("nan"), dtype=torch.float32, device=qi8.device)
+    _need(out, "out", dtype=torch.float32, device=qi8.device)
+    w = (ws or Workspace(qi8.device)).get(256)
+    rc = _lib.lib().csa_index_scores_fp8(_ptr(qi8), _ptr(sq), _ptr(wi), _ptr(ki8), _ptr(sk), _ptr(n_cmp), _ptr(out),
+                                         Q, B, Hi, Di, N_max, qps, _ptr(w), w.numel(), _stream(qi8.device))
+    _lib.check("csa_index_scores_fp8", rc)
+    return out
+
+
+def index_topk_fp8(qi8, sq, wi, ki8, sk, n_cmp, k: int, q_per_seq=None, out=None, ws: Workspace | None = None):
+    """FP8 indexer scores + top-k (csa_index_topk_fp8). Returns int32 [Q, k]."""
+    Q, Hi, Di, B, N_max, qps = _index_fp8_common(qi8, sq, wi, ki8, sk, n_cmp, q_per_seq)
+    if out is None:
+        out = torch.empty((Q, k), dtype=torch.int32, device=qi8.device)
+    _need(out, "out", dtype=torch.int32, device=qi8.device)
+    L = _lib.lib()
+    w = (ws or Workspace(qi8.device)).get(L.csa_index_topk_workspace_bytes(Q, N_max, k))
+    rc = L.csa_index_topk_fp8(_ptr(qi8), _ptr(sq), _ptr(wi), _ptr(ki8), _ptr(sk), _ptr(n_cmp), int(k), _ptr(out),
+                              Q, B, Hi, Di, N_max, qps, _ptr(w), w.numel(), _stream(qi8.device))
+    _lib.check("csa_index_topk_fp8", rc)
+    return out
+
+
 # ------------------------------------------------------------- A4 / A5
 
 def _mqa_common(q, kv_cmp, kv_win, win_end, sink, q_per_seq):

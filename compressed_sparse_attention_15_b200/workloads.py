@@ -17,8 +17,13 @@ Recipe (tensor id: distribution):
   9 gate   [B, T_c, D]    N(0,1)      gate logits of the tokens compressed in a step
  10 ape    [win, D]       N(0,0.1)    in-window position embedding (fp32)
  12 gate_raw [1, bulk_T, D] N(0,1)    gate logits of the bulk-compressed sequence
+ 13 qi8    [Q, Hi, Di]    E4M3 codes of 64 * N(0,1)   FP8 indexer queries (|64 x| <= 384 < 448)
+ 14 sq     [Q, Hi]        U(0,1)/64 + 1/256            their per-row scales (fp32)
+ 15 ki8    [B, N, Di]     E4M3 codes of 64 * N(0,1)   FP8 indexer keys
+ 16 sk     [B, N]         U(0,1)/64 + 1/256            their per-row scales (fp32)
     norm_w [D]            1.0         RMSNorm weight (fp32)
-bf16 tensors are drawn in fp32 and rounded once to bf16 (RNE).
+bf16 tensors are drawn in fp32 and rounded once to bf16 (RNE); FP8 codes are
+fp32 draws rounded once to E4M3 (RNE, torch's float8_e4m3fn conversion).
 """
 from __future__ import annotations
 
@@ -30,7 +35,8 @@ import torch
 from . import synth
 
 TID = {"q": 1, "kv_cmp": 2, "kv_win": 3, "qi": 4, "wi": 5, "ki": 6, "sink": 7, "kv_raw": 8, "gate": 9, "ape": 10,
-       "gate_raw": 12}
+       "gate_raw": 12, "qi8": 13, "sq": 14, "ki8": 15, "sk": 16}
+FP8_CODE_STD = 64.0  # FP8 code draws are FP8_CODE_STD * N(0,1), inside the E4M3 range (448)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -61,6 +67,7 @@ class Workload:
     # sequence 0's cache, reported apart from the decode step
     bulk_T: int = 0
     seed: int = 0
+    index_fmt: str = "bf16"  # indexer keys / queries: "bf16", or "e4m3" FP8 codes with per-row scales
 
     @property
     def scale(self) -> float:
@@ -109,6 +116,9 @@ WORKLOADS = {
         name="csa_decode_1m", dtype=torch.bfloat16, B=8, Q=8, H=64, D=512, Hi=64, Di=128, k=1024, W=128,
         N=262143, T_raw=128, pos0=1048575, raw0=1048448, T_c=8, c_src0=120, c_dst0=262142, bulk_T=1048576),
 }
+# The 64K decode batch with the FP8 (E4M3) indexer.
+WORKLOADS["csa_decode_64k_fp8"] = dataclasses.replace(WORKLOADS["csa_decode_64k"], name="csa_decode_64k_fp8",
+                                                      index_fmt="e4m3")
 
 
 def tensor_shape(w: Workload, name: str):
@@ -116,12 +126,19 @@ def tensor_shape(w: Workload, name: str):
         "q": (w.Q, w.H, w.D), "kv_cmp": (w.B, w.N, w.D), "kv_win": (w.B, w.T_raw, w.D),
         "qi": (w.Q, w.Hi, w.Di), "wi": (w.Q, w.Hi), "ki": (w.B, w.N, w.Di), "sink": (w.H,),
         "kv_raw": (1, w.bulk_T, w.D), "gate_raw": (1, w.bulk_T, w.D), "ape": (w.win, w.D),
-        "gate": (w.B, w.T_c, w.D),
+        "gate": (w.B, w.T_c, w.D), "qi8": (w.Q, w.Hi, w.Di), "sq": (w.Q, w.Hi), "ki8": (w.B, w.N, w.Di),
+        "sk": (w.B, w.N),
     }[name]
 
 
 def _dtype_of(w: Workload, name: str):
-    return torch.float32 if name in ("wi", "sink", "ape", "norm_w") else w.dtype
+    if name in ("qi8", "ki8"):
+        return torch.uint8
+    return torch.float32 if name in ("wi", "sink", "ape", "norm_w", "sq", "sk") else w.dtype
+
+
+def _codes(x: torch.Tensor) -> torch.Tensor:
+    return (x * FP8_CODE_STD).to(torch.float8_e4m3fn).view(torch.uint8)
 
 
 def make(w: Workload, name: str, device="cpu") -> torch.Tensor:
@@ -130,6 +147,10 @@ def make(w: Workload, name: str, device="cpu") -> torch.Tensor:
     dt = _dtype_of(w, name)
     if name == "wi":
         return synth.uniform(w.seed, TID[name], shape, dtype=dt, device=device)
+    if name in ("sq", "sk"):
+        return synth.uniform(w.seed, TID[name], shape, device=device) / 64 + 1.0 / 256
+    if name in ("qi8", "ki8"):
+        return _codes(synth.normal(w.seed, TID[name], shape, device=device))
     std = 0.1 if name == "ape" else 1.0
     return synth.normal(w.seed, TID[name], shape, std=std, dtype=dt, device=device)
 
@@ -138,6 +159,11 @@ def rows(w: Workload, name: str, flat_rows) -> torch.Tensor:
     """Rows of a tensor (index into its flattened leading dims), regenerated
     on the host in the workload dtype."""
     shape = tensor_shape(w, name)
+    if name in ("qi8", "ki8"):
+        return _codes(synth.normal_rows(w.seed, TID[name], shape, flat_rows))
+    if name in ("sq", "sk"):
+        flat = torch.as_tensor(flat_rows, dtype=torch.int64)
+        return synth.uniform_at(w.seed, TID[name], flat) / 64 + 1.0 / 256
     std = 0.1 if name == "ape" else 1.0
     return synth.normal_rows(w.seed, TID[name], shape, flat_rows, std=std, dtype=_dtype_of(w, name))
 

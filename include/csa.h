@@ -60,7 +60,7 @@ enum {
 };
 
 /* Element types of the dtype-typed tensors. */
-enum { CSA_DTYPE_F32 = 0, CSA_DTYPE_BF16 = 1 };
+enum { CSA_DTYPE_F32 = 0, CSA_DTYPE_BF16 = 1, CSA_DTYPE_E4M3 = 2 /* FP8 indexer entry points only */ };
 
 /* Bits of the workspace status word. */
 enum {
@@ -145,6 +145,38 @@ int csa_index_scores(const void *qi, const float *wi, const void *ki, const int3
 size_t csa_topk_workspace_bytes(int Q, int N_max, int k);
 int csa_topk(const float *scores, const int32_t *n_cmp, int k, int32_t *out_idx,
              int Q, int N_max, void *ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa_index_scores_fp8 / csa_index_topk_fp8 -- the indexer on FP8 inputs.
+ *
+ * "deepseek-ai/DeepSeek-V4-Flash-0731", table "Config changes": the model's
+ * quantization_config is fmt e4m3, quant_method fp8, dynamic activation
+ * scales; "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: the
+ * indexer is trained quantization-aware. Keys and queries arrive as OCP FP8
+ * E4M3 codes (1 byte: sign, 4-bit exponent with bias 7, 3-bit mantissa; NaN
+ * at S.1111.111, no infinities) with one positive fp32 scale per row:
+ *     qi[q,h,:] = sq[q,h] * e4m3(qi8[q,h,:]),  ki[b,j,:] = sk[b,j] * e4m3(ki8[b,j,:])
+ * and the scores and the selection are those of csa_index_scores /
+ * csa_index_topk on these values.
+ *
+ *   qi8 : [Q, Hi, Di] uint8 codes.   sq : [Q, Hi] float32 (> 0).
+ *   wi  : [Q, Hi] float32.
+ *   ki8 : [B, N_max, Di] uint8 codes. sk : [B, N_max] float32 (> 0).
+ *   n_cmp, k, out_idx, scores, q_per_seq, workspace: as for the bf16 calls
+ *   (csa_index_topk_workspace_bytes(Q, N_max, k) for the _topk call, 256
+ *   bytes for the _scores call).
+ * Limits: Hi <= 128, Di <= 256, N_max <= 2^22; the tensor-core path takes
+ * Hi = 64, Di = 128 with 16-byte aligned qi8 / ki8 / wi / sq.
+ * Returns CSA_ERR_INVALID (null pointer, bad shape, misaligned float or
+ * int32 array, k outside 1..CSA_MAX_TOPK) or CSA_ERR_WORKSPACE before any
+ * launch.
+ * ---------------------------------------------------------------------- */
+int csa_index_scores_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                         const int32_t *n_cmp, float *scores, int Q, int B, int Hi, int Di, int N_max, int q_per_seq,
+                         void *ws, size_t ws_bytes, csa_stream_t stream);
+int csa_index_topk_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                       const int32_t *n_cmp, int k, int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max,
+                       int q_per_seq, void *ws, size_t ws_bytes, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * csa_sparse_mqa -- MQA over the selected compressed entries, the sliding

@@ -76,6 +76,25 @@ def test_index_topk_rejects_bad_arguments(L):
     assert call(ws=ctypes.c_void_p(4096 + 128)) == 3  # not 256-byte aligned
 
 
+def test_index_fp8_rejects_bad_arguments(L):
+    ws_ok = L.csa_index_topk_workspace_bytes(4, 100, 16)
+
+    def topk(k=16, Hi=4, Di=16, q_per_seq=4, sq=P, sk=P, ws_bytes=ws_ok):
+        return L.csa_index_topk_fp8(P, sq, P, P, sk, P, k, P, 4, 1, Hi, Di, 100, q_per_seq, P, ws_bytes, NULL)
+    assert topk(k=0) == 1
+    assert topk(Hi=129) == 1
+    assert topk(Di=257) == 1
+    assert topk(q_per_seq=1) == 1
+    assert topk(sq=NULL) == 1 and topk(sk=NULL) == 1          # the scales are required
+    assert topk(sk=ctypes.c_void_p(4096 + 2)) == 1           # misaligned float array
+    assert topk(ws_bytes=ws_ok - 1) == 3
+
+    def scores(scores_ptr=P, ws_bytes=256):
+        return L.csa_index_scores_fp8(P, P, P, P, P, P, scores_ptr, 4, 1, 4, 16, 100, 4, P, ws_bytes, NULL)
+    assert scores(scores_ptr=NULL) == 1
+    assert scores(ws_bytes=255) == 3
+
+
 def test_mqa_rejects_bad_arguments(L):
     ws = L.csa_mqa_workspace_bytes(2, 4, 16, 32)
     assert ws >= 256

@@ -77,3 +77,17 @@ def test_device_bytes_equal_host_bytes(cuda_device):
         assert torch.equal(h.view(torch.int16 if dt == torch.bfloat16 else torch.int32),
                            d.view(torch.int16 if dt == torch.bfloat16 else torch.int32))
     assert torch.equal(synth.uniform(5, 4, (999,)), synth.uniform(5, 4, (999,), device=cuda_device).cpu())
+
+
+def test_fp8_code_draws_stay_inside_the_e4m3_range():
+    import numpy as np
+
+    import oracle as O
+    from compressed_sparse_attention_15_b200 import workloads as WL
+    w = WL.small(WL.WORKLOADS["csa_decode_64k"], Q=2, B=2, N=4096)
+    for name in ("qi8", "ki8"):
+        v = O.e4m3_decode(WL.make(w, name).numpy())
+        assert np.isfinite(v).all() and np.abs(v).max() <= 448
+    for name in ("sq", "sk"):
+        s = WL.make(w, name)
+        assert (s > 0).all()
