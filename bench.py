@@ -66,7 +66,11 @@ def algo_bytes(w: WL.Workload):
     b["compress"] = w.B * (2 * w.T_c * w.D * e + w.win * w.D * 4 + w.D * 4
                            + ((w.T_c - w.win) // w.stride + 1) * w.D * e)
     if w.mode == "csa":
-        b["index_scores"] = w.Q * (n_vis * w.Di * e + w.Hi * w.Di * e + w.Hi * 4)
+        if w.index_fmt == "e4m3":
+            # FP8 key rows + one fp32 scale per entry; FP8 query heads + scales + weights
+            b["index_scores"] = w.Q * (n_vis * (w.Di + 4) + w.Hi * w.Di + 2 * w.Hi * 4)
+        else:
+            b["index_scores"] = w.Q * (n_vis * w.Di * e + w.Hi * w.Di * e + w.Hi * 4)
         b["topk"] = w.Q * w.k * 4
         rows = w.k + w.W
         b["mqa"] = w.Q * (rows * w.D * e + 2 * w.H * w.D * e + w.k * 4 + w.H * 4)
@@ -103,10 +107,12 @@ class Step:
         self.w = w
         self.dev = device
         self.graph = graph
-        names = [n for n in self.PER_STEP if w.mode == "csa" or n not in ("qi", "wi")]
+        fp8 = w.index_fmt == "e4m3"
+        per_step = self.PER_STEP if not fp8 else ("q", "gate", "qi8", "sq", "wi")
+        names = [n for n in per_step if w.mode == "csa" or n not in ("qi", "wi", "qi8", "sq")]
         shapes = {n: WL.tensor_shape(w, n) for n in names}
         shapes["kv_new"] = (w.B, w.D)  # the newest raw token of each sequence
-        dts = {n: torch.float32 if n == "wi" else w.dtype for n in shapes}
+        dts = {n: (torch.float32 if n in ("wi", "sq") else torch.uint8 if n == "qi8" else w.dtype) for n in shapes}
         offs, total = {}, 0
         for n, shp in shapes.items():
             offs[n] = total
@@ -119,7 +125,8 @@ class Step:
         if caches is None:
             caches = {n: WL.make(w, n, device) for n in ("kv_cmp", "kv_win", "sink", "ape")}
             if w.mode == "csa":
-                caches["ki"] = WL.make(w, "ki", device)
+                for n in (("ki8", "sk") if fp8 else ("ki",)):
+                    caches[n] = WL.make(w, n, device)
         self.caches = caches
         self.t.update(caches)
         for n in names:
@@ -131,7 +138,8 @@ class Step:
             win_end=w.win_end().to(device), n_cmp=ops.visible_entries(w.positions(), w.win, w.stride).to(device),
             ape=t["ape"], norm_w=WL.norm_w(w, device), gate=t["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
             win=w.win, stride=w.stride, qi=t.get("qi"), wi=t.get("wi"), ki=t.get("ki"),
-            k=w.k if w.mode == "csa" else None, graph=graph)
+            k=w.k if w.mode == "csa" else None, graph=graph,
+            qi8=t.get("qi8"), sq=t.get("sq"), ki8=t.get("ki8"), sk=t.get("sk"))
         self.out = self.ds.out
         self._scores = None
 
@@ -151,8 +159,12 @@ class Step:
             self._scores = torch.empty((self.w.Q, self.w.N), dtype=torch.float32, device=self.dev)
             self._ws_s, self._ws_t = ops.Workspace(self.dev), ops.Workspace(self.dev)
         sc = self._scores
+        if ds.fp8:
+            score = lambda: ops.index_scores_fp8(ds.qi8, ds.sq, ds.wi, ds.ki8, ds.sk, ds.n_cmp, out=sc, ws=self._ws_s)
+        else:
+            score = lambda: ops.index_scores(ds.qi, ds.wi, ds.ki, ds.n_cmp, out=sc, ws=self._ws_s)
         return [("compress", ds.append),
-                ("index_scores", lambda: ops.index_scores(ds.qi, ds.wi, ds.ki, ds.n_cmp, out=sc, ws=self._ws_s)),
+                ("index_scores", score),
                 ("topk", lambda: ops.topk(sc, ds.n_cmp, ds.k, out=ds.idx, ws=self._ws_t)),
                 ("mqa", ds.attend)]
 
@@ -424,9 +436,10 @@ def e2e_ours(args, w: WL.Workload, step: Step, device):
 def oracle_step_inputs(w: WL.Workload):
     import numpy as np
 
-    host = {n: WL.make(w, n) for n in ("q", "sink", "ape", "qi", "wi") if n != "qi" or w.mode == "csa"}
+    host = {n: WL.make(w, n) for n in ("q", "sink", "ape")}
     if w.mode == "csa":
-        host["ki"] = WL.make(w, "ki")
+        names = ("qi8", "sq", "wi", "ki8", "sk") if w.index_fmt == "e4m3" else ("qi", "wi", "ki")
+        host.update({n: WL.make(w, n) for n in names})
     host["np"] = np
     return host
 
@@ -454,7 +467,11 @@ def time_oracle(w: WL.Workload, steps: int, budget_s: float):
             gate = WL.rows(w, "gate", b * w.T_c + torch.arange(w.T_c))
             t0 = time.perf_counter()
             new = O.round_to(O.compress(raw, gate, ape, np.ones(w.D), w.win, w.stride), "bf16")
-            if w.mode == "csa":
+            if w.mode == "csa" and w.index_fmt == "e4m3":
+                idx, _ = O.index_topk_fp8(host["qi8"][q].numpy(), host["sq"][q], host["wi"][q], host["ki8"][b].numpy(),
+                                          host["sk"][b], int(w.positions()[q]), w.k, w.win, w.stride)
+                sel = idx[idx >= 0]
+            elif w.mode == "csa":
                 idx, _ = O.index_topk(host["qi"][q], host["wi"][q], host["ki"][b], int(w.positions()[q]), w.k,
                                       w.win, w.stride)
                 sel = idx[idx >= 0]
@@ -480,7 +497,7 @@ def time_oracle(w: WL.Workload, steps: int, budget_s: float):
 
 def workload_config(w: WL.Workload):
     return {"workload": w.name, "batch": w.Q, "context": w.pos0 + 1, "heads": f"{w.H}q:1kv", "head_dim": w.D,
-            "indexer": f"{w.Hi}x{w.Di}" if w.mode == "csa" else None, "topk": w.k or None, "window": w.W,
+            "indexer": f"{w.Hi}x{w.Di} {w.index_fmt}" if w.mode == "csa" else None, "topk": w.k or None, "window": w.W,
             "compress": f"win {w.win} stride {w.stride}", "l2": "flushed before every timed step: 256 MB write, then 256 MB read (clean eviction)",
             "inputs": "seeded synthetic (counter-based generator), resident in HBM"}
 
@@ -549,7 +566,7 @@ def main():
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
-        for name in ("hca_decode_1m", "csa_decode_1m"):
+        for name in ("hca_decode_1m", "csa_decode_1m", "csa_decode_64k_fp8"):
             if name == w.name:
                 continue
             sw = WL.WORKLOADS[name]

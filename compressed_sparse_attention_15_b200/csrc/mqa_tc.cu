@@ -30,9 +30,10 @@
 // tiles, one CTA each, the CTAs of a query forming one thread-block cluster
 // (the largest size for which every query's cluster is resident at once).
 // With one split the CTA folds in the sink and writes the output; otherwise
-// every CTA stages its unnormalised (m, l, O) in shared memory and, after a
-// cluster barrier, merges 1/splits of the output from all of them through
-// distributed shared memory.
+// every CTA writes its unnormalised (m, l, O) to the workspace and, after a
+// cluster barrier, merges 1/splits of the output from all of them (L2 reads;
+// distributed-shared-memory reads of the same data measured several times
+// slower).
 // Roles (224 threads): warps 0-1 load (one per tile buffer), warp 2 issues
 // the MMAs and owns TMEM, warps 3-6 run the softmax and the epilogue. All
 // mbarrier waits are bounded; the softmax warps take every decision to stop
@@ -106,6 +107,19 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool v
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// L2 prefetch of one TMA box of `map` at (c0, c1) (out-of-range parts are
+// ignored, as for loads), and of `bytes` contiguous bytes at p (16-byte
+// aligned, a multiple of 16).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap *map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // 2^x on the SFU (relative error about 2^-22; flushes subnormal results to
 // zero, which only ever meets weights far below the bf16 resolution of P).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -144,6 +158,44 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// out[h][d..d+3] = sum_r coef[r][h] * O_r[h][d..d+3] for the 4-dim groups
+// [g0, g1) of one query (O_r: the split partials, [64][512] fp32 each). Each
+// thread takes kB groups per round, all kB * splits loads issued first.
+template <int kB, int kS>
+__device__ __forceinline__ void merge_groups(const float *po, const float *coef, bf16 *out, int splits, int g0,
+                                             int g1) {
+  for (int base = g0 + threadIdx.x; base < g1; base += kThreads * kB) {
+    float4 v[kB][kS];
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int gi = base + i * kThreads;
+      const int h = gi / (kD / 4), d = 4 * (gi % (kD / 4));
+#pragma unroll
+      for (int r = 0; r < kS; ++r)
+        if (r < splits && gi < g1) v[i][r] = __ldcg(reinterpret_cast<const float4 *>(po + ((size_t)r * kH + h) * kD + d));
+    }
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int gi = base + i * kThreads;
+      if (gi >= g1) break;
+      const int h = gi / (kD / 4), d = 4 * (gi % (kD / 4));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < kS; ++r)
+        if (r < splits) {
+          const float c = coef[r * kH + h];
+          acc.x = fmaf(c, v[i][r].x, acc.x);
+          acc.y = fmaf(c, v[i][r].y, acc.y);
+          acc.z = fmaf(c, v[i][r].z, acc.z);
+          acc.w = fmaf(c, v[i][r].w, acc.w);
+        }
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+      *reinterpret_cast<uint2 *>(out + h * kD + d) =
+          make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+    }
+  }
+}
+
 // tcgen05.ld of 16 TMEM lanes x 64 columns (16x256b shape, 8 repeats): for
 // column group c, thread t gets r[4c + e] = (lane t/4, column 8c + 2(t%4) + e)
 // and r[4c + 2 + e] = (lane t/4 + 8, same column), e = 0, 1.
@@ -162,7 +214,7 @@ __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)
 __global__ void __launch_bounds__(kThreads, 1)
     mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp_t,
                   const __grid_constant__ CUtensorMap tm_win_t, MqaArgs a, int splits, int tiles_per_split,
-                  float scale_log2) {
+                  float scale_log2, float *part_o, float *part_ml) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *kv = smem;                              // [2 tiles][8 boxes][64 rows][128 B]
@@ -220,34 +272,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::prefetch_tmap(&tm_cmp_t);
       tc::prefetch_tmap(&tm_win_t);
     }
+    // Source row of list position r (null: padding or an unused slot).
+    auto src_row = [&](int r) -> const bf16 * {
+      if (r < L.nsel) {
+        int j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
+        if (j < -1 || j >= a.N_max) {
+          raise_status(a.status, CSA_STATUS_BAD_INDEX);
+          j = -1;
+        }
+        return j >= 0 ? static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + j) * kD : nullptr;
+      }
+      if (r >= L.nsel4 && r < L.R)
+        return static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + L.wlo + (r - L.nsel4)) * kD;
+      return nullptr;
+    };
+    // A tile is one contiguous run when it lies in the window part, or in the
+    // compressed part of a dense (HCA) row list.
+    auto is_run = [&](int r0, bool &win_run) {
+      win_run = r0 >= L.nsel4;
+      return win_run || (!a.idx && r0 + kRows <= L.nsel4);
+    };
+    // Bring tile li into L2 ahead of its load, which can only start once the
+    // tile buffer is free: the load then waits on L2, not on HBM.
+    auto prefetch_l2 = [&](int li) {
+      if (li >= ntiles) return;
+      const int r0 = (t0 + li) * kRows;
+      bool win_run;
+      if (is_run(r0, win_run)) {
+        if (lane == 0) {
+          const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
+          for (int bx = 0; bx < 8; ++bx) tma_prefetch_l2(win_run ? &tm_win_t : &tm_cmp_t, 64 * bx, row);
+        }
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          if (const bf16 *p = src_row(r0 + lane + 32 * hh)) bulk_prefetch_l2(p, kD * 2);
+      }
+    };
     int last = -1;
     for (int li = g; li < ntiles; li += 2) {
       const int r0 = (t0 + li) * kRows;
-      // A tile is one contiguous run when it lies in the window part, or in
-      // the compressed part of a dense (HCA) row list.
-      const bool win_run = r0 >= L.nsel4;
-      const bool cmp_run = !a.idx && r0 + kRows <= L.nsel4;
+      bool win_run;
+      const bool run = is_run(r0, win_run);
       __syncwarp();  // the previous tile's copies have read rowp[g]
-      if (!win_run && !cmp_run) {
+      if (!run) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int r = r0 + lane + 32 * hh;
-          const bf16 *p = nullptr;
-          if (r < L.nsel) {
-            int j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
-            if (j < -1 || j >= a.N_max) {
-              raise_status(a.status, CSA_STATUS_BAD_INDEX);
-              j = -1;
-            }
-            if (j >= 0) p = static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + j) * kD;
-          } else if (r >= L.nsel4 && r < L.R) {
-            p = static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + L.wlo + (r - L.nsel4)) * kD;
-          }
-          sm->rowp[g][lane + 32 * hh] = p;
-        }
+        for (int hh = 0; hh < 2; ++hh) sm->rowp[g][lane + 32 * hh] = src_row(r0 + lane + 32 * hh);
       }
+      if (li == g) prefetch_l2(li + 2);  // later tiles are prefetched one round ahead, below
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status))) break;
-      if (win_run || cmp_run) {
+      if (run) {
         if (lane == 0) {
           tc::mbar_arrive_expect_tx(&sm->kv_full[g], kTileBytes);
           const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
@@ -266,6 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t dst = buf_base + (c16 >> 3) * kBoxBytes + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
           cp_async16(dst, src ? src + c16 * 8 : static_cast<const bf16 *>(a.kv_win), src != nullptr);
         }
+      }
+      if (li > g) prefetch_l2(li + 2);
+      if (!run) {
         cp_async_wait_all();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc::mbar_arrive(&sm->kv_full[g]);
@@ -537,10 +614,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_sync(1, 128);
     const int orow = quarter * 32 + lane;  // O^T row (dims) within a 128-dim chunk
     if (splits > 1) {
-      // Stage this split's unnormalised O (fp32, [64 heads][512 dims]) in
-      // the tile buffers, which no copy or MMA touches any more, for the
-      // cluster merge below; its (mref, lsum) stay in shared memory.
-      float *ostage = reinterpret_cast<float *>(kv);
+      // This split's unnormalised O (fp32, [64 heads][512 dims]) and its
+      // (mref, lsum) go to the workspace, for the cluster merge below.
+      const size_t pidx = (size_t)qq * splits + split;
+      if (leader) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int h = 2 * lane + i;
+          part_ml[(pidx * 2) * kH + h] = sm->mref[h];
+          part_ml[(pidx * 2 + 1) * kH + h] = sm->lsum[h];
+        }
+      }
+      float *po = part_o + pidx * (size_t)kH * kD;
 #pragma unroll 1
       for (int m = 0; m < 4; ++m) {
         const int d = 128 * m + orow;
@@ -555,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 32; ++c) v[c] = 0u;
           }
 #pragma unroll
-          for (int c = 0; c < 32; ++c) ostage[(32 * half + c) * kD + d] = __uint_as_float(v[c]);
+          for (int c = 0; c < 32; ++c) po[(size_t)(32 * half + c) * kD + d] = __uint_as_float(v[c]);
         }
       }
     } else if (ok) {
@@ -594,20 +679,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tmem_dealloc(tmem, kTmemCols);
   }
   if (splits > 1) {
-    // The splits of query qq are the blocks of one cluster (rank = split).
-    // Merge with the sink, every block taking 1/splits of the outputs:
+    // The splits of query qq are the blocks of one cluster (rank = split):
+    // the cluster barrier orders every split's partials (global memory) before
+    // the merge. Every block merges 1/splits of the outputs with the sink:
     //   M = max(max_s m_s, sink), L = sum_s l_s 2^(m_s - M) + 2^(sink - M),
     //   out = sum_s O_s 2^(m_s - M) / L   (m and sink in log2 units).
-    cluster_sync();  // every split's O, mref and lsum are staged
+    cluster_sync();
     float *coef = reinterpret_cast<float *>(ps);  // [splits][64]: 2^(m_s - M) / L
+    const float *pml = part_ml + (size_t)qq * splits * 2 * kH;
     if (threadIdx.x < kH) {
       const int h = threadIdx.x;
       float mr[kMaxSplits], lr[kMaxSplits];
 #pragma unroll
       for (int r = 0; r < kMaxSplits; ++r)
         if (r < splits) {
-          mr[r] = ld_peer_f(&sm->mref[h], r);
-          lr[r] = ld_peer_f(&sm->lsum[h], r);
+          mr[r] = pml[(2 * r) * kH + h];
+          lr[r] = pml[(2 * r + 1) * kH + h];
         }
       const float sk = a.sink[h] * kLog2e;
       float M = sk;
@@ -627,31 +714,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (r < splits) coef[r * kH + h] = w[r] * inv;
     }
     __syncthreads();
-    const float *ostage = reinterpret_cast<const float *>(kv);
+    const float *po = part_o + (size_t)qq * splits * kH * kD;
     bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qq * kH * kD;
     constexpr int kGroups = kH * kD / 4;  // 4-dim groups of the output
-    const int g1 = (split + 1) * kGroups / splits;
-    for (int gi = split * kGroups / splits + threadIdx.x; gi < g1; gi += kThreads) {
-      const int h = gi / (kD / 4), d = 4 * (gi % (kD / 4));
-      float4 v[kMaxSplits];
-#pragma unroll
-      for (int r = 0; r < kMaxSplits; ++r)
-        if (r < splits) v[r] = ld_peer_f4(ostage + h * kD + d, r);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int r = 0; r < kMaxSplits; ++r)
-        if (r < splits) {
-          const float c = coef[r * kH + h];
-          acc.x = fmaf(c, v[r].x, acc.x);
-          acc.y = fmaf(c, v[r].y, acc.y);
-          acc.z = fmaf(c, v[r].z, acc.z);
-          acc.w = fmaf(c, v[r].w, acc.w);
-        }
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-      *reinterpret_cast<uint2 *>(out + h * kD + d) =
-          make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-    }
-    cluster_sync();  // no block leaves while a peer may still read its staging buffer
+    const int g0 = split * kGroups / splits, g1 = (split + 1) * kGroups / splits;
+    // Batches of groups with every partial load in flight before the sums
+    // (a group at a time waits out one L2 latency per group).
+    if (splits <= 4)
+      merge_groups<4, 4>(po, coef, out, splits, g0, g1);
+    else if (splits <= 8)
+      merge_groups<2, 8>(po, coef, out, splits, g0, g1);
+    else
+      merge_groups<1, kMaxSplits>(po, coef, out, splits, g0, g1);
   }
 }
 
@@ -735,9 +809,17 @@ int rows_max_of(const MqaArgs &a) { return (((a.idx ? a.k : a.N_max) + 3) & ~3) 
 
 }  // namespace
 
-// The splits of a query merge through distributed shared memory: no
-// workspace beyond the status word.
-size_t mqa_tc_partial_bytes(int, int, int, int) { return 0; }
+// Upper bound on the split partials for any row list of at most rows_max
+// rows (+3 rows of padding): Q x min(tiles, SMs / Q, 16) x 64 x (512 + 2) fp32.
+size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
+  if (H != kH || D != kD || Q < 1) return 0;
+  const int tiles = (rows_max + 3 + kRows - 1) / kRows;
+  int s = num_sms_cached() / Q;
+  s = s > kMaxSplits ? kMaxSplits : s;
+  s = s < 1 ? 1 : (s > tiles ? tiles : s);
+  if (s <= 1) return 0;
+  return (size_t)Q * s * kH * (kD + 2) * sizeof(float);
+}
 
 cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   *taken = false;
@@ -750,10 +832,14 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
       !make_tmap_bf16_2d(&tm_cmp_t, a.kv_cmp, kD, cmp_rows, kD * 2, 64, kRows) ||
       !make_tmap_bf16_2d(&tm_win_t, a.kv_win, kD, win_rows, kD * 2, 64, kRows))
     return cudaSuccess;
+  const size_t need = splits > 1 ? (size_t)a.Q * splits * kH * (kD + 2) * sizeof(float) : 0;
+  if (need > a.partial_bytes) return cudaSuccess;  // cannot happen with the documented workspace size
+  float *part_o = static_cast<float *>(a.partials);
+  float *part_ml = part_o + (size_t)a.Q * splits * kH * kD;
   set_kernel_attributes();
   *taken = true;
   return launch_pdl_cluster(mqa_tc_kernel, dim3(splits, a.Q), dim3(kThreads), kSmemBytes, stream, (unsigned)splits,
-                            tm_q, tm_cmp_t, tm_win_t, a, splits, tps, a.scale * kLog2e);
+                            tm_q, tm_cmp_t, tm_win_t, a, splits, tps, a.scale * kLog2e, part_o, part_ml);
 }
 
 }  // namespace csa

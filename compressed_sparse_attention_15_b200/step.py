@@ -6,7 +6,7 @@ The step over device-resident caches is:
      (csa_compress; CSA every 4 tokens, HCA every 128) -- on a forked stream,
      concurrently with 2 when the layer is CSA;
   2. CSA only: score every visible compressed entry and select the top-k
-     (csa_index_topk);
+     (csa_index_topk, or csa_index_topk_fp8 with FP8 indexer inputs);
   3. attend over the selected (CSA) or all visible (HCA) entries + the
      sliding window + the per-head sink (csa_sparse_mqa / hca_mqa).
 The library never allocates or synchronises, so the launches are captured
@@ -23,8 +23,10 @@ from . import ops
 class DecodeStep:
     def __init__(self, *, q, kv_cmp, kv_win, sink, scale: float, win_len: int, win_end, n_cmp,
                  ape, norm_w, gate, append_src0: int, append_dst0: int, win: int, stride: int,
-                 qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True):
-        self.csa = qi is not None
+                 qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True,
+                 qi8=None, sq=None, ki8=None, sk=None):
+        self.fp8 = qi8 is not None
+        self.csa = qi is not None or self.fp8
         self.q, self.kv_cmp, self.kv_win, self.sink = q, kv_cmp, kv_win, sink
         self.scale, self.win_len, self.win_end, self.n_cmp = float(scale), int(win_len), win_end, n_cmp
         self.ape, self.norm_w, self.gate = ape, norm_w, gate
@@ -34,6 +36,7 @@ class DecodeStep:
         self.kv_src = kv_win[:, append_src0:append_src0 + T_c]
         self.cmp_dst = kv_cmp[:, append_dst0:append_dst0 + n_new]
         self.qi, self.wi, self.ki, self.k = qi, wi, ki, k
+        self.qi8, self.sq, self.ki8, self.sk = qi8, sq, ki8, sk
         dev = q.device
         self.out = out if out is not None else torch.empty_like(q)
         self.idx = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev) if self.csa else None
@@ -54,7 +57,11 @@ class DecodeStep:
         ops.compress(self.kv_src, self.gate, self.ape, self.norm_w, self.win, self.stride, out=self.cmp_dst)
 
     def select(self):
-        ops.index_topk(self.qi, self.wi, self.ki, self.n_cmp, self.k, out=self.idx, ws=self.ws_index)
+        if self.fp8:
+            ops.index_topk_fp8(self.qi8, self.sq, self.wi, self.ki8, self.sk, self.n_cmp, self.k, out=self.idx,
+                               ws=self.ws_index)
+        else:
+            ops.index_topk(self.qi, self.wi, self.ki, self.n_cmp, self.k, out=self.idx, ws=self.ws_index)
 
     def attend(self):
         if self.csa:

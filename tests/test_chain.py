@@ -7,6 +7,7 @@ import torch
 
 import oracle as O
 from compressed_sparse_attention_15_b200 import ops, workloads as WL
+from compressed_sparse_attention_15_b200.step import DecodeStep
 from helpers import assert_close, check_topk_set
 
 pytestmark = pytest.mark.gpu
@@ -72,6 +73,47 @@ def test_csa_decode_step_chain(cuda_device):
         qh = WL.rows(w, "q", q * w.H + torch.arange(w.H))
         ref = O.attend(qh, np.concatenate([rows_c, rows_w]), sink, w.scale)[0]
         assert_close(out[q], ref, torch.bfloat16, f"decode chain q={q}")
+
+
+def test_fp8_indexer_decode_step_chain(cuda_device):
+    # The 64 K decode step with the FP8 indexer, run as one graph replay of
+    # DecodeStep (append, FP8 select, attend); checked against the oracle chain
+    # on four queries.
+    w = WL.WORKLOADS["csa_decode_64k_fp8"]
+    names = ("q", "kv_cmp", "kv_win", "sink", "gate", "ape", "qi8", "sq", "wi", "ki8", "sk")
+    d = {t: WL.make(w, t, cuda_device) for t in names}
+    ds = DecodeStep(q=d["q"], kv_cmp=d["kv_cmp"], kv_win=d["kv_win"], sink=d["sink"], scale=w.scale, win_len=w.W,
+                    win_end=w.win_end().to(cuda_device),
+                    n_cmp=ops.visible_entries(w.positions(), w.win, w.stride).to(cuda_device), ape=d["ape"],
+                    norm_w=WL.norm_w(w, cuda_device), gate=d["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
+                    win=w.win, stride=w.stride, qi8=d["qi8"], sq=d["sq"], wi=d["wi"], ki8=d["ki8"], sk=d["sk"],
+                    k=w.k)
+    out = ds.run()
+    torch.cuda.synchronize()
+    assert ds.status() == 0
+    idx_h = ds.idx.cpu().numpy()
+    ape, sink = WL.make(w, "ape"), WL.make(w, "sink")
+    qi8, sq, wi = (WL.make(w, t) for t in ("qi8", "sq", "wi"))
+    compared = 0
+    for q in (0, 9, 18, 27):
+        b = q
+        rows = torch.arange(b * w.N, (b + 1) * w.N)
+        ref_s = O.index_scores_fp8(qi8[q].numpy(), sq[q], wi[q], WL.rows(w, "ki8", rows).numpy(),
+                                   WL.rows(w, "sk", rows), w.N)
+        ref_idx = O.topk(ref_s, w.k)
+        if check_topk_set(idx_h[q], ref_idx, ref_s, w.k, w.N):
+            continue
+        sel = ref_idx[ref_idx >= 0]
+        rows_c = O.round_to(WL.rows(w, "kv_cmp", b * w.N + torch.as_tensor(sel)), "bf16")
+        raw = WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.c_src0, w.c_src0 + w.T_c))
+        gate = WL.rows(w, "gate", b * w.T_c + torch.arange(w.T_c))
+        rows_c[sel == w.c_dst0] = O.round_to(O.compress(raw, gate, ape, np.ones(w.D), w.win, w.stride), "bf16")[0]
+        rows_w = O.as_f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.T_raw)))
+        qh = WL.rows(w, "q", q * w.H + torch.arange(w.H))
+        ref = O.attend(qh, np.concatenate([rows_c, rows_w]), sink, w.scale)[0]
+        assert_close(out[q], ref, torch.bfloat16, f"FP8 decode chain q={q}")
+        compared += 1
+    assert compared >= 3
 
 
 def test_status_word_flags_bad_device_values(cuda_device):
