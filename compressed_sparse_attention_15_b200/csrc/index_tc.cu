@@ -15,9 +15,9 @@
 // the weighted ReLU sum over heads is thread-local.
 //
 // Pipeline (persistent, one CTA per SM, 192 threads):
-//   warp 0      TMA producer: key tiles (32 KB bf16 / 16 KB FP8) into a ring
-//               of 5 / 10 stages, and the query's head block (16 / 8 KB) into
-//               one of two query slots;
+//   warp 0      TMA producer: 32 KB key tiles (128 bf16 / 256 FP8 entries)
+//               into a 5-stage ring, and the query's head block (16 / 8 KB)
+//               into one of two query slots;
 //   warp 1      MMA issuer (one thread) and TMEM owner (2 accumulators);
 //   warps 2..5  epilogue: tcgen05.ld, ReLU, weighted sum, coalesced store.
 // Each CTA walks a contiguous range of the flat (query, tile) space. Every
@@ -33,22 +33,27 @@ namespace csa {
 namespace {
 
 constexpr int kHi = 64, kDi = 128;
-constexpr int kTileM = 128;
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 128;
 
-// Per element format: a tile is 128 entries x 128 dims; a TMA box carries 64
-// bf16 / 128 FP8 dims (128 bytes, the swizzle span) of 128 rows = 16 KB.
+// Per element format: a stage is 32 KB of keys in two TMA boxes of 128 rows x
+// 128 bytes (the swizzle span): bf16 tiles are 128 entries split along the
+// dims (64 + 64), E4M3 tiles are 256 entries split along the rows (128 +
+// 128, one MMA row block each), so both formats pay the per-tile costs
+// (barriers, MMA issue, epilogue hand-off) once per 32 KB.
 template <bool kFp8>
 struct Fmt {
   static constexpr int kElem = kFp8 ? 1 : 2;
-  static constexpr int kStages = kFp8 ? 10 : 5;
-  static constexpr int kBoxes = kFp8 ? 1 : 2;              // boxes per tile / per query block
-  static constexpr int kKSteps = kFp8 ? 4 : 8;             // MMAs per tile (32 bytes of K each)
-  static constexpr uint32_t kTileBytes = kTileM * kDi * kElem;
-  static constexpr uint32_t kBoxBytes = kTileBytes / kBoxes;  // 16 KB
+  static constexpr int kStages = 5;
+  static constexpr int kSub = kFp8 ? 2 : 1;                // 128-row MMA blocks per tile
+  static constexpr int kTileRows = 128 * kSub;
+  static constexpr int kKBoxes = kFp8 ? 1 : 2;             // 128-byte K boxes per row (query block too)
+  static constexpr int kKSteps = kFp8 ? 4 : 8;             // MMAs per row block (32 bytes of K each)
+  static constexpr uint32_t kBoxBytes = 128 * 128;         // 16 KB
+  static constexpr uint32_t kTileBytes = 2 * kBoxBytes;    // 32 KB
   static constexpr uint32_t kQBytes = kHi * kDi * kElem;
-  static constexpr uint32_t kQBox = kQBytes / kBoxes;         // 8 KB
+  static constexpr uint32_t kQBox = kQBytes / kKBoxes;      // 8 KB
+  static constexpr uint32_t kAccCols = 64 * kSub;          // TMEM columns of one accumulator
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static constexpr uint32_t kIdesc = kFp8 ? tc::idesc_e4m3(128, 64) : tc::idesc_bf16(128, 64, 0, 0);
 };
 
@@ -72,10 +77,10 @@ struct Tile {
 // row is loaded and multiplied; entries at or past the query's visible count
 // are only masked in the epilogue, so that no role waits on that count
 // before its first copy or MMA.
-__device__ __forceinline__ Tile tile_of(long long t, int tiles_per_q) {
+__device__ __forceinline__ Tile tile_of(long long t, int tiles_per_q, int tile_rows) {
   Tile r;
   r.q = (int)(t / tiles_per_q);
-  r.j0 = (int)(t - (long long)r.q * tiles_per_q) * kTileM;
+  r.j0 = (int)(t - (long long)r.q * tiles_per_q) * tile_rows;
   return r;
 }
 
@@ -110,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
+  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, F::kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -127,13 +132,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;  // per stage: a load was issued, with this parity
       for (long long t = t_begin; t < t_end && !*abort; ++t) {
-        const Tile tl = tile_of(t, tiles_per_q);
+        const Tile tl = tile_of(t, tiles_per_q, F::kTileRows);
         if (tl.q != cur_q) {
           const int slot = nq & 1;
           const uint32_t qph = (nq >> 1) & 1;
           if (!tc::mbar_wait(&bars->qempty[slot], qph ^ 1, abort, a.status)) break;
           tc::mbar_arrive_expect_tx(&bars->qfull[slot], kQBytes);
-          for (int bx = 0; bx < F::kBoxes; ++bx)
+          for (int bx = 0; bx < F::kKBoxes; ++bx)
             tc::tma_load_2d(q_buf + slot * kQBytes + bx * F::kQBox, &tm_qi, bx * 64, tl.q * kHi, &bars->qfull[slot]);
           ++nq;
           cur_q = tl.q;
@@ -141,8 +146,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort, a.status)) break;
         tc::mbar_arrive_expect_tx(&bars->full[stage], kTileBytes);
         const int row = (tl.q / a.q_per_seq) * a.N_max + tl.j0;
-        for (int bx = 0; bx < F::kBoxes; ++bx)
-          tc::tma_load_2d(stage_buf + stage * kTileBytes + bx * F::kBoxBytes, &tm_ki, bx * 64, row, &bars->full[stage]);
+        for (int bx = 0; bx < 2; ++bx)  // bf16: dims 64 bx.., E4M3: rows 128 bx..
+          tc::tma_load_2d(stage_buf + stage * kTileBytes + bx * F::kBoxBytes, &tm_ki, kFp8 ? 0 : 64 * bx,
+                          kFp8 ? row + 128 * bx : row, &bars->full[stage]);
         issued_mask |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages) {
@@ -162,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, acc = 0, nq = 0, cur_q = -1, slot = 0;
       uint32_t phase = 0, accph = 0;
       for (long long t = t_begin; t < t_end && !*abort; ++t) {
-        const Tile tl = tile_of(t, tiles_per_q);
+        const Tile tl = tile_of(t, tiles_per_q, F::kTileRows);
         if (tl.q != cur_q) {
           if (cur_q >= 0) tc::commit(&bars->qempty[slot]);  // old head block free once its MMAs finish
           slot = nq & 1;
@@ -176,13 +182,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_base = tc::smem_u32(stage_buf + stage * kTileBytes);
         const uint32_t b_base = tc::smem_u32(q_buf + slot * kQBytes);
 #pragma unroll
-        for (int kk = 0; kk < F::kKSteps; ++kk) {  // 32 bytes of K per MMA, 4 per 128-byte box
-          const uint64_t ad = tc::sw128_desc(a_base + (kk >> 2) * F::kBoxBytes + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = tc::sw128_desc(b_base + (kk >> 2) * F::kQBox + (kk & 3) * 32, 16, 1024);
-          if constexpr (kFp8)
-            tc::mma_f8(tmem + acc * 64, ad, bd, idesc, kk > 0);
-          else
-            tc::mma_bf16(tmem + acc * 64, ad, bd, idesc, kk > 0);
+        for (int sub = 0; sub < F::kSub; ++sub) {
+#pragma unroll
+          for (int kk = 0; kk < F::kKSteps; ++kk) {  // 32 bytes of K per MMA, 4 per 128-byte box
+            const uint32_t box = kFp8 ? sub : (kk >> 2);
+            const uint64_t ad = tc::sw128_desc(a_base + box * F::kBoxBytes + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = tc::sw128_desc(b_base + (kk >> 2) * F::kQBox + (kk & 3) * 32, 16, 1024);
+            const uint32_t d = tmem + acc * F::kAccCols + 64 * sub;
+            if constexpr (kFp8)
+              tc::mma_f8(d, ad, bd, idesc, kk > 0);
+            else
+              tc::mma_bf16(d, ad, bd, idesc, kk > 0);
+          }
         }
         tc::commit(&bars->empty[stage]);
         tc::commit(&bars->accfull[acc]);
@@ -206,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t accph = 0;
     float w[kHi];
     for (long long t = t_begin; t < t_end && !*abort; ++t) {
-      const Tile tl = tile_of(t, tiles_per_q);
+      const Tile tl = tile_of(t, tiles_per_q, F::kTileRows);
       if (tl.q != cur_q) {
         const int raw = a.n_cmp[tl.q];
         if ((raw < 0 || raw > a.N_max) && row == 0) raise_status(a.status, CSA_STATUS_BAD_COUNT);
@@ -231,22 +242,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc::fence_after_sync();
-      uint32_t v0[32], v1[32];
-      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * 64;
-      tc::tmem_ld32(taddr, v0);
-      tc::tmem_ld32(taddr + 32, v1);
-      tc::tmem_ld_wait();
+      float sc[F::kSub];
+#pragma unroll
+      for (int sub = 0; sub < F::kSub; ++sub) {
+        uint32_t v0[32], v1[32];
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * F::kAccCols + 64 * sub;
+        tc::tmem_ld32(taddr, v0);
+        tc::tmem_ld32(taddr + 32, v1);
+        tc::tmem_ld_wait();
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) s = fmaf(w[h], fmaxf(__uint_as_float(v0[h]), 0.f), s);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) s = fmaf(w[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s);
+        sc[sub] = s;
+      }
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->accempty[acc]);
-      float s = 0.f;
 #pragma unroll
-      for (int h = 0; h < 32; ++h) s = fmaf(w[h], fmaxf(__uint_as_float(v0[h]), 0.f), s);
-#pragma unroll
-      for (int h = 0; h < 32; ++h) s = fmaf(w[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s);
-      const int j = tl.j0 + row;
-      if (j < cur_n) {
-        if constexpr (kFp8) s *= a.sk[(size_t)(tl.q / a.q_per_seq) * a.N_max + j];
-        a.scores[(size_t)tl.q * a.N_max + j] = s;
+      for (int sub = 0; sub < F::kSub; ++sub) {
+        const int j = tl.j0 + 128 * sub + row;
+        if (j < cur_n) {
+          float s = sc[sub];
+          if constexpr (kFp8) s *= a.sk[(size_t)(tl.q / a.q_per_seq) * a.N_max + j];
+          a.scores[(size_t)tl.q * a.N_max + j] = s;
+        }
       }
       if (++acc == 2) {
         acc = 0;
@@ -258,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, kTmemCols);
+    tc::tmem_dealloc(tmem, F::kTmemCols);
   }
 }
 
@@ -286,9 +306,10 @@ cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool
   CUtensorMap tm_ki, tm_qi;
   const int esz = fp8 ? 1 : 2, box = fp8 ? 128 : 64;
   auto mk = fp8 ? make_tmap_u8_2d : make_tmap_bf16_2d;
-  if (!mk(&tm_ki, a.ki, kDi, (uint64_t)a.B * a.N_max, kDi * esz, box, kTileM)) return cudaSuccess;
+  if (!mk(&tm_ki, a.ki, kDi, (uint64_t)a.B * a.N_max, kDi * esz, box, 128)) return cudaSuccess;
   if (!mk(&tm_qi, a.qi, kDi, (uint64_t)a.Q * kHi, kDi * esz, box, kHi)) return cudaSuccess;
-  const int tiles_per_q = (a.N_max + kTileM - 1) / kTileM;
+  const int tile_rows = fp8 ? Fmt<true>::kTileRows : Fmt<false>::kTileRows;
+  const int tiles_per_q = (a.N_max + tile_rows - 1) / tile_rows;
   const long long total = (long long)a.Q * tiles_per_q;
   long long grid = num_sms_cached();
   if (grid > total) grid = total;

@@ -23,7 +23,7 @@
 //
 // Loads: contiguous runs of 64 rows (HCA entries, window rows) are single TMA
 // boxes of 64 rows; top-k rows are gathered with 16-byte cp.async copies by
-// the two loader warps (TMA gathers issue too slowly for 1 KB rows). The
+// the loader warps (TMA gathers issue too slowly for 1 KB rows). The
 // compressed segment is padded to a multiple of 4 rows (unused, masked).
 //
 // Work split: query q's row list is cut into `splits` (<= 16) runs of whole
@@ -34,8 +34,8 @@
 // cluster barrier, merges 1/splits of the output from all of them (L2 reads;
 // distributed-shared-memory reads of the same data measured several times
 // slower).
-// Roles (224 threads): warps 0-1 load (one per tile buffer), warp 2 issues
-// the MMAs and owns TMEM, warps 3-6 run the softmax and the epilogue. All
+// Roles (288 threads): warps 0-3 load (two per tile buffer), warp 4 issues
+// the MMAs and owns TMEM, warps 5-8 run the softmax and the epilogue. All
 // mbarrier waits are bounded; the softmax warps take every decision to stop
 // together (a barrier reduction), so no named barrier is left half-joined.
 #include "common.cuh"
@@ -54,10 +54,10 @@ constexpr uint32_t kTileBytes = 8 * kBoxBytes;      // 64 rows x 512 dims: 64 KB
 constexpr uint32_t kQBoxBytes = kH * 128;           // 64 heads x 64 dims: 8 KB
 constexpr uint32_t kQBytes = 8 * kQBoxBytes;        // 64 KB
 constexpr uint32_t kPBytes = kRows * kH * 2;        // 8 KB
-constexpr int kLoadWarps = 2;
-constexpr int kThreads = 224;
-constexpr int kMmaWarp = 2;
-constexpr int kSoftWarp0 = 3;
+constexpr int kLoadWarps = 4;                       // two per tile buffer, 32 rows each
+constexpr int kThreads = 288;
+constexpr int kMmaWarp = 4;
+constexpr int kSoftWarp0 = 5;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSplits = 16;                      // splits of one query form one cluster (<= 16 CTAs)
 constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m (M = 128 layout)
@@ -75,7 +75,7 @@ struct Small {
   int abort;
   int rescale;
   int need[4];  // per tile (mod 4): some logit exceeded the running maximum by more than 2^8
-  const bf16 *rowp[2][kRows];  // gathered tiles: source row of each tile row (null: zero-fill)
+  const bf16 *rowp[kLoadWarps][32];  // gathered tiles: source row of each of a loader warp's rows (null: zero-fill)
 };
 
 constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kQBytes + 2 * kPBytes + sizeof(Small);
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tc::mbar_init(&sm->q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&sm->kv_full[i], 32);
+      tc::mbar_init(&sm->kv_full[i], 64);
       tc::mbar_init(&sm->kv_empty[i], 1);
       tc::mbar_init(&sm->s_full[i], 1);
       tc::mbar_init(&sm->p_full[i], 4 * 32);
@@ -261,14 +261,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kLoadWarps) {
     // ------------------------------------------------------------ loaders
-    // Warp g fills tile buffer g (tiles g, g + 2, ...). A contiguous run is 8
-    // TMA boxes issued by lane 0. A gathered tile is 4096 16-byte cp.async
-    // copies, 128 per lane, each warp instruction moving 512 contiguous bytes
-    // of one row; every lane waits for its own copies, fences them for the
-    // tensor core and arrives, so kv_full expects 32 arrivals either way.
-    const int g = warp;
+    // Warps 2g and 2g + 1 fill tile buffer g (tiles g, g + 2, ...), rows
+    // 0-31 and 32-63 of each tile. A contiguous run is 8 TMA boxes issued by
+    // lane 0 of warp 2g. A gathered tile is 16-byte cp.async copies, 64 per
+    // lane, each warp instruction moving 512 contiguous bytes of one row;
+    // every lane waits for its own copies, fences them for the tensor core
+    // and arrives, so kv_full expects 64 arrivals either way. Each warp also
+    // prefetches its rows of its next tile into L2 while the buffer is busy.
+    const int g = warp >> 1, half = warp & 1;
     const uint32_t buf_base = tc::smem_u32(kv) + g * kTileBytes;
-    if (lane == 0) {
+    if (warp == 0 && lane == 0) {
       tc::prefetch_tmap(&tm_cmp_t);
       tc::prefetch_tmap(&tm_win_t);
     }
@@ -292,21 +294,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       win_run = r0 >= L.nsel4;
       return win_run || (!a.idx && r0 + kRows <= L.nsel4);
     };
-    // Bring tile li into L2 ahead of its load, which can only start once the
-    // tile buffer is free: the load then waits on L2, not on HBM.
+    // Bring this warp's rows of tile li into L2 ahead of their load, which can
+    // only start once the tile buffer is free: the load then waits on L2.
     auto prefetch_l2 = [&](int li) {
       if (li >= ntiles) return;
       const int r0 = (t0 + li) * kRows;
       bool win_run;
       if (is_run(r0, win_run)) {
         if (lane == 0) {
-          const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
+          const int row = (win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0) + 32 * half;
           for (int bx = 0; bx < 8; ++bx) tma_prefetch_l2(win_run ? &tm_win_t : &tm_cmp_t, 64 * bx, row);
         }
-      } else {
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-          if (const bf16 *p = src_row(r0 + lane + 32 * hh)) bulk_prefetch_l2(p, kD * 2);
+      } else if (const bf16 *p = src_row(r0 + 32 * half + lane)) {
+        bulk_prefetch_l2(p, kD * 2);
       }
     };
     int last = -1;
@@ -314,15 +314,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r0 = (t0 + li) * kRows;
       bool win_run;
       const bool run = is_run(r0, win_run);
-      __syncwarp();  // the previous tile's copies have read rowp[g]
-      if (!run) {
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) sm->rowp[g][lane + 32 * hh] = src_row(r0 + lane + 32 * hh);
-      }
+      __syncwarp();  // the previous tile's copies have read rowp[warp]
+      if (!run) sm->rowp[warp][lane] = src_row(r0 + 32 * half + lane);
       if (li == g) prefetch_l2(li + 2);  // later tiles are prefetched one round ahead, below
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status))) break;
       if (run) {
-        if (lane == 0) {
+        if (half == 0 && lane == 0) {
           tc::mbar_arrive_expect_tx(&sm->kv_full[g], kTileBytes);
           const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
           for (int bx = 0; bx < 8; ++bx)
@@ -332,11 +329,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::mbar_arrive(&sm->kv_full[g]);
         }
       } else {
-        __syncwarp();  // rowp[g] written by every lane
+        __syncwarp();  // rowp[warp] written by every lane
 #pragma unroll 8
-        for (int i = 0; i < 2 * kRows; ++i) {
-          const int row = i >> 1, c16 = lane + 32 * (i & 1);  // 16-byte piece c16 of the 1 KB row
-          const bf16 *src = sm->rowp[g][row];
+        for (int i = 0; i < 64; ++i) {
+          const int rw = i >> 1, c16 = lane + 32 * (i & 1);  // 16-byte piece c16 of this warp's row rw
+          const int row = 32 * half + rw;                     // row within the tile
+          const bf16 *src = sm->rowp[warp][rw];
           const uint32_t dst = buf_base + (c16 >> 3) * kBoxBytes + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
           cp_async16(dst, src ? src + c16 * 8 : static_cast<const bf16 *>(a.kv_win), src != nullptr);
         }
@@ -350,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       last = li;
     }
     // Drain: a TMA tile still in flight must land before the CTA exits.
-    if (lane == 0 && last >= 0) tc::mbar_drain(&sm->kv_full[g], (last >> 1) & 1);
+    if (half == 0 && lane == 0 && last >= 0) tc::mbar_drain(&sm->kv_full[g], (last >> 1) & 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
