@@ -424,12 +424,13 @@ cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
     if ((a.D / 8) % 32 == 0) {
       const int nvec = a.D / 8;
       // Long windows and few entries: a cluster of C blocks per entry, at
-      // least 16 positions each, about two blocks per SM in all.
-      // (C a power of two, so that it divides D)
+      // least 16 positions each, about two blocks per SM in all. C is a power
+      // of two (it divides D) and at most 4: a block fills an SM, and
+      // clusters of 8 such blocks do not all fit in the GPCs at once.
       int C = 1;
       if (a.win >= 32) {
         const long long fill = (2LL * num_sms() + total - 1) / total;
-        while (2 * C <= 8 && 2 * C <= a.win / 16 && 2 * C <= fill) C *= 2;
+        while (2 * C <= 4 && 2 * C <= a.win / 16 && 2 * C <= fill) C *= 2;
       }
       const int P = (a.win + C - 1) / C;
       int G = P < 16 ? P : 16;

@@ -216,6 +216,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0, cur_q = -1, cur_n = 0;
     uint32_t accph = 0;
     float w[kHi];
+    float sk_next[F::kSub];
+    auto load_sk = [&](long long tt) {  // key scales of tile tt's rows of this thread (1 past the cache)
+      const Tile tn = tile_of(tt, tiles_per_q, F::kTileRows);
+#pragma unroll
+      for (int sub = 0; sub < F::kSub; ++sub) {
+        const int j = tn.j0 + 128 * sub + row;
+        sk_next[sub] = j < a.N_max ? __ldg(a.sk + (size_t)(tn.q / a.q_per_seq) * a.N_max + j) : 1.f;
+      }
+    };
+#pragma unroll
+    for (int sub = 0; sub < F::kSub; ++sub) sk_next[sub] = 1.f;
+    if constexpr (kFp8) {
+      if (t_begin < t_end) load_sk(t_begin);
+    }
     for (long long t = t_begin; t < t_end && !*abort; ++t) {
       const Tile tl = tile_of(t, tiles_per_q, F::kTileRows);
       if (tl.q != cur_q) {
@@ -238,6 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           w[h + 3] = v.w;
         }
         cur_q = tl.q;
+      }
+      // E4M3: the key scales of this tile were loaded one tile ahead; start
+      // the next tile's now, so their latency hides behind this tile's work.
+      float skv[F::kSub];
+#pragma unroll
+      for (int sub = 0; sub < F::kSub; ++sub) skv[sub] = sk_next[sub];
+      if constexpr (kFp8) {
+        if (t + 1 < t_end) load_sk(t + 1);
       }
       const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
@@ -263,9 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int sub = 0; sub < F::kSub; ++sub) {
         const int j = tl.j0 + 128 * sub + row;
         if (j < cur_n) {
-          float s = sc[sub];
-          if constexpr (kFp8) s *= a.sk[(size_t)(tl.q / a.q_per_seq) * a.N_max + j];
-          a.scores[(size_t)tl.q * a.N_max + j] = s;
+          a.scores[(size_t)tl.q * a.N_max + j] = kFp8 ? sc[sub] * skv[sub] : sc[sub];
         }
       }
       if (++acc == 2) {
