@@ -27,13 +27,15 @@
 // compressed segment is padded to a multiple of 4 rows (unused, masked).
 //
 // Work split: query q's row list is cut into `splits` (<= 16) runs of whole
-// tiles, one CTA each, the CTAs of a query forming one thread-block cluster
-// (the largest size for which every query's cluster is resident at once).
+// tiles, one CTA each. Normally the CTAs of a query form one thread-block
+// cluster (the largest size for which every query's cluster is resident at
+// once); when that caps the splits well below SMs / Q, they are plain blocks
+// and mqa_combine_kernel merges their partials.
 // With one split the CTA folds in the sink and writes the output; otherwise
-// every CTA writes its unnormalised (m, l, O) to the workspace and, after a
-// cluster barrier, merges 1/splits of the output from all of them (L2 reads;
-// distributed-shared-memory reads of the same data measured several times
-// slower).
+// every CTA writes its unnormalised (m, l, O) to the workspace and, in a
+// cluster, after a cluster barrier merges 1/splits of the output from all of
+// them (L2 reads; distributed-shared-memory reads of the same data measured
+// several times slower).
 // Roles (288 threads): warps 0-3 load (two per tile buffer), warp 4 issues
 // the MMAs and owns TMEM, warps 5-8 run the softmax and the epilogue. All
 // mbarrier waits are bounded; the softmax warps take every decision to stop
@@ -214,7 +216,7 @@ __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)
 __global__ void __launch_bounds__(kThreads, 1)
     mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp_t,
                   const __grid_constant__ CUtensorMap tm_win_t, MqaArgs a, int splits, int tiles_per_split,
-                  float scale_log2, float *part_o, float *part_ml) {
+                  float scale_log2, float *part_o, float *part_ml, int cluster_merge) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *kv = smem;                              // [2 tiles][8 boxes][64 rows][128 B]
@@ -676,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
-  if (splits > 1) {
+  if (splits > 1 && cluster_merge) {
     // The splits of query qq are the blocks of one cluster (rank = split):
     // the cluster barrier orders every split's partials (global memory) before
     // the merge. Every block merges 1/splits of the outputs with the sink:
@@ -727,6 +729,53 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Merge of the split partials when the splits of a query are not one
+// cluster (more splits than cluster residency allows): one block per
+// (query, head); thread t owns dims 4t..4t+3 and issues the loads of all
+// splits at once. Same formula as the in-kernel merge.
+__global__ void __launch_bounds__(128) mqa_combine_kernel(const float *part_o, const float *part_ml,
+                                                          const float *sink, bf16 *out, int splits) {
+  extern __shared__ float w[];  // [splits] weights, then [2][splits] (m, l)
+  const int qq = blockIdx.x, h = blockIdx.y;
+  pdl_wait();
+  pdl_release();
+  float *ml = w + splits;
+  for (int i = threadIdx.x; i < 2 * splits; i += blockDim.x) {
+    const int which = i / splits, sp = i - which * splits;
+    ml[i] = part_ml[(((size_t)qq * splits + sp) * 2 + which) * kH + h];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const float sk = sink[h] * kLog2e;
+    float M = sk;
+    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, ml[sp]);
+    float Lsum = exp2f(sk - M);
+    for (int sp = 0; sp < splits; ++sp) {
+      const float ww = ml[sp] == -INFINITY ? 0.f : exp2f(ml[sp] - M);
+      w[sp] = ww;
+      Lsum += ml[splits + sp] * ww;
+    }
+    const float inv = 1.f / Lsum;
+    for (int sp = 0; sp < splits; ++sp) w[sp] *= inv;
+  }
+  __syncthreads();
+  const int d = 4 * threadIdx.x;
+  const float *src = part_o + ((size_t)qq * splits * kH + h) * kD + d;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int sp = 0; sp < splits; ++sp) {
+    const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)sp * kH * kD));
+    const float ww = w[sp];
+    acc.x = fmaf(ww, v.x, acc.x);
+    acc.y = fmaf(ww, v.y, acc.y);
+    acc.z = fmaf(ww, v.z, acc.z);
+    acc.w = fmaf(ww, v.w, acc.w);
+  }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+  *reinterpret_cast<uint2 *>(out + ((size_t)qq * kH + h) * kD + d) =
+      make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+}
+
 int num_sms_cached() {
   static int n = 0;
   if (!n) {
@@ -775,25 +824,40 @@ int max_active_clusters(int size) {
   return cache[size] > 0 ? cache[size] : 0;
 }
 
-// Split query rows into runs of whole tiles: the largest cluster size (up to
-// SMs / Q and 16) for which all Q clusters are resident at once; one split
-// when no cluster size fits.
-void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split) {
+// Split query rows into runs of whole tiles. Preferred: the largest
+// cluster size (up to SMs / Q and 16) for which all Q clusters are resident
+// at once, merged inside the kernel. When cluster residency caps the splits
+// well below SMs / Q (1.25x or more), the splits are plain blocks instead and
+// a combine kernel merges them.
+void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split, bool *cluster_merge) {
   const int tiles = (rows_max + kRows - 1) / kRows;
   int hi = num_sms_cached() / (Q > 0 ? Q : 1);
   hi = hi > kMaxSplits ? kMaxSplits : hi;
   hi = hi > tiles ? tiles : hi;
+  int cl = 1, cl_tps = tiles > 0 ? tiles : 1;
   for (int s = hi; s >= 2; --s) {
     const int tps = (tiles + s - 1) / s;
     const int sp = (tiles + tps - 1) / tps;
     if (sp >= 2 && max_active_clusters(sp) >= Q) {
-      *splits = sp;
-      *tiles_per_split = tps;
-      return;
+      cl = sp;
+      cl_tps = tps;
+      break;
     }
   }
-  *splits = 1;
-  *tiles_per_split = tiles > 0 ? tiles : 1;
+  int fr = 1, fr_tps = tiles > 0 ? tiles : 1;
+  if (hi >= 2) {
+    fr_tps = (tiles + hi - 1) / hi;
+    fr = (tiles + fr_tps - 1) / fr_tps;
+  }
+  if (fr >= 2 && 4 * fr >= 5 * cl) {
+    *splits = fr;
+    *tiles_per_split = fr_tps;
+    *cluster_merge = false;
+  } else {
+    *splits = cl;
+    *tiles_per_split = cl_tps;
+    *cluster_merge = cl > 1;
+  }
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -823,7 +887,8 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   *taken = false;
   if (!tc_shape(a)) return cudaSuccess;
   int splits, tps;
-  plan_splits(a.Q, rows_max_of(a), &splits, &tps);
+  bool cluster_merge;
+  plan_splits(a.Q, rows_max_of(a), &splits, &tps, &cluster_merge);
   CUtensorMap tm_q, tm_cmp_t, tm_win_t;
   const uint64_t cmp_rows = (uint64_t)a.B * a.N_max, win_rows = (uint64_t)a.B * a.T_raw;
   if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * kH, kD * 2, 64, kH) ||
@@ -836,8 +901,12 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   float *part_ml = part_o + (size_t)a.Q * splits * kH * kD;
   set_kernel_attributes();
   *taken = true;
-  return launch_pdl_cluster(mqa_tc_kernel, dim3(splits, a.Q), dim3(kThreads), kSmemBytes, stream, (unsigned)splits,
-                            tm_q, tm_cmp_t, tm_win_t, a, splits, tps, a.scale * kLog2e, part_o, part_ml);
+  cudaError_t e = launch_pdl_cluster(mqa_tc_kernel, dim3(splits, a.Q), dim3(kThreads), kSmemBytes, stream,
+                                     cluster_merge ? (unsigned)splits : 1u, tm_q, tm_cmp_t, tm_win_t, a, splits, tps,
+                                     a.scale * kLog2e, part_o, part_ml, (int)cluster_merge);
+  if (e != cudaSuccess || splits <= 1 || cluster_merge) return e;
+  return launch_pdl(mqa_combine_kernel, dim3(a.Q, kH), dim3(kD / 4), splits * 3 * sizeof(float), stream,
+                    (const float *)part_o, (const float *)part_ml, a.sink, static_cast<bf16 *>(a.out), splits);
 }
 
 }  // namespace csa
