@@ -9,13 +9,18 @@ from .csa_oracle import (  # noqa: F401
     attend,
     compress,
     e4m3_decode,
+    e4m3_encode,
+    hadamard_matrix,
+    hadamard_rotate,
     hca_mqa,
+    index_compress,
     index_scores,
     index_scores_fp8,
     index_topk,
     index_topk_fp8,
     n_entries,
     n_visible,
+    quantize_rows_e4m3,
     rms_norm,
     round_to,
     sparse_mqa,

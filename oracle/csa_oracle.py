@@ -53,6 +53,14 @@ the design notes):
   Architecture analysis INNOVATIONS section 1) with one positive fp32 scale
   per row: per compressed entry for the keys, per (query, head) for the
   queries; value = scale * decoded code. The score is R9 on those values.
+* R19 the indexer's own compressor (the next row f2; Architecture analysis
+  INNOVATIONS section 1: "its own dedicated KV compressor with Hadamard
+  rotation"): the A1 pool + RMSNorm at the indexer head dim, followed by the
+  orthonormal Sylvester-Hadamard rotation x -> x H_n / sqrt(n) of each row; the
+  queries take the same rotation, so scores are unchanged in exact
+  arithmetic. Rows become FP8 codes with one scale per row, amax / 448
+  (dynamic scaling; a zero row gets scale 1), each value rounded to the
+  nearest E4M3 value, ties to even, magnitudes above 448 saturating to 448.
 
 Pins (tests/test_oracle_pins.py) tie every function to something other than
 itself: closed forms, textbook/library special cases (torch rms_norm,
@@ -179,6 +187,58 @@ def e4m3_decode(codes) -> np.ndarray:
     m = (c & 0x7).astype(np.float64)
     mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
     return np.where((c & 0x7F) == 0x7F, np.nan, sign * mag)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest OCP FP8 E4M3 code of each value (ties to the even code),
+    magnitudes above 448 saturating to 448, the sign kept (a negative value
+    that rounds to zero gives -0, 0x80); written from the format's value set:
+    the 127 non-negative finite codes 0x00..0x7E in increasing order."""
+    x = np.asarray(x, dtype=np.float64)
+    pos = e4m3_decode(np.arange(0x7F, dtype=np.uint8))          # 0 .. 448, increasing
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(pos, a, side="left"), 0, 0x7E)   # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - pos[lo], pos[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))   # ties: even code (even mantissa)
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(a == pos[hi], hi, code).astype(np.uint8)      # exact values
+    return np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)  # the sign is kept, zero included
+
+
+def quantize_rows_e4m3(x):
+    """Per-row dynamic FP8 quantization (reading R19), in fp32 like the GPU
+    (the codes are integers decided by fp32 arithmetic on both sides):
+        scale = fp32(amax_row / 448) (1 for an all-zero row),
+        code  = e4m3_encode(fp32(x_f32 / scale)).
+    x: [rows, n]. Returns (codes uint8 [rows, n], scales float32 [rows])."""
+    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    amax = np.abs(x32).max(axis=1)
+    scale = np.where(amax > 0, (amax / np.float32(448.0)).astype(np.float32), np.float32(1.0)).astype(np.float32)
+    y = (x32 / scale[:, None]).astype(np.float32)
+    return e4m3_encode(y), scale
+
+
+def hadamard_matrix(n: int) -> np.ndarray:
+    """Sylvester's Hadamard matrix: H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]]."""
+    assert n >= 1 and n & (n - 1) == 0
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def hadamard_rotate(x) -> np.ndarray:
+    """Orthonormal Hadamard rotation of each row (reading R19): x H_n / sqrt(n)."""
+    x = as_f64(x)
+    n = x.shape[-1]
+    return x @ hadamard_matrix(n) / np.sqrt(n)
+
+
+def index_compress(kv, gate, ape, norm_w, win: int, stride: int, eps: float = RMS_EPS) -> np.ndarray:
+    """The indexer's keys from its own raw KV (reading R19): the A1 pool +
+    RMSNorm at the indexer head dim, then the Hadamard rotation of each entry."""
+    return hadamard_rotate(compress(kv, gate, ape, norm_w, win, stride, eps))
 
 
 def index_scores_fp8(qi8, sq, wi, ki8, sk, n_vis: int) -> np.ndarray:

@@ -236,6 +236,90 @@ def test_index_fp8_unit_scales_single_head_is_a_plain_dot_of_decoded_codes():
     assert np.allclose(got, (tk @ tq[0]).numpy(), rtol=1e-15)
 
 
+# ------------------------------------------- indexer compressor and FP8 codes (R19)
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = np.arange(0x7F, dtype=np.uint8)
+    vals = O.e4m3_decode(codes)
+    assert np.array_equal(O.e4m3_encode(vals), codes)
+    assert np.array_equal(O.e4m3_encode(-vals), codes | 0x80)
+
+
+def test_e4m3_encode_matches_torch_float8_on_fp32_values_in_range():
+    # torch's cast rounds to nearest, ties to even, on fp32 inputs
+    x = np.linspace(-448, 448, 400001).astype(np.float32)
+    x = np.concatenate([x, (rng.standard_normal(100000) * 30).astype(np.float32).clip(-448, 448)])
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x.astype(np.float64)), ref)
+
+
+def test_e4m3_encode_ties_saturation_and_underflow():
+    # 84 lies halfway between 80 (mantissa 010) and 88 (011): the even one
+    assert O.e4m3_decode(O.e4m3_encode([84.0, -84.0])).tolist() == [80.0, -80.0]
+    # 1.0625 halfway between 1 (000) and 1.125 (001); 1.1875 between 1.125 and 1.25 (010)
+    assert O.e4m3_decode(O.e4m3_encode([1.0625, 1.1875])).tolist() == [1.0, 1.25]
+    assert O.e4m3_encode([448.0, 460.0, 1e6, -1e6]).tolist() == [0x7E, 0x7E, 0x7E, 0xFE]
+    # half the smallest subnormal (2^-10) ties to 0 (even); just above it goes to 2^-9
+    assert O.e4m3_encode([2.0 ** -10, 2.0 ** -10 * 1.01, -1e-30]).tolist() == [0x00, 0x01, 0x80]
+
+
+def test_quantize_rows_maps_the_row_maximum_to_448_and_bounds_the_error():
+    x = rng.standard_normal((20, 128)) * rng.uniform(0.01, 100, (20, 1))
+    x[3] = 0.0
+    codes, scales = O.quantize_rows_e4m3(x)
+    assert scales.dtype == np.float32 and scales[3] == 1.0 and (codes[3] & 0x7F == 0).all()
+    deq = O.e4m3_decode(codes) * scales[:, None].astype(np.float64)
+    for r in range(20):
+        if r == 3:
+            continue
+        j = np.argmax(np.abs(x[r]))
+        assert codes[r, j] & 0x7F == 0x7E                     # the largest magnitude becomes +-448
+        # nearest-value rounding: error at most half the E4M3 spacing at that magnitude (<= 2^-4 relative),
+        # or half the smallest subnormal step
+        err = np.abs(deq[r] - x[r])
+        assert np.all(err <= np.maximum(np.abs(x[r]) * 2.0 ** -4, 2.0 ** -10 * scales[r]) * 1.0001)
+
+
+def test_hadamard_is_sylvester_and_orthonormal():
+    import scipy.linalg
+    for n in (1, 2, 16, 128):
+        assert np.array_equal(O.hadamard_matrix(n), scipy.linalg.hadamard(n))
+    h = O.hadamard_matrix(128)
+    assert np.array_equal(h @ h.T, 128 * np.eye(128))
+    x = rng.standard_normal((7, 128))
+    y = O.hadamard_rotate(x)
+    assert np.allclose(O.hadamard_rotate(y), x, atol=1e-12)                 # H / sqrt(n) is its own inverse
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1))
+    e0 = np.zeros((1, 128))
+    e0[0, 0] = 1
+    assert np.allclose(O.hadamard_rotate(e0), np.full((1, 128), 1 / np.sqrt(128)))
+
+
+def test_rotation_leaves_indexer_scores_unchanged():
+    Hi, n = 4, 30
+    qi, ki, wi = rng.standard_normal((Hi, 128)), rng.standard_normal((n, 128)), rng.uniform(0, 1, Hi)
+    assert np.allclose(O.index_scores(O.hadamard_rotate(qi), wi, O.hadamard_rotate(ki), n),
+                       O.index_scores(qi, wi, ki, n), rtol=1e-12, atol=1e-12)
+
+
+def test_index_compress_is_the_rotated_pool():
+    # constant raw KV rows: the pool returns the row before the norm, so each
+    # entry is the rotation of norm(c) -- an explicit closed form through H
+    T, D = 20, 128
+    c = rng.standard_normal(D)
+    kv = np.tile(c, (T, 1))
+    gate, ape = rng.standard_normal((T, D)), rng.standard_normal((8, D)) * 0.1
+    out = O.index_compress(kv, gate, ape, np.ones(D), 8, 4)
+    want = (c / np.sqrt(np.mean(c * c) + 1e-6)) @ scipy_hadamard(D) / np.sqrt(D)
+    assert out.shape == (O.n_entries(T, 8, 4), D)
+    assert np.allclose(out, np.tile(want, (out.shape[0], 1)), rtol=1e-12, atol=1e-12)
+
+
+def scipy_hadamard(n):
+    import scipy.linalg
+    return scipy.linalg.hadamard(n).astype(np.float64)
+
+
 def test_topk_closed_form_ties():
     g = _golden("topk_ties.json")
     for case in g["cases"]:
