@@ -109,15 +109,8 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool v
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// L2 prefetch of one TMA box of `map` at (c0, c1) (out-of-range parts are
-// ignored, as for loads), and of `bytes` contiguous bytes at p (16-byte
-// aligned, a multiple of 16).
-__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap *map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1)
-               : "memory");
-}
-
+// L2 prefetch of `bytes` contiguous bytes at p (16-byte aligned, a multiple
+// of 16).
 __device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -298,14 +291,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // Bring this warp's rows of tile li into L2 ahead of their load, which can
     // only start once the tile buffer is free: the load then waits on L2.
+    // (A run's rows are contiguous in memory: one bulk prefetch of this
+    // warp's 32 rows streams them from HBM in order, where the tile's TMA
+    // boxes each read 128 bytes of every row.)
     auto prefetch_l2 = [&](int li) {
       if (li >= ntiles) return;
       const int r0 = (t0 + li) * kRows;
       bool win_run;
       if (is_run(r0, win_run)) {
         if (lane == 0) {
-          const int row = (win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0) + 32 * half;
-          for (int bx = 0; bx < 8; ++bx) tma_prefetch_l2(win_run ? &tm_win_t : &tm_cmp_t, 64 * bx, row);
+          // first row of this warp's half, and how many rows of the sequence's buffer remain from it
+          const int first = win_run ? L.wlo + (r0 - L.nsel4) + 32 * half : r0 + 32 * half;
+          const int avail = (win_run ? a.T_raw : a.N_max) - first;
+          const int rows = avail < 32 ? avail : 32;
+          if (rows > 0) {
+            const bf16 *base = win_run ? static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + first) * kD
+                                       : static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + first) * kD;
+            bulk_prefetch_l2(base, (uint32_t)rows * kD * 2);
+          }
         }
       } else if (const bf16 *p = src_row(r0 + 32 * half + lane)) {
         bulk_prefetch_l2(p, kD * 2);
@@ -318,7 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool run = is_run(r0, win_run);
       __syncwarp();  // the previous tile's copies have read rowp[warp]
       if (!run) sm->rowp[warp][lane] = src_row(r0 + 32 * half + lane);
-      if (li == g) prefetch_l2(li + 2);  // later tiles are prefetched one round ahead, below
+      if (li == g) {  // the first tile streams in order too; later tiles are prefetched one round ahead, below
+        if (run) prefetch_l2(li);
+        prefetch_l2(li + 2);
+      }
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status))) break;
       if (run) {
         if (half == 0 && lane == 0) {
