@@ -81,6 +81,48 @@ int csa_compress(const void *kv, const void *gate, const float *ape, const float
   return cuda_rc(launch_compress(a, (cudaStream_t)stream));
 }
 
+static bool pow2_dim(int D) { return D == 64 || D == 128 || D == 256 || D == 512; }
+
+int csa_index_compress(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
+                       int stride, void *out, float *out_scales, int B, int T, int D, long long kv_seq_stride,
+                       long long gate_seq_stride, long long out_seq_stride, int dtype, int out_dtype,
+                       csa_stream_t stream) {
+  if (!kv || !gate || !ape || !norm_w || !out) return CSA_ERR_INVALID;
+  if (!dtype_ok(dtype) || !pow2_dim(D) || B < 1 || win < 1 || win > 128 || stride < 1) return CSA_ERR_INVALID;
+  const bool fp8 = out_dtype == CSA_DTYPE_E4M3;
+  if (!fp8 && out_dtype != dtype) return CSA_ERR_INVALID;
+  if (fp8 && (!out_scales || (reinterpret_cast<uintptr_t>(out_scales) & 3))) return CSA_ERR_INVALID;
+  if (ratio != stride || T < win) return CSA_ERR_INVALID;
+  if (kv_seq_stride < 0 || gate_seq_stride < 0 || out_seq_stride < 0) return CSA_ERR_INVALID;
+  if (!elem_aligned(kv, dtype) || !elem_aligned(gate, dtype) || (!fp8 && !elem_aligned(out, dtype)) ||
+      (fp8 && (reinterpret_cast<uintptr_t>(out) & 1)))
+    return CSA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(ape) | reinterpret_cast<uintptr_t>(norm_w)) & 3) return CSA_ERR_INVALID;
+  const int N = (T - win) / stride + 1;
+  const long long kv_ss = kv_seq_stride ? kv_seq_stride : (long long)T * D;
+  const long long g_ss = gate_seq_stride ? gate_seq_stride : (long long)T * D;
+  const long long o_ss = out_seq_stride ? out_seq_stride : (long long)N * D;
+  if (B > 1 && (kv_ss < (long long)T * D || g_ss < (long long)T * D || o_ss < (long long)N * D)) return CSA_ERR_INVALID;
+  if (o_ss % D) return CSA_ERR_INVALID;
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  CompressArgs a{kv, gate, ape, norm_w, out, B, T, D, win, stride, N, kv_ss, g_ss, o_ss, dtype};
+  return cuda_rc(launch_index_compress(a, fp8 ? static_cast<uint8_t *>(out) : nullptr, fp8 ? out_scales : nullptr,
+                                       o_ss / D, (cudaStream_t)stream));
+}
+
+int csa_hadamard_rows(const void *x, void *out, float *out_scales, long long rows, int D, int dtype, int out_dtype,
+                      csa_stream_t stream) {
+  if (!x || !out || rows < 0 || !dtype_ok(dtype) || !pow2_dim(D)) return CSA_ERR_INVALID;
+  const bool fp8 = out_dtype == CSA_DTYPE_E4M3;
+  if (!fp8 && out_dtype != dtype) return CSA_ERR_INVALID;
+  if (fp8 && (!out_scales || (reinterpret_cast<uintptr_t>(out_scales) & 3))) return CSA_ERR_INVALID;
+  if (!elem_aligned(x, dtype) || (!fp8 && !elem_aligned(out, dtype)) || (fp8 && (reinterpret_cast<uintptr_t>(out) & 1)))
+    return CSA_ERR_INVALID;
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  return cuda_rc(launch_hadamard_rows(x, fp8 ? nullptr : out, fp8 ? static_cast<uint8_t *>(out) : nullptr,
+                                      fp8 ? out_scales : nullptr, rows, D, dtype, (cudaStream_t)stream));
+}
+
 size_t csa_topk_workspace_bytes(int Q, int N_max, int k) {
   if (Q < 1 || N_max < 1 || k < 1) return kStatusBytes;
   return kStatusBytes + align256(topk_scratch_bytes(Q, N_max, k));

@@ -56,6 +56,15 @@ struct CompressArgs {
   int dtype;
 };
 cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream);
+// The indexer's compressor (pool + RMSNorm + Hadamard rotation; D in 64..512,
+// a power of two): rows to a.out in a.dtype, or, with codes != nullptr, E4M3
+// codes at the same offsets and one scale per entry (sequence stride scale_ss).
+cudaError_t launch_index_compress(const CompressArgs &a, uint8_t *codes, float *scales, long long scale_ss,
+                                  cudaStream_t stream);
+// Hadamard rotation of rows x [rows, D] into out (dtype), or into E4M3 codes
+// + per-row scales when codes != nullptr.
+cudaError_t launch_hadamard_rows(const void *x, void *out, uint8_t *codes, float *scales, long long rows, int D,
+                                 int dtype, cudaStream_t stream);
 
 struct ScoreArgs {
   const void *qi;

@@ -118,6 +118,45 @@ def compress(kv, gate, ape, norm_w, win: int, stride: int, out=None, ratio=None)
     return out[0] if squeeze else out
 
 
+def index_compress(kv, gate, ape, norm_w, win: int, stride: int, fp8: bool = False):
+    """The indexer's own compressor (csa_index_compress): csa_compress's
+    entries rotated by the orthonormal Hadamard matrix. Returns [B, N, D] in
+    the input dtype, or (E4M3 codes uint8 [B, N, D], scales fp32 [B, N])."""
+    squeeze = kv.dim() == 2
+    if squeeze:
+        kv, gate = kv.unsqueeze(0), gate.unsqueeze(0)
+    _need(kv, "kv")
+    _need(gate, "gate", dtype=kv.dtype, device=kv.device)
+    _need(ape, "ape", dtype=torch.float32, device=kv.device)
+    _need(norm_w, "norm_w", dtype=torch.float32, device=kv.device)
+    B, T, D = kv.shape
+    N = (T - win) // stride + 1 if T >= win else 0
+    out = torch.empty((B, N, D), dtype=torch.uint8 if fp8 else kv.dtype, device=kv.device)
+    scales = torch.empty((B, N), dtype=torch.float32, device=kv.device) if fp8 else None
+    rc = _lib.lib().csa_index_compress(
+        _ptr(kv), _ptr(gate), _ptr(ape), _ptr(norm_w), int(stride), int(win), int(stride), _ptr(out),
+        _ptr(scales) if fp8 else None, B, T, D, 0, 0, 0, _dtype_code(kv),
+        _lib.CSA_DTYPE_E4M3 if fp8 else _dtype_code(kv), _stream(kv.device))
+    _lib.check("csa_index_compress", rc)
+    if squeeze:
+        return (out[0], scales[0]) if fp8 else out[0]
+    return (out, scales) if fp8 else out
+
+
+def hadamard_rows(x, fp8: bool = False):
+    """Orthonormal Hadamard rotation of the last dimension of x (csa_hadamard_rows):
+    same shape and dtype, or (E4M3 codes uint8, scales fp32 [x.shape[:-1]])."""
+    _need(x, "x")
+    D = x.shape[-1]
+    rows = x.numel() // D
+    out = torch.empty(x.shape, dtype=torch.uint8 if fp8 else x.dtype, device=x.device)
+    scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if fp8 else None
+    rc = _lib.lib().csa_hadamard_rows(_ptr(x), _ptr(out), _ptr(scales) if fp8 else None, rows, D, _dtype_code(x),
+                                      _lib.CSA_DTYPE_E4M3 if fp8 else _dtype_code(x), _stream(x.device))
+    _lib.check("csa_hadamard_rows", rc)
+    return (out, scales) if fp8 else out
+
+
 # ------------------------------------------------------------- A2 + A3
 
 def _index_common(qi, wi, ki, n_cmp, q_per_seq):

@@ -108,6 +108,34 @@ int csa_compress(const void *kv, const void *gate, const float *ape, const float
                  int dtype, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * csa_index_compress -- the indexer's own KV compressor, and
+ * csa_hadamard_rows -- the rotation of indexer query rows.
+ *
+ * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: the indexer
+ * "has its own dedicated KV compressor with Hadamard rotation". Entry j is
+ * csa_compress's entry (same windows, pool, RMSNorm, arguments and
+ * strides) rotated by the orthonormal Sylvester-Hadamard matrix:
+ *     out[b, j, :] = compress(...)[b, j, :] H_D / sqrt(D).
+ * csa_hadamard_rows rotates each row of x [rows, D] the same way (the
+ * indexer queries: scores are unchanged in exact arithmetic).
+ * out_dtype = dtype writes rows in the input dtype. out_dtype =
+ * CSA_DTYPE_E4M3 writes FP8 codes (uint8, same layout) and one float32 scale
+ * per row to out_scales ([B, N] with sequence stride out_seq_stride / D, or
+ * [rows]): scale = amax|row| / 448 (1 for a zero row), code = E4M3(v / scale)
+ * rounded to nearest even, saturating -- the inputs of csa_index_topk_fp8
+ * (the model's quantization_config: fmt e4m3, dynamic activation scales,
+ * "deepseek-ai/DeepSeek-V4-Flash-0731", table "Config changes").
+ * D must be 64, 128, 256 or 512; other limits and errors as csa_compress;
+ * out_scales must be a 4-byte aligned device pointer for FP8 output.
+ * ---------------------------------------------------------------------- */
+int csa_index_compress(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
+                       int stride, void *out, float *out_scales, int B, int T, int D, long long kv_seq_stride,
+                       long long gate_seq_stride, long long out_seq_stride, int dtype, int out_dtype,
+                       csa_stream_t stream);
+int csa_hadamard_rows(const void *x, void *out, float *out_scales, long long rows, int D, int dtype, int out_dtype,
+                      csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * csa_index_topk -- indexer scores and top-k selection of compressed entries.
  *
  * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1, Indexer: a
