@@ -8,6 +8,7 @@ from .csa_oracle import (  # noqa: F401
     as_f64,
     attend,
     compress,
+    compress_rope,
     e4m3_decode,
     e4m3_encode,
     hadamard_matrix,
@@ -22,6 +23,7 @@ from .csa_oracle import (  # noqa: F401
     n_visible,
     quantize_rows_e4m3,
     rms_norm,
+    rope_last_dims,
     round_to,
     sparse_mqa,
     topk,

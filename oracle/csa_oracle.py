@@ -61,6 +61,14 @@ the design notes):
   arithmetic. Rows become FP8 codes with one scale per row, amax / 448
   (dynamic scaling; a zero row gets scale 1), each value rounded to the
   nearest E4M3 value, ties to even, magnitudes above 448 saturating to 448.
+* R20 RoPE on the compressed entries (the next row f3; Architecture analysis,
+  INNOVATIONS section 1: "RoPE on rope dimensions of compressed KV", section
+  2: the last 64 of the 512 dims are the rope dims; ARCHITECTURE_SPEC:
+  compress_rope_theta 160000): after the pool + RMSNorm, the last 64 dims of
+  entry j are rotated in adjacent pairs (d, d + 1) by the angle
+  p_j * theta^(-2i / 64) for pair i, with p_j = pos0 + j * stride + win - 1,
+  the absolute position of the entry's last token (pos0: the position of the
+  sequence's raw token 0). Plain RoPE, no frequency scaling.
 
 Pins (tests/test_oracle_pins.py) tie every function to something other than
 itself: closed forms, textbook/library special cases (torch rms_norm,
@@ -147,6 +155,32 @@ def compress(kv, gate, ape, norm_w, win: int, stride: int, eps: float = RMS_EPS,
 # ---------------------------------------------------------------------------
 # Causal visibility of compressed entries
 # ---------------------------------------------------------------------------
+
+def rope_last_dims(x, positions, theta: float, rope_dims: int = 64) -> np.ndarray:
+    """Rotate the last `rope_dims` dims of each row of x in adjacent pairs
+    (reading R20): pair i = (d, d + 1), d = D - rope_dims + 2 i, by the angle
+    positions[row] * theta^(-2 i / rope_dims)."""
+    y = as_f64(x).copy()
+    pos = np.asarray(positions, dtype=np.float64)
+    D = y.shape[-1]
+    i = np.arange(rope_dims // 2, dtype=np.float64)
+    ang = pos[:, None] * theta ** (-2.0 * i / rope_dims)[None, :]        # [rows, pairs]
+    c, s_ = np.cos(ang), np.sin(ang)
+    a = y[:, D - rope_dims::2].copy()
+    b = y[:, D - rope_dims + 1::2].copy()
+    y[:, D - rope_dims::2] = a * c - b * s_
+    y[:, D - rope_dims + 1::2] = a * s_ + b * c
+    return y
+
+
+def compress_rope(kv, gate, ape, norm_w, win: int, stride: int, pos0: int, theta: float, rope_dims: int = 64,
+                  eps: float = RMS_EPS) -> np.ndarray:
+    """A1 followed by RoPE on the entries' last dims (reading R20): entry j at
+    the position of its last token, pos0 + j * stride + win - 1."""
+    c = compress(kv, gate, ape, norm_w, win, stride, eps)
+    p = pos0 + np.arange(c.shape[0]) * stride + win - 1
+    return rope_last_dims(c, p, theta, rope_dims)
+
 
 def n_visible(p: int, win: int, stride: int) -> int:
     """Entries whose every token is at or before position p (reading R6):

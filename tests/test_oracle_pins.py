@@ -320,6 +320,49 @@ def scipy_hadamard(n):
     return scipy.linalg.hadamard(n).astype(np.float64)
 
 
+# ------------------------------------------------------- RoPE on compressed entries (R20)
+
+def test_rope_closed_form_one_pair():
+    # rope_dims 2: the single pair rotates by the angle p * theta^0 = p
+    x = np.array([[0.0, 0.0, 3.0, 4.0]])
+    for p in (0.0, 1.0, 2.5):
+        y = O.rope_last_dims(x, [p], 160000.0, rope_dims=2)
+        assert np.allclose(y[0], [0.0, 0.0, 3 * math.cos(p) - 4 * math.sin(p), 3 * math.sin(p) + 4 * math.cos(p)],
+                           rtol=0, atol=1e-15)
+
+
+def test_rope_frequencies_follow_theta():
+    # pair i of 64 rope dims turns by p * theta^(-i/32): a unit vector on pair i
+    # ends at angle p * theta^(-i/32) (complex multiplication by e^{i angle})
+    theta, p = 160000.0, 37.0
+    for i in (0, 1, 17, 31):
+        x = np.zeros((1, 512))
+        x[0, 448 + 2 * i] = 1.0
+        y = O.rope_last_dims(x, [p], theta)
+        z = complex(y[0, 448 + 2 * i], y[0, 449 + 2 * i])
+        ang = p * theta ** (-i / 32)
+        assert abs(z - complex(math.cos(ang), math.sin(ang))) < 1e-12
+
+
+def test_rope_dot_products_depend_only_on_the_offset():
+    q, k = rng.standard_normal((1, 512)), rng.standard_normal((1, 512))
+    dots = [float((O.rope_last_dims(q, [p + 100.0], 160000.0) @ O.rope_last_dims(k, [p], 160000.0).T)[0, 0])
+            for p in (0.0, 1000.0, 123456.0)]
+    assert np.allclose(dots, dots[0], rtol=1e-9)
+    assert np.allclose(np.linalg.norm(O.rope_last_dims(q, [5e5], 160000.0)), np.linalg.norm(q))
+
+
+def test_compress_rope_positions_are_the_last_tokens():
+    T, D = 40, 128
+    kv, gate = rng.standard_normal((T, D)), rng.standard_normal((T, D))
+    ape = rng.standard_normal((8, D)) * 0.1
+    base = O.compress(kv, gate, ape, np.ones(D), 8, 4)
+    got = O.compress_rope(kv, gate, ape, np.ones(D), 8, 4, pos0=1000, theta=160000.0)
+    assert np.array_equal(got[:, :64], base[:, :64])
+    want = O.rope_last_dims(base, 1000 + 4 * np.arange(base.shape[0]) + 7, 160000.0)
+    assert np.allclose(got, want, rtol=0, atol=1e-15)
+
+
 def test_topk_closed_form_ties():
     g = _golden("topk_ties.json")
     for case in g["cases"]:
