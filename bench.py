@@ -566,7 +566,7 @@ def main():
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
-        for name in ("hca_decode_1m", "csa_decode_1m", "csa_decode_64k_fp8"):
+        for name in ("hca_decode_1m", "csa_decode_1m", "csa_decode_64k_fp8", "csa_decode_64k_pro"):
             if name == w.name:
                 continue
             sw = WL.WORKLOADS[name]

@@ -1,5 +1,7 @@
 // A4 / A5 on the tensor cores for the Flash attention shape: 64 query heads,
-// one shared KV head, head_dim 512, K = V, bf16 in, fp32 accumulation
+// one shared KV head, head_dim 512, K = V, bf16 in, fp32 accumulation; the
+// V4-Pro shape (128 heads) runs as two 64-head groups per query, one block
+// row each, reading the same KV rows (the second read mostly from L2)
 // ("DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: sliding window
 // + compressed rows + per-head attention sink; section 2: keys and values
 // share one 512-dim representation).
@@ -217,7 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *ps = qs + kQBytes;                      // [2][64 rows][128 B]  (P^T, MN-major)
   Small *sm = reinterpret_cast<Small *>(ps + 2 * kPBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, qq = blockIdx.y;
+  // blockIdx.y = qv: one group of 64 heads of query qq (H = 64 G)
+  const int G = a.H / kH;
+  const int split = blockIdx.x, qv = blockIdx.y, qq = qv / G, hg = qv - qq * G;
   const int b = qq / a.q_per_seq;
 
   if (threadIdx.x == 0) {
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::prefetch_tmap(&tm_q);
         tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
         for (int bx = 0; bx < kD / 64; ++bx)
-          tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qq * kH, &sm->q_full);
+          tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qv * kH, &sm->q_full);
         q_issued = true;
       }
       constexpr uint32_t idesc_s = tc::idesc_bf16(64, 64, 0, 0);
@@ -622,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (splits > 1) {
       // This split's unnormalised O (fp32, [64 heads][512 dims]) and its
       // (mref, lsum) go to the workspace, for the cluster merge below.
-      const size_t pidx = (size_t)qq * splits + split;
+      const size_t pidx = (size_t)qv * splits + split;
       if (leader) {
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -655,14 +659,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int h = 2 * lane + i;
-          const float mr = sm->mref[h], sk = a.sink[h] * kLog2e;
+          const float mr = sm->mref[h], sk = a.sink[hg * kH + h] * kLog2e;
           const float M = fmaxf(mr, sk);
           const float wm = mr == -INFINITY ? 0.f : exp2f(mr - M);
           sm->alpha[h] = wm / (sm->lsum[h] * wm + exp2f(sk - M));
         }
       }
       named_sync(1, 128);
-      bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qq * kH * kD;
+      bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qv * kH * kD;
 #pragma unroll 1
       for (int m = 0; m < 4; ++m) {
         const int d = 128 * m + orow;
@@ -692,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     //   out = sum_s O_s 2^(m_s - M) / L   (m and sink in log2 units).
     cluster_sync();
     float *coef = reinterpret_cast<float *>(ps);  // [splits][64]: 2^(m_s - M) / L
-    const float *pml = part_ml + (size_t)qq * splits * 2 * kH;
+    const float *pml = part_ml + (size_t)qv * splits * 2 * kH;
     if (threadIdx.x < kH) {
       const int h = threadIdx.x;
       float mr[kMaxSplits], lr[kMaxSplits];
@@ -702,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mr[r] = pml[(2 * r) * kH + h];
           lr[r] = pml[(2 * r + 1) * kH + h];
         }
-      const float sk = a.sink[h] * kLog2e;
+      const float sk = a.sink[hg * kH + h] * kLog2e;
       float M = sk;
 #pragma unroll
       for (int r = 0; r < kMaxSplits; ++r)
@@ -720,8 +724,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (r < splits) coef[r * kH + h] = w[r] * inv;
     }
     __syncthreads();
-    const float *po = part_o + (size_t)qq * splits * kH * kD;
-    bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qq * kH * kD;
+    const float *po = part_o + (size_t)qv * splits * kH * kD;
+    bf16 *out = static_cast<bf16 *>(a.out) + (size_t)qv * kH * kD;
     constexpr int kGroups = kH * kD / 4;  // 4-dim groups of the output
     const int g0 = split * kGroups / splits, g1 = (split + 1) * kGroups / splits;
     // Batches of groups with every partial load in flight before the sums
@@ -740,9 +744,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (query, head); thread t owns dims 4t..4t+3 and issues the loads of all
 // splits at once. Same formula as the in-kernel merge.
 __global__ void __launch_bounds__(128) mqa_combine_kernel(const float *part_o, const float *part_ml,
-                                                          const float *sink, bf16 *out, int splits) {
+                                                          const float *sink, bf16 *out, int splits, int G) {
   extern __shared__ float w[];  // [splits] weights, then [2][splits] (m, l)
-  const int qq = blockIdx.x, h = blockIdx.y;
+  const int qq = blockIdx.x, h = blockIdx.y;  // qq: a group of 64 heads of query qq / G
   pdl_wait();
   pdl_release();
   float *ml = w + splits;
@@ -752,7 +756,7 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const float *part_o, c
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const float sk = sink[h] * kLog2e;
+    const float sk = sink[(qq % G) * kH + h] * kLog2e;
     float M = sk;
     for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, ml[sp]);
     float Lsum = exp2f(sk - M);
@@ -869,7 +873,8 @@ void plan_splits(int Q, int rows_max, int *splits, int *tiles_per_split, bool *c
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 bool tc_shape(const MqaArgs &a) {
-  return a.dtype == CSA_DTYPE_BF16 && a.H == kH && a.D == kD && a.Q <= 65535 && aligned16(a.q) &&
+  return a.dtype == CSA_DTYPE_BF16 && (a.H == kH || a.H == 2 * kH) && a.D == kD &&
+         (long long)a.Q * (a.H / kH) <= 65535 && aligned16(a.q) &&
          aligned16(a.kv_cmp) && aligned16(a.kv_win) && aligned16(a.out);
 }
 
@@ -880,7 +885,8 @@ int rows_max_of(const MqaArgs &a) { return (((a.idx ? a.k : a.N_max) + 3) & ~3) 
 // Upper bound on the split partials for any row list of at most rows_max
 // rows (+3 rows of padding): Q x min(tiles, SMs / Q, 16) x 64 x (512 + 2) fp32.
 size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
-  if (H != kH || D != kD || Q < 1) return 0;
+  if ((H != kH && H != 2 * kH) || D != kD || Q < 1) return 0;
+  Q *= H / kH;  // one row list per group of 64 heads
   const int tiles = (rows_max + 3 + kRows - 1) / kRows;
   int s = num_sms_cached() / Q;
   s = s > kMaxSplits ? kMaxSplits : s;
@@ -894,25 +900,26 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   if (!tc_shape(a)) return cudaSuccess;
   int splits, tps;
   bool cluster_merge;
-  plan_splits(a.Q, rows_max_of(a), &splits, &tps, &cluster_merge);
+  const int G = a.H / kH, QV = a.Q * G;  // blocks per split: one per group of 64 heads of a query
+  plan_splits(QV, rows_max_of(a), &splits, &tps, &cluster_merge);
   CUtensorMap tm_q, tm_cmp_t, tm_win_t;
   const uint64_t cmp_rows = (uint64_t)a.B * a.N_max, win_rows = (uint64_t)a.B * a.T_raw;
-  if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * kH, kD * 2, 64, kH) ||
+  if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * a.H, kD * 2, 64, kH) ||
       !make_tmap_bf16_2d(&tm_cmp_t, a.kv_cmp, kD, cmp_rows, kD * 2, 64, kRows) ||
       !make_tmap_bf16_2d(&tm_win_t, a.kv_win, kD, win_rows, kD * 2, 64, kRows))
     return cudaSuccess;
-  const size_t need = splits > 1 ? (size_t)a.Q * splits * kH * (kD + 2) * sizeof(float) : 0;
+  const size_t need = splits > 1 ? (size_t)QV * splits * kH * (kD + 2) * sizeof(float) : 0;
   if (need > a.partial_bytes) return cudaSuccess;  // cannot happen with the documented workspace size
   float *part_o = static_cast<float *>(a.partials);
-  float *part_ml = part_o + (size_t)a.Q * splits * kH * kD;
+  float *part_ml = part_o + (size_t)QV * splits * kH * kD;
   set_kernel_attributes();
   *taken = true;
-  cudaError_t e = launch_pdl_cluster(mqa_tc_kernel, dim3(splits, a.Q), dim3(kThreads), kSmemBytes, stream,
+  cudaError_t e = launch_pdl_cluster(mqa_tc_kernel, dim3(splits, QV), dim3(kThreads), kSmemBytes, stream,
                                      cluster_merge ? (unsigned)splits : 1u, tm_q, tm_cmp_t, tm_win_t, a, splits, tps,
                                      a.scale * kLog2e, part_o, part_ml, (int)cluster_merge);
   if (e != cudaSuccess || splits <= 1 || cluster_merge) return e;
-  return launch_pdl(mqa_combine_kernel, dim3(a.Q, kH), dim3(kD / 4), splits * 3 * sizeof(float), stream,
-                    (const float *)part_o, (const float *)part_ml, a.sink, static_cast<bf16 *>(a.out), splits);
+  return launch_pdl(mqa_combine_kernel, dim3(QV, kH), dim3(kD / 4), splits * 3 * sizeof(float), stream,
+                    (const float *)part_o, (const float *)part_ml, a.sink, static_cast<bf16 *>(a.out), splits, G);
 }
 
 }  // namespace csa

@@ -116,6 +116,11 @@ WORKLOADS = {
         name="csa_decode_1m", dtype=torch.bfloat16, B=8, Q=8, H=64, D=512, Hi=64, Di=128, k=1024, W=128,
         N=262143, T_raw=128, pos0=1048575, raw0=1048448, T_c=8, c_src0=120, c_dst0=262142, bulk_T=1048576),
 }
+# The 64K decode batch in the V4-Pro attention shape: 128 query heads, top-1024
+# ("DeepSeek-V4 Architecture Analysis", ARCHITECTURE_SPEC["DeepSeek-V4-Pro"]:
+# num_heads 128, index_topk 1024, the same 512-dim head and 64 x 128 indexer).
+WORKLOADS["csa_decode_64k_pro"] = dataclasses.replace(WORKLOADS["csa_decode_64k"], name="csa_decode_64k_pro",
+                                                      H=128, k=1024)
 # The 64K decode batch with the FP8 (E4M3) indexer.
 WORKLOADS["csa_decode_64k_fp8"] = dataclasses.replace(WORKLOADS["csa_decode_64k"], name="csa_decode_64k_fp8",
                                                       index_fmt="e4m3")

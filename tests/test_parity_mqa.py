@@ -32,6 +32,7 @@ def _dev(cuda_device, *ts):
     (4, 2, 100, 64, 64, 512, 40, 128, torch.bfloat16),   # window clipped by T_raw/sequence start
     (3, 1, 50, 30, 8, 64, 7, 5, torch.bfloat16),         # small odd shapes (generic kernel)
     (4, 4, 300, 40, 64, 512, 200, 16, torch.float32),
+    (4, 2, 2000, 200, 128, 512, 1024, 128, torch.bfloat16),  # V4-Pro: 128 heads (two 64-head groups), top-1024
 ])
 def test_sparse_mqa_matches_oracle(cuda_device, Q, B, N, T_raw, H, D, k, W, dtype):
     q, kv_cmp, kv_win, sink = _mqa_inputs(1, Q, B, N, T_raw, H, D, dtype)
@@ -54,6 +55,7 @@ def test_sparse_mqa_matches_oracle(cuda_device, Q, B, N, T_raw, H, D, k, W, dtyp
     (8, 8, 1000, 128, 64, 512, 128, torch.bfloat16),
     (6, 2, 333, 150, 64, 512, 128, torch.bfloat16),
     (16, 1, 40, 64, 4, 16, 16, torch.float32),
+    (5, 5, 700, 128, 128, 512, 128, torch.bfloat16),    # V4-Pro: 128 heads
 ])
 def test_hca_mqa_matches_oracle(cuda_device, Q, B, N, T_raw, H, D, W, dtype):
     q, kv_cmp, kv_win, sink = _mqa_inputs(2, Q, B, N, T_raw, H, D, dtype)
