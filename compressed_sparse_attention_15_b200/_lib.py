@@ -26,6 +26,8 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "csa_strerror": (ctypes.c_char_p, [_I]),
     "csa_compress": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _LL, _LL, _LL, _I, _P]),
+    "csa_compress_rope": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _LL, _LL, _LL, _I, ctypes.c_double, _P, _I,
+                               _P]),
     "csa_index_compress": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _LL, _LL, _LL, _I, _I, _P]),
     "csa_hadamard_rows": (_I, [_P, _P, _P, _LL, _I, _I, _I, _P]),
     "csa_index_topk_workspace_bytes": (_SZ, [_I, _I, _I]),

@@ -34,6 +34,30 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRmsEps = 1e-6f;
 
+// RoPE of the pair (x0, x1) = dims (d, d + 1), d even, of entry j of sequence
+// b when d lies in the rope dims (the last a.rope_dims). The angle is formed
+// and reduced in double: positions reach 2^20 and beyond, where a float angle
+// would keep no fractional bits.
+__device__ __forceinline__ void rope_pair(const CompressArgs &a, int b, int j, int d, float &x0, float &x1) {
+  const int d0 = a.D - a.rope_dims;
+  if (a.rope_dims == 0 || d < d0) return;
+  const double p = (double)((a.pos0 ? a.pos0[b] : 0) + (long long)j * a.stride + a.win - 1);
+  const double ang = p * pow(a.rope_theta, -(double)(d - d0) / a.rope_dims);  // pair (d - d0) / 2
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  const float c = (float)cs, s = (float)sn;
+  const float y0 = x0 * c - x1 * s, y1 = x0 * s + x1 * c;
+  x0 = y0;
+  x1 = y1;
+}
+
+// RoPE of 8 consecutive dims [d, d + 8) held by one thread (d a multiple of 8).
+__device__ __forceinline__ void rope8(const CompressArgs &a, int b, int j, int d, float (&c)[8]) {
+  if (a.rope_dims == 0 || d + 8 <= a.D - a.rope_dims) return;
+#pragma unroll
+  for (int m = 0; m < 8; m += 2) rope_pair(a, b, j, d + m, c[m], c[m + 1]);
+}
+
 // ------------------------------------------------------------------ generic
 
 template <typename T>
@@ -73,7 +97,19 @@ __global__ void __launch_bounds__(256) compress_generic_kernel(CompressArgs a) {
     const float r = 1.0f / sqrtf(ss / (float)a.D + kRmsEps);
     __syncwarp();
     T *o = out + b * a.out_ss + (long long)j * a.D;
-    for (int d = lane; d < a.D; d += 32) o[d] = from_f<T>(c[d] * r * a.norm_w[d]);
+    for (int d = lane; d < a.D; d += 32) {
+      float x = c[d] * r * a.norm_w[d];
+      if (a.rope_dims) {  // the pair partner comes from shared memory
+        const int dp = d ^ 1;
+        float y = c[dp] * r * a.norm_w[dp];
+        if (d & 1) {
+          rope_pair(a, b, j, dp, y, x);
+        } else {
+          rope_pair(a, b, j, d, x, y);
+        }
+      }
+      o[d] = from_f<T>(x);
+    }
     __syncwarp();
   }
 }
@@ -252,7 +288,15 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
         if (r < (int)C) tot += sr[r];
       const float rn = 1.0f / sqrtf(tot / (float)a.D + kRmsEps);
       bf16 *o = static_cast<bf16 *>(a.out) + b * a.out_ss + (long long)j * a.D;
-      o[d] = __float2bfloat16_rn(cd * rn * a.norm_w[d]);
+      float x = cd * rn * a.norm_w[d];
+      if (a.rope_dims) {  // the pair partner is the neighbouring thread's dim
+        float y = __shfl_xor_sync(0xffffffffu, x, 1);
+        if (d & 1)
+          rope_pair(a, b, j, d - 1, y, x);
+        else
+          rope_pair(a, b, j, d, x, y);
+      }
+      o[d] = __float2bfloat16_rn(x);
     }
     cluster_sync();  // no block leaves while a peer may still read its share
     return;
@@ -271,6 +315,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
 #pragma unroll
     for (int k = 0; k < 8; ++k) c[k] = blk[k * nvec + t] * rn * nw[k];
     bf16 *o = static_cast<bf16 *>(a.out) + b * a.out_ss + (long long)j * a.D;
+    rope8(a, b, j, 8 * t, c);
     reinterpret_cast<uint4 *>(o)[t] = pack8(c);
   }
 }
@@ -373,6 +418,7 @@ __global__ void __launch_bounds__(256) compress_stream_kernel(CompressArgs a, lo
     const float r = 1.0f / sqrtf(ss / (float)D + kRmsEps);
 #pragma unroll
     for (int k = 0; k < 8; ++k) c[k] = c[k] * r * nw[k];
+    rope8(a, b, j, 8 * v, c);
     reinterpret_cast<uint4 *>(out + b * a.out_ss + (long long)j * D)[v] = pack8(c);
 #pragma unroll
     for (int i = 0; i < S; ++i) {

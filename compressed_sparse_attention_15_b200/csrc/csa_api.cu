@@ -62,15 +62,19 @@ const char *csa_strerror(int code) {
   }
 }
 
-int csa_compress(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
-                 int stride, void *out, int B, int T, int D, long long kv_seq_stride, long long gate_seq_stride,
-                 long long out_seq_stride, int dtype, csa_stream_t stream) {
+static int compress_common(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio,
+                           int win, int stride, void *out, int B, int T, int D, long long kv_seq_stride,
+                           long long gate_seq_stride, long long out_seq_stride, int dtype, int rope_dims,
+                           double rope_theta, const int64_t *pos0, csa_stream_t stream) {
   if (!kv || !gate || !ape || !norm_w || !out) return CSA_ERR_INVALID;
   if (!dtype_ok(dtype) || B < 1 || D < 1 || D > 4096 || win < 1 || win > 128 || stride < 1) return CSA_ERR_INVALID;
   if (ratio != stride || T < win) return CSA_ERR_INVALID;
   if (kv_seq_stride < 0 || gate_seq_stride < 0 || out_seq_stride < 0) return CSA_ERR_INVALID;
   if (!elem_aligned(kv, dtype) || !elem_aligned(gate, dtype) || !elem_aligned(out, dtype)) return CSA_ERR_INVALID;
   if ((reinterpret_cast<uintptr_t>(ape) | reinterpret_cast<uintptr_t>(norm_w)) & 3) return CSA_ERR_INVALID;
+  if (rope_dims < 0 || rope_dims > D || rope_dims % 8 || (rope_dims && !(rope_theta > 1.0)) ||
+      (reinterpret_cast<uintptr_t>(pos0) & 7))
+    return CSA_ERR_INVALID;
   const int N = (T - win) / stride + 1;
   const long long kv_ss = kv_seq_stride ? kv_seq_stride : (long long)T * D;
   const long long g_ss = gate_seq_stride ? gate_seq_stride : (long long)T * D;
@@ -78,7 +82,25 @@ int csa_compress(const void *kv, const void *gate, const float *ape, const float
   if (B > 1 && (kv_ss < (long long)T * D || g_ss < (long long)T * D || o_ss < (long long)N * D)) return CSA_ERR_INVALID;
   if (!device_ok()) return CSA_ERR_UNSUPPORTED;
   CompressArgs a{kv, gate, ape, norm_w, out, B, T, D, win, stride, N, kv_ss, g_ss, o_ss, dtype};
+  a.rope_dims = rope_dims;
+  a.rope_theta = rope_theta;
+  a.pos0 = pos0;
   return cuda_rc(launch_compress(a, (cudaStream_t)stream));
+}
+
+int csa_compress(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
+                 int stride, void *out, int B, int T, int D, long long kv_seq_stride, long long gate_seq_stride,
+                 long long out_seq_stride, int dtype, csa_stream_t stream) {
+  return compress_common(kv, gate, ape, norm_w, ratio, win, stride, out, B, T, D, kv_seq_stride, gate_seq_stride,
+                         out_seq_stride, dtype, 0, 0.0, nullptr, stream);
+}
+
+int csa_compress_rope(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
+                      int stride, void *out, int B, int T, int D, long long kv_seq_stride, long long gate_seq_stride,
+                      long long out_seq_stride, int rope_dims, double rope_theta, const int64_t *pos0, int dtype,
+                      csa_stream_t stream) {
+  return compress_common(kv, gate, ape, norm_w, ratio, win, stride, out, B, T, D, kv_seq_stride, gate_seq_stride,
+                         out_seq_stride, dtype, rope_dims, rope_theta, pos0, stream);
 }
 
 static bool pow2_dim(int D) { return D == 64 || D == 128 || D == 256 || D == 512; }

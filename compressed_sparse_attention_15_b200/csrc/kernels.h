@@ -54,6 +54,12 @@ struct CompressArgs {
   int B, T, D, win, stride, N;
   long long kv_ss, gate_ss, out_ss;  // sequence strides in elements
   int dtype;
+  // RoPE on the last rope_dims dims of each entry (0: none): entry j of
+  // sequence b at position pos0[b] + j * stride + win - 1, pair i turning by
+  // that position times rope_theta^(-2 i / rope_dims).
+  int rope_dims = 0;
+  double rope_theta = 0.0;
+  const int64_t *pos0 = nullptr;
 };
 cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream);
 // The indexer's compressor (pool + RMSNorm + Hadamard rotation; D in 64..512,

@@ -83,8 +83,10 @@ def visible_entries(p: torch.Tensor, win: int, stride: int) -> torch.Tensor:
 
 # ------------------------------------------------------------------ A1
 
-def compress(kv, gate, ape, norm_w, win: int, stride: int, out=None, ratio=None):
-    """Gated-pooling compressor + RMSNorm (csa_compress).
+def compress(kv, gate, ape, norm_w, win: int, stride: int, out=None, ratio=None, rope=None):
+    """Gated-pooling compressor + RMSNorm (csa_compress); with
+    rope = (rope_dims, theta, pos0 int64 [B] or None), RoPE on the entries'
+    last rope_dims dims as well (csa_compress_rope).
 
     kv, gate: [B, T, D] (or [T, D]) with contiguous rows and any sequence
     stride; ape [win, D] fp32; norm_w [D] fp32. Returns / fills out
@@ -110,11 +112,21 @@ def compress(kv, gate, ape, norm_w, win: int, stride: int, out=None, ratio=None)
         _need(out, "out", dtype=kv.dtype, device=kv.device, contiguous=False)
         if out.shape != (B, N, D) or out.stride(2) != 1 or out.stride(1) != D:
             raise ValueError("out must be [B, N, D] with contiguous [N, D] rows")
-    rc = _lib.lib().csa_compress(
-        _ptr(kv), _ptr(gate), _ptr(ape), _ptr(norm_w), int(stride if ratio is None else ratio), int(win),
-        int(stride), _ptr(out), B, T, D, kv.stride(0), gate.stride(0), out.stride(0), _dtype_code(kv),
-        _stream(kv.device))
-    _lib.check("csa_compress", rc)
+    if rope is None:
+        rc = _lib.lib().csa_compress(
+            _ptr(kv), _ptr(gate), _ptr(ape), _ptr(norm_w), int(stride if ratio is None else ratio), int(win),
+            int(stride), _ptr(out), B, T, D, kv.stride(0), gate.stride(0), out.stride(0), _dtype_code(kv),
+            _stream(kv.device))
+        _lib.check("csa_compress", rc)
+    else:
+        rope_dims, theta, pos0 = rope
+        if pos0 is not None:
+            _need(pos0, "pos0", dtype=torch.int64, device=kv.device)
+        rc = _lib.lib().csa_compress_rope(
+            _ptr(kv), _ptr(gate), _ptr(ape), _ptr(norm_w), int(stride if ratio is None else ratio), int(win),
+            int(stride), _ptr(out), B, T, D, kv.stride(0), gate.stride(0), out.stride(0), int(rope_dims),
+            float(theta), _ptr(pos0) if pos0 is not None else None, _dtype_code(kv), _stream(kv.device))
+        _lib.check("csa_compress_rope", rc)
     return out[0] if squeeze else out
 
 

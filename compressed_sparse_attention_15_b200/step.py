@@ -3,7 +3,8 @@ CUDA graph.
 
 The step over device-resident caches is:
   1. fold the newest raw window of every sequence into its compressed cache
-     (csa_compress; CSA every 4 tokens, HCA every 128) -- on a forked stream,
+     (csa_compress, or csa_compress_rope with RoPE on the new entry's rope
+     dims; CSA every 4 tokens, HCA every 128) -- on a forked stream,
      concurrently with 2 when the layer is CSA;
   2. CSA only: score every visible compressed entry and select the top-k
      (csa_index_topk, or csa_index_topk_fp8 with FP8 indexer inputs);
@@ -24,7 +25,7 @@ class DecodeStep:
     def __init__(self, *, q, kv_cmp, kv_win, sink, scale: float, win_len: int, win_end, n_cmp,
                  ape, norm_w, gate, append_src0: int, append_dst0: int, win: int, stride: int,
                  qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True,
-                 qi8=None, sq=None, ki8=None, sk=None):
+                 qi8=None, sq=None, ki8=None, sk=None, append_rope=None):
         self.fp8 = qi8 is not None
         self.csa = qi is not None or self.fp8
         self.q, self.kv_cmp, self.kv_win, self.sink = q, kv_cmp, kv_win, sink
@@ -37,6 +38,7 @@ class DecodeStep:
         self.cmp_dst = kv_cmp[:, append_dst0:append_dst0 + n_new]
         self.qi, self.wi, self.ki, self.k = qi, wi, ki, k
         self.qi8, self.sq, self.ki8, self.sk = qi8, sq, ki8, sk
+        self.append_rope = append_rope  # (rope_dims, theta, pos0 int64 [B]): RoPE fused into the append
         dev = q.device
         self.out = out if out is not None else torch.empty_like(q)
         self.idx = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev) if self.csa else None
@@ -54,7 +56,8 @@ class DecodeStep:
 
     # -- the parts, on the current stream --------------------------------
     def append(self):
-        ops.compress(self.kv_src, self.gate, self.ape, self.norm_w, self.win, self.stride, out=self.cmp_dst)
+        ops.compress(self.kv_src, self.gate, self.ape, self.norm_w, self.win, self.stride, out=self.cmp_dst,
+                     rope=self.append_rope)
 
     def select(self):
         if self.fp8:

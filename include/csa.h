@@ -108,6 +108,29 @@ int csa_compress(const void *kv, const void *gate, const float *ape, const float
                  int dtype, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * csa_compress_rope -- csa_compress with RoPE on the entries' rope dims,
+ * fused: the cache append of a decode step.
+ *
+ * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1 (the compressor
+ * applies "RoPE on rope dimensions of compressed KV"), section 2 (the last
+ * qk_rope_head_dim = 64 of the 512 dims are the rope dims) and
+ * ARCHITECTURE_SPEC (compress_rope_theta = 160000). After the pool and the
+ * RMSNorm, the last rope_dims dims of entry j of sequence b are rotated in
+ * adjacent pairs (d, d + 1), pair i by the angle
+ *     (pos0[b] + j * stride + win - 1) * rope_theta^(-2 i / rope_dims),
+ * the position of the entry's last raw token (pos0[b]: the absolute position
+ * of kv[b, 0]; the angle is formed in double precision).
+ * Arguments as csa_compress, plus rope_dims (a multiple of 8, <= D; 0 gives
+ * csa_compress), rope_theta (> 1) and pos0 (int64 [B] device array, 8-byte
+ * aligned, or NULL for all zeros). Errors as csa_compress, CSA_ERR_INVALID
+ * also for a bad rope_dims / rope_theta / pos0.
+ * ---------------------------------------------------------------------- */
+int csa_compress_rope(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
+                      int stride, void *out, int B, int T, int D, long long kv_seq_stride, long long gate_seq_stride,
+                      long long out_seq_stride, int rope_dims, double rope_theta, const int64_t *pos0, int dtype,
+                      csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * csa_index_compress -- the indexer's own KV compressor, and
  * csa_hadamard_rows -- the rotation of indexer query rows.
  *

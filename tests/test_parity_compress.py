@@ -97,3 +97,26 @@ def test_compress_full_1m_tokens_sampled(cuda_device):
         toks = torch.arange(4 * j, 4 * j + 8)
         ref.append(O.compress(WL.rows(w, "kv_raw", toks), WL.rows(w, "gate_raw", toks), ape_h, np.ones(512), 8, 4)[0])
     assert_close(got, np.stack(ref), torch.bfloat16, "compress 1M sampled")
+
+
+@pytest.mark.parametrize("B,T,D,win,stride,dtype", [
+    (3, 1003, 512, 8, 4, torch.bfloat16),     # many entries: the streaming kernel
+    (32, 8, 512, 8, 4, torch.bfloat16),       # the decode append: one entry per sequence (window kernel)
+    (2, 1000, 512, 128, 128, torch.bfloat16),  # HCA windows: a cluster of blocks per entry
+    (2, 300, 64, 8, 4, torch.float32),        # the generic kernel (pairs split across lanes)
+    (2, 100, 128, 8, 4, torch.bfloat16),      # generic kernel, bf16
+])
+def test_compress_rope_matches_oracle(cuda_device, B, T, D, win, stride, dtype):
+    # row f3 (reading R20): the pool + RMSNorm + RoPE on the last 64 dims at
+    # each entry's last-token position, with large absolute positions
+    kv, gate, ape, w, dev = _inputs(5, B, T, D, win, dtype, cuda_device)
+    pos0 = torch.tensor([[0, 65408 + 120, 1048448, 7][b % 4] + 3 * b for b in range(B)], dtype=torch.int64)
+    rd = min(64, D)
+    out = ops.compress(*dev, win, stride, rope=(rd, 160000.0, pos0.to(cuda_device)))
+    torch.cuda.synchronize()
+    ref = np.stack([O.compress_rope(kv[b], gate[b], ape, w, win, stride, int(pos0[b]), 160000.0, rd)
+                    for b in range(B)])
+    assert_close(out, ref, dtype, f"compress+rope B{B} T{T} D{D} win{win}")
+    # the dims before the rope dims are exactly csa_compress's
+    plain = ops.compress(*dev, win, stride)
+    assert torch.equal(out[..., :D - rd], plain[..., :D - rd])
