@@ -74,6 +74,8 @@ def algo_bytes(w: WL.Workload):
         b["topk"] = w.Q * w.k * 4
         rows = w.k + w.W
         b["mqa"] = w.Q * (rows * w.D * e + 2 * w.H * w.D * e + w.k * 4 + w.H * 4)
+        # selection inside the attention: the indices are written, not read back
+        b["topk_mqa"] = b["mqa"]
     else:
         rows = n_vis + w.W
         b["mqa"] = w.Q * (rows * w.D * e + 2 * w.H * w.D * e + w.H * 4)
@@ -88,6 +90,8 @@ def algo_flops(w: WL.Workload):
     else:
         rows = w.N + w.W
     f["mqa"] = w.Q * rows * w.H * w.D * 4
+    if w.mode == "csa":
+        f["topk_mqa"] = f["mqa"]
     return f
 
 
@@ -150,10 +154,11 @@ class Step:
 
     def parts(self):
         """The step's kernels one call at a time (per-kernel timing and the
-        profiling aid). The CSA select call is split into its two kernels,
-        scores then top-k, through their own entry points."""
+        profiling aid). Without the fused selection, the CSA select call is
+        split into its two kernels, scores then top-k, through their own entry
+        points."""
         ds = self.ds
-        if not ds.csa:
+        if not ds.csa or ds.fuse_select:
             return ds.parts()
         if self._scores is None:
             self._scores = torch.empty((self.w.Q, self.w.N), dtype=torch.float32, device=self.dev)

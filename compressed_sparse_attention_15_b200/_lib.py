@@ -40,6 +40,9 @@ SIGNATURES = {
     "csa_mqa_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "csa_sparse_mqa": (_I, [_P, _P, _P, _P, _P, _F, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _P, _SZ, _P]),
     "hca_mqa": (_I, [_P, _P, _P, _P, _F, _P, _I, _I, _I, _I, _I, _P, _I, _P, _I, _I, _I, _P, _SZ, _P]),
+    "csa_topk_sparse_mqa_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "csa_topk_sparse_mqa": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _F, _P, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _P,
+                                 _SZ, _P]),
     "csa_workspace_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "csa_launch_count": (ctypes.c_ulonglong, []),
     "csa_index_topk_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),

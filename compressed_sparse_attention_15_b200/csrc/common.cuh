@@ -97,6 +97,14 @@ __device__ __forceinline__ uint32_t ld_peer(const void *local, uint32_t rank) {
   return v;
 }
 
+// Store a 32-bit word to the shared memory of block `rank` of this cluster.
+__device__ __forceinline__ void st_peer(void *local, uint32_t rank, uint32_t v) {
+  const uint32_t la = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ float ld_peer_f(const float *local, uint32_t rank) {
   return __uint_as_float(ld_peer(local, rank));
 }

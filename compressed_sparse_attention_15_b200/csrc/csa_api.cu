@@ -288,6 +288,43 @@ int csa_sparse_mqa(const void *q, const void *kv_cmp, const int32_t *idx, const 
   return cuda_rc(launch_mqa(a, (cudaStream_t)stream));
 }
 
+size_t csa_topk_sparse_mqa_workspace_bytes(int Q, int H, int D, int N_max, int k, int win_len) {
+  if (Q < 1 || H < 1 || D < 1 || N_max < 1 || k < 1 || win_len < 0) return kStatusBytes;
+  // the selection's scratch and the attention's partials are used one after the other
+  const size_t t = topk_scratch_bytes(Q, N_max, k), m = mqa_partial_bytes(Q, H, D, k + win_len);
+  return kStatusBytes + align256(t > m ? t : m);
+}
+
+int csa_topk_sparse_mqa(const float *scores, const int32_t *n_cmp, int k, int32_t *idx_out, const void *q,
+                        const void *kv_cmp, const void *kv_win, const float *sink, float scale, void *out, int Q,
+                        int B, int H, int D, int N_max, int win_len, const int32_t *win_end, int T_raw,
+                        int q_per_seq, int dtype, void *ws, size_t ws_bytes, csa_stream_t stream) {
+  int rc = check_mqa(q, kv_cmp, kv_win, sink, out, Q, B, H, D, N_max, win_len, win_end, T_raw, q_per_seq, dtype);
+  if (rc) return rc;
+  if (!scores || !n_cmp || !idx_out || k < 1 || k > CSA_MAX_TOPK || (long long)k + win_len > 65536)
+    return CSA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(n_cmp) |
+       reinterpret_cast<uintptr_t>(idx_out)) & 3)
+    return CSA_ERR_INVALID;
+  if (!ws || !ws_aligned(ws) || ws_bytes < csa_topk_sparse_mqa_workspace_bytes(Q, H, D, N_max, k, win_len))
+    return CSA_ERR_WORKSPACE;
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  char *scratch = static_cast<char *>(ws) + kStatusBytes;
+  const size_t scratch_bytes = ws_bytes - kStatusBytes;
+  MqaArgs a{q, kv_cmp, kv_win, nullptr, n_cmp, win_end, sink, scale, out, Q, B, H, D, N_max, k, win_len, T_raw,
+            q_per_seq, dtype, scratch, scratch_bytes, status_of(ws), scores, idx_out};
+  bool taken = false;
+  cudaError_t e = launch_topk_mqa_tc(a, (cudaStream_t)stream, &taken);
+  if (taken) return cuda_rc(e);
+  TopkArgs ta{scores, n_cmp, idx_out, Q, N_max, k, status_of(ws)};
+  e = launch_topk(ta, (cudaStream_t)stream, scratch, scratch_bytes);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  a.idx = idx_out;
+  a.scores = nullptr;
+  a.idx_out = nullptr;
+  return cuda_rc(launch_mqa(a, (cudaStream_t)stream));
+}
+
 int hca_mqa(const void *q, const void *kv_cmp, const void *kv_win, const float *sink, float scale, void *out, int Q,
             int B, int H, int D, int N_max, const int32_t *n_cmp, int win_len, const int32_t *win_end, int T_raw,
             int q_per_seq, int dtype, void *ws, size_t ws_bytes, csa_stream_t stream) {

@@ -109,8 +109,13 @@ struct MqaArgs {
   void *partials;          // split-K scratch inside the workspace
   size_t partial_bytes;
   uint32_t *status;
+  const float *scores;     // non-null: select the top-k of these indexer scores in the kernel (idx unused)
+  int32_t *idx_out;        // ... and write the selection here
 };
 cudaError_t launch_mqa(const MqaArgs &a, cudaStream_t stream);
+// Top-k selection fused into the tensor-core MQA (a.scores set); *taken is
+// false when the shape or the launch plan does not allow it.
+cudaError_t launch_topk_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken);
 size_t mqa_partial_bytes(int Q, int H, int D, int rows_max);
 
 }  // namespace csa

@@ -42,6 +42,7 @@
 // the MMAs and owns TMEM, warps 5-8 run the softmax and the epilogue. All
 // mbarrier waits are bounded; the softmax warps take every decision to stop
 // together (a barrier reduction), so no named barrier is left half-joined.
+#include "cluster_select.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -68,6 +69,8 @@ constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64
 constexpr uint32_t kColS = 256;                     // S^T buffer j at 256 + 64j (M = 64 layout)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kSelMax = 1024;                       // largest k selected inside the kernel
+constexpr int kSelKeys = 2 * kTileBytes / 4;        // slice keys that fit in the tile buffers
 
 struct Small {
   uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done, o_done;
@@ -80,9 +83,13 @@ struct Small {
   int rescale;
   int need[4];  // per tile (mod 4): some logit exceeded the running maximum by more than 2^8
   const bf16 *rowp[kLoadWarps][32];  // gathered tiles: source row of each of a loader warp's rows (null: zero-fill)
+  sel::Shared cs;                    // in-kernel top-k: cluster exchange
+  int32_t sel[kSelMax];              // in-kernel top-k: the selected entry of each list position of this split
 };
 
 constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kQBytes + 2 * kPBytes + sizeof(Small);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
+static_assert(2 * kPBytes == 2 * sel::kBins * 4, "the P buffers hold the two selection histograms");
 
 // Row list of one query: compressed rows [0, nsel) (padded with unused rows
 // up to nsel4, a multiple of 4), then the window rows [nsel4, R).
@@ -92,7 +99,7 @@ struct RowList {
 
 __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *status) {
   RowList L;
-  L.nsel = a.idx ? a.k : clamp_count(a.n_cmp[qq], a.N_max, status);
+  L.nsel = (a.idx || a.scores) ? a.k : clamp_count(a.n_cmp[qq], a.N_max, status);
   int e = a.win_end[qq];
   if (e < 0 || e >= a.T_raw) {
     raise_status(status, CSA_STATUS_BAD_WINDOW);
@@ -208,6 +215,46 @@ __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// Top-k of query qq's indexer scores by the cluster of its splits, all
+// threads taking part (the selection csa_topk makes). List position r of the
+// selection lands in sel[r] of the split whose tiles hold it, and in idx_out
+// (written by head group 0); each selected row is prefetched into L2 as it is
+// found. The slice's keys use the tile buffers and the histograms the P
+// buffers, neither in use yet.
+__device__ void select_rows(const MqaArgs &a, Small *sm, uint8_t *kv, uint8_t *ps, int qq, int hg, int b,
+                            int tiles_per_split) {
+  const uint32_t C = cluster_size(), c = cluster_rank();
+  const int n = clamp_count(a.n_cmp[qq], a.N_max, (threadIdx.x == 0 && c == 0) ? a.status : nullptr);
+  const int k = a.k;
+  int32_t *out = hg == 0 ? a.idx_out + (size_t)qq * k : nullptr;
+  if (n <= k) {  // the same in every block of the cluster: no block touches a peer
+    for (int i = threadIdx.x; i < k; i += kThreads) {
+      const int j = i < n ? i : -1;
+      sm->sel[i] = j;
+      if (out && c == 0) out[i] = j;
+    }
+  } else {
+    const int S = ((n + (int)C - 1) / (int)C + 31) & ~31;
+    const int j0 = (int)c * S, len = max(0, min(S, n - j0));
+    uint32_t *keys = reinterpret_cast<uint32_t *>(kv);
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    sel::cache_keys<kThreads>(keys, a.scores + (size_t)qq * a.N_max + j0, len, lo, hi);
+    const bf16 *rows = static_cast<const bf16 *>(a.kv_cmp) + (size_t)b * a.N_max * kD;
+    const int rows_per_split = kRows * tiles_per_split;
+    sel::cluster_select<kThreads, 8, kMaxSplits>(
+        sm->cs, reinterpret_cast<uint32_t *>(ps), keys, len, j0, k, C, c, lo, hi, [&](uint32_t slot, int j) {
+          st_peer(&sm->sel[slot], slot / (uint32_t)rows_per_split, (uint32_t)j);
+          if (out) out[slot] = j;
+          bulk_prefetch_l2(rows + (size_t)j * kD, kD * 2);
+        });
+    cluster_wait();  // every selected position is in its split's sel; no peer reads this block any more
+  }
+  // the keys were written through the generic proxy; the tile buffers are
+  // next written by TMA and cp.async
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp_t,
                   const __grid_constant__ CUtensorMap tm_win_t, MqaArgs a, int splits, int tiles_per_split,
@@ -257,6 +304,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t0 = split * tiles_per_split;
   const int t1 = min(tiles_all, t0 + tiles_per_split);
   const int ntiles = max(0, t1 - t0);
+  const bool fused = a.scores != nullptr;  // the row selection is made here (sel), not read from idx
+  const bool sparse = fused || a.idx != nullptr;
+  if (warp == kMmaWarp && lane == 0 && ntiles > 0) {
+    tc::prefetch_tmap(&tm_q);
+    tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
+    for (int bx = 0; bx < kD / 64; ++bx) tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qv * kH, &sm->q_full);
+  }
+  if (fused) select_rows(a, sm, kv, ps, qq, hg, b, tiles_per_split);
+  // entry of the selection at list position r < nsel
+  auto sel_at = [&](int r) -> int { return fused ? sm->sel[r] : a.idx[(size_t)qq * a.k + r]; };
 
   if (warp < kLoadWarps) {
     // ------------------------------------------------------------ loaders
@@ -276,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Source row of list position r (null: padding or an unused slot).
     auto src_row = [&](int r) -> const bf16 * {
       if (r < L.nsel) {
-        int j = a.idx ? a.idx[(size_t)qq * a.k + r] : r;
+        int j = sparse ? sel_at(r) : r;
         if (j < -1 || j >= a.N_max) {
           raise_status(a.status, CSA_STATUS_BAD_INDEX);
           j = -1;
@@ -291,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // compressed part of a dense (HCA) row list.
     auto is_run = [&](int r0, bool &win_run) {
       win_run = r0 >= L.nsel4;
-      return win_run || (!a.idx && r0 + kRows <= L.nsel4);
+      return win_run || (!sparse && r0 + kRows <= L.nsel4);
     };
     // Bring this warp's rows of tile li into L2 ahead of their load, which can
     // only start once the tile buffer is free: the load then waits on L2.
@@ -364,14 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool q_issued = false;
-      if (ntiles > 0) {
-        tc::prefetch_tmap(&tm_q);
-        tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
-        for (int bx = 0; bx < kD / 64; ++bx)
-          tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qv * kH, &sm->q_full);
-        q_issued = true;
-      }
+      const bool q_issued = ntiles > 0;  // the Q load was issued above
       constexpr uint32_t idesc_s = tc::idesc_bf16(64, 64, 0, 0);
       constexpr uint32_t idesc_pv = tc::idesc_bf16(128, 64, 1, 1);
       const uint32_t kv_base = tc::smem_u32(kv), q_base = tc::smem_u32(qs), p_base = tc::smem_u32(ps);
@@ -455,21 +505,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 16; ++i) l[i] = 0.f;
     bool ok = true;
     int idxA = 0, idxB = 0;
-    if (ntiles > 0 && a.idx) {
+    if (ntiles > 0 && sparse) {
       const int r = t0 * kRows + rowA;
-      if (r < L.nsel) idxA = a.idx[(size_t)qq * a.k + r];
-      if (r + 8 < L.nsel) idxB = a.idx[(size_t)qq * a.k + r + 8];
+      if (r < L.nsel) idxA = sel_at(r);
+      if (r + 8 < L.nsel) idxB = sel_at(r + 8);
     }
     for (int li = 0; li < ntiles; ++li) {
       const int buf = li & 1;
       const bool got = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full[buf], (li >> 1) & 1, abort, a.status));
       tc::fence_after_sync();
       const int rA = (t0 + li) * kRows + rowA, rB = rA + 8;
-      const bool validA = rA < L.nsel4 ? (rA < L.nsel && (!a.idx || (idxA >= 0 && idxA < a.N_max))) : rA < L.R;
-      const bool validB = rB < L.nsel4 ? (rB < L.nsel && (!a.idx || (idxB >= 0 && idxB < a.N_max))) : rB < L.R;
-      if (li + 1 < ntiles && a.idx) {  // the next tile's indices, loaded while this tile is processed
-        idxA = rA + kRows < L.nsel ? a.idx[(size_t)qq * a.k + rA + kRows] : 0;
-        idxB = rB + kRows < L.nsel ? a.idx[(size_t)qq * a.k + rB + kRows] : 0;
+      const bool validA = rA < L.nsel4 ? (rA < L.nsel && (!sparse || (idxA >= 0 && idxA < a.N_max))) : rA < L.R;
+      const bool validB = rB < L.nsel4 ? (rB < L.nsel && (!sparse || (idxB >= 0 && idxB < a.N_max))) : rB < L.R;
+      if (li + 1 < ntiles && sparse) {  // the next tile's indices, loaded while this tile is processed
+        idxA = rA + kRows < L.nsel ? sel_at(rA + kRows) : 0;
+        idxB = rB + kRows < L.nsel ? sel_at(rB + kRows) : 0;
       }
       uint32_t v[32];
       tmem_ld_16x256b_x8(tmem + lane_off + kColS + 64 * buf, v);
@@ -878,7 +928,7 @@ bool tc_shape(const MqaArgs &a) {
          aligned16(a.kv_cmp) && aligned16(a.kv_win) && aligned16(a.out);
 }
 
-int rows_max_of(const MqaArgs &a) { return (((a.idx ? a.k : a.N_max) + 3) & ~3) + a.win_len; }
+int rows_max_of(const MqaArgs &a) { return ((((a.idx || a.scores) ? a.k : a.N_max) + 3) & ~3) + a.win_len; }
 
 }  // namespace
 
@@ -895,13 +945,20 @@ size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
   return (size_t)Q * s * kH * (kD + 2) * sizeof(float);
 }
 
-cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
+namespace {
+
+cudaError_t launch_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   *taken = false;
   if (!tc_shape(a)) return cudaSuccess;
   int splits, tps;
   bool cluster_merge;
   const int G = a.H / kH, QV = a.Q * G;  // blocks per split: one per group of 64 heads of a query
   plan_splits(QV, rows_max_of(a), &splits, &tps, &cluster_merge);
+  // In-kernel selection: the splits of a query must be one cluster, and each
+  // block's slice of the scores must fit in its tile buffers.
+  if (a.scores && (!cluster_merge || a.k > kSelMax || (((a.N_max + splits - 1) / splits + 31) & ~31) > kSelKeys ||
+                   !a.idx_out || !a.n_cmp))
+    return cudaSuccess;
   CUtensorMap tm_q, tm_cmp_t, tm_win_t;
   const uint64_t cmp_rows = (uint64_t)a.B * a.N_max, win_rows = (uint64_t)a.B * a.T_raw;
   if (!make_tmap_bf16_2d(&tm_q, a.q, kD, (uint64_t)a.Q * a.H, kD * 2, 64, kH) ||
@@ -920,6 +977,22 @@ cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   if (e != cudaSuccess || splits <= 1 || cluster_merge) return e;
   return launch_pdl(mqa_combine_kernel, dim3(QV, kH), dim3(kD / 4), splits * 3 * sizeof(float), stream,
                     (const float *)part_o, (const float *)part_ml, a.sink, static_cast<bf16 *>(a.out), splits, G);
+}
+
+}  // namespace
+
+cudaError_t launch_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
+  MqaArgs b = a;
+  b.scores = nullptr;
+  return launch_tc(b, stream, taken);
+}
+
+cudaError_t launch_topk_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
+  *taken = false;
+  if (!a.scores) return cudaSuccess;
+  MqaArgs b = a;
+  b.idx = nullptr;
+  return launch_tc(b, stream, taken);
 }
 
 }  // namespace csa

@@ -320,6 +320,31 @@ def sparse_mqa(q, kv_cmp, idx, kv_win, win_end, sink, scale: float, win_len: int
     return out
 
 
+def topk_sparse_mqa(scores, n_cmp, k: int, q, kv_cmp, kv_win, win_end, sink, scale: float, win_len: int,
+                    q_per_seq=None, out=None, idx_out=None, ws: Workspace | None = None):
+    """Top-k of the indexer scores, then CSA attention over the selection
+    (csa_topk_sparse_mqa: one kernel where the launch plan allows). Returns
+    (out [Q, H, D], idx [Q, k] int32)."""
+    Q, H, D, B, N_max, T_raw, qps = _mqa_common(q, kv_cmp, kv_win, win_end, sink, q_per_seq)
+    _need(scores, "scores", dtype=torch.float32, device=q.device)
+    _need(n_cmp, "n_cmp", dtype=torch.int32, device=q.device)
+    if scores.shape != (Q, N_max) or n_cmp.shape != (Q,):
+        raise ValueError("scores must be [Q, N_max] and n_cmp [Q]")
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is None:
+        idx_out = torch.empty((Q, k), dtype=torch.int32, device=q.device)
+    _need(out, "out", dtype=q.dtype, device=q.device)
+    _need(idx_out, "idx_out", dtype=torch.int32, device=q.device)
+    L = _lib.lib()
+    w = (ws or Workspace(q.device)).get(L.csa_topk_sparse_mqa_workspace_bytes(Q, H, D, N_max, int(k), int(win_len)))
+    rc = L.csa_topk_sparse_mqa(_ptr(scores), _ptr(n_cmp), int(k), _ptr(idx_out), _ptr(q), _ptr(kv_cmp), _ptr(kv_win),
+                               _ptr(sink), float(scale), _ptr(out), Q, B, H, D, N_max, int(win_len), _ptr(win_end),
+                               T_raw, qps, _dtype_code(q), _ptr(w), w.numel(), _stream(q.device))
+    _lib.check("csa_topk_sparse_mqa", rc)
+    return out, idx_out
+
+
 def hca_mqa(q, kv_cmp, n_cmp, kv_win, win_end, sink, scale: float, win_len: int, q_per_seq=None, out=None,
             ws: Workspace | None = None):
     """HCA attention over every visible entry + window + sink (hca_mqa)."""

@@ -10,6 +10,9 @@ The step over device-resident caches is:
      (csa_index_topk, or csa_index_topk_fp8 with FP8 indexer inputs);
   3. attend over the selected (CSA) or all visible (HCA) entries + the
      sliding window + the per-head sink (csa_sparse_mqa / hca_mqa).
+With fuse_select=True, a CSA step only scores in 2 (csa_index_scores(_fp8))
+and 3 is csa_topk_sparse_mqa, which makes the selection inside the attention
+kernel where its launch plan allows.
 The library never allocates or synchronises, so the launches are captured
 once into a CUDA graph and each step is one graph launch. Buffers are bound
 at construction; later steps see whatever the caller wrote into them.
@@ -25,7 +28,7 @@ class DecodeStep:
     def __init__(self, *, q, kv_cmp, kv_win, sink, scale: float, win_len: int, win_end, n_cmp,
                  ape, norm_w, gate, append_src0: int, append_dst0: int, win: int, stride: int,
                  qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True,
-                 qi8=None, sq=None, ki8=None, sk=None, append_rope=None):
+                 qi8=None, sq=None, ki8=None, sk=None, append_rope=None, fuse_select: bool = False):
         self.fp8 = qi8 is not None
         self.csa = qi is not None or self.fp8
         self.q, self.kv_cmp, self.kv_win, self.sink = q, kv_cmp, kv_win, sink
@@ -42,6 +45,9 @@ class DecodeStep:
         dev = q.device
         self.out = out if out is not None else torch.empty_like(q)
         self.idx = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev) if self.csa else None
+        self.fuse_select = bool(fuse_select) and self.csa
+        self.scores = (torch.empty((q.shape[0], kv_cmp.shape[1]), dtype=torch.float32, device=dev)
+                       if self.fuse_select else None)
         self.ws_index = ops.Workspace(dev)
         self.ws_mqa = ops.Workspace(dev)
         self.side = torch.cuda.Stream(dev)
@@ -60,14 +66,23 @@ class DecodeStep:
                      rope=self.append_rope)
 
     def select(self):
-        if self.fp8:
+        if self.fuse_select:  # scores only; the selection is made with the attention
+            if self.fp8:
+                ops.index_scores_fp8(self.qi8, self.sq, self.wi, self.ki8, self.sk, self.n_cmp, out=self.scores,
+                                     ws=self.ws_index)
+            else:
+                ops.index_scores(self.qi, self.wi, self.ki, self.n_cmp, out=self.scores, ws=self.ws_index)
+        elif self.fp8:
             ops.index_topk_fp8(self.qi8, self.sq, self.wi, self.ki8, self.sk, self.n_cmp, self.k, out=self.idx,
                                ws=self.ws_index)
         else:
             ops.index_topk(self.qi, self.wi, self.ki, self.n_cmp, self.k, out=self.idx, ws=self.ws_index)
 
     def attend(self):
-        if self.csa:
+        if self.fuse_select:
+            ops.topk_sparse_mqa(self.scores, self.n_cmp, self.k, self.q, self.kv_cmp, self.kv_win, self.win_end,
+                                self.sink, self.scale, self.win_len, out=self.out, idx_out=self.idx, ws=self.ws_mqa)
+        elif self.csa:
             ops.sparse_mqa(self.q, self.kv_cmp, self.idx, self.kv_win, self.win_end, self.sink, self.scale,
                            self.win_len, out=self.out, ws=self.ws_mqa)
         else:
@@ -76,6 +91,9 @@ class DecodeStep:
 
     def parts(self):
         p = [("compress", self.append)]
+        if self.fuse_select:
+            p += [("index_scores", self.select), ("topk_mqa", self.attend)]
+            return p
         if self.csa:
             p.append(("index_topk", self.select))
         p.append(("mqa", self.attend))

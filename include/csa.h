@@ -261,6 +261,35 @@ int csa_sparse_mqa(const void *q, const void *kv_cmp, const int32_t *idx, const 
                    void *ws, size_t ws_bytes, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * csa_topk_sparse_mqa -- csa_topk followed by csa_sparse_mqa, as one call.
+ *
+ * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: the indexer's
+ * top-k picks the compressed entries the core attention reads. Given the
+ * indexer scores, this call selects with csa_topk's rule, writes the
+ * selection to idx_out, and computes csa_sparse_mqa over it; results are
+ * those of the two calls in sequence. Where the tensor-core attention runs
+ * each query's splits as one thread-block cluster (H = 64 or 128, D = 512,
+ * bf16, k <= 1024, slices of at most 32,768 scores per block), the selection
+ * is made inside the attention kernel, by the cluster, and the attention
+ * starts from it without a kernel boundary; otherwise the two kernels run.
+ *
+ *   scores  : [Q, N_max] float32 (row stride N_max); entries j < n_cmp[q] read.
+ *   n_cmp   : [Q] int32 device array (0 .. N_max), visible entries per query.
+ *   idx_out : [Q, k] int32, written (ascending, -1 padded, as csa_topk).
+ *   q, kv_cmp, kv_win, win_end, sink, scale, out, shapes, dtype: as
+ *   csa_sparse_mqa.
+ * Limits: those of csa_topk and csa_sparse_mqa.
+ * Workspace: csa_topk_sparse_mqa_workspace_bytes(Q, H, D, N_max, k, win_len).
+ * Returns CSA_ERR_INVALID / CSA_ERR_WORKSPACE before any launch.
+ * ---------------------------------------------------------------------- */
+size_t csa_topk_sparse_mqa_workspace_bytes(int Q, int H, int D, int N_max, int k, int win_len);
+int csa_topk_sparse_mqa(const float *scores, const int32_t *n_cmp, int k, int32_t *idx_out,
+                        const void *q, const void *kv_cmp, const void *kv_win, const float *sink,
+                        float scale, void *out, int Q, int B, int H, int D, int N_max, int win_len,
+                        const int32_t *win_end, int T_raw, int q_per_seq, int dtype,
+                        void *ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * hca_mqa -- the dense (heavily compressed, 128 tokens -> 1) variant: as
  * csa_sparse_mqa but over every visible compressed entry j < n_cmp[q]
  * instead of an index list ("DeepSeek-V4 Architecture Analysis",
