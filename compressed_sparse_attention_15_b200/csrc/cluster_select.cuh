@@ -286,14 +286,22 @@ __device__ void cluster_select(Shared &cs, uint32_t *hist2, const uint32_t *keys
     cs.warp_eq[warp] = e;
   }
   __syncthreads();
-  if (warp == 0) {
-    uint32_t x = lane < NW ? cs.warp_gt[lane] : 0u, y = lane < NW ? cs.warp_eq[lane] : 0u;
+  if (warp == 0) {  // each warp's offset within the slice, and the slice's totals
+    const uint32_t x0 = lane < NW ? cs.warp_gt[lane] : 0u, y0 = lane < NW ? cs.warp_eq[lane] : 0u;
+    uint32_t x = x0, y = y0;  // inclusive scans over the warps
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      x += __shfl_xor_sync(0xffffffffu, x, o);
-      y += __shfl_xor_sync(0xffffffffu, y, o);
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t xs = __shfl_up_sync(0xffffffffu, x, o), ys = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) {
+        x += xs;
+        y += ys;
+      }
     }
-    if (lane == 0) {
+    if (lane < NW) {
+      cs.warp_gt[lane] = x - x0;
+      cs.warp_eq[lane] = y - y0;
+    }
+    if (lane == 31) {
       cs.cnt_gt = x;
       cs.cnt_eq = y;
     }
@@ -316,11 +324,7 @@ __device__ void cluster_select(Shared &cs, uint32_t *hist2, const uint32_t *keys
     }
   }
   __syncthreads();
-  uint32_t G = cs.base_gt, E = cs.base_eq;
-  for (int w = 0; w < warp; ++w) {
-    G += cs.warp_gt[w];
-    E += cs.warp_eq[w];
-  }
+  uint32_t G = cs.base_gt + cs.warp_gt[warp], E = cs.base_eq + cs.warp_eq[warp];
   const uint32_t lt = (1u << lane) - 1u;
   for (int base = lo; base < hi; base += 32) {
     const int j = base + lane;

@@ -255,6 +255,10 @@ __device__ void select_rows(const MqaArgs &a, Small *sm, uint8_t *kv, uint8_t *p
   __syncthreads();
 }
 
+// kFused: the selection is made here from a.scores (select_rows) instead of
+// read from a.idx; a separate instantiation, so the plain kernel carries none
+// of its code.
+template <bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     mqa_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_cmp_t,
                   const __grid_constant__ CUtensorMap tm_win_t, MqaArgs a, int splits, int tiles_per_split,
@@ -304,14 +308,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t0 = split * tiles_per_split;
   const int t1 = min(tiles_all, t0 + tiles_per_split);
   const int ntiles = max(0, t1 - t0);
-  const bool fused = a.scores != nullptr;  // the row selection is made here (sel), not read from idx
+  constexpr bool fused = kFused;
   const bool sparse = fused || a.idx != nullptr;
   if (warp == kMmaWarp && lane == 0 && ntiles > 0) {
     tc::prefetch_tmap(&tm_q);
     tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
     for (int bx = 0; bx < kD / 64; ++bx) tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qv * kH, &sm->q_full);
   }
-  if (fused) select_rows(a, sm, kv, ps, qq, hg, b, tiles_per_split);
+  if constexpr (kFused) select_rows(a, sm, kv, ps, qq, hg, b, tiles_per_split);
   // entry of the selection at list position r < nsel
   auto sel_at = [&](int r) -> int { return fused ? sm->sel[r] : a.idx[(size_t)qq * a.k + r]; };
 
@@ -850,8 +854,10 @@ int num_sms_cached() {
 void set_kernel_attributes() {
   static bool done = false;
   if (!done) {
-    cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    for (auto kern : {mqa_tc_kernel<false>, mqa_tc_kernel<true>}) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    }
     done = true;
   }
 }
@@ -875,7 +881,8 @@ int max_active_clusters(int size) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel, &cfg) != cudaSuccess) {
+    // (both instantiations: one block per SM, the same shared memory)
+    if (cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel<false>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
@@ -971,7 +978,7 @@ cudaError_t launch_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   float *part_ml = part_o + (size_t)QV * splits * kH * kD;
   set_kernel_attributes();
   *taken = true;
-  cudaError_t e = launch_pdl_cluster(mqa_tc_kernel, dim3(splits, QV), dim3(kThreads), kSmemBytes, stream,
+  cudaError_t e = launch_pdl_cluster(a.scores ? mqa_tc_kernel<true> : mqa_tc_kernel<false>, dim3(splits, QV), dim3(kThreads), kSmemBytes, stream,
                                      cluster_merge ? (unsigned)splits : 1u, tm_q, tm_cmp_t, tm_win_t, a, splits, tps,
                                      a.scale * kLog2e, part_o, part_ml, (int)cluster_merge);
   if (e != cudaSuccess || splits <= 1 || cluster_merge) return e;

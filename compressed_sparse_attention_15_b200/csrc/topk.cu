@@ -162,11 +162,22 @@ __device__ void select_and_emit(TopkShared &sh, const uint32_t *keys, const floa
     sh.warp_eq[warp] = e;
   }
   __syncthreads();
-  uint32_t G = 0, E = 0;
-  for (int w = 0; w < warp; ++w) {
-    G += sh.warp_gt[w];
-    E += sh.warp_eq[w];
+  if (warp == 0) {  // exclusive scans over the warps: each warp's first output slot
+    const uint32_t x0 = sh.warp_gt[lane], y0 = sh.warp_eq[lane];
+    uint32_t x = x0, y = y0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t xs = __shfl_up_sync(0xffffffffu, x, o), ys = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) {
+        x += xs;
+        y += ys;
+      }
+    }
+    sh.warp_gt[lane] = x - x0;
+    sh.warp_eq[lane] = y - y0;
   }
+  __syncthreads();
+  uint32_t G = sh.warp_gt[warp], E = sh.warp_eq[warp];
   const uint32_t lt = (1u << lane) - 1u;
   for (int base = lo; base < hi; base += 32) {
     const int j = base + lane;
