@@ -38,8 +38,8 @@
 // cluster, after a cluster barrier merges 1/splits of the output from all of
 // them (L2 reads; distributed-shared-memory reads of the same data measured
 // several times slower).
-// Roles (288 threads): warps 0-3 load (two per tile buffer), warp 4 issues
-// the MMAs and owns TMEM, warps 5-8 run the softmax and the epilogue. All
+// Roles (416 threads): warps 0-7 load (four per tile buffer), warp 8 issues
+// the MMAs and owns TMEM, warps 9-12 run the softmax and the epilogue. All
 // mbarrier waits are bounded; the softmax warps take every decision to stop
 // together (a barrier reduction), so no named barrier is left half-joined.
 #include "cluster_select.cuh"
@@ -59,10 +59,12 @@ constexpr uint32_t kTileBytes = 8 * kBoxBytes;      // 64 rows x 512 dims: 64 KB
 constexpr uint32_t kQBoxBytes = kH * 128;           // 64 heads x 64 dims: 8 KB
 constexpr uint32_t kQBytes = 8 * kQBoxBytes;        // 64 KB
 constexpr uint32_t kPBytes = kRows * kH * 2;        // 8 KB
-constexpr int kLoadWarps = 4;                       // two per tile buffer, 32 rows each
-constexpr int kThreads = 288;
-constexpr int kMmaWarp = 4;
-constexpr int kSoftWarp0 = 5;
+constexpr int kLoadWarps = 8;                       // four per tile buffer
+constexpr int kWarpsPerBuf = kLoadWarps / 2;
+constexpr int kRowsPerWarp = kRows / kWarpsPerBuf;  // 16 rows of a tile per loader warp
+constexpr int kMmaWarp = kLoadWarps;
+constexpr int kSoftWarp0 = kLoadWarps + 1;          // 4 softmax warps: one per TMEM lane quarter
+constexpr int kThreads = 32 * (kSoftWarp0 + 4);
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSplits = 16;                      // splits of one query form one cluster (<= 16 CTAs)
 constexpr uint32_t kColO = 0;                       // O^T chunk m at columns 64m (M = 128 layout)
@@ -82,7 +84,7 @@ struct Small {
   int abort;
   int rescale;
   int need[4];  // per tile (mod 4): some logit exceeded the running maximum by more than 2^8
-  const bf16 *rowp[kLoadWarps][32];  // gathered tiles: source row of each of a loader warp's rows (null: zero-fill)
+  const bf16 *rowp[kLoadWarps][kRowsPerWarp];  // gathered tiles: source of each of a loader warp's rows (null: zero-fill)
   sel::Shared cs;                    // in-kernel top-k: cluster exchange
   int32_t sel[kSelMax];              // in-kernel top-k: the selected entry of each list position of this split
 };
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tc::mbar_init(&sm->q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&sm->kv_full[i], 64);
+      tc::mbar_init(&sm->kv_full[i], 32 * kWarpsPerBuf);
       tc::mbar_init(&sm->kv_empty[i], 1);
       tc::mbar_init(&sm->s_full[i], 1);
       tc::mbar_init(&sm->p_full[i], 4 * 32);
@@ -321,14 +323,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kLoadWarps) {
     // ------------------------------------------------------------ loaders
-    // Warps 2g and 2g + 1 fill tile buffer g (tiles g, g + 2, ...), rows
-    // 0-31 and 32-63 of each tile. A contiguous run is 8 TMA boxes issued by
-    // lane 0 of warp 2g. A gathered tile is 16-byte cp.async copies, 64 per
-    // lane, each warp instruction moving 512 contiguous bytes of one row;
-    // every lane waits for its own copies, fences them for the tensor core
-    // and arrives, so kv_full expects 64 arrivals either way. Each warp also
-    // prefetches its rows of its next tile into L2 while the buffer is busy.
-    const int g = warp >> 1, half = warp & 1;
+    // Warps 4g .. 4g + 3 fill tile buffer g (tiles g, g + 2, ...), 16 rows
+    // of each tile each (part = warp % 4: rows 16 part .. 16 part + 15). A
+    // contiguous run is 8 TMA boxes issued by lane 0 of warp 4g. A gathered
+    // tile is 16-byte cp.async copies, 32 per lane, each warp instruction
+    // moving 512 contiguous bytes of one row; every lane waits for its own
+    // copies, fences them for the tensor core and arrives, so kv_full
+    // expects 128 arrivals either way. Each warp also prefetches its rows of
+    // its next tile into L2 while the buffer is busy.
+    const int g = warp / kWarpsPerBuf, part = warp % kWarpsPerBuf;
     const uint32_t buf_base = tc::smem_u32(kv) + g * kTileBytes;
     if (warp == 0 && lane == 0) {
       tc::prefetch_tmap(&tm_cmp_t);
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Bring this warp's rows of tile li into L2 ahead of their load, which can
     // only start once the tile buffer is free: the load then waits on L2.
     // (A run's rows are contiguous in memory: one bulk prefetch of this
-    // warp's 32 rows streams them from HBM in order, where the tile's TMA
+    // warp's 16 rows streams them from HBM in order, where the tile's TMA
     // boxes each read 128 bytes of every row.)
     auto prefetch_l2 = [&](int li) {
       if (li >= ntiles) return;
@@ -365,18 +368,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool win_run;
       if (is_run(r0, win_run)) {
         if (lane == 0) {
-          // first row of this warp's half, and how many rows of the sequence's buffer remain from it
-          const int first = win_run ? L.wlo + (r0 - L.nsel4) + 32 * half : r0 + 32 * half;
+          // first row of this warp's part, and how many rows of the sequence's buffer remain from it
+          const int first = win_run ? L.wlo + (r0 - L.nsel4) + kRowsPerWarp * part : r0 + kRowsPerWarp * part;
           const int avail = (win_run ? a.T_raw : a.N_max) - first;
-          const int rows = avail < 32 ? avail : 32;
+          const int rows = avail < kRowsPerWarp ? avail : kRowsPerWarp;
           if (rows > 0) {
             const bf16 *base = win_run ? static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + first) * kD
                                        : static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + first) * kD;
             bulk_prefetch_l2(base, (uint32_t)rows * kD * 2);
           }
         }
-      } else if (const bf16 *p = src_row(r0 + 32 * half + lane)) {
-        bulk_prefetch_l2(p, kD * 2);
+      } else if (lane < kRowsPerWarp) {
+        if (const bf16 *p = src_row(r0 + kRowsPerWarp * part + lane)) bulk_prefetch_l2(p, kD * 2);
       }
     };
     int last = -1;
@@ -385,14 +388,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool win_run;
       const bool run = is_run(r0, win_run);
       __syncwarp();  // the previous tile's copies have read rowp[warp]
-      if (!run) sm->rowp[warp][lane] = src_row(r0 + 32 * half + lane);
+      if (!run && lane < kRowsPerWarp) sm->rowp[warp][lane] = src_row(r0 + kRowsPerWarp * part + lane);
       if (li == g) {  // the first tile streams in order too; later tiles are prefetched one round ahead, below
         if (run) prefetch_l2(li);
         prefetch_l2(li + 2);
       }
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status))) break;
       if (run) {
-        if (half == 0 && lane == 0) {
+        if (part == 0 && lane == 0) {
           tc::mbar_arrive_expect_tx(&sm->kv_full[g], kTileBytes);
           const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
           for (int bx = 0; bx < 8; ++bx)
@@ -404,9 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         __syncwarp();  // rowp[warp] written by every lane
 #pragma unroll 8
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 2 * kRowsPerWarp; ++i) {
           const int rw = i >> 1, c16 = lane + 32 * (i & 1);  // 16-byte piece c16 of this warp's row rw
-          const int row = 32 * half + rw;                     // row within the tile
+          const int row = kRowsPerWarp * part + rw;           // row within the tile
           const bf16 *src = sm->rowp[warp][rw];
           const uint32_t dst = buf_base + (c16 >> 3) * kBoxBytes + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
           cp_async16(dst, src ? src + c16 * 8 : static_cast<const bf16 *>(a.kv_win), src != nullptr);
@@ -421,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       last = li;
     }
     // Drain: a TMA tile still in flight must land before the CTA exits.
-    if (half == 0 && lane == 0 && last >= 0) tc::mbar_drain(&sm->kv_full[g], (last >> 1) & 1);
+    if (part == 0 && lane == 0 && last >= 0) tc::mbar_drain(&sm->kv_full[g], (last >> 1) & 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
