@@ -144,6 +144,10 @@ __device__ __forceinline__ uint4 pack8(const float f[8]) {
 // ... < i1. One cluster of C blocks per (sequence, entry): block c of the
 // cluster takes positions [c P, c P + P), P = ceil(win / C); the C partial
 // states are merged by block 0 through distributed shared memory.
+// kRope: rotate the rope dims of each written entry (a.rope_dims > 0); its
+// own instantiation, so the plain kernel carries none of the rotation's code
+// or registers.
+template <bool kRope>
 __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, int G) {
   extern __shared__ float ws[];  // [G][3][8][nvec] partial states, then [32] sums, then [3][8][nvec] block state
   pdl_wait();
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
       const float rn = 1.0f / sqrtf(tot / (float)a.D + kRmsEps);
       bf16 *o = static_cast<bf16 *>(a.out) + b * a.out_ss + (long long)j * a.D;
       float x = cd * rn * a.norm_w[d];
-      if (a.rope_dims) {  // the pair partner is the neighbouring thread's dim
+      if constexpr (kRope) {  // the pair partner is the neighbouring thread's dim
         float y = __shfl_xor_sync(0xffffffffu, x, 1);
         if (d & 1)
           rope_pair(a, b, j, d - 1, y, x);
@@ -315,7 +319,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
 #pragma unroll
     for (int k = 0; k < 8; ++k) c[k] = blk[k * nvec + t] * rn * nw[k];
     bf16 *o = static_cast<bf16 *>(a.out) + b * a.out_ss + (long long)j * a.D;
-    rope8(a, b, j, 8 * t, c);
+    if constexpr (kRope) rope8(a, b, j, 8 * t, c);
     reinterpret_cast<uint4 *>(o)[t] = pack8(c);
   }
 }
@@ -325,8 +329,9 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
 // WPR warps own one row (8 dims per lane, D = 256 * WPR); each group of WPR
 // warps walks a contiguous run of the flattened (sequence, entry) space.
 // S = stride, window = 2 S; ape (pre-scaled by log2 e) lives in shared memory.
-template <int WPR, int S>
+template <int WPR, int S, bool kRope>
 __global__ void __launch_bounds__(256) compress_stream_kernel(CompressArgs a, long long per_group) {
+  // (kRope as for compress_window_kernel)
   constexpr int W = 2 * S;
   extern __shared__ float ape_s[];  // [W][D] * log2 e
   __shared__ float grp_sum[8];
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(256) compress_stream_kernel(CompressArgs a, lo
     const float r = 1.0f / sqrtf(ss / (float)D + kRmsEps);
 #pragma unroll
     for (int k = 0; k < 8; ++k) c[k] = c[k] * r * nw[k];
-    rope8(a, b, j, 8 * v, c);
+    if constexpr (kRope) rope8(a, b, j, 8 * v, c);
     reinterpret_cast<uint4 *>(out + b * a.out_ss + (long long)j * D)[v] = pack8(c);
 #pragma unroll
     for (int i = 0; i < S; ++i) {
@@ -452,7 +457,8 @@ cudaError_t launch_stream(const CompressArgs &a, cudaStream_t stream) {
   groups = (total + per - 1) / per;
   const long long blocks = (groups + groups_per_block - 1) / groups_per_block;
   const size_t smem = (size_t)2 * S * a.D * sizeof(float);
-  return launch_pdl(compress_stream_kernel<WPR, S>, dim3((unsigned)blocks), dim3(256), smem, stream, a, per);
+  return launch_pdl(a.rope_dims ? compress_stream_kernel<WPR, S, true> : compress_stream_kernel<WPR, S, false>,
+                    dim3((unsigned)blocks), dim3(256), smem, stream, a, per);
 }
 
 }  // namespace
@@ -484,12 +490,13 @@ cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
       const size_t smem = ((size_t)(G + 1) * 3 * 8 * nvec + 32) * sizeof(float);
       static bool attr_set = false;
       if (!attr_set) {
-        cudaFuncSetAttribute(compress_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(((size_t)4 * 8 * 512 + 32) * sizeof(float)));
+        for (auto kern : {compress_window_kernel<false>, compress_window_kernel<true>})
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(((size_t)4 * 8 * 512 + 32) * sizeof(float)));
         attr_set = true;
       }
-      return launch_pdl_cluster(compress_window_kernel, dim3((unsigned)(total * C)), dim3(G * nvec), smem, stream,
-                                (unsigned)C, a, G);
+      return launch_pdl_cluster(a.rope_dims ? compress_window_kernel<true> : compress_window_kernel<false>,
+                                dim3((unsigned)(total * C)), dim3(G * nvec), smem, stream, (unsigned)C, a, G);
     }
   }
   const int threads = 256, wpb = threads / 32;
