@@ -113,3 +113,24 @@ def test_topk_rejects_bad_arguments(L):
     assert L.csa_topk(P, P, 0, P, 2, 10, P, 256, NULL) == 1
     assert L.csa_topk(NULL, P, 4, P, 2, 10, P, 256, NULL) == 1
     assert L.csa_topk(P, P, 4, P, 2, 10, P, 0, NULL) == 3
+
+
+def test_topk_sparse_mqa_rejects_bad_arguments(L):
+    # scores [2, 63], k 16, window 16, 4 heads x 16 dims, one sequence of 2 queries
+    ws = L.csa_topk_sparse_mqa_workspace_bytes(2, 4, 16, 63, 16, 16)
+    assert ws >= L.csa_topk_workspace_bytes(2, 63, 16)
+    assert ws >= L.csa_mqa_workspace_bytes(2, 4, 16, 16 + 16)
+
+    def call(scores=P, n=P, k=16, idx_out=P, W=16, H=4, ws_bytes=ws, ws_ptr=P):
+        return L.csa_topk_sparse_mqa(scores, n, k, idx_out, P, P, P, P, 0.25, P, 2, 1, H, 16, 63, W, P, 256, 2, 0,
+                                     ws_ptr, ws_bytes, NULL)
+    assert call(scores=NULL) == 1
+    assert call(n=NULL) == 1
+    assert call(idx_out=NULL) == 1
+    assert call(k=0) == 1
+    assert call(k=4097) == 1
+    assert call(idx_out=ctypes.c_void_p(4096 + 2)) == 1  # misaligned int32 array
+    assert call(W=0) == 1
+    assert call(H=129) == 1
+    assert call(ws_bytes=ws - 1) == 3
+    assert call(ws_ptr=ctypes.c_void_p(4096 + 128)) == 3  # not 256-byte aligned
