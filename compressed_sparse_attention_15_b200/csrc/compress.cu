@@ -433,17 +433,7 @@ __global__ void __launch_bounds__(256) compress_stream_kernel(CompressArgs a, lo
   }
 }
 
-int g_num_sms = 0;
-
-int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    g_num_sms = n > 0 ? n : 148;
-  }
-  return g_num_sms;
-}
+int num_sms() { return device_sm_count(); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -488,13 +478,12 @@ cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
       int G = P < 16 ? P : 16;
       while (G > 1 && G * nvec > 512) G >>= 1;
       const size_t smem = ((size_t)(G + 1) * 3 * 8 * nvec + 32) * sizeof(float);
-      static bool attr_set = false;
-      if (!attr_set) {
+      static DeviceOnce attr;
+      once_per_device(attr, [] {
         for (auto kern : {compress_window_kernel<false>, compress_window_kernel<true>})
           cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(((size_t)4 * 8 * 512 + 32) * sizeof(float)));
-        attr_set = true;
-      }
+      });
       return launch_pdl_cluster(a.rope_dims ? compress_window_kernel<true> : compress_window_kernel<false>,
                                 dim3((unsigned)(total * C)), dim3(G * nvec), smem, stream, (unsigned)C, a, G);
     }
@@ -503,12 +492,11 @@ cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream) {
   const size_t smem = (size_t)wpb * a.D * sizeof(float);
   long long blocks = (total + wpb - 1) / wpb;
   if (blocks > 65535LL * 16) blocks = 65535LL * 16;
-  static bool attr_set = false;  // the attribute is a per-function fact: set it once
-  if (!attr_set) {
+  static DeviceOnce attr;
+  once_per_device(attr, [] {
     cudaFuncSetAttribute(compress_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * 4096 * 4);
     cudaFuncSetAttribute(compress_generic_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * 4096 * 4);
-    attr_set = true;
-  }
+  });
   if (a.dtype == CSA_DTYPE_F32)
     return launch_pdl(compress_generic_kernel<float>, dim3((unsigned)blocks), dim3(threads), smem, stream, a);
   return launch_pdl(compress_generic_kernel<bf16>, dim3((unsigned)blocks), dim3(threads), smem, stream, a);

@@ -90,14 +90,13 @@ cudaError_t launch_index_scores(const ScoreArgs &a, cudaStream_t stream) {
   if (taken) return err;
   const size_t smem = ((size_t)a.Hi * a.Di + (size_t)kTileJ * (a.Di + 1) + a.Hi + 4 * kTileJ) * sizeof(float);
   dim3 grid(a.Q, (a.N_max + kTileJ - 1) / kTileJ);
-  static bool attr_set = false;  // set once for the largest size the ABI admits
-  if (!attr_set) {
+  static DeviceOnce attr;  // set for the largest size the ABI admits
+  once_per_device(attr, [] {
     const int max_smem = (128 * 256 + kTileJ * 257 + 128 + 4 * kTileJ) * 4;
     cudaFuncSetAttribute(index_scores_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     cudaFuncSetAttribute(index_scores_generic_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     cudaFuncSetAttribute(index_scores_generic_kernel<uint8_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    attr_set = true;
-  }
+  });
   if (a.dtype == CSA_DTYPE_E4M3)
     return launch_pdl(index_scores_generic_kernel<uint8_t>, grid, dim3(256), smem, stream, a);
   if (a.dtype == CSA_DTYPE_F32) return launch_pdl(index_scores_generic_kernel<float>, grid, dim3(256), smem, stream, a);

@@ -302,16 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int num_sms_cached() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+int num_sms_cached() { return device_sm_count(); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -335,14 +326,13 @@ cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool
   if (grid > total) grid = total;
   const long long per_cta = (total + grid - 1) / grid;
   grid = (total + per_cta - 1) / per_cta;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static DeviceOnce attr;
+  once_per_device(attr, [] {
     cudaFuncSetAttribute(index_scores_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem_bytes<false>());
     cudaFuncSetAttribute(index_scores_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem_bytes<true>());
-    attr_set = true;
-  }
+  });
   *taken = true;
   if (fp8)
     return launch_pdl(index_scores_tc_kernel<true>, dim3((unsigned)grid), dim3(kThreads), smem_bytes<true>(), stream,

@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include <utility>
 
 namespace csa {
@@ -96,6 +99,45 @@ struct TopkArgs {
 // lists, at least topk_scratch_bytes() bytes; without it one stage is used.
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, size_t scratch_bytes);
 size_t topk_scratch_bytes(int Q, int N_max, int k);
+
+// ---------------------------------------------------------------- per-device setup
+// Kernel attributes are set, and device facts cached, once per device (a
+// process may drive several GPUs, from several host threads).
+constexpr int kMaxDevices = 64;
+
+struct DeviceOnce {
+  std::mutex m;
+  bool done[kMaxDevices] = {};
+};
+
+// Runs fn on the current device the first time this site is reached there;
+// every caller returns only after it has run.
+template <class F>
+inline void once_per_device(DeviceOnce &o, F fn) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    fn();
+    return;
+  }
+  std::lock_guard<std::mutex> g(o.m);
+  if (!o.done[dev]) {
+    fn();
+    o.done[dev] = true;
+  }
+}
+
+// SM count of the current device (148 on a B200), cached per device.
+inline int device_sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
 
 struct MqaArgs {
   const void *q, *kv_cmp, *kv_win;

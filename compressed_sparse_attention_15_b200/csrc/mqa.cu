@@ -143,12 +143,11 @@ __global__ void __launch_bounds__(kThreads) mqa_generic_kernel(MqaArgs a) {
 template <typename T, int HG>
 cudaError_t launch_generic(const MqaArgs &a, cudaStream_t stream) {
   const size_t smem = ((size_t)(HG + kRC) * a.D + HG * kRC) * sizeof(float);
-  static bool attr_set = false;  // set once for the largest D the ABI admits
-  if (!attr_set) {
+  static DeviceOnce attr;  // set for the largest D the ABI admits
+  once_per_device(attr, [] {
     cudaFuncSetAttribute(mqa_generic_kernel<T, HG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)(((size_t)(HG + kRC) * 1024 + HG * kRC) * sizeof(float)));
-    attr_set = true;
-  }
+  });
   dim3 grid(a.Q, a.H / HG);
   return launch_pdl(mqa_generic_kernel<T, HG>, grid, dim3(kThreads), smem, stream, a);
 }

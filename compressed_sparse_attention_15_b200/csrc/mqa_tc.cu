@@ -843,34 +843,27 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const float *part_o, c
       make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
 }
 
-int num_sms_cached() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+int num_sms_cached() { return device_sm_count(); }
 
 void set_kernel_attributes() {
-  static bool done = false;
-  if (!done) {
+  static DeviceOnce attr;
+  once_per_device(attr, [] {
     for (auto kern : {mqa_tc_kernel<false>, mqa_tc_kernel<true>}) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
       cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     }
-    done = true;
-  }
+  });
 }
 
 // How many clusters of `size` CTAs of this kernel the GPU holds at once
 // (one CTA per SM, and a cluster must fit in one GPC).
 int max_active_clusters(int size) {
-  static int cache[kMaxSplits + 1] = {0};
+  static std::atomic<int> cache[kMaxDevices][kMaxSplits + 1];  // per device: 0 unknown, -1 none
   if (size < 1 || size > kMaxSplits) return 0;
-  if (cache[size] == 0) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  int c = cache[dev][size].load(std::memory_order_relaxed);
+  if (c == 0) {
     set_kernel_attributes();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(size, 1);
@@ -889,9 +882,10 @@ int max_active_clusters(int size) {
       cudaGetLastError();
       n = 0;
     }
-    cache[size] = n > 0 ? n : -1;
+    c = n > 0 ? n : -1;
+    cache[dev][size].store(c, std::memory_order_relaxed);
   }
-  return cache[size] > 0 ? cache[size] : 0;
+  return c > 0 ? c : 0;
 }
 
 // Split query rows into runs of whole tiles. Preferred: the largest

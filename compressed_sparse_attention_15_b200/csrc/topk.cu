@@ -343,10 +343,7 @@ __global__ void __launch_bounds__(kThreads) topk_stage2_kernel(TopkArgs a, const
 // least 2K entries per CTA, the slice's keys within the shared-memory cache.
 int plan_cluster(int Q, int N_max, int k) {
   if (Q < 1 || N_max <= k || N_max < 4096) return 0;
-  int sms = 0, dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int C = sms / Q;
+  int C = device_sm_count() / Q;
   C = C > 8 ? 8 : C;
   const int by_len = (N_max + 2047) / 2048;
   C = C > by_len ? by_len : C;
@@ -361,14 +358,13 @@ size_t topk_scratch_bytes(int Q, int N_max, int k) {
 }
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, size_t scratch_bytes) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static DeviceOnce attr;
+  once_per_device(attr, [] {
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     cudaFuncSetAttribute(topk_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 * 4);
     cudaFuncSetAttribute(topk_stage2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
-    attr_set = true;
-  }
+  });
   if (const int C = plan_cluster(a.Q, a.N_max, a.k)) {
     const int S = ((a.N_max + C - 1) / C + 31) & ~31;
     return launch_pdl_cluster(topk_cluster_kernel, dim3(C, a.Q), dim3(kThreads), (size_t)S * 4, stream, (unsigned)C,
