@@ -74,8 +74,6 @@ def algo_bytes(w: WL.Workload):
         b["topk"] = w.Q * w.k * 4
         rows = w.k + w.W
         b["mqa"] = w.Q * (rows * w.D * e + 2 * w.H * w.D * e + w.k * 4 + w.H * 4)
-        # selection inside the attention: the indices are written, not read back
-        b["topk_mqa"] = b["mqa"]
     else:
         rows = n_vis + w.W
         b["mqa"] = w.Q * (rows * w.D * e + 2 * w.H * w.D * e + w.H * 4)
@@ -83,16 +81,28 @@ def algo_bytes(w: WL.Workload):
 
 
 def algo_flops(w: WL.Workload):
+    """Per-step FLOPs of the contractions: the indexer's products over every
+    visible entry of every query, and QK^T + PV over each query's rows."""
+    n_vis = ops.visible_entries(w.positions(), w.win, w.stride).double()
     f = {}
     if w.mode == "csa":
-        f["index_scores"] = w.Q * w.N * w.Hi * w.Di * 2
-        rows = w.k + w.W
+        f["index_scores"] = float(n_vis.sum()) * w.Hi * w.Di * 2
+        rows = float(torch.clamp(n_vis, max=w.k).sum()) + w.Q * w.W
     else:
-        rows = w.N + w.W
-    f["mqa"] = w.Q * rows * w.H * w.D * 4
-    if w.mode == "csa":
-        f["topk_mqa"] = f["mqa"]
+        rows = float(n_vis.sum()) + w.Q * w.W
+    f["mqa"] = rows * w.H * w.D * 4
     return f
+
+
+# A step part whose algorithmic bytes and FLOPs are another's: the attention
+# with the selection made inside it moves what the attention moves.
+PART_ALIAS = {"topk_mqa": "mqa"}
+
+
+def prefill(w: WL.Workload) -> bool:
+    """Several queries of one sequence share its compressed keys (a causal
+    prefill chunk): the indexer is then tensor-bound, not HBM-bound."""
+    return w.q_per_seq > 1
 
 
 # --------------------------------------------------------------------------
@@ -350,11 +360,21 @@ def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
             "frac": round(gbps / hbm_gbs, 4), "bytes": nbytes, "tokens_per_s": round(w.bulk_T / (ms * 1e-3), 1)}
 
 
-def roofline_of(w, per_kernel_ms, hbm_gbs, traffic=None):
-    """Roofline of the kernel with the most algorithmic bytes in the step.
-    ``traffic`` maps a part name to its measured DRAM bytes per launch."""
+def roofline_of(w, per_kernel_ms, hbm_gbs, traffic=None, tflops=None):
+    """Roofline of the kernel with the most algorithmic bytes in the step
+    (decode: HBM-bound), or with the most FLOPs against the bf16 tensor peak
+    (prefill, given ``tflops``). ``traffic`` maps a part name to its measured
+    DRAM bytes per launch."""
+    if prefill(w) and tflops:
+        af = algo_flops(w)
+        name, fl = max(((k, af[PART_ALIAS.get(k, k)]) for k in per_kernel_ms if PART_ALIAS.get(k, k) in af),
+                       key=lambda x: x[1])
+        achieved = fl / (per_kernel_ms[name] * 1e-3) / 1e12
+        return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1), "peak": tflops, "unit": "TFLOP/s",
+                "frac": round(achieved / tflops, 4), "traffic": (traffic or {}).get(name), "flops_per_launch": int(fl)}
     ab = algo_bytes(w)
-    best = max(((k, ab[k]) for k in per_kernel_ms if k in ab), key=lambda x: x[1])
+    best = max(((k, ab[PART_ALIAS.get(k, k)]) for k in per_kernel_ms if PART_ALIAS.get(k, k) in ab),
+               key=lambda x: x[1])
     name, nbytes = best
     traffic = (traffic or {}).get(name)
     ms = per_kernel_ms[name]
@@ -563,7 +583,7 @@ def main():
     w = WL.shard(w, rank)  # this rank's own sequences (same shapes)
     r = time_ours(args, w, device, dist_on, rank, world)
     traffic = load_traffic(args.traffic_json, w.name)
-    roof = roofline_of(w, r["per_kernel_ms"], hbm, traffic)
+    roof = roofline_of(w, r["per_kernel_ms"], hbm, traffic, tflops)
     roof["peak_kind"] = f"{peak_kind} HBM copy bandwidth"
     e2e = e2e_ours(args, w, r["step"], device)
     del r["step"]
@@ -571,20 +591,24 @@ def main():
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
-        for name in ("hca_decode_1m", "csa_decode_1m", "csa_decode_64k_fp8", "csa_decode_64k_pro"):
+        for name in ("hca_decode_1m", "csa_decode_1m", "csa_decode_64k_fp8", "csa_decode_64k_pro", "csa_prefill_chunk_4k"):
             if name == w.name:
                 continue
             sw = WL.WORKLOADS[name]
             try:
                 s = time_ours(args, sw, device, False, 0, 1, secondary=True)
                 del s["step"]
-                rf = roofline_of(sw, s["per_kernel_ms"], hbm, load_traffic(args.traffic_json, name))
-                step_bytes = sum(algo_bytes(sw).values())
-                secondary[name] = {"queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1), "ms_per_step": round(s["ms"], 4),
-                                   "per_kernel_ms": {k: round(v, 4) for k, v in s["per_kernel_ms"].items()},
-                                   "step_GBps": round(step_bytes / (s["ms"] * 1e-3) / 1e9, 1),
-                                   "step_frac": round(step_bytes / (s["ms"] * 1e-3) / 1e9 / hbm, 4),
-                                   "roofline": rf, "status": s["status"]}
+                rf = roofline_of(sw, s["per_kernel_ms"], hbm, load_traffic(args.traffic_json, name), tflops)
+                line = {"queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1), "ms_per_step": round(s["ms"], 4),
+                        "per_kernel_ms": {k: round(v, 4) for k, v in s["per_kernel_ms"].items()}}
+                if prefill(sw):  # tensor-bound: the step's FLOPs against the bf16 peak
+                    step_tf = sum(algo_flops(sw).values()) / (s["ms"] * 1e-3) / 1e12
+                    line.update(step_TFLOPs=round(step_tf, 1), step_frac=round(step_tf / tflops, 4))
+                else:
+                    step_gbs = sum(algo_bytes(sw).values()) / (s["ms"] * 1e-3) / 1e9
+                    line.update(step_GBps=round(step_gbs, 1), step_frac=round(step_gbs / hbm, 4))
+                line.update(roofline=rf, status=s["status"])
+                secondary[name] = line
             except Exception as ex:  # report, do not hide
                 secondary[name] = {"error": repr(ex)}
             torch.cuda.empty_cache()
