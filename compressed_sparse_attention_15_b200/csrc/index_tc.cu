@@ -23,6 +23,13 @@
 // Each CTA walks a contiguous range of the flat (query, tile) space. Every
 // wait is bounded; a timeout raises CSA_STATUS_WAIT_TIMEOUT, all roles stop,
 // in-flight copies and MMAs are drained (bounded) and TMEM is freed.
+//
+// Prefill (several queries per sequence, bf16): kG = 4 queries of one
+// sequence share each key tile. Their 4 x 64 heads are the MMA's N (256):
+// one tile load and one M128 N256 product per 4 queries instead of four of
+// each, so the kernel becomes tensor-bound instead of tile-bound. The four
+// head blocks take 64 KB, so there is one query slot (a new group's block
+// loads once the last group's MMAs are done) and four key stages.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -40,21 +47,25 @@ constexpr int kThreads = 192;
 // dims (64 + 64), E4M3 tiles are 256 entries split along the rows (128 +
 // 128, one MMA row block each), so both formats pay the per-tile costs
 // (barriers, MMA issue, epilogue hand-off) once per 32 KB.
-template <bool kFp8>
+template <bool kFp8, int kG>
 struct Fmt {
+  static_assert(kG == 1 || (kG == 4 && !kFp8), "query groups: bf16 only");
   static constexpr int kElem = kFp8 ? 1 : 2;
-  static constexpr int kStages = 5;
+  static constexpr int kStages = kG == 1 ? 5 : 4;
+  static constexpr int kQSlots = kG == 1 ? 2 : 1;
   static constexpr int kSub = kFp8 ? 2 : 1;                // 128-row MMA blocks per tile
   static constexpr int kTileRows = 128 * kSub;
   static constexpr int kKBoxes = kFp8 ? 1 : 2;             // 128-byte K boxes per row (query block too)
   static constexpr int kKSteps = kFp8 ? 4 : 8;             // MMAs per row block (32 bytes of K each)
   static constexpr uint32_t kBoxBytes = 128 * 128;         // 16 KB
   static constexpr uint32_t kTileBytes = 2 * kBoxBytes;    // 32 KB
-  static constexpr uint32_t kQBytes = kHi * kDi * kElem;
-  static constexpr uint32_t kQBox = kQBytes / kKBoxes;      // 8 KB
-  static constexpr uint32_t kAccCols = 64 * kSub;          // TMEM columns of one accumulator
+  static constexpr uint32_t kQBytes = kG * kHi * kDi * kElem;  // one query group's head blocks
+  static constexpr uint32_t kQBox = kQBytes / kKBoxes;      // 8 KB (32 KB for 4 queries)
+  static constexpr uint32_t kAccCols = 64 * kSub * kG;     // TMEM columns of one accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
-  static constexpr uint32_t kIdesc = kFp8 ? tc::idesc_e4m3(128, 64) : tc::idesc_bf16(128, 64, 0, 0);
+  static constexpr uint32_t kIdesc = kFp8 ? tc::idesc_e4m3(128, 64) : tc::idesc_bf16(128, 64 * kG, 0, 0);
+  // per epilogue warp: its group's head weights and visible counts
+  static constexpr uint32_t kWBytes = kG == 1 ? 0 : 4 * (kG * kHi * 4 + kG * 4);
 };
 
 template <int kStages>
@@ -64,16 +75,20 @@ struct Bars {
   int abort;
 };
 
-template <bool kFp8>
+template <bool kFp8, int kG>
 constexpr size_t smem_bytes() {
-  return 1024 + Fmt<kFp8>::kStages * Fmt<kFp8>::kTileBytes + 2 * Fmt<kFp8>::kQBytes + sizeof(Bars<Fmt<kFp8>::kStages>);
+  using F = Fmt<kFp8, kG>;
+  return 1024 + F::kStages * F::kTileBytes + F::kQSlots * F::kQBytes + F::kWBytes + sizeof(Bars<F::kStages>);
 }
+static_assert(smem_bytes<false, 1>() <= 227 * 1024 && smem_bytes<true, 1>() <= 227 * 1024 &&
+                  smem_bytes<false, 4>() <= 227 * 1024,
+              "shared memory per block");
 
 struct Tile {
   int q, j0;
 };
 
-// Tile t of the flat (query, 128-entry tile) space. Every tile of a query's
+// Tile t of the flat (query group, 128-entry tile) space (q: the group). Every tile of a query's
 // row is loaded and multiplied; entries at or past the query's visible count
 // are only masked in the epilogue, so that no role waits on that count
 // before its first copy or MMA.
@@ -84,18 +99,19 @@ __device__ __forceinline__ Tile tile_of(long long t, int tiles_per_q, int tile_r
   return r;
 }
 
-template <bool kFp8>
+template <bool kFp8, int kG>
 __global__ void __launch_bounds__(kThreads, 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
                            ScoreArgs a, int tiles_per_q, long long total, long long per_cta) {
-  using F = Fmt<kFp8>;
+  using F = Fmt<kFp8, kG>;
   constexpr int kStages = F::kStages;
   constexpr uint32_t kTileBytes = F::kTileBytes, kQBytes = F::kQBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stage_buf = smem;
   uint8_t *q_buf = smem + kStages * kTileBytes;
-  Bars<kStages> *bars = reinterpret_cast<Bars<kStages> *>(q_buf + 2 * kQBytes);
+  float *w_buf = reinterpret_cast<float *>(q_buf + F::kQSlots * kQBytes);  // kG > 1: [4 warps][kG x 64 + kG]
+  Bars<kStages> *bars = reinterpret_cast<Bars<kStages> *>(q_buf + F::kQSlots * kQBytes + F::kWBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long t_begin = (long long)blockIdx.x * per_cta;
   const long long t_end = min(total, t_begin + per_cta);
@@ -134,18 +150,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (long long t = t_begin; t < t_end && !*abort; ++t) {
         const Tile tl = tile_of(t, tiles_per_q, F::kTileRows);
         if (tl.q != cur_q) {
-          const int slot = nq & 1;
-          const uint32_t qph = (nq >> 1) & 1;
+          const int slot = nq % F::kQSlots;
+          const uint32_t qph = (nq / F::kQSlots) & 1;
           if (!tc::mbar_wait(&bars->qempty[slot], qph ^ 1, abort, a.status)) break;
           tc::mbar_arrive_expect_tx(&bars->qfull[slot], kQBytes);
           for (int bx = 0; bx < F::kKBoxes; ++bx)
-            tc::tma_load_2d(q_buf + slot * kQBytes + bx * F::kQBox, &tm_qi, bx * 64, tl.q * kHi, &bars->qfull[slot]);
+            tc::tma_load_2d(q_buf + slot * kQBytes + bx * F::kQBox, &tm_qi, bx * 64, tl.q * kG * kHi,
+                            &bars->qfull[slot]);
           ++nq;
           cur_q = tl.q;
         }
         if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort, a.status)) break;
         tc::mbar_arrive_expect_tx(&bars->full[stage], kTileBytes);
-        const int row = (tl.q / a.q_per_seq) * a.N_max + tl.j0;
+        const int row = (tl.q * kG / a.q_per_seq) * a.N_max + tl.j0;
         for (int bx = 0; bx < 2; ++bx)  // bf16: dims 64 bx.., E4M3: rows 128 bx..
           tc::tma_load_2d(stage_buf + stage * kTileBytes + bx * F::kBoxBytes, &tm_ki, kFp8 ? 0 : 64 * bx,
                           kFp8 ? row + 128 * bx : row, &bars->full[stage]);
@@ -160,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // A phase that was already consumed completes the wait at once.
       for (int s = 0; s < kStages; ++s)
         if (issued_mask & (1u << s)) tc::mbar_drain(&bars->full[s], (issued_phase >> s) & 1);
-      for (int i = nq - 1; i >= 0 && i >= nq - 2; --i) tc::mbar_drain(&bars->qfull[i & 1], (i >> 1) & 1);
+      for (int i = nq - 1; i >= 0 && i >= nq - F::kQSlots; --i)
+        tc::mbar_drain(&bars->qfull[i % F::kQSlots], (i / F::kQSlots) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -171,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile tl = tile_of(t, tiles_per_q, F::kTileRows);
         if (tl.q != cur_q) {
           if (cur_q >= 0) tc::commit(&bars->qempty[slot]);  // old head block free once its MMAs finish
-          slot = nq & 1;
-          if (!tc::mbar_wait(&bars->qfull[slot], (nq >> 1) & 1, abort, a.status)) break;
+          slot = nq % F::kQSlots;
+          if (!tc::mbar_wait(&bars->qfull[slot], (nq / F::kQSlots) & 1, abort, a.status)) break;
           ++nq;
           cur_q = tl.q;
         }
@@ -209,6 +227,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       tc::commit(&bars->mma_done);
       tc::mbar_drain(&bars->mma_done, 0);
+    }
+  } else if constexpr (kG > 1) {
+    // Query groups: thread `row` owns one entry's 4 x 64 head products. Each
+    // epilogue warp keeps its own copy of the group's head weights in shared
+    // memory (no warp waits on another when the group changes).
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;
+    float *wq = w_buf + (warp - 2) * (kG * kHi + kG);
+    int *nq = reinterpret_cast<int *>(wq + kG * kHi);  // the group's visible counts
+    int acc = 0, cur_g = -1;
+    uint32_t accph = 0;
+    for (long long t = t_begin; t < t_end && !*abort; ++t) {
+      const Tile tl = tile_of(t, tiles_per_q, F::kTileRows);
+      if (tl.q != cur_g) {
+        __syncwarp();  // every lane is done with the previous group's weights
+        for (int i = lane; i < kG * kHi; i += 32) wq[i] = __ldg(a.wi + (size_t)tl.q * kG * kHi + i);
+        if (lane < kG) {
+          const int raw = a.n_cmp[tl.q * kG + lane];
+          if ((raw < 0 || raw > a.N_max) && row == lane) raise_status(a.status, CSA_STATUS_BAD_COUNT);
+          nq[lane] = raw < 0 ? 0 : (raw > a.N_max ? a.N_max : raw);
+        }
+        __syncwarp();
+        cur_g = tl.q;
+      }
+      const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
+      tc::fence_after_sync();
+      const int j = tl.j0 + row;
+#pragma unroll 1
+      for (int g = 0; g < kG; ++g) {
+        uint32_t v0[32], v1[32];
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * F::kAccCols + 64 * g;
+        tc::tmem_ld32(taddr, v0);
+        tc::tmem_ld32(taddr + 32, v1);
+        tc::tmem_ld_wait();
+        const float *wg = wq + g * kHi;
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) s = fmaf(wg[h], fmaxf(__uint_as_float(v0[h]), 0.f), s);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) s = fmaf(wg[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s);
+        if (j < nq[g]) a.scores[(size_t)(tl.q * kG + g) * a.N_max + j] = s;
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars->accempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        accph ^= 1;
+      }
     }
   } else {
     const int quarter = warp & 3;  // TMEM lanes this warp may access
@@ -308,37 +375,46 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 }  // namespace
 
-cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool *taken) {
-  *taken = false;
-  const bool fp8 = a.dtype == CSA_DTYPE_E4M3;
-  if (!(fp8 || a.dtype == CSA_DTYPE_BF16) || a.Hi != kHi || a.Di != kDi) return cudaSuccess;
-  if (!aligned16(a.qi) || !aligned16(a.ki) || (reinterpret_cast<uintptr_t>(a.wi) & 15)) return cudaSuccess;
-  if (fp8 && (reinterpret_cast<uintptr_t>(a.sq) & 15)) return cudaSuccess;
+namespace {
+
+// *taken stays false when no tensor map can describe these pointers (the
+// generic kernel then serves the call).
+template <bool kFp8, int kG>
+cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t stream, bool *taken) {
+  using F = Fmt<kFp8, kG>;
   CUtensorMap tm_ki, tm_qi;
-  const int esz = fp8 ? 1 : 2, box = fp8 ? 128 : 64;
-  auto mk = fp8 ? make_tmap_u8_2d : make_tmap_bf16_2d;
+  const int esz = kFp8 ? 1 : 2, box = kFp8 ? 128 : 64;
+  auto mk = kFp8 ? make_tmap_u8_2d : make_tmap_bf16_2d;
   if (!mk(&tm_ki, a.ki, kDi, (uint64_t)a.B * a.N_max, kDi * esz, box, 128)) return cudaSuccess;
-  if (!mk(&tm_qi, a.qi, kDi, (uint64_t)a.Q * kHi, kDi * esz, box, kHi)) return cudaSuccess;
-  const int tile_rows = fp8 ? Fmt<true>::kTileRows : Fmt<false>::kTileRows;
-  const int tiles_per_q = (a.N_max + tile_rows - 1) / tile_rows;
-  const long long total = (long long)a.Q * tiles_per_q;
+  if (!mk(&tm_qi, a.qi, kDi, (uint64_t)a.Q * kHi, kDi * esz, box, kG * kHi)) return cudaSuccess;
+  const int tiles_per_q = (a.N_max + F::kTileRows - 1) / F::kTileRows;
+  const long long total = (long long)(a.Q / kG) * tiles_per_q;
   long long grid = num_sms_cached();
   if (grid > total) grid = total;
   const long long per_cta = (total + grid - 1) / grid;
   grid = (total + per_cta - 1) / per_cta;
   static DeviceOnce attr;
   once_per_device(attr, [] {
-    cudaFuncSetAttribute(index_scores_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes<false>());
-    cudaFuncSetAttribute(index_scores_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes<true>());
+    cudaFuncSetAttribute(index_scores_tc_kernel<kFp8, kG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes<kFp8, kG>());
   });
   *taken = true;
-  if (fp8)
-    return launch_pdl(index_scores_tc_kernel<true>, dim3((unsigned)grid), dim3(kThreads), smem_bytes<true>(), stream,
-                      tm_ki, tm_qi, a, tiles_per_q, total, per_cta);
-  return launch_pdl(index_scores_tc_kernel<false>, dim3((unsigned)grid), dim3(kThreads), smem_bytes<false>(), stream,
-                    tm_ki, tm_qi, a, tiles_per_q, total, per_cta);
+  return launch_pdl(index_scores_tc_kernel<kFp8, kG>, dim3((unsigned)grid), dim3(kThreads), smem_bytes<kFp8, kG>(),
+                    stream, tm_ki, tm_qi, a, tiles_per_q, total, per_cta);
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores_tc(const ScoreArgs &a, cudaStream_t stream, bool *taken) {
+  *taken = false;
+  const bool fp8 = a.dtype == CSA_DTYPE_E4M3;
+  if (!(fp8 || a.dtype == CSA_DTYPE_BF16) || a.Hi != kHi || a.Di != kDi) return cudaSuccess;
+  if (!aligned16(a.qi) || !aligned16(a.ki) || (reinterpret_cast<uintptr_t>(a.wi) & 15)) return cudaSuccess;
+  if (fp8 && (reinterpret_cast<uintptr_t>(a.sq) & 15)) return cudaSuccess;
+  // Groups of 4 queries of one sequence share each key tile (prefill).
+  const bool groups = !fp8 && a.q_per_seq % 4 == 0 && a.Q % 4 == 0;
+  return fp8 ? launch_tc<true, 1>(a, stream, taken) : groups ? launch_tc<false, 4>(a, stream, taken)
+                                                           : launch_tc<false, 1>(a, stream, taken);
 }
 
 }  // namespace csa

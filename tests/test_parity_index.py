@@ -22,6 +22,8 @@ def _score_inputs(seed, Q, B, N, Hi, Di, dtype):
     (6, 3, 1000, 64, 128, torch.bfloat16),   # Flash indexer shape, ragged tail
     (5, 5, 300, 8, 32, torch.bfloat16),
     (4, 2, 129, 64, 128, torch.float32),
+    (16, 2, 1000, 64, 128, torch.bfloat16),  # 8 queries per sequence: groups of 4 share each key tile
+    (8, 1, 129, 64, 128, torch.bfloat16),    # one group pair over a full tile + 1 entry
 ])
 def test_index_scores_match_oracle(cuda_device, Q, B, N, Hi, Di, dtype):
     qi, wi, ki = _score_inputs(1, Q, B, N, Hi, Di, dtype)
