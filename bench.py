@@ -28,6 +28,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -194,13 +195,14 @@ class Clocks:
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device):
+    def __init__(self, device, path=None):
         try:
             self.idx = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
             self.idx = str(torch.cuda.current_device())
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # the raw samples (the JSON line carries their summary)
+        self.path = path or os.path.join(tempfile.gettempdir(), f"csa_bench_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
@@ -294,7 +296,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
 
     K = args.steps if not secondary else max(10, args.steps // 4)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    clocks = Clocks(device)
+    clocks = Clocks(device, args.clock_log)
     _sync_barrier(dist_on)
     wall0 = time.perf_counter()
     with clocks:
@@ -536,6 +538,8 @@ def main():
     ap.add_argument("--workload", default="csa_decode_64k", choices=[n for n in WL.WORKLOADS if n != "tiny_csa_prefill_fp32"])
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None,
+                    help="file for the nvidia-smi samples taken during the timed region (default: a temporary file)")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
     ap.add_argument("--once", action="store_true",
                     help="profiling aid: build the step without a graph and launch each of its kernels once more")
