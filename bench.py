@@ -150,7 +150,7 @@ class Step:
         t = self.t
         self.ds = DecodeStep(
             q=t["q"], kv_cmp=t["kv_cmp"], kv_win=t["kv_win"], sink=t["sink"], scale=w.scale, win_len=w.W,
-            win_end=w.win_end().to(device), n_cmp=ops.visible_entries(w.positions(), w.win, w.stride).to(device),
+            win_end=w.win_end().to(device), n_cmp=ops.visible_entries(w.positions().to(device), w.win, w.stride),
             ape=t["ape"], norm_w=WL.norm_w(w, device), gate=t["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
             win=w.win, stride=w.stride, qi=t.get("qi"), wi=t.get("wi"), ki=t.get("ki"),
             k=w.k if w.mode == "csa" else None, graph=graph,

@@ -15,6 +15,7 @@ from .ops import (  # noqa: F401
     index_topk,
     sparse_mqa,
     topk,
+    num_entries,
     visible_entries,
     workspace_status,
 )

@@ -46,6 +46,9 @@ SIGNATURES = {
     "csa_workspace_status": (_I, [_P, _P, ctypes.POINTER(ctypes.c_uint32)]),
     "csa_launch_count": (ctypes.c_ulonglong, []),
     "csa_index_topk_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "csa_num_entries": (_LL, [_LL, _I, _I]),
+    "csa_visible_counts_host": (_I, [_P, _LL, _I, _I, _P]),
+    "csa_visible_counts": (_I, [_P, _LL, _I, _I, _P, _P]),
 }
 
 _lib = None

@@ -194,6 +194,22 @@ int csa_topk(const float *scores, const int32_t *n_cmp, int k, int32_t *out_idx,
                              ws_bytes - kStatusBytes));
 }
 
+}  // extern "C"
+
+// The host-side checks of csa_index_topk's arguments other than the
+// workspace (also run by the entry point without allocation before it
+// touches its built-in buffer).
+int csa::check_index_topk(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int k,
+                          const int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max, int q_per_seq, int dtype) {
+  int rc = check_scores(qi, wi, ki, n_cmp, Q, B, Hi, Di, N_max, q_per_seq, dtype);
+  if (rc) return rc;
+  if (!out_idx || (reinterpret_cast<uintptr_t>(out_idx) & 3) || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  return CSA_OK;
+}
+
+extern "C" {
+
 int csa_index_topk(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int k, int32_t *out_idx,
                    int Q, int B, int Hi, int Di, int N_max, int q_per_seq, int dtype, void *ws, size_t ws_bytes,
                    csa_stream_t stream) {

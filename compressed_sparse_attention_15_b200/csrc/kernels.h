@@ -100,6 +100,11 @@ struct TopkArgs {
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, size_t scratch_bytes);
 size_t topk_scratch_bytes(int Q, int N_max, int k);
 
+// Host-side checks of csa_index_topk's arguments other than the workspace
+// (CSA_OK or the code csa_index_topk would return).
+int check_index_topk(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int k,
+                     const int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max, int q_per_seq, int dtype);
+
 // ---------------------------------------------------------------- per-device setup
 // Kernel attributes are set, and device facts cached, once per device (a
 // process may drive several GPUs, from several host threads).

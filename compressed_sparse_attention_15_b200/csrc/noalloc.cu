@@ -28,19 +28,28 @@ namespace {
 constexpr size_t kScratchBytes = CSA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void *g_scratch_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+// Device address of g_noalloc_scratch, per device: looked up once per device
+// (the lookup runs under the lock of once_per_device, so concurrent first
+// calls from several host threads see one lookup) and read lock-free after.
+std::atomic<void *> g_scratch_ptr[csa::kMaxDevices];
 
-// Looks up (once per device) the device address of the scratch array.
 int scratch_on_current_device(void **out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA_ERR_CUDA;
-  if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CSA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= csa::kMaxDevices) return CSA_ERR_CUDA;
+  void *p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    static csa::DeviceOnce once;
+    csa::once_per_device(once, [dev] {
+      void *a = nullptr;
+      if (cudaGetSymbolAddress(&a, g_noalloc_scratch) == cudaSuccess && a)
+        g_scratch_ptr[dev].store(a, std::memory_order_release);
+      else
+        cudaGetLastError();
+    });
+    p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!p) return CSA_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return CSA_OK;
 }
 
@@ -51,6 +60,10 @@ extern "C" int csa_index_topk_noalloc(const void *qi, const float *wi, const voi
                                       int dtype, csa_stream_t stream) {
   if (Q < 1 || N_max < 1 || k < 1) return CSA_ERR_INVALID;
   if (csa_index_topk_workspace_bytes(Q, N_max, k) > kScratchBytes) return CSA_ERR_SCRATCH_LIMIT;
+  // csa_index_topk's own argument checks, before anything is written to the
+  // shared buffer: a rejected call leaves it untouched.
+  const int chk = csa::check_index_topk(qi, wi, ki, n_cmp, k, out_idx, Q, B, Hi, Di, N_max, q_per_seq, dtype);
+  if (chk != CSA_OK) return chk;
   void *scratch = nullptr;
   const int rc = scratch_on_current_device(&scratch);
   if (rc != CSA_OK) return rc;

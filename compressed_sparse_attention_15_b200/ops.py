@@ -74,11 +74,27 @@ def workspace_status(ws: torch.Tensor) -> int:
 
 
 def visible_entries(p: torch.Tensor, win: int, stride: int) -> torch.Tensor:
-    """int32 count of compressed entries whose window ends at or before each
-    position p (entry j covers tokens j*stride .. j*stride + win - 1)."""
-    p = torch.as_tensor(p, dtype=torch.int64)
-    n = torch.div(p + 1 - win, stride, rounding_mode="floor") + 1
-    return n.clamp_min(0).to(torch.int32)
+    """int32 count of compressed entries visible at each position p
+    (csa_visible_counts on a CUDA tensor, one kernel on the current stream;
+    csa_visible_counts_host on a CPU tensor). Returns a tensor on p's device."""
+    p = torch.as_tensor(p, dtype=torch.int64).contiguous()
+    out = torch.empty(p.shape, dtype=torch.int32, device=p.device)
+    L = _lib.lib()
+    if p.is_cuda:
+        rc = L.csa_visible_counts(_ptr(p), p.numel(), int(win), int(stride), _ptr(out), _stream(p.device))
+        _lib.check("csa_visible_counts", rc)
+    else:
+        rc = L.csa_visible_counts_host(_ptr(p), p.numel(), int(win), int(stride), _ptr(out))
+        _lib.check("csa_visible_counts_host", rc)
+    return out
+
+
+def num_entries(T: int, win: int, stride: int) -> int:
+    """Entries a compressor run over T raw tokens makes (csa_num_entries)."""
+    n = _lib.lib().csa_num_entries(int(T), int(win), int(stride))
+    if n < 0:
+        raise ValueError(f"invalid window geometry win={win} stride={stride} T={T}")
+    return int(n)
 
 
 # ------------------------------------------------------------------ A1
@@ -103,7 +119,7 @@ def compress(kv, gate, ape, norm_w, win: int, stride: int, out=None, ratio=None,
     for t, nm in ((kv, "kv"), (gate, "gate")):
         if t.shape != (B, T, D) or t.stride(2) != 1 or t.stride(1) != D:
             raise ValueError(f"{nm} must be [B, T, D] with contiguous [T, D] rows")
-    N = (T - win) // stride + 1 if T >= win else 0
+    N = num_entries(T, win, stride)
     if out is None:
         out = torch.empty((B, N, D), dtype=kv.dtype, device=kv.device)
     else:
@@ -142,7 +158,7 @@ def index_compress(kv, gate, ape, norm_w, win: int, stride: int, fp8: bool = Fal
     _need(ape, "ape", dtype=torch.float32, device=kv.device)
     _need(norm_w, "norm_w", dtype=torch.float32, device=kv.device)
     B, T, D = kv.shape
-    N = (T - win) // stride + 1 if T >= win else 0
+    N = num_entries(T, win, stride)
     out = torch.empty((B, N, D), dtype=torch.uint8 if fp8 else kv.dtype, device=kv.device)
     scales = torch.empty((B, N), dtype=torch.float32, device=kv.device) if fp8 else None
     rc = _lib.lib().csa_index_compress(

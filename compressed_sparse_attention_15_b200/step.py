@@ -36,7 +36,7 @@ class DecodeStep:
         self.ape, self.norm_w, self.gate = ape, norm_w, gate
         self.win, self.stride = int(win), int(stride)
         T_c = gate.shape[1]
-        n_new = (T_c - self.win) // self.stride + 1
+        n_new = ops.num_entries(T_c, self.win, self.stride)
         self.kv_src = kv_win[:, append_src0:append_src0 + T_c]
         self.cmp_dst = kv_cmp[:, append_dst0:append_dst0 + n_new]
         self.qi, self.wi, self.ki, self.k = qi, wi, ki, k

@@ -77,6 +77,35 @@ enum {
 const char *csa_strerror(int code);
 
 /* ------------------------------------------------------------------------
+ * csa_num_entries, csa_visible_counts -- how many compressed entries exist,
+ * and how many a query may read.
+ *
+ * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: the compressor
+ * folds each window of raw tokens into one entry (CSA: windows of 8 tokens
+ * every 4, overlapping; HCA: 128 every 128). Entry j covers tokens
+ * j*stride .. j*stride + win - 1 (the reading of the window geometry used by
+ * csa_compress), and a query at position p may read it iff its whole window
+ * lies at or before p:  j*stride + win - 1 <= p.  Hence
+ *     n(p) = 0 if p + 1 < win,  else (p + 1 - win) / stride + 1,
+ * the number of complete windows in the first p + 1 tokens.
+ *
+ * csa_num_entries: entries a compressor run over T tokens makes (n(T - 1));
+ *   host-only, no GPU needed. Returns -1 if win < 1, stride < 1 or T < 0.
+ * csa_visible_counts_host: n_cmp[q] = n(pos[q]) for q < Q on HOST arrays
+ *   (pos int64, 8-byte aligned; n_cmp int32); no GPU needed.
+ * csa_visible_counts: the same on DEVICE arrays, one kernel on `stream`;
+ *   the result is the n_cmp argument of csa_index_topk / hca_mqa /
+ *   csa_topk_sparse_mqa for queries at positions pos.
+ * Negative positions count 0; counts above INT32_MAX are clamped to it.
+ * Both return CSA_ERR_INVALID (Q < 0, win < 1, stride < 1, a null or
+ * misaligned pointer with Q > 0) before any work, CSA_ERR_CUDA if the launch
+ * fails (for example without an sm_100 device), else CSA_OK. Q = 0 does nothing.
+ * ---------------------------------------------------------------------- */
+long long csa_num_entries(long long T, int win, int stride);
+int csa_visible_counts_host(const int64_t *pos, long long Q, int win, int stride, int32_t *n_cmp);
+int csa_visible_counts(const int64_t *pos, long long Q, int win, int stride, int32_t *n_cmp, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * csa_compress -- gated-pooling KV compressor followed by RMSNorm.
  *
  * Defined by "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: a

@@ -49,7 +49,7 @@ def test_csa_decode_step_chain(cuda_device):
     nw = WL.norm_w(w, cuda_device)
     ops.compress(d["kv_win"][:, w.c_src0:w.c_src0 + w.T_c], d["gate"], d["ape"], nw, w.win, w.stride,
                  out=d["kv_cmp"][:, w.c_dst0:w.c_dst0 + 1])
-    n = ops.visible_entries(w.positions(), w.win, w.stride).to(cuda_device)
+    n = ops.visible_entries(w.positions().to(cuda_device), w.win, w.stride)
     idx = ops.index_topk(d["qi"], d["wi"], d["ki"], n, w.k)
     out = ops.sparse_mqa(d["q"], d["kv_cmp"], idx, d["kv_win"], w.win_end().to(cuda_device), d["sink"], w.scale, w.W)
     torch.cuda.synchronize()
@@ -84,7 +84,7 @@ def test_fp8_indexer_decode_step_chain(cuda_device):
     d = {t: WL.make(w, t, cuda_device) for t in names}
     ds = DecodeStep(q=d["q"], kv_cmp=d["kv_cmp"], kv_win=d["kv_win"], sink=d["sink"], scale=w.scale, win_len=w.W,
                     win_end=w.win_end().to(cuda_device),
-                    n_cmp=ops.visible_entries(w.positions(), w.win, w.stride).to(cuda_device), ape=d["ape"],
+                    n_cmp=ops.visible_entries(w.positions().to(cuda_device), w.win, w.stride), ape=d["ape"],
                     norm_w=WL.norm_w(w, cuda_device), gate=d["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
                     win=w.win, stride=w.stride, qi8=d["qi8"], sq=d["sq"], wi=d["wi"], ki8=d["ki8"], sk=d["sk"],
                     k=w.k)

@@ -280,6 +280,30 @@ def test_quantize_rows_maps_the_row_maximum_to_448_and_bounds_the_error():
         assert np.all(err <= np.maximum(np.abs(x[r]) * 2.0 ** -4, 2.0 ** -10 * scales[r]) * 1.0001)
 
 
+def test_quantize_rows_scale_reproduces_the_row_maximum():
+    # Reading R19: the scale maps each row's largest magnitude onto the largest
+    # finite E4M3 value (448, S.1111.110), so decoding that code and
+    # multiplying by the scale gives the row maximum back, up to fp32
+    # rounding. A scale with another denominator (amax / 440, amax / 512)
+    # misses it by 2 % or more.
+    x = rng.standard_normal((64, 128)) * rng.uniform(1e-3, 1e3, (64, 1))
+    codes, scales = O.quantize_rows_e4m3(x)
+    amax = np.abs(x.astype(np.float32)).max(axis=1).astype(np.float64)
+    top = O.e4m3_decode(np.array([0x7E], dtype=np.uint8))[0]
+    assert top == 448.0
+    assert np.all(np.abs(top * scales.astype(np.float64) - amax) <= amax * 2.0 ** -22)
+
+
+def test_quantize_rows_hand_example():
+    # Row (3.5, -7, 1, 0): amax 7, scale 7 / 448 = 2^-6 exactly; the scaled
+    # values 224, -448, 64, 0 are all E4M3 values:
+    #   224 = 1.75 * 2^7 -> exponent field 7 + 7 = 14, mantissa .110 -> 0 1110 110 = 0x76
+    #  -448 = -1.75 * 2^8 -> 1 1111 110 = 0xFE;   64 = 2^6 -> 0 1101 000 = 0x68;   0 -> 0x00
+    codes, scales = O.quantize_rows_e4m3(np.array([[3.5, -7.0, 1.0, 0.0]]))
+    assert scales[0] == np.float32(2.0 ** -6)
+    assert codes[0].tolist() == [0x76, 0xFE, 0x68, 0x00]
+
+
 def test_hadamard_is_sylvester_and_orthonormal():
     import scipy.linalg
     for n in (1, 2, 16, 128):

@@ -36,6 +36,10 @@ def _inputs(seed, Q, B, N, Hi, Di, dtype, dev):
 @pytest.mark.parametrize("Q,B,N,Hi,Di,k,dtype", [
     (32, 32, 16383, 64, 128, 512, torch.bfloat16),   # the 64 K-context decode batch (tensor-core scorer)
     (12, 3, 3001, 4, 16, 16, torch.float32),         # small fp32 case (generic scorer)
+    # no cluster fits (75 queries on 148 SMs) and the lists exceed the one-block
+    # key cache: the two-stage selection, whose segment winners live in the
+    # shared buffer beyond the scores
+    (75, 75, 52000, 4, 16, 16, torch.float32),
 ])
 def test_noalloc_matches_the_workspace_entry_point_twice(cuda_device, Q, B, N, Hi, Di, k, dtype):
     L = _lib.lib()
@@ -66,3 +70,18 @@ def test_noalloc_rejects_requests_beyond_its_scratch(cuda_device):
     assert rc == CSA_ERR_SCRATCH_LIMIT
     assert "scratch" in _lib.strerror(rc)
     assert L.csa_launch_count() == before  # nothing was launched
+
+
+@pytest.mark.gpu
+def test_noalloc_rejects_bad_arguments_before_any_work(cuda_device):
+    L = _lib.lib()
+    x = torch.zeros(16, dtype=torch.int32, device=cuda_device)
+    before = L.csa_launch_count()
+    # Hi above the limit, then a misaligned output: rejected on the host like csa_index_topk
+    rc = L.csa_index_topk_noalloc(_p(x), _p(x), _p(x), _p(x), 8, _p(x), 4, 1, 129, 16, 64, 4, _lib.CSA_DTYPE_F32,
+                                  ctypes.c_void_p(0))
+    assert rc == 1
+    rc = L.csa_index_topk_noalloc(_p(x), _p(x), _p(x), _p(x), 8, ctypes.c_void_p(x.data_ptr() + 2), 4, 1, 4, 16, 64,
+                                  4, _lib.CSA_DTYPE_F32, ctypes.c_void_p(0))
+    assert rc == 1
+    assert L.csa_launch_count() == before
