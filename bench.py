@@ -98,6 +98,15 @@ def algo_flops(w: WL.Workload):
 # A step part whose algorithmic bytes and FLOPs are another's: the attention
 # with the selection made inside it moves what the attention moves.
 PART_ALIAS = {"topk_mqa": "mqa"}
+# The fused decode-step kernel moves the whole step's bytes.
+WHOLE_STEP = "decode_step"
+
+
+def part_amount(table, name):
+    """Algorithmic bytes (or FLOPs) of one step part."""
+    if name == WHOLE_STEP:
+        return sum(table.values())
+    return table.get(PART_ALIAS.get(name, name))
 
 
 def prefill(w: WL.Workload) -> bool:
@@ -169,7 +178,7 @@ class Step:
         split into its two kernels, scores then top-k, through their own entry
         points."""
         ds = self.ds
-        if not ds.csa or ds.fuse_select:
+        if not ds.csa or ds.fuse_select or ds.fused:
             return ds.parts()
         if self._scores is None:
             self._scores = torch.empty((self.w.Q, self.w.N), dtype=torch.float32, device=self.dev)
@@ -370,13 +379,13 @@ def roofline_of(w, per_kernel_ms, hbm_gbs, traffic=None, tflops=None):
     DRAM bytes per launch."""
     if prefill(w) and tflops:
         af = algo_flops(w)
-        name, fl = max(((k, af[PART_ALIAS.get(k, k)]) for k in per_kernel_ms if PART_ALIAS.get(k, k) in af),
+        name, fl = max(((k, part_amount(af, k)) for k in per_kernel_ms if part_amount(af, k) is not None),
                        key=lambda x: x[1])
         achieved = fl / (per_kernel_ms[name] * 1e-3) / 1e12
         return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1), "peak": tflops, "unit": "TFLOP/s",
                 "frac": round(achieved / tflops, 4), "traffic": (traffic or {}).get(name), "flops_per_launch": int(fl)}
     ab = algo_bytes(w)
-    best = max(((k, ab[PART_ALIAS.get(k, k)]) for k in per_kernel_ms if PART_ALIAS.get(k, k) in ab),
+    best = max(((k, part_amount(ab, k)) for k in per_kernel_ms if part_amount(ab, k) is not None),
                key=lambda x: x[1])
     name, nbytes = best
     traffic = (traffic or {}).get(name)

@@ -47,9 +47,32 @@ SIGNATURES = {
     "csa_launch_count": (ctypes.c_ulonglong, []),
     "csa_index_topk_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "csa_num_entries": (_LL, [_LL, _I, _I]),
+    "csa_last_cuda_error": (_I, []),
+    "csa_cuda_error_string": (ctypes.c_char_p, [_I]),
     "csa_visible_counts_host": (_I, [_P, _LL, _I, _I, _P]),
     "csa_visible_counts": (_I, [_P, _LL, _I, _I, _P, _P]),
 }
+
+
+
+class DecodeStepArgs(ctypes.Structure):
+    """csa_decode_step_args (include/csa.h), field for field."""
+    _fields_ = [
+        ("q", _P), ("kv_cmp", _P), ("kv_win", _P), ("win_end", _P), ("sink", _P), ("out", _P), ("n_cmp", _P),
+        ("qi", _P), ("sq", _P), ("wi", _P), ("ki", _P), ("sk", _P), ("idx_out", _P),
+        ("app_kv", _P), ("app_gate", _P), ("ape", _P), ("norm_w", _P), ("pos0", _P),
+        ("scale", _F),
+        ("Q", _I), ("B", _I), ("H", _I), ("D", _I), ("N_max", _I), ("win_len", _I), ("T_raw", _I),
+        ("q_per_seq", _I), ("dtype", _I),
+        ("index_dtype", _I), ("Hi", _I), ("Di", _I), ("k", _I),
+        ("app_win", _I), ("app_stride", _I), ("app_T", _I), ("rope_dims", _I),
+        ("app_kv_seq_stride", _LL), ("app_gate_seq_stride", _LL), ("app_row0", _LL),
+        ("rope_theta", ctypes.c_double),
+    ]
+
+
+SIGNATURES["csa_decode_step_workspace_bytes"] = (_SZ, [ctypes.POINTER(DecodeStepArgs)])
+SIGNATURES["csa_decode_step"] = (_I, [ctypes.POINTER(DecodeStepArgs), _P, _SZ, _P])
 
 _lib = None
 
@@ -57,7 +80,11 @@ _lib = None
 class CsaError(RuntimeError):
     def __init__(self, fn: str, code: int):
         self.code = code
-        super().__init__(f"{fn} failed: {strerror(code)}")
+        msg = f"{fn} failed: {strerror(code)}"
+        if code == 4:  # CSA_ERR_CUDA: name the CUDA error behind it
+            e = lib().csa_last_cuda_error()
+            msg += f" ({e}: {lib().csa_cuda_error_string(e).decode()})"
+        super().__init__(msg)
 
 
 def lib() -> ctypes.CDLL:

@@ -13,6 +13,8 @@ using namespace csa;
 namespace csa {
 static unsigned long long g_launches = 0;
 void note_launches(unsigned n) { __atomic_fetch_add(&g_launches, (unsigned long long)n, __ATOMIC_RELAXED); }
+static thread_local int g_last_cuda_error = 0;
+void note_cuda_error(cudaError_t e) { g_last_cuda_error = (int)e; }
 }  // namespace csa
 
 namespace {
@@ -42,7 +44,11 @@ bool elem_aligned(const void *p, int dtype) {
 }
 uint32_t *status_of(void *ws) { return static_cast<uint32_t *>(ws); }
 
-int cuda_rc(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+int cuda_rc(cudaError_t e) {
+  if (e == cudaSuccess) return CSA_OK;
+  note_cuda_error(e);
+  return CSA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -355,6 +361,10 @@ int hca_mqa(const void *q, const void *kv_cmp, const void *kv_win, const float *
 }
 
 unsigned long long csa_launch_count(void) { return __atomic_load_n(&csa::g_launches, __ATOMIC_RELAXED); }
+
+int csa_last_cuda_error(void) { return csa::g_last_cuda_error; }
+
+const char *csa_cuda_error_string(int code) { return cudaGetErrorString((cudaError_t)code); }
 
 int csa_workspace_status(void *ws, csa_stream_t stream, uint32_t *status) {
   if (!ws || !status) return CSA_ERR_INVALID;

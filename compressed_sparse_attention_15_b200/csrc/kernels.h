@@ -15,6 +15,8 @@ namespace csa {
 
 // Process-wide count of kernel launches made by the library.
 void note_launches(unsigned n);
+// Remember (per host thread) a CUDA error a call returns as CSA_ERR_CUDA.
+void note_cuda_error(cudaError_t e);
 
 // Launch with programmatic stream serialization: the kernel may begin while
 // its predecessor in the stream finishes (it calls pdl_wait() before reading

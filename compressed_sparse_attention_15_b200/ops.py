@@ -54,8 +54,8 @@ class Workspace:
     def get(self, nbytes: int) -> torch.Tensor:
         nbytes = max(256, int(nbytes))
         if self.buf is None or self.buf.numel() < nbytes:
-            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-            self.buf[:256].zero_()
+            # zero-filled: the status word, and the counters of csa_decode_step
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         return self.buf
 
     def status(self) -> int:
@@ -375,4 +375,79 @@ def hca_mqa(q, kv_cmp, n_cmp, kv_win, win_end, sink, scale: float, win_len: int,
                    _ptr(n_cmp), int(win_len), _ptr(win_end), T_raw, qps, _dtype_code(q), _ptr(w), w.numel(),
                    _stream(q.device))
     _lib.check("hca_mqa", rc)
+    return out
+
+
+# ------------------------------------------------------- the whole decode step
+
+def decode_step(q, kv_cmp, kv_win, win_end, sink, scale: float, win_len: int, n_cmp, *, qi=None, wi=None, ki=None,
+                k: int | None = None, qi8=None, sq=None, ki8=None, sk=None, append=None, out=None, idx_out=None,
+                q_per_seq=None, ws: Workspace | None = None):
+    """One decode step in one call (csa_decode_step): the cache append, then
+    for CSA (qi or qi8 given) the indexer top-k and the sparse attention, for
+    HCA the dense attention over the n_cmp visible entries.
+
+    append = None or a dict with kv, gate ([B, T, D], rows contiguous, any
+    sequence stride), ape, norm_w, win, stride, row0 (first cache row written)
+    and optionally rope = (rope_dims, theta, pos0 int64 [B] or None).
+    Returns out [Q, H, D] (and fills idx_out [Q, k] for CSA)."""
+    Q, H, D, B, N_max, T_raw, qps = _mqa_common(q, kv_cmp, kv_win, win_end, sink, q_per_seq)
+    _need(n_cmp, "n_cmp", dtype=torch.int32, device=q.device)
+    if n_cmp.shape != (Q,):
+        raise ValueError("n_cmp must be [Q]")
+    a = _lib.DecodeStepArgs()
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", dtype=q.dtype, device=q.device)
+    a.q, a.kv_cmp, a.kv_win, a.win_end, a.sink, a.out, a.n_cmp = (
+        _ptr(q), _ptr(kv_cmp), _ptr(kv_win), _ptr(win_end), _ptr(sink), _ptr(out), _ptr(n_cmp))
+    a.scale = float(scale)
+    a.Q, a.B, a.H, a.D, a.N_max, a.win_len, a.T_raw, a.q_per_seq = Q, B, H, D, N_max, int(win_len), T_raw, qps
+    a.dtype = _dtype_code(q)
+    fp8 = qi8 is not None
+    if qi is not None or fp8:
+        if k is None:
+            raise ValueError("k is required for a CSA step")
+        if fp8:
+            _index_fp8_common(qi8, sq, wi, ki8, sk, n_cmp, qps)
+            a.qi, a.sq, a.wi, a.ki, a.sk = _ptr(qi8), _ptr(sq), _ptr(wi), _ptr(ki8), _ptr(sk)
+            a.index_dtype = _lib.CSA_DTYPE_E4M3
+            a.Hi, a.Di = qi8.shape[1], qi8.shape[2]
+        else:
+            _index_common(qi, wi, ki, n_cmp, qps)
+            a.qi, a.wi, a.ki = _ptr(qi), _ptr(wi), _ptr(ki)
+            a.index_dtype = _dtype_code(qi)
+            a.Hi, a.Di = qi.shape[1], qi.shape[2]
+        if idx_out is None:
+            idx_out = torch.empty((Q, int(k)), dtype=torch.int32, device=q.device)
+        _need(idx_out, "idx_out", dtype=torch.int32, device=q.device)
+        if idx_out.shape != (Q, int(k)):
+            raise ValueError("idx_out must be [Q, k]")
+        a.idx_out = _ptr(idx_out)
+        a.k = int(k)
+    if append is not None:
+        kv, gate = append["kv"], append["gate"]
+        _need(kv, "append kv", dtype=q.dtype, device=q.device, contiguous=False)
+        _need(gate, "append gate", dtype=q.dtype, device=q.device, contiguous=False)
+        _need(append["ape"], "ape", dtype=torch.float32, device=q.device)
+        _need(append["norm_w"], "norm_w", dtype=torch.float32, device=q.device)
+        if kv.dim() != 3 or kv.shape[0] != B or kv.shape[2] != D or kv.stride(2) != 1 or kv.stride(1) != D:
+            raise ValueError("append kv must be [B, T, D] with contiguous [T, D] rows")
+        if gate.shape != kv.shape or gate.stride(2) != 1 or gate.stride(1) != D:
+            raise ValueError("append gate must match append kv")
+        a.app_kv, a.app_gate, a.ape, a.norm_w = _ptr(kv), _ptr(gate), _ptr(append["ape"]), _ptr(append["norm_w"])
+        a.app_win, a.app_stride, a.app_T = int(append["win"]), int(append["stride"]), kv.shape[1]
+        a.app_kv_seq_stride, a.app_gate_seq_stride = kv.stride(0), gate.stride(0)
+        a.app_row0 = int(append["row0"])
+        rope = append.get("rope")
+        if rope is not None:
+            rope_dims, theta, pos0 = rope
+            if pos0 is not None:
+                _need(pos0, "pos0", dtype=torch.int64, device=q.device)
+                a.pos0 = _ptr(pos0)
+            a.rope_dims, a.rope_theta = int(rope_dims), float(theta)
+    L = _lib.lib()
+    w = (ws or Workspace(q.device)).get(L.csa_decode_step_workspace_bytes(ctypes.byref(a)))
+    rc = L.csa_decode_step(ctypes.byref(a), _ptr(w), w.numel(), _stream(q.device))
+    _lib.check("csa_decode_step", rc)
     return out

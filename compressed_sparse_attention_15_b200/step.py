@@ -10,9 +10,13 @@ The step over device-resident caches is:
      (csa_index_topk, or csa_index_topk_fp8 with FP8 indexer inputs);
   3. attend over the selected (CSA) or all visible (HCA) entries + the
      sliding window + the per-head sink (csa_sparse_mqa / hca_mqa).
-With fuse_select=True, a CSA step only scores in 2 (csa_index_scores(_fp8))
-and 3 is csa_topk_sparse_mqa, which makes the selection inside the attention
-kernel where its launch plan allows.
+With fused=True (the default) the whole step is one csa_decode_step call:
+one persistent kernel in which the selection and attention of some queries
+overlap the indexer key scan of others (the separate kernels serve shapes it
+does not take). With fused=False the parts are separate calls; there,
+fuse_select=True makes a CSA step only score in 2 (csa_index_scores(_fp8))
+and run 3 as csa_topk_sparse_mqa, the selection inside the attention kernel
+where its launch plan allows.
 The library never allocates or synchronises, so the launches are captured
 once into a CUDA graph and each step is one graph launch. Buffers are bound
 at construction; later steps see whatever the caller wrote into them.
@@ -28,7 +32,8 @@ class DecodeStep:
     def __init__(self, *, q, kv_cmp, kv_win, sink, scale: float, win_len: int, win_end, n_cmp,
                  ape, norm_w, gate, append_src0: int, append_dst0: int, win: int, stride: int,
                  qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True,
-                 qi8=None, sq=None, ki8=None, sk=None, append_rope=None, fuse_select: bool = False):
+                 qi8=None, sq=None, ki8=None, sk=None, append_rope=None, fuse_select: bool = False,
+                 fused: bool = True):
         self.fp8 = qi8 is not None
         self.csa = qi is not None or self.fp8
         self.q, self.kv_cmp, self.kv_win, self.sink = q, kv_cmp, kv_win, sink
@@ -45,7 +50,9 @@ class DecodeStep:
         dev = q.device
         self.out = out if out is not None else torch.empty_like(q)
         self.idx = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev) if self.csa else None
-        self.fuse_select = bool(fuse_select) and self.csa
+        self.fused = bool(fused)
+        self.fuse_select = bool(fuse_select) and self.csa and not self.fused
+        self.append_src0, self.append_dst0 = int(append_src0), int(append_dst0)
         self.scores = (torch.empty((q.shape[0], kv_cmp.shape[1]), dtype=torch.float32, device=dev)
                        if self.fuse_select else None)
         self.ws_index = ops.Workspace(dev)
@@ -89,7 +96,25 @@ class DecodeStep:
             ops.hca_mqa(self.q, self.kv_cmp, self.n_cmp, self.kv_win, self.win_end, self.sink, self.scale,
                         self.win_len, out=self.out, ws=self.ws_mqa)
 
+    def step(self):
+        """The whole step as one csa_decode_step call."""
+        append = {"kv": self.kv_src, "gate": self.gate, "ape": self.ape, "norm_w": self.norm_w, "win": self.win,
+                  "stride": self.stride, "row0": self.append_dst0, "rope": self.append_rope}
+        if self.fp8:
+            ops.decode_step(self.q, self.kv_cmp, self.kv_win, self.win_end, self.sink, self.scale, self.win_len,
+                            self.n_cmp, qi8=self.qi8, sq=self.sq, wi=self.wi, ki8=self.ki8, sk=self.sk, k=self.k,
+                            append=append, out=self.out, idx_out=self.idx, ws=self.ws_index)
+        elif self.csa:
+            ops.decode_step(self.q, self.kv_cmp, self.kv_win, self.win_end, self.sink, self.scale, self.win_len,
+                            self.n_cmp, qi=self.qi, wi=self.wi, ki=self.ki, k=self.k, append=append, out=self.out,
+                            idx_out=self.idx, ws=self.ws_index)
+        else:
+            ops.decode_step(self.q, self.kv_cmp, self.kv_win, self.win_end, self.sink, self.scale, self.win_len,
+                            self.n_cmp, append=append, out=self.out, ws=self.ws_index)
+
     def parts(self):
+        if self.fused:
+            return [("decode_step", self.step)]
         p = [("compress", self.append)]
         if self.fuse_select:
             p += [("index_scores", self.select), ("topk_mqa", self.attend)]
@@ -100,6 +125,9 @@ class DecodeStep:
         return p
 
     def _launch(self):
+        if self.fused:
+            self.step()
+            return
         main = torch.cuda.current_stream()
         if self.csa:
             # the append only feeds the attention: overlap it with the indexer

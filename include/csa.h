@@ -359,9 +359,86 @@ int csa_index_topk_noalloc(const void *qi, const float *wi, const void *ki, cons
                            int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max, int q_per_seq,
                            int dtype, csa_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * csa_decode_step -- one whole decode step of a CSA or HCA layer in one call:
+ * the cache append, then (CSA) the indexer scores and top-k, then the
+ * attention over the selection (CSA) or all visible entries (HCA) plus the
+ * window and the sink.
+ *
+ * "DeepSeek-V4 Architecture Analysis", INNOVATIONS section 1: each step
+ * folds the newest raw window into the compressed cache, the indexer selects
+ * the top-k compressed entries (CSA), and the core attention reads them with
+ * the 128-token sliding window and the per-head sink; HCA attends to every
+ * compressed entry. The results are those of the separate calls in order:
+ *   1. if app_kv != NULL: csa_compress (csa_compress_rope if rope_dims > 0)
+ *      of app_kv / app_gate [B, app_T, D] (sequence strides app_kv_seq_stride,
+ *      app_gate_seq_stride; 0 = app_T * D) with ape [app_win, D], norm_w [D],
+ *      window app_win, stride app_stride (= ratio), writing its
+ *      N_new = (app_T - app_win) / app_stride + 1 entries of sequence b to
+ *      kv_cmp[b, app_row0 .. app_row0 + N_new) (app_row0 + N_new <= N_max);
+ *   2. CSA (qi != NULL): csa_index_topk (index_dtype CSA_DTYPE_BF16) or
+ *      csa_index_topk_fp8 (CSA_DTYPE_E4M3, with sq / sk) into idx_out [Q, k],
+ *      then csa_sparse_mqa over idx_out;
+ *      HCA (qi == NULL): hca_mqa over the entries j < n_cmp[q].
+ * Every argument keeps the meaning, layout and limits it has in those calls.
+ *
+ * For bf16 attention with H = 64 or 128, D = 512, one query per sequence
+ * (q_per_seq = 1) and the indexer shape 64 x 128, the step is ONE persistent
+ * kernel: each SM pulls tasks (append, key-tile chunks, top-k, attention
+ * splits, split merges) from device-side queues as their inputs complete,
+ * so the selection and attention of some queries overlap the key scan of
+ * others. Other shapes run the separate kernels. Split plans differ from the
+ * separate calls', so outputs agree with them to rounding, not bit for bit.
+ *
+ * Workspace: csa_decode_step_workspace_bytes(args) bytes, 256-byte aligned,
+ * zero-filled before the first call (cudaMemset once); the step leaves its
+ * counters at zero for the next call. Bytes 0..3 hold the status word (as for
+ * every call); bytes 8..15 may hold a limit in nanoseconds for every bounded
+ * wait of the fused kernel (0 = 2 s; for tests of the timeout path).
+ * Calls sharing one workspace must not overlap on the GPU.
+ * Returns CSA_ERR_INVALID / CSA_ERR_WORKSPACE before any launch.
+ * ---------------------------------------------------------------------- */
+typedef struct csa_decode_step_args {
+  /* attention: as csa_sparse_mqa / hca_mqa */
+  const void *q;           /* [Q, H, D] */
+  const void *kv_cmp;      /* [B, N_max, D] (the append writes into it) */
+  const void *kv_win;      /* [B, T_raw, D] */
+  const int32_t *win_end;  /* [Q] */
+  const float *sink;       /* [H] */
+  void *out;               /* [Q, H, D] */
+  const int32_t *n_cmp;    /* [Q] visible entries per query */
+  /* indexer (CSA): qi == NULL selects HCA */
+  const void *qi;          /* [Q, Hi, Di] (uint8 codes for E4M3) */
+  const float *sq;         /* [Q, Hi] (E4M3 only) */
+  const float *wi;         /* [Q, Hi] */
+  const void *ki;          /* [B, N_max, Di] (uint8 codes for E4M3) */
+  const float *sk;         /* [B, N_max] (E4M3 only) */
+  int32_t *idx_out;        /* [Q, k] the selection */
+  /* append (app_kv == NULL: none) */
+  const void *app_kv;
+  const void *app_gate;
+  const float *ape;
+  const float *norm_w;
+  const int64_t *pos0;     /* RoPE positions (csa_compress_rope), may be NULL */
+  float scale;
+  int Q, B, H, D, N_max, win_len, T_raw, q_per_seq, dtype;
+  int index_dtype, Hi, Di, k;
+  int app_win, app_stride, app_T, rope_dims;
+  long long app_kv_seq_stride, app_gate_seq_stride, app_row0;
+  double rope_theta;
+} csa_decode_step_args;
+
+size_t csa_decode_step_workspace_bytes(const csa_decode_step_args *args);
+int csa_decode_step(const csa_decode_step_args *args, void *ws, size_t ws_bytes, csa_stream_t stream);
+
 /* Number of kernels this library has launched in this process so far
  * (a monotonically increasing counter, for profiling and tests). */
 unsigned long long csa_launch_count(void);
+
+/* The CUDA error code (cudaError_t) behind the last CSA_ERR_CUDA this host
+ * thread received from the library (0 if none), and its text. */
+int csa_last_cuda_error(void);
+const char *csa_cuda_error_string(int code);
 
 /* Synchronises `stream`, copies the workspace status word into *status and
  * clears it. Returns CSA_OK if it was zero, CSA_ERR_DEVICE if not,

@@ -1,0 +1,285 @@
+"""The whole decode step in one call (csa_decode_step, the persistent fused
+kernel): the cache append, the indexer top-k and the sparse attention (CSA),
+or the append and the dense attention (HCA), against the fp64 oracle's chain
+on the same seeded inputs, and against the separate kernels."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from compressed_sparse_attention_15_b200 import _lib, ops, synth, workloads as WL
+from compressed_sparse_attention_15_b200.step import DecodeStep
+from helpers import assert_close, check_topk_set
+
+pytestmark = pytest.mark.gpu
+
+
+# ---------------------------------------------------------------- oracle side
+
+def oracle_selection(qi, wi, ki_b, n, k, fp8=None):
+    """The oracle's indexer scores and top-k of one query over n entries."""
+    if fp8 is not None:
+        sq, sk_b = fp8
+        s = O.index_scores_fp8(qi.numpy(), sq, wi, ki_b.numpy(), sk_b, n)
+    else:
+        s = O.index_scores(qi, wi, ki_b, n)
+    return O.topk(s, k), s
+
+
+def oracle_out(q_heads, rows_cmp, kv_win_b, e, W, sink, scale):
+    rows = np.concatenate([np.asarray(rows_cmp, dtype=np.float64).reshape(-1, q_heads.shape[-1]),
+                           O.window_rows(kv_win_b, e, W)])
+    return O.attend(q_heads, rows, sink, scale)[0]
+
+
+def appended_rows(raw, gate, ape, win, stride, rope=None):
+    """The oracle's entries of the step's append, rounded to the cache dtype."""
+    c = O.compress(raw, gate, ape, np.ones(raw.shape[-1]), win, stride)
+    if rope is not None:
+        rope_dims, theta, p0 = rope
+        c = O.rope_last_dims(c, p0 + np.arange(c.shape[0]) * stride + win - 1, theta, rope_dims)
+    return O.round_to(c, "bf16")
+
+
+# ---------------------------------------------------------------- full size
+
+def _decode_step(w, dev, fused=True):
+    fp8 = w.index_fmt == "e4m3"
+    names = ["q", "kv_cmp", "kv_win", "sink", "gate", "ape"]
+    if w.mode == "csa":
+        names += ["qi8", "sq", "wi", "ki8", "sk"] if fp8 else ["qi", "wi", "ki"]
+    d = {t: WL.make(w, t, dev) for t in names}
+    ds = DecodeStep(q=d["q"], kv_cmp=d["kv_cmp"], kv_win=d["kv_win"], sink=d["sink"], scale=w.scale, win_len=w.W,
+                    win_end=w.win_end().to(dev), n_cmp=ops.visible_entries(w.positions().to(dev), w.win, w.stride),
+                    ape=d["ape"], norm_w=WL.norm_w(w, dev), gate=d["gate"], append_src0=w.c_src0,
+                    append_dst0=w.c_dst0, win=w.win, stride=w.stride, qi=d.get("qi"), wi=d.get("wi"),
+                    ki=d.get("ki"), qi8=d.get("qi8"), sq=d.get("sq"), ki8=d.get("ki8"), sk=d.get("sk"),
+                    k=w.k if w.mode == "csa" else None, fused=fused)
+    return ds, d
+
+
+def _check_full(w, ds, queries):
+    out = ds.out.cpu()
+    idx_h = ds.idx.cpu().numpy() if ds.idx is not None else None
+    ape, sink = WL.make(w, "ape"), WL.make(w, "sink")
+    fp8 = w.index_fmt == "e4m3"
+    if fp8:
+        qi8, sq, wi = (WL.make(w, t) for t in ("qi8", "sq", "wi"))
+    compared = 0
+    for q in queries:
+        b = q
+        raw = WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.c_src0, w.c_src0 + w.T_c))
+        gate = WL.rows(w, "gate", b * w.T_c + torch.arange(w.T_c))
+        new = appended_rows(raw, gate, ape, w.win, w.stride)[0]
+        kv_win_b = WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.T_raw))
+        qh = WL.rows(w, "q", q * w.H + torch.arange(w.H))
+        e = int(w.win_end()[q])
+        if w.mode == "csa":
+            rows = torch.arange(b * w.N, (b + 1) * w.N)
+            if fp8:
+                ref_idx, ref_s = oracle_selection(qi8[q], wi[q], WL.rows(w, "ki8", rows), w.N, w.k,
+                                                  fp8=(sq[q], WL.rows(w, "sk", rows)))
+            else:
+                ref_idx, ref_s = oracle_selection(WL.rows(w, "qi", q * w.Hi + torch.arange(w.Hi)),
+                                                  WL.make(w, "wi")[q], WL.rows(w, "ki", rows), w.N, w.k)
+            if check_topk_set(idx_h[q], ref_idx, ref_s, w.k, w.N):
+                continue  # a legitimate boundary tie: outputs not comparable
+            sel = np.sort(ref_idx[ref_idx >= 0])
+            rows_c = O.round_to(WL.rows(w, "kv_cmp", b * w.N + torch.as_tensor(sel)), "bf16")
+            rows_c[sel == w.c_dst0] = new
+        else:
+            rows_c = O.round_to(WL.rows(w, "kv_cmp", b * w.N + torch.arange(w.N)), "bf16")
+            rows_c[w.c_dst0] = new
+        ref = oracle_out(qh, rows_c, kv_win_b, e, w.W, sink, w.scale)
+        assert_close(out[q], ref, torch.bfloat16, f"{w.name} q={q}")
+        compared += 1
+    return compared
+
+
+FULL = {
+    "csa_decode_64k": (0, 5, 13, 22, 31),
+    "csa_decode_64k_fp8": (0, 17, 31),
+    "csa_decode_64k_pro": (0, 19, 31),
+    "hca_decode_1m": (0, 7, 15),
+    "csa_decode_1m": (0, 7),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FULL))
+def test_full_size_step_matches_oracle(cuda_device, name):
+    # The benchmark's workloads in its launch configuration (the step replayed
+    # from its CUDA graph, twice: the second replay starts from the counters
+    # the first left), sampled queries against the oracle chain.
+    w = WL.WORKLOADS[name]
+    ds, _ = _decode_step(w, cuda_device)
+    ds.run()
+    first = ds.out.clone()
+    ds.run()
+    torch.cuda.synchronize()
+    assert ds.status() == 0
+    assert torch.equal(first, ds.out), "a second replay of the step changed the output"
+    queries = FULL[name]
+    assert _check_full(w, ds, queries) >= len(queries) - 1
+
+
+@pytest.mark.parametrize("name", ["csa_decode_64k", "hca_decode_1m", "csa_decode_64k_fp8"])
+def test_fused_step_matches_separate_kernels(cuda_device, name):
+    # The same step through the separate kernels: the selections are the same
+    # sets (the scores are computed by the same products in the same order),
+    # the outputs agree within the bf16 tolerance.
+    w = WL.WORKLOADS[name]
+    ds_f, d = _decode_step(w, cuda_device, fused=True)
+    out_f = ds_f.run().clone()
+    idx_f = ds_f.idx.clone() if ds_f.idx is not None else None
+    ds_s, _ = _decode_step(w, cuda_device, fused=False)
+    out_s = ds_s.run()
+    torch.cuda.synchronize()
+    if idx_f is not None:
+        assert torch.equal(torch.sort(idx_f, dim=1).values, torch.sort(ds_s.idx, dim=1).values)
+    err = (out_f.float() - out_s.float()).abs()
+    assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
+
+
+# ---------------------------------------------------------------- small cases
+
+def _small_case(dev, *, Q, N, k, H=64, W=128, n=None, ends=None, T_raw=160, fp8=False, hca=False, seed=3,
+                append=True, rope=None, check=None):
+    """One fused step on seeded synthetic inputs; every (or check[]) query's
+    output and selection against the oracle."""
+    B, D, Hi, Di = Q, 512, 64, 128
+    g = lambda tid, shape, **kw: synth.normal(seed, tid, shape, **kw)
+    q = g(1, (Q, H, D), dtype=torch.bfloat16)
+    kv_cmp = g(2, (B, N, D), dtype=torch.bfloat16)
+    kv_win = g(3, (B, T_raw, D), dtype=torch.bfloat16)
+    sink = g(7, (H,))
+    n = torch.as_tensor(n if n is not None else [N] * Q, dtype=torch.int32)
+    ends = torch.as_tensor(ends if ends is not None else [T_raw - 1] * Q, dtype=torch.int32)
+    win, stride = (128, 128) if hca else (8, 4)
+    T_c = win
+    gate = g(9, (B, T_c, D), dtype=torch.bfloat16)
+    ape = synth.normal(seed, 10, (win, D), std=0.1)
+    nw = torch.ones(D)
+    row0 = max(0, N - 1)
+    src0 = T_raw - T_c
+    kw = {}
+    if not hca:
+        if fp8:
+            qi8 = WL._codes(g(13, (Q, Hi, Di)))
+            ki8 = WL._codes(g(15, (B, N, Di)))
+            sq = synth.uniform(seed, 14, (Q, Hi)) / 64 + 1.0 / 256
+            sk = synth.uniform(seed, 16, (B, N)) / 64 + 1.0 / 256
+            wi = synth.uniform(seed, 5, (Q, Hi))
+            kw = dict(qi8=qi8.to(dev), sq=sq.to(dev), wi=wi.to(dev), ki8=ki8.to(dev), sk=sk.to(dev), k=k)
+        else:
+            qi = g(4, (Q, Hi, Di), dtype=torch.bfloat16)
+            wi = synth.uniform(seed, 5, (Q, Hi))
+            ki = g(6, (B, N, Di), dtype=torch.bfloat16)
+            kw = dict(qi=qi.to(dev), wi=wi.to(dev), ki=ki.to(dev), k=k)
+    kv_cmp_d, kv_win_d = kv_cmp.to(dev), kv_win.to(dev)
+    app = None
+    pos0 = None
+    if append:
+        app = {"kv": kv_win_d[:, src0:src0 + T_c], "gate": gate.to(dev), "ape": ape.to(dev), "norm_w": nw.to(dev),
+               "win": win, "stride": stride, "row0": row0}
+        if rope is not None:
+            pos0 = torch.arange(B, dtype=torch.int64) * 1000 + 5000
+            app["rope"] = (rope[0], rope[1], pos0.to(dev))
+    ws = ops.Workspace(dev)
+    out = ops.decode_step(q.to(dev), kv_cmp_d, kv_win_d, ends.to(dev), sink.to(dev), D ** -0.5, W, n.to(dev),
+                          append=app, ws=ws, **kw)
+    idx = None
+    if not hca:
+        # the selection comes back through idx_out; run once more into a known buffer
+        idx = torch.full((Q, k), -7, dtype=torch.int32, device=dev)
+        out = ops.decode_step(q.to(dev), kv_cmp_d, kv_win_d, ends.to(dev), sink.to(dev), D ** -0.5, W, n.to(dev),
+                              append=app, ws=ws, idx_out=idx, **kw)
+    torch.cuda.synchronize()
+    assert ops.workspace_status(ws.get(0)) == 0
+    out_h = out.cpu()
+    idx_h = idx.cpu().numpy() if idx is not None else None
+    compared = 0
+    for qq in (check if check is not None else range(Q)):
+        b, nv, e = qq, int(n[qq]), int(ends[qq])
+        new = None
+        if append:
+            raw = kv_win[b, src0:src0 + T_c]
+            new = appended_rows(raw, gate[b], ape, win, stride,
+                                rope=None if rope is None else (rope[0], rope[1], int(pos0[b])))[0]
+        if hca:
+            rows_c = O.round_to(kv_cmp[b, :nv], "bf16")
+            if append and row0 < nv:
+                rows_c[row0] = new
+        else:
+            if fp8:
+                ref_idx, ref_s = oracle_selection(qi8[qq], wi[qq], ki8[b], nv, k, fp8=(sq[qq], sk[b]))
+            else:
+                ref_idx, ref_s = oracle_selection(qi[qq], wi[qq], ki[b], nv, k)
+            if check_topk_set(idx_h[qq], ref_idx, ref_s, k, nv):
+                continue
+            sel = np.sort(ref_idx[ref_idx >= 0])
+            rows_c = O.round_to(kv_cmp[b][torch.as_tensor(sel, dtype=torch.int64)], "bf16").reshape(-1, D)
+            if append:
+                rows_c[sel == row0] = new
+        ref = oracle_out(q[qq], rows_c, kv_win[b], e, W, sink, D ** -0.5)
+        assert_close(out_h[qq], ref, torch.bfloat16, f"query {qq} (n={nv}, end={e})")
+        compared += 1
+    return compared
+
+
+def test_ragged_counts_and_short_lists(cuda_device):
+    # 3001 entries (a ragged last key tile); n above, at and below k, one and
+    # zero visible entries (the attention then reads the window and the sink)
+    n = [3001, 513, 512, 1, 0, 2000]
+    assert _small_case(cuda_device, Q=6, N=3001, k=512, n=n) >= 5
+
+
+def test_short_windows(cuda_device):
+    # windows of 1, 5, 64, 65 and 128 rows (queries near the start of their
+    # raw buffer), the window split then partly or mostly masked
+    ends = [0, 4, 63, 64, 159]
+    assert _small_case(cuda_device, Q=5, N=2500, k=256, ends=ends, W=128) >= 4
+
+
+def test_window_of_64(cuda_device):
+    assert _small_case(cuda_device, Q=4, N=1800, k=128, W=64, ends=[30, 63, 100, 159]) >= 3
+
+
+def test_pro_heads_and_top_1024(cuda_device):
+    assert _small_case(cuda_device, Q=3, N=4000, k=1024, H=128) >= 2
+
+
+def test_fp8_indexer(cuda_device):
+    assert _small_case(cuda_device, Q=5, N=3001, k=512, fp8=True, n=[3001, 600, 512, 9, 2999]) >= 4
+
+
+def test_hca_dense_ragged(cuda_device):
+    # dense lists of 700 entries (not a multiple of the 64-row tile), counts
+    # down to zero; the appended entry is the last row
+    assert _small_case(cuda_device, Q=6, N=700, k=0, hca=True, n=[700, 699, 65, 64, 1, 0]) == 6
+
+
+def test_hca_without_append(cuda_device):
+    assert _small_case(cuda_device, Q=4, N=1500, k=0, hca=True, append=False) == 4
+
+
+def test_append_with_rope(cuda_device):
+    # the append rotates the new entry's last 64 dims (theta 160000)
+    assert _small_case(cuda_device, Q=4, N=2048, k=256, rope=(64, 160000.0), n=[2048] * 4) >= 3
+
+
+def test_many_queries(cuda_device):
+    # 200 queries: many tasks of every kind per CTA, the queues wrap many times
+    assert _small_case(cuda_device, Q=200, N=1500, k=64, check=range(0, 200, 23)) >= 8
+
+
+def test_two_segment_selection(cuda_device):
+    # lists longer than one block's key cache take the two-stage selection
+    # (per-segment winners, then the winners' top-k)
+    assert _small_case(cuda_device, Q=2, N=60000, k=512, append=False) >= 1
+
+
+def test_rejects_bad_arguments(cuda_device):
+    a = _lib.DecodeStepArgs()
+    L = _lib.lib()
+    import ctypes
+    assert L.csa_decode_step(ctypes.byref(a), ctypes.c_void_p(0), 0, ctypes.c_void_p(0)) == 1  # Q = 0 etc.

@@ -142,7 +142,8 @@ def test_decode_step_with_the_fused_selection(cuda_device):
     ds = DecodeStep(q=d["q"], kv_cmp=d["kv_cmp"], kv_win=d["kv_win"], sink=d["sink"], scale=w.scale, win_len=w.W,
                     win_end=w.win_end().to(cuda_device), n_cmp=n.to(cuda_device), ape=d["ape"],
                     norm_w=WL.norm_w(w, cuda_device), gate=d["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
-                    win=w.win, stride=w.stride, qi=d["qi"], wi=d["wi"], ki=d["ki"], k=w.k, fuse_select=True)
+                    win=w.win, stride=w.stride, qi=d["qi"], wi=d["wi"], ki=d["ki"], k=w.k, fuse_select=True,
+                    fused=False)
     out = ds.run().cpu()
     assert ds.status() == 0
     idx_h = ds.idx.cpu().numpy()
