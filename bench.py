@@ -127,10 +127,11 @@ class Step:
     # that the end-to-end run moves them with a single host-to-device copy
     PER_STEP = ("q", "gate", "qi", "wi")
 
-    def __init__(self, w: WL.Workload, device, graph: bool = True, caches=None):
+    def __init__(self, w: WL.Workload, device, graph: bool = True, caches=None, fused: bool = True):
         self.w = w
         self.dev = device
         self.graph = graph
+        self.fused = fused
         fp8 = w.index_fmt == "e4m3"
         per_step = self.PER_STEP if not fp8 else ("q", "gate", "qi8", "sq", "wi")
         names = [n for n in per_step if w.mode == "csa" or n not in ("qi", "wi", "qi8", "sq")]
@@ -163,14 +164,14 @@ class Step:
             ape=t["ape"], norm_w=WL.norm_w(w, device), gate=t["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
             win=w.win, stride=w.stride, qi=t.get("qi"), wi=t.get("wi"), ki=t.get("ki"),
             k=w.k if w.mode == "csa" else None, graph=graph,
-            qi8=t.get("qi8"), sq=t.get("sq"), ki8=t.get("ki8"), sk=t.get("sk"))
+            qi8=t.get("qi8"), sq=t.get("sq"), ki8=t.get("ki8"), sk=t.get("sk"), fused=fused)
         self.out = self.ds.out
         self._scores = None
 
     def twin(self):
         """A second step over the same caches with its own input staging
         buffer and output (double buffering for the end-to-end pipeline)."""
-        return Step(self.w, self.dev, graph=self.graph, caches=self.caches)
+        return Step(self.w, self.dev, graph=self.graph, caches=self.caches, fused=self.fused)
 
     def parts(self):
         """The step's kernels one call at a time (per-kernel timing and the
@@ -294,17 +295,45 @@ def job_value(world: int, q_per_rank: int, ms_max: float) -> float:
     return world * q_per_rank / (ms_max * 1e-3)
 
 
+def _time_steps(step, flush, stream, K):
+    """Mean device time (ms) of K graph replays, L2 flushed before each."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush()
+        evs[i][0].record(stream)
+        step.run()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / K
+
+
 def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=False):
-    n0 = _lib.lib().csa_launch_count()
-    step = Step(w, device)  # runs the step once eagerly, then captures it
-    launches_per_step = (_lib.lib().csa_launch_count() - n0) // 2
+    """Times the step on both paths (the whole step as one fused kernel, and
+    the separate kernels), reports the faster; the other path's time and the
+    separate kernels' per-kernel times are kept for the record."""
     flush = L2Flush(device)
     stream = torch.cuda.current_stream(device)
-    for _ in range(max(3, args.warmup)):
-        step.run()
+    steps, launches = {}, {}
+    for fused in (True, False):
+        if args.path != "both" and (args.path == "fused") != fused:
+            continue
+        n0 = _lib.lib().csa_launch_count()
+        caches = steps[True].caches if True in steps else None
+        steps[fused] = Step(w, device, caches=caches, fused=fused)  # runs the step once eagerly, then captures it
+        launches[fused] = (_lib.lib().csa_launch_count() - n0) // 2
+        for _ in range(max(3, args.warmup)):
+            steps[fused].run()
     torch.cuda.synchronize()
+    K0 = max(5, args.steps // 5)
+    trial = {f: _time_steps(st, flush, stream, K0) for f, st in steps.items()}
+    fused = min(trial, key=trial.get)
+    step = steps[fused]
+    launches_per_step = launches[fused]
 
     K = args.steps if not secondary else max(10, args.steps // 4)
+    for st in steps.values():
+        if st is not step:
+            st.ds.graph = None  # release the other path's graph before the timed region
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     clocks = Clocks(device, args.clock_log)
     _sync_barrier(dist_on)
@@ -323,24 +352,31 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     ms_max = max_over_ranks(ms, dist_on, device)
 
     # Per-kernel durations: the same kernels launched one by one with events
-    # between them (a host-side head start keeps the launches queued).
-    names = [n for n, _ in step.parts()]
-    per = {n: 0.0 for n in names}
-    Kp = max(5, K // 2)
-    for _ in range(Kp):
-        flush()
-        torch.cuda._sleep(2_000_000)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-        ev[0].record(stream)
-        for i, (_, f) in enumerate(step.parts()):
-            f()
-            ev[i + 1].record(stream)
-        torch.cuda.synchronize()
-        for i, n in enumerate(names):
-            per[n] += ev[i].elapsed_time(ev[i + 1]) / Kp
+    # between them (a host-side head start keeps the launches queued); for
+    # both paths when both were built.
+    per = {}
+    for st in steps.values():
+        parts = st.parts()
+        names = [n for n, _ in parts]
+        acc = {n: 0.0 for n in names}
+        Kp = max(5, K // 2)
+        for _ in range(Kp):
+            flush()
+            torch.cuda._sleep(2_000_000)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+            ev[0].record(stream)
+            for i, (_, f) in enumerate(st.parts()):
+                f()
+                ev[i + 1].record(stream)
+            torch.cuda.synchronize()
+            for i, n in enumerate(names):
+                acc[n] += ev[i].elapsed_time(ev[i + 1]) / Kp
+        per.update(acc)
     status = step.ds.status()
+    paths = {("fused" if f else "separate"): round(v, 4) for f, v in trial.items()}
     return {"ms": ms_max, "ms_local": ms, "per_kernel_ms": per, "launches_per_step": int(launches_per_step),
-            "wall_s": wall, "clocks": clocks.summary(), "status": status, "K": K, "step": step}
+            "wall_s": wall, "clocks": clocks.summary(), "status": status, "K": K, "step": step,
+            "path": "fused" if fused else "separate", "paths_ms": paths}
 
 
 def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
@@ -370,6 +406,14 @@ def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
     gbps = nbytes / (ms * 1e-3) / 1e9
     return {"tokens": w.bulk_T, "entries": n, "ms": round(ms, 4), "GBps": round(gbps, 1),
             "frac": round(gbps / hbm_gbs, 4), "bytes": nbytes, "tokens_per_s": round(w.bulk_T / (ms * 1e-3), 1)}
+
+
+def path_parts(per_kernel_ms, path):
+    """The per-kernel times of the path that was timed: the fused kernel, or
+    the separate kernels."""
+    if path == "fused":
+        return {k: v for k, v in per_kernel_ms.items() if k == WHOLE_STEP}
+    return {k: v for k, v in per_kernel_ms.items() if k != WHOLE_STEP}
 
 
 def roofline_of(w, per_kernel_ms, hbm_gbs, traffic=None, tflops=None):
@@ -551,6 +595,8 @@ def main():
     ap.add_argument("--clock-log", default=None,
                     help="file for the nvidia-smi samples taken during the timed region (default: a temporary file)")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    ap.add_argument("--path", default="both", choices=["both", "fused", "separate"],
+                    help="the decode step as one fused kernel, as the separate kernels, or the faster of both")
     ap.add_argument("--once", action="store_true",
                     help="profiling aid: build the step without a graph and launch each of its kernels once more")
     args = ap.parse_args()
@@ -597,7 +643,7 @@ def main():
     w = WL.shard(w, rank)  # this rank's own sequences (same shapes)
     r = time_ours(args, w, device, dist_on, rank, world)
     traffic = load_traffic(args.traffic_json, w.name)
-    roof = roofline_of(w, r["per_kernel_ms"], hbm, traffic, tflops)
+    roof = roofline_of(w, path_parts(r["per_kernel_ms"], r["path"]), hbm, traffic, tflops)
     roof["peak_kind"] = f"{peak_kind} HBM copy bandwidth"
     e2e = e2e_ours(args, w, r["step"], device)
     del r["step"]
@@ -612,8 +658,10 @@ def main():
             try:
                 s = time_ours(args, sw, device, False, 0, 1, secondary=True)
                 del s["step"]
-                rf = roofline_of(sw, s["per_kernel_ms"], hbm, load_traffic(args.traffic_json, name), tflops)
+                rf = roofline_of(sw, path_parts(s["per_kernel_ms"], s["path"]), hbm,
+                                 load_traffic(args.traffic_json, name), tflops)
                 line = {"queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1), "ms_per_step": round(s["ms"], 4),
+                        "path": s["path"], "paths_ms": s["paths_ms"],
                         "per_kernel_ms": {k: round(v, 4) for k, v in s["per_kernel_ms"].items()}}
                 if prefill(sw):  # tensor-bound: the step's FLOPs against the bf16 peak
                     step_tf = sum(algo_flops(sw).values()) / (s["ms"] * 1e-3) / 1e12
@@ -646,6 +694,7 @@ def main():
             "parallelism": f"replicas x{world} (independent sequences per GPU, no collective)",
             "step_GBps": round(step_bytes / (r["ms"] * 1e-3) / 1e9, 1),
             "step_roofline_frac": round(step_bytes / (r["ms"] * 1e-3) / 1e9 / hbm, 4),
+            "path": r["path"], "paths_ms": r["paths_ms"],
             "per_kernel_ms": {k: round(v, 4) for k, v in r["per_kernel_ms"].items()},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": r["launches_per_step"] * r["K"], "launches_per_step": r["launches_per_step"],

@@ -73,6 +73,7 @@ constexpr uint32_t kTmemCols = 512, kColO = 0, kColS = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kMaxSplits = 32;
+constexpr int kAhead = 1;  // rounds of tiles prefetched into L2 ahead of their load (see the stand-alone kernel)
 
 // scorer (indexer 64 heads x 128 dims)
 constexpr int kHi = 64, kDi = 128;
@@ -114,7 +115,7 @@ struct Hdr {
   int4 smeta[kStages];
   int4 ameta[2];
   // attention pipeline
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done, o_done;
+  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[4], o_done;
   uint64_t mma_drain;
   float red[4][kH];
   alignas(16) float mref[kH];
@@ -369,49 +370,42 @@ __device__ __forceinline__ int4 static_task(const StepPlan &P, int t) {
 }
 
 // The ready-queue warp: while the workers run a scoring run or wait for
-// work (not busy), it takes the next queued task and leaves it in the
-// mailbox; once every queued task of the launch is taken it leaves EXIT.
+// work (not busy), it takes a ticket (the next queue position, one atomic
+// add: tickets never fail or retry) and waits for that position to be
+// filled, then leaves the task in the mailbox. Every queued task is filled
+// by a running task and taken by exactly one ticket, so a waiting ticket is
+// always served; a ticket past the last queued task of the launch means EXIT.
+// The workers keep taking static work while the ticket waits.
 __device__ void scheduler(const StepArgs &a, const StepPlan &P, Hdr *h) {
   if ((threadIdx.x & 31) != 0) return;
   volatile int *mb_full = &h->mb_full, *busy = &h->busy, *abort = &h->abort;
   unsigned long long *qu = ready_queue(a, P);
-  uint32_t backoff = 64;
   for (;;) {
-    while (*mb_full) {
+    while (*mb_full || *busy) {  // (a busy CTA would sit on a ready task)
       if (*abort) return;
       __nanosleep(128);
     }
-    int4 task;
-    for (;;) {
-      if (*abort) return;
-      const unsigned long long hr = ld_acquire_u64(a.ctr + K_HEAD);
-      const uint32_t head = (uint32_t)hr, reserved = (uint32_t)(hr >> 32);
-      if ((int)head >= P.D || ld_relaxed(a.ctr + K_ABORT)) {
-        task = make_int4(T_EXIT, 0, 0, 0);
-        break;
-      }
-      if (head < reserved && !*busy) {
-        if (atomicCAS(a.ctr + K_HEAD, head, head + 1) == head) {
-          // the slot is reserved: its pusher is writing it
-          unsigned long long v;
-          const uint64_t t0 = tc::globaltimer_ns();
-          while ((v = ld_acquire_u64(qu + head)) == 0) {
-            if (tc::globaltimer_ns() - t0 > h->wait_ns) {
-              raise_status(a.status, CSA_STATUS_WAIT_TIMEOUT);
-              atomicExch(a.ctr + K_ABORT, 1u);
-              *abort = 1;
-              return;
-            }
+    const uint32_t ticket = atomicAdd(a.ctr + K_HEAD, 1u);
+    int4 task = make_int4(T_EXIT, 0, 0, 0);
+    if ((int)ticket < P.D) {
+      unsigned long long v;
+      uint64_t t0 = 0;
+      for (uint32_t i = 0; (v = ld_acquire_u64(qu + ticket)) == 0; ++i) {
+        if (*abort) return;
+        __nanosleep(64);
+        if ((i & 15) == 15) {
+          if (ld_relaxed(a.ctr + K_ABORT)) break;  // another CTA gave up: EXIT
+          const uint64_t now = tc::globaltimer_ns();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > h->wait_ns) {
+            raise_status(a.status, CSA_STATUS_WAIT_TIMEOUT);
+            atomicExch(a.ctr + K_ABORT, 1u);
+            break;
           }
-          task = dec_task(v);
-          backoff = 64;
-          break;
         }
-        __nanosleep(backoff);  // another CTA took it: back off a little
-        backoff = backoff < 1024 ? 2 * backoff : 1024;
-        continue;
       }
-      __nanosleep(256);
+      if (v != 0) task = dec_task(v);
     }
     h->mb_task = task;
     __threadfence_block();
@@ -906,11 +900,11 @@ __device__ void topk1_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t
     wbar();
     if (single) {
       int32_t *out = a.idx + (size_t)q * k;
-      bsel::select<kWorkers, kHist1>(h->sel, hist, len, k, kBarWork, [&](int j) { return keys[j]; },
+      bsel::select<kWorkers, kHist1>(h->sel, hist, keys, len, k, kBarWork,
                                      [&](uint32_t slot, int j) { out[slot] = j; });
     } else {
       const size_t cb = ((size_t)q * P.nseg + g) * k;
-      bsel::select<kWorkers, kHist1>(h->sel, hist, len, k, kBarWork, [&](int j) { return keys[j]; },
+      bsel::select<kWorkers, kHist1>(h->sel, hist, keys, len, k, kBarWork,
                                      [&](uint32_t slot, int j) {
                                        a.cand_key[cb + slot] = keys[j];
                                        a.cand_idx[cb + slot] = j0 + j;
@@ -964,7 +958,7 @@ __device__ void topk2_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t
   if (total <= k) {
     for (int i = threadIdx.x; i < k; i += kWorkers) out[i] = i < total ? pos[i] : -1;
   } else {
-    bsel::select<kWorkers, kHist2>(h->sel, hist, total, k, kBarWork, [&](int j) { return keys[j]; },
+    bsel::select<kWorkers, kHist2>(h->sel, hist, keys, total, k, kBarWork,
                                    [&](uint32_t slot, int j) { out[slot] = pos[j]; });
   }
   wbar();
@@ -1125,9 +1119,9 @@ __device__ void mqa_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t *
       const bool run = is_run(r0, win_run, srow);
       __syncwarp();
       if (!run && lane < kRowsPerWarp) h->rowp[warp][lane] = src_row(r0 + kRowsPerWarp * part + lane);
-      if (li < 2) {
+      if (li < 2) {  // the first tile streams in order too; later tiles are prefetched kAhead rounds ahead
         if (run) prefetch_l2(li);
-        prefetch_l2(li + 2);
+        for (int r = 1; r <= kAhead; ++r) prefetch_l2(li + 2 * r);
       }
       if (!__all_sync(0xffffffffu, mwait(&h->kv_empty[g], ((LI >> 1) & 1) ^ 1, abort, a.status, lim))) break;
       if (run) {
@@ -1150,7 +1144,7 @@ __device__ void mqa_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t *
           cp_async16(dst, src ? src + c16 * 8 : static_cast<const bf16 *>(a.kv_win), src != nullptr);
         }
       }
-      if (li >= 2) prefetch_l2(li + 2);
+      if (li >= 2) prefetch_l2(li + 2 * kAhead);
       if (!run) {
         cp_async_wait_all();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1167,6 +1161,10 @@ __device__ void mqa_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t *
       bool ok = ntiles == 0 || mwait(&h->q_full, mq & 1, abort, a.status, lim);
       const uint64_t ad_kv = tc::sw128_desc(kv_base, 16, 1024), bd_q = tc::sw128_desc(q_base, 16, 1024);
       const uint64_t ad_v = tc::sw128_desc(kv_base, kBoxBytes, 1024), bd_p = tc::sw128_desc(p_base, kPBytes, 1024);
+      // Two streams of work, issued as soon as each is ready: S^T(ns) once
+      // tile ns has landed (and the softmax is done with S^T(ns - 2)), and
+      // P.V(np) once P(np) is written. Neither waits behind the other, so the
+      // P.V that frees a tile buffer is never held up by the next tile's load.
       int ns = 0, np = 0;
       uint32_t idle = 0;
       uint64_t t_idle = 0;
@@ -1185,10 +1183,12 @@ __device__ void mqa_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t *
                            bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv, np > 0 || j > 0);
           }
           tc::commit(&h->kv_empty[pb]);
-          tc::commit(&h->pv_done);
+          tc::commit(&h->pv_done[LP & 3]);
           ++np;
           progressed = true;
         }
+        // S^T(ns) overwrites the S^T buffer of tile ns - 2: P.V(ns - 2) must
+        // have been issued, i.e. its softmax has finished reading it.
         if (ns < ntiles && ns <= np + 1 && tc::mbar_test_wait(&h->kv_full[LS & 1], (LS >> 1) & 1)) {
           const int buf = LS & 1;
           tc::fence_after_sync();
@@ -1208,7 +1208,10 @@ __device__ void mqa_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t *
         }
         if (*abort) {
           ok = false;
-        } else if ((++idle & 63) == 0) {
+        } else {
+          __nanosleep(32);  // neither product is ready: leave the issue slots to the other warps
+        }
+        if (ok && (++idle & 63) == 0) {
           const uint64_t now = tc::globaltimer_ns();
           if (t_idle == 0) {
             t_idle = now;
@@ -1348,10 +1351,13 @@ __device__ void mqa_task(const StepArgs &a, const StepPlan &P, Hdr *h, uint8_t *
                        : "memory");
         }
       }
-      if (li > 0) {
-        ok = __all_sync(0xffffffffu, mwait(&h->pv_done, (LI - 1) & 1, abort, a.status, lim));
+      if (li > 0 && rescale) {
+        // O^T is rescaled in TMEM: P.V of the previous tile must be complete
+        // first (only then: see the stand-alone attention kernel; one barrier
+        // per tile slot mod 4)
+        ok = __all_sync(0xffffffffu, mwait(&h->pv_done[(LI - 1) & 3], ((LI - 1) >> 2) & 1, abort, a.status, lim));
         tc::fence_after_sync();
-        if (ok && rescale) {
+        if (ok) {
 #pragma unroll 1
           for (int m = 0; m < 4; ++m) {
 #pragma unroll 1
@@ -1552,7 +1558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&h->p_full[s], 4 * 32);
     }
     tc::mbar_init(&h->q_full, 1);
-    tc::mbar_init(&h->pv_done, 1);
+    for (int i = 0; i < 4; ++i) tc::mbar_init(&h->pv_done[i], 1);
     tc::mbar_init(&h->o_done, 1);
     tc::mbar_init(&h->mma_drain, 1);
     for (int i = 0; i < 4; ++i) h->need[i] = 0;

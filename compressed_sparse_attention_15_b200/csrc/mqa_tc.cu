@@ -73,9 +73,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSelMax = 1024;                       // largest k selected inside the kernel
 constexpr int kSelKeys = 2 * kTileBytes / 4;        // slice keys that fit in the tile buffers
+// Rounds of tiles whose rows the loaders bring into L2 ahead of their load:
+// with two tile buffers a tile's load can only start once the buffer is
+// free, so the L2 prefetches are what keeps more of the stream in flight.
+constexpr int kAhead = 1;
 
 struct Small {
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done, o_done;
+  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[4], o_done;
   float red[4][kH];
   alignas(16) float mref[kH];
   float alpha[kH];
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&sm->s_full[i], 1);
       tc::mbar_init(&sm->p_full[i], 4 * 32);
     }
-    tc::mbar_init(&sm->pv_done, 1);
+    for (int i = 0; i < 4; ++i) tc::mbar_init(&sm->pv_done[i], 1);
     tc::mbar_init(&sm->o_done, 1);
     sm->abort = 0;
     sm->rescale = 0;
@@ -330,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // moving 512 contiguous bytes of one row; every lane waits for its own
     // copies, fences them for the tensor core and arrives, so kv_full
     // expects 128 arrivals either way. Each warp also prefetches its rows of
-    // its next tile into L2 while the buffer is busy.
+    // its next kAhead tiles into L2 while the buffer is busy.
     const int g = warp / kWarpsPerBuf, part = warp % kWarpsPerBuf;
     const uint32_t buf_base = tc::smem_u32(kv) + g * kTileBytes;
     if (warp == 0 && lane == 0) {
@@ -389,9 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool run = is_run(r0, win_run);
       __syncwarp();  // the previous tile's copies have read rowp[warp]
       if (!run && lane < kRowsPerWarp) sm->rowp[warp][lane] = src_row(r0 + kRowsPerWarp * part + lane);
-      if (li == g) {  // the first tile streams in order too; later tiles are prefetched one round ahead, below
+      if (li == g) {  // the first tile streams in order too; later tiles are prefetched kAhead rounds ahead
         if (run) prefetch_l2(li);
-        prefetch_l2(li + 2);
+        for (int r = 1; r <= kAhead; ++r) prefetch_l2(li + 2 * r);
       }
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status))) break;
       if (run) {
@@ -415,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           cp_async16(dst, src ? src + c16 * 8 : static_cast<const bf16 *>(a.kv_win), src != nullptr);
         }
       }
-      if (li > g) prefetch_l2(li + 2);
+      if (li > g) prefetch_l2(li + 2 * kAhead);
       if (!run) {
         cp_async_wait_all();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -457,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            bd0 + (uint64_t)((j * 2048) >> 4), idesc_pv, np > 0 || j > 0);
           }
           tc::commit(&sm->kv_empty[pb]);
-          tc::commit(&sm->pv_done);
+          tc::commit(&sm->pv_done[np & 3]);
           ++np;
           progressed = true;
         }
@@ -482,7 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (*abort) {
           ok = false;
-        } else if ((++idle & 63) == 0) {
+        } else {
+          __nanosleep(32);  // neither product is ready: leave the issue slots to the other warps
+        }
+        if (ok && (++idle & 63) == 0) {
           const uint64_t now = tc::globaltimer_ns();
           if (t_idle == 0) {
             t_idle = now;
@@ -631,12 +638,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                        : "memory");
         }
       }
-      if (li > 0) {
-        // P.V of the previous tile must be complete before O^T may be
-        // touched; consumed every tile so the barrier phases stay in step.
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->pv_done, (li - 1) & 1, abort, a.status));
+      if (li > 0 && rescale) {
+        // O^T is rescaled in TMEM: P.V of the previous tile must be complete
+        // first. (Only then: S^T(li) completing implied every earlier P.V
+        // but that one, and a P(li) that needs no rescale does not wait. One
+        // barrier per tile slot mod 4, so a skipped phase is never mistaken
+        // for another: slot (li - 1) mod 4 next completes for tile li + 3.)
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->pv_done[(li - 1) & 3], ((li - 1) >> 2) & 1, abort, a.status));
         tc::fence_after_sync();
-        if (ok && rescale) {
+        if (ok) {
 #pragma unroll 1
           for (int m = 0; m < 4; ++m) {
 #pragma unroll 1

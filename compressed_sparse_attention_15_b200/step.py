@@ -10,13 +10,14 @@ The step over device-resident caches is:
      (csa_index_topk, or csa_index_topk_fp8 with FP8 indexer inputs);
   3. attend over the selected (CSA) or all visible (HCA) entries + the
      sliding window + the per-head sink (csa_sparse_mqa / hca_mqa).
-With fused=True (the default) the whole step is one csa_decode_step call:
-one persistent kernel in which the selection and attention of some queries
-overlap the indexer key scan of others (the separate kernels serve shapes it
-does not take). With fused=False the parts are separate calls; there,
-fuse_select=True makes a CSA step only score in 2 (csa_index_scores(_fp8))
-and run 3 as csa_topk_sparse_mqa, the selection inside the attention kernel
-where its launch plan allows.
+With fused=True the whole step is one csa_decode_step call: one persistent
+kernel in which the selection and attention of some queries overlap the
+indexer key scan of others (the separate kernels serve shapes it does not
+take). With fused=False (the default; measured faster on the benchmark
+workloads) the parts are separate calls; there, fuse_select=True makes a CSA
+step only score in 2 (csa_index_scores(_fp8)) and run 3 as
+csa_topk_sparse_mqa, the selection inside the attention kernel where its
+launch plan allows.
 The library never allocates or synchronises, so the launches are captured
 once into a CUDA graph and each step is one graph launch. Buffers are bound
 at construction; later steps see whatever the caller wrote into them.
@@ -33,7 +34,7 @@ class DecodeStep:
                  ape, norm_w, gate, append_src0: int, append_dst0: int, win: int, stride: int,
                  qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True,
                  qi8=None, sq=None, ki8=None, sk=None, append_rope=None, fuse_select: bool = False,
-                 fused: bool = True):
+                 fused: bool = False):
         self.fp8 = qi8 is not None
         self.csa = qi is not None or self.fp8
         self.q, self.kv_cmp, self.kv_win, self.sink = q, kv_cmp, kv_win, sink
