@@ -95,6 +95,15 @@ def algo_flops(w: WL.Workload):
     return f
 
 
+# The other workloads, each one line of "secondary": (label, workload, append
+# RoPE (rope_dims, theta) or None). The RoPE line is the 64 K decode step with
+# the cache append rotating the new entry's last 64 dims (qk_rope_head_dim 64,
+# compress_rope_theta 160000 of the Flash configuration).
+SECONDARY = (("hca_decode_1m", "hca_decode_1m", None), ("csa_decode_1m", "csa_decode_1m", None),
+             ("csa_decode_64k_fp8", "csa_decode_64k_fp8", None), ("csa_decode_64k_pro", "csa_decode_64k_pro", None),
+             ("csa_prefill_chunk_4k", "csa_prefill_chunk_4k", None),
+             ("csa_decode_64k_append_rope", "csa_decode_64k", (64, 160000.0)))
+
 # A step part whose algorithmic bytes and FLOPs are another's: the attention
 # with the selection made inside it moves what the attention moves.
 PART_ALIAS = {"topk_mqa": "mqa"}
@@ -127,11 +136,12 @@ class Step:
     # that the end-to-end run moves them with a single host-to-device copy
     PER_STEP = ("q", "gate", "qi", "wi")
 
-    def __init__(self, w: WL.Workload, device, graph: bool = True, caches=None, fused: bool = True):
+    def __init__(self, w: WL.Workload, device, graph: bool = True, caches=None, fused: bool = True, rope=None):
         self.w = w
         self.dev = device
         self.graph = graph
         self.fused = fused
+        self.rope = rope  # (rope_dims, theta): RoPE fused into the append
         fp8 = w.index_fmt == "e4m3"
         per_step = self.PER_STEP if not fp8 else ("q", "gate", "qi8", "sq", "wi")
         names = [n for n in per_step if w.mode == "csa" or n not in ("qi", "wi", "qi8", "sq")]
@@ -164,14 +174,16 @@ class Step:
             ape=t["ape"], norm_w=WL.norm_w(w, device), gate=t["gate"], append_src0=w.c_src0, append_dst0=w.c_dst0,
             win=w.win, stride=w.stride, qi=t.get("qi"), wi=t.get("wi"), ki=t.get("ki"),
             k=w.k if w.mode == "csa" else None, graph=graph,
-            qi8=t.get("qi8"), sq=t.get("sq"), ki8=t.get("ki8"), sk=t.get("sk"), fused=fused)
+            qi8=t.get("qi8"), sq=t.get("sq"), ki8=t.get("ki8"), sk=t.get("sk"), fused=fused,
+            append_rope=None if rope is None else
+            (rope[0], rope[1], torch.full((w.B,), w.raw0 + w.c_src0, dtype=torch.int64, device=device)))
         self.out = self.ds.out
         self._scores = None
 
     def twin(self):
         """A second step over the same caches with its own input staging
         buffer and output (double buffering for the end-to-end pipeline)."""
-        return Step(self.w, self.dev, graph=self.graph, caches=self.caches, fused=self.fused)
+        return Step(self.w, self.dev, graph=self.graph, caches=self.caches, fused=self.fused, rope=self.rope)
 
     def parts(self):
         """The step's kernels one call at a time (per-kernel timing and the
@@ -307,7 +319,7 @@ def _time_steps(step, flush, stream, K):
     return sum(a.elapsed_time(b) for a, b in evs) / K
 
 
-def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=False):
+def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=False, rope=None):
     """Times the step on both paths (the whole step as one fused kernel, and
     the separate kernels), reports the faster; the other path's time and the
     separate kernels' per-kernel times are kept for the record."""
@@ -319,7 +331,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
             continue
         n0 = _lib.lib().csa_launch_count()
         caches = steps[True].caches if True in steps else None
-        steps[fused] = Step(w, device, caches=caches, fused=fused)  # runs the step once eagerly, then captures it
+        steps[fused] = Step(w, device, caches=caches, fused=fused, rope=rope)  # runs once eagerly, then captured
         launches[fused] = (_lib.lib().csa_launch_count() - n0) // 2
         for _ in range(max(3, args.warmup)):
             steps[fused].run()
@@ -406,6 +418,49 @@ def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
     gbps = nbytes / (ms * 1e-3) / 1e9
     return {"tokens": w.bulk_T, "entries": n, "ms": round(ms, 4), "GBps": round(gbps, 1),
             "frac": round(gbps / hbm_gbs, 4), "bytes": nbytes, "tokens_per_s": round(w.bulk_T / (ms * 1e-3), 1)}
+
+
+def time_index_compress(args, w: WL.Workload, device, hbm_gbs):
+    """The indexer's own compressor over the 1 M-token indexer stream
+    (ikv_raw, igate_raw [1, bulk_T, 128] bf16 -> Hadamard-rotated E4M3 codes
+    [1, (bulk_T - 8)/4 + 1, 128] + one fp32 scale per entry), then the Hadamard
+    rotation + E4M3 quantisation of one decode batch's indexer queries
+    ([Q * Hi, 128] bf16), each timed alone."""
+    kv = WL.make(w, "ikv_raw", device)
+    gate = WL.make(w, "igate_raw", device)
+    ape = WL.make(w, "iape", device)
+    nw = torch.ones(w.Di, dtype=torch.float32, device=device)
+    qi = WL.make(WL.WORKLOADS["csa_decode_64k"], "qi", device).reshape(-1, w.Di)
+    n = ops.num_entries(w.bulk_T, w.win, w.stride)
+    flush = L2Flush(device)
+    stream = torch.cuda.current_stream(device)
+
+    def timed(f):
+        for _ in range(3):
+            f()
+        K = max(5, args.steps // 4)
+        ms = 0.0
+        for _ in range(K):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            f()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms += a.elapsed_time(b) / K
+        return ms
+
+    ms_c = timed(lambda: ops.index_compress(kv, gate, ape, nw, w.win, w.stride, fp8=True))
+    ms_h = timed(lambda: ops.hadamard_rows(qi, fp8=True))
+    by_c = 2 * w.bulk_T * w.Di * 2 + n * (w.Di + 4) + w.win * w.Di * 4 + w.Di * 4
+    by_h = qi.shape[0] * (w.Di * 2 + w.Di + 4)
+    gc, gh = by_c / (ms_c * 1e-3) / 1e9, by_h / (ms_h * 1e-3) / 1e9
+    return {"csa_index_compress": {"tokens": w.bulk_T, "entries": n, "out": "e4m3 codes + fp32 scales",
+                                   "ms": round(ms_c, 4), "GBps": round(gc, 1), "frac": round(gc / hbm_gbs, 4),
+                                   "bytes": by_c, "tokens_per_s": round(w.bulk_T / (ms_c * 1e-3), 1)},
+            "csa_hadamard_rows": {"rows": qi.shape[0], "dim": w.Di, "out": "e4m3 codes + fp32 scales",
+                                  "ms": round(ms_h, 4), "GBps": round(gh, 1), "bytes": by_h,
+                                  "note": "one decode batch's query rows: launch-latency bound"}}
 
 
 def path_parts(per_kernel_ms, path):
@@ -514,64 +569,131 @@ def e2e_ours(args, w: WL.Workload, step: Step, device):
 # The oracle on the host (CPU baseline and --impl reference)
 # --------------------------------------------------------------------------
 
-def oracle_step_inputs(w: WL.Workload):
-    import numpy as np
-
-    host = {n: WL.make(w, n) for n in ("q", "sink", "ape")}
-    if w.mode == "csa":
-        names = ("qi8", "sq", "wi", "ki8", "sk") if w.index_fmt == "e4m3" else ("qi", "wi", "ki")
-        host.update({n: WL.make(w, n) for n in names})
-    host["np"] = np
-    return host
+def _oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count()
 
 
-def time_oracle(w: WL.Workload, steps: int, budget_s: float):
-    """Time the fp64 oracle on the host over up to `steps` full batches, stopping
-    once `budget_s` of oracle time has been spent. Input regeneration and row
-    gathering happen outside the timed sections."""
+def time_oracle(w: WL.Workload, steps: int, budget_s: float, queries=None, rope=None):
+    """Time the fp64 oracle on the host over the step's work: per sequence the
+    append (the compressor over the step's raw tokens, with RoPE when ``rope``
+    = (rope_dims, theta) is given), per query the indexer top-k (CSA) and the
+    attention. ``queries`` (default: all) is the subset run; the time is
+    extrapolated to the whole batch (sequences x append time + queries x query
+    time). Up to ``steps`` passes; stops once ``budget_s`` of oracle time is
+    spent (after at least one query). Input regeneration and row gathering are
+    not timed."""
     import numpy as np
 
     import oracle as O
 
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
-    host = oracle_step_inputs(w)
-    ape = host["ape"]
-    total, done = 0.0, 0
+    qs = list(range(w.Q)) if queries is None else list(queries)
+    ape = WL.make(w, "ape")
+    sink = WL.make(w, "sink")
+    fp8 = w.mode == "csa" and w.index_fmt == "e4m3"
+    if w.mode == "csa":
+        iq = {n: WL.make(w, n) for n in (("sq", "wi") if fp8 else ("wi",))}
+    knames = (("ki8", "sk") if fp8 else ("ki",)) if w.mode == "csa" else ()
+    # every sequence's indexer keys at once when they fit in a few hundred MB
+    keys_all = {n: WL.make(w, n) for n in knames} if w.B * w.N * w.Di <= (80 << 20) else None
+    t_app, n_app, t_q, n_q = 0.0, 0, 0.0, 0
+    seq_cache, q_cache, raw_cache = {}, {}, {}  # regenerated inputs, kept for the next pass
     for _ in range(max(1, steps)):
-        for q in range(w.Q):
+        for q in qs:
             b = q // w.q_per_seq
-            raw = WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.c_src0, w.c_src0 + w.T_c))
-            gate = WL.rows(w, "gate", b * w.T_c + torch.arange(w.T_c))
+            if b not in seq_cache:
+                seq_cache.clear()
+                if b not in raw_cache:
+                    raw_cache[b] = (WL.rows(w, "kv_win", b * w.T_raw + torch.arange(w.c_src0, w.c_src0 + w.T_c)),
+                                    WL.rows(w, "gate", b * w.T_c + torch.arange(w.T_c)))
+                raw, gate = raw_cache[b]
+                t0 = time.perf_counter()
+                if rope:
+                    new = O.compress_rope(raw, gate, ape, np.ones(w.D), w.win, w.stride, w.raw0 + w.c_src0, rope[1],
+                                          rope[0])
+                else:
+                    new = O.compress(raw, gate, ape, np.ones(w.D), w.win, w.stride)
+                new = O.round_to(new, "bf16")
+                t_app += time.perf_counter() - t0
+                n_app += 1
+                if keys_all is not None:
+                    keys = {n: t[b] for n, t in keys_all.items()}
+                else:
+                    keys = {n: WL.rows(w, n, b * w.N + torch.arange(w.N)) for n in knames}
+                seq_cache[b] = (new, keys)
+            new, keys = seq_cache[b]
+            p = int(w.positions()[q])
+            if q not in q_cache:
+                q_cache[q] = {"q": WL.rows(w, "q", q * w.H + torch.arange(w.H))}
+                if w.mode == "csa":
+                    q_cache[q]["qi"] = WL.rows(w, "qi8" if fp8 else "qi", q * w.Hi + torch.arange(w.Hi))
+            qc = q_cache[q]
+            q_rows, qi_rows = qc["q"], qc.get("qi")
             t0 = time.perf_counter()
-            new = O.round_to(O.compress(raw, gate, ape, np.ones(w.D), w.win, w.stride), "bf16")
-            if w.mode == "csa" and w.index_fmt == "e4m3":
-                idx, _ = O.index_topk_fp8(host["qi8"][q].numpy(), host["sq"][q], host["wi"][q], host["ki8"][b].numpy(),
-                                          host["sk"][b], int(w.positions()[q]), w.k, w.win, w.stride)
+            if fp8:
+                idx, _ = O.index_topk_fp8(qi_rows.numpy(), iq["sq"][q], iq["wi"][q], keys["ki8"].numpy(),
+                                          keys["sk"], p, w.k, w.win, w.stride)
                 sel = idx[idx >= 0]
             elif w.mode == "csa":
-                idx, _ = O.index_topk(host["qi"][q], host["wi"][q], host["ki"][b], int(w.positions()[q]), w.k,
-                                      w.win, w.stride)
+                idx, _ = O.index_topk(qi_rows, iq["wi"][q], keys["ki"], p, w.k, w.win, w.stride)
                 sel = idx[idx >= 0]
             else:
-                sel = np.arange(w.N)
-            total += time.perf_counter() - t0
-            rows_c = O.round_to(WL.rows(w, "kv_cmp", b * w.N + torch.as_tensor(sel)), "bf16")
-            rows_c[sel == w.c_dst0] = new[0]
-            e = int(w.win_end()[q])
-            rows_w = O.as_f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(max(0, e - w.W + 1), e + 1)))
+                sel = np.arange(O.n_visible(p, w.win, w.stride))
+            t_q += time.perf_counter() - t0
+            if "rows" not in qc:
+                rows_c = O.round_to(WL.rows(w, "kv_cmp", b * w.N + torch.as_tensor(sel)), "bf16")
+                fresh = (sel >= w.c_dst0) & (sel < w.c_dst0 + len(new))
+                rows_c[fresh] = new[sel[fresh] - w.c_dst0]
+                e = int(w.win_end()[q])
+                rows_w = O.as_f64(WL.rows(w, "kv_win", b * w.T_raw + torch.arange(max(0, e - w.W + 1), e + 1)))
+                qc["rows"] = np.concatenate([rows_c, rows_w])
             t0 = time.perf_counter()
-            O.attend(host["q"][q], np.concatenate([rows_c, rows_w]), host["sink"], w.scale)
-            total += time.perf_counter() - t0
-            done += 1
-        if total >= budget_s:
+            O.attend(q_rows, qc["rows"], sink, w.scale)
+            t_q += time.perf_counter() - t0
+            n_q += 1
+            if t_app + t_q >= budget_s:
+                break
+        if t_app + t_q >= budget_s:
             break
-    return {"value": done / total, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": f"{done} queries ({done // w.Q} full batches of {w.Q}) of {w.name}, fp64 numpy; "
-                      f"input regeneration untimed", "seconds": round(total, 2)}
+    step_s = w.B * (t_app / n_app) + w.Q * (t_q / n_q)
+    subset = "all queries" if queries is None else f"{len(qs)} evenly spaced queries"
+    return {"value": w.Q / step_s, "unit": UNIT, "cores": int(_oracle_cores()), "kind": "oracle",
+            "sample": f"{n_q} queries ({subset}, {n_app} appends) of {w.name}"
+                      f"{' with RoPE append' if rope else ''}, fp64 numpy, extrapolated to the batch of {w.Q}; "
+                      f"input regeneration untimed", "seconds": round(t_app + t_q, 2)}
+
+
+def time_oracle_compress(w: WL.Workload, budget_s: float, indexer: bool = False):
+    """Time the oracle's compressor over consecutive chunks of the 1 M-token
+    raw sequence (4,096 entries a chunk) until ``budget_s`` is spent; tokens/s.
+    ``indexer``: the indexer's compressor (Hadamard rotation, E4M3 codes) on
+    its 128-dim stream."""
+    import numpy as np
+
+    import oracle as O
+
+    D = w.Di if indexer else w.D
+    names = ("ikv_raw", "igate_raw") if indexer else ("kv_raw", "gate_raw")
+    ape = WL.make(w, "iape" if indexer else "ape")
+    per = 4096 * w.stride + w.win - w.stride  # tokens of a 4,096-entry chunk
+    t, toks, i = 0.0, 0, 0
+    while t < budget_s and (i + 1) * 4096 * w.stride <= w.bulk_T:
+        r = torch.arange(i * 4096 * w.stride, min(w.bulk_T, i * 4096 * w.stride + per))
+        kv, gate = WL.rows(w, names[0], r), WL.rows(w, names[1], r)
+        t0 = time.perf_counter()
+        if indexer:
+            O.quantize_rows_e4m3(O.index_compress(kv, gate, ape, np.ones(D), w.win, w.stride))
+        else:
+            O.round_to(O.compress(kv, gate, ape, np.ones(D), w.win, w.stride), "bf16")
+        t += time.perf_counter() - t0
+        toks += 4096 * w.stride
+        i += 1
+    return {"value": round(toks / t, 1), "unit": "tokens/s", "cores": int(_oracle_cores()), "kind": "oracle",
+            "sample": f"{i} chunks of 4,096 entries ({toks} tokens) of the {w.bulk_T}-token "
+                      f"{'indexer ' if indexer else ''}stream, fp64 numpy", "seconds": round(t, 2)}
 
 
 # --------------------------------------------------------------------------
@@ -599,6 +721,8 @@ def main():
                     help="the decode step as one fused kernel, as the separate kernels, or the faster of both")
     ap.add_argument("--once", action="store_true",
                     help="profiling aid: build the step without a graph and launch each of its kernels once more")
+    ap.add_argument("--once-bulk", default=None, choices=["compress", "index_compress"],
+                    help="profiling aid: run the 1 M-token bulk compression (or the indexer's) twice, untimed")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -624,8 +748,23 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
         return 1
+    if args.once_bulk:
+        wb, dev = WL.WORKLOADS["csa_decode_1m"], torch.device("cuda", 0)
+        ix = args.once_bulk == "index_compress"
+        kv = WL.make(wb, "ikv_raw" if ix else "kv_raw", dev)
+        gate = WL.make(wb, "igate_raw" if ix else "gate_raw", dev)
+        ape = WL.make(wb, "iape" if ix else "ape", dev)
+        nw = torch.ones(kv.shape[-1], dtype=torch.float32, device=dev)
+        for _ in range(2):
+            if ix:
+                ops.index_compress(kv, gate, ape, nw, wb.win, wb.stride, fp8=True)
+            else:
+                ops.compress(kv, gate, ape, nw, wb.win, wb.stride)
+        torch.cuda.synchronize()
+        print(json.dumps({"once_bulk": args.once_bulk, "tokens": wb.bulk_T}))
+        return 0
     if args.once:
-        step = Step(w, torch.device("cuda", 0), graph=False)  # runs the step once while building it
+        step = Step(w, torch.device("cuda", 0), graph=False, fused=args.path == "fused")  # runs the step once
         torch.cuda.synchronize()
         for _, f in step.parts():
             f()
@@ -651,18 +790,20 @@ def main():
 
     secondary = {}
     if not args.no_secondary and rank == 0 and not dist_on:
-        for name in ("hca_decode_1m", "csa_decode_1m", "csa_decode_64k_fp8", "csa_decode_64k_pro", "csa_prefill_chunk_4k"):
-            if name == w.name:
+        for label, name, rope in SECONDARY:
+            if name == w.name and rope is None:
                 continue
             sw = WL.WORKLOADS[name]
             try:
-                s = time_ours(args, sw, device, False, 0, 1, secondary=True)
+                s = time_ours(args, sw, device, False, 0, 1, secondary=True, rope=rope)
                 del s["step"]
                 rf = roofline_of(sw, path_parts(s["per_kernel_ms"], s["path"]), hbm,
-                                 load_traffic(args.traffic_json, name), tflops)
-                line = {"queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1), "ms_per_step": round(s["ms"], 4),
-                        "path": s["path"], "paths_ms": s["paths_ms"],
+                                 load_traffic(args.traffic_json, label), tflops)
+                line = {"workload": name, "queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1),
+                        "ms_per_step": round(s["ms"], 4), "path": s["path"], "paths_ms": s["paths_ms"],
                         "per_kernel_ms": {k: round(v, 4) for k, v in s["per_kernel_ms"].items()}}
+                if rope:
+                    line["append"] = f"csa_compress_rope: rope_dims {rope[0]}, theta {rope[1]:g}"
                 if prefill(sw):  # tensor-bound: the step's FLOPs against the bf16 peak
                     step_tf = sum(algo_flops(sw).values()) / (s["ms"] * 1e-3) / 1e12
                     line.update(step_TFLOPs=round(step_tf, 1), step_frac=round(step_tf / tflops, 4))
@@ -670,15 +811,33 @@ def main():
                     step_gbs = sum(algo_bytes(sw).values()) / (s["ms"] * 1e-3) / 1e9
                     line.update(step_GBps=round(step_gbs, 1), step_frac=round(step_gbs / hbm, 4))
                 line.update(roofline=rf, status=s["status"])
-                secondary[name] = line
+                secondary[label] = line
             except Exception as ex:  # report, do not hide
-                secondary[name] = {"error": repr(ex)}
+                secondary[label] = {"error": repr(ex)}
             torch.cuda.empty_cache()
-        try:
-            secondary["compress_1m_tokens"] = time_bulk_compress(args, WL.WORKLOADS["csa_decode_1m"], device, hbm)
-        except Exception as ex:
-            secondary["compress_1m_tokens"] = {"error": repr(ex)}
-        torch.cuda.empty_cache()
+        w1m = WL.WORKLOADS["csa_decode_1m"]
+        for label, fn in (("compress_1m_tokens", time_bulk_compress), ("indexer_compress_1m_tokens", time_index_compress)):
+            try:
+                secondary[label] = fn(args, w1m, device, hbm)
+            except Exception as ex:
+                secondary[label] = {"error": repr(ex)}
+            torch.cuda.empty_cache()
+        if not args.no_cpu_baseline:  # the oracle on the host cores, per line (bounded samples)
+            for label, name, rope in SECONDARY:
+                if label not in secondary or "error" in secondary[label]:
+                    continue
+                sw = WL.WORKLOADS[name]
+                qs = None if not prefill(sw) else [round(i * (sw.Q - 1) / 63) for i in range(64)]
+                try:
+                    secondary[label]["cpu_baseline"] = time_oracle(sw, 1, budget_s=60.0, queries=qs, rope=rope)
+                except Exception as ex:
+                    secondary[label]["cpu_baseline"] = {"error": repr(ex)}
+            for label, ix in (("compress_1m_tokens", False), ("indexer_compress_1m_tokens", True)):
+                if "error" not in secondary.get(label, {"error": 1}):
+                    try:
+                        secondary[label]["cpu_baseline"] = time_oracle_compress(w1m, 3.0, indexer=ix)
+                    except Exception as ex:
+                        secondary[label]["cpu_baseline"] = {"error": repr(ex)}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline and not dist_on:

@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort = &bars->abort;
   pdl_wait();  // inputs may come from the previous kernel in the stream
   pdl_release();
+  const uint64_t lim = tc::wait_limit_of(a.status);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tl.q != cur_q) {
           const int slot = nq % F::kQSlots;
           const uint32_t qph = (nq / F::kQSlots) & 1;
-          if (!tc::mbar_wait(&bars->qempty[slot], qph ^ 1, abort, a.status)) break;
+          if (!tc::mbar_wait(&bars->qempty[slot], qph ^ 1, abort, a.status, lim)) break;
           tc::mbar_arrive_expect_tx(&bars->qfull[slot], kQBytes);
           for (int bx = 0; bx < F::kKBoxes; ++bx)
             tc::tma_load_2d(q_buf + slot * kQBytes + bx * F::kQBox, &tm_qi, bx * 64, tl.q * kG * kHi,
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++nq;
           cur_q = tl.q;
         }
-        if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort, a.status)) break;
+        if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort, a.status, lim)) break;
         tc::mbar_arrive_expect_tx(&bars->full[stage], kTileBytes);
         const int row = (tl.q * kG / a.q_per_seq) * a.N_max + tl.j0;
         for (int bx = 0; bx < 2; ++bx)  // bf16: dims 64 bx.., E4M3: rows 128 bx..
@@ -190,12 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tl.q != cur_q) {
           if (cur_q >= 0) tc::commit(&bars->qempty[slot]);  // old head block free once its MMAs finish
           slot = nq % F::kQSlots;
-          if (!tc::mbar_wait(&bars->qfull[slot], (nq / F::kQSlots) & 1, abort, a.status)) break;
+          if (!tc::mbar_wait(&bars->qfull[slot], (nq / F::kQSlots) & 1, abort, a.status, lim)) break;
           ++nq;
           cur_q = tl.q;
         }
-        if (!tc::mbar_wait(&bars->accempty[acc], accph ^ 1, abort, a.status)) break;
-        if (!tc::mbar_wait(&bars->full[stage], phase, abort, a.status)) break;
+        if (!tc::mbar_wait(&bars->accempty[acc], accph ^ 1, abort, a.status, lim)) break;
+        if (!tc::mbar_wait(&bars->full[stage], phase, abort, a.status, lim)) break;
         tc::fence_after_sync();
         const uint32_t a_base = tc::smem_u32(stage_buf + stage * kTileBytes);
         const uint32_t b_base = tc::smem_u32(q_buf + slot * kQBytes);
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         cur_g = tl.q;
       }
-      const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status);
+      const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status, lim);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc::fence_after_sync();
       const int j = tl.j0 + row;
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (kFp8) {
         if (t + 1 < t_end) load_sk(t + 1);
       }
-      const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status);
+      const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status, lim);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc::fence_after_sync();
       float sc[F::kSub];

@@ -307,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm->tmem_base;
   volatile int *abort = &sm->abort;
   pdl_wait();  // inputs (indices, queries, caches) may come from the previous kernel
+  const uint64_t lim = tc::wait_limit_of(a.status);
   pdl_release();
 
   const RowList L = row_list(a, qq, threadIdx.x == 0 ? a.status : nullptr);
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (run) prefetch_l2(li);
         for (int r = 1; r <= kAhead; ++r) prefetch_l2(li + 2 * r);
       }
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status))) break;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm->kv_empty[g], ((li >> 1) & 1) ^ 1, abort, a.status, lim))) break;
       if (run) {
         if (part == 0 && lane == 0) {
           tc::mbar_arrive_expect_tx(&sm->kv_full[g], kTileBytes);
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = tc::idesc_bf16(64, 64, 0, 0);
       constexpr uint32_t idesc_pv = tc::idesc_bf16(128, 64, 1, 1);
       const uint32_t kv_base = tc::smem_u32(kv), q_base = tc::smem_u32(qs), p_base = tc::smem_u32(ps);
-      bool ok = ntiles == 0 || tc::mbar_wait(&sm->q_full, 0, abort, a.status);
+      bool ok = ntiles == 0 || tc::mbar_wait(&sm->q_full, 0, abort, a.status, lim);
       const uint64_t ad_kv = tc::sw128_desc(kv_base, 16, 1024), bd_q = tc::sw128_desc(q_base, 16, 1024);
       const uint64_t ad_v = tc::sw128_desc(kv_base, kBoxBytes, 1024), bd_p = tc::sw128_desc(p_base, kPBytes, 1024);
       // Two streams of work, issued as soon as each is ready: S^T(ns) once
@@ -493,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t now = tc::globaltimer_ns();
           if (t_idle == 0) {
             t_idle = now;
-          } else if (now - t_idle > tc::kWaitLimitNs) {
+          } else if (now - t_idle > lim) {
             raise_status(a.status, CSA_STATUS_WAIT_TIMEOUT);
             *abort = 1;
             ok = false;
@@ -526,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int li = 0; li < ntiles; ++li) {
       const int buf = li & 1;
-      const bool got = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full[buf], (li >> 1) & 1, abort, a.status));
+      const bool got = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full[buf], (li >> 1) & 1, abort, a.status, lim));
       tc::fence_after_sync();
       const int rA = (t0 + li) * kRows + rowA, rB = rA + 8;
       const bool validA = rA < L.nsel4 ? (rA < L.nsel && (!sparse || (idxA >= 0 && idxA < a.N_max))) : rA < L.R;
@@ -644,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // but that one, and a P(li) that needs no rescale does not wait. One
         // barrier per tile slot mod 4, so a skipped phase is never mistaken
         // for another: slot (li - 1) mod 4 next completes for tile li + 3.)
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->pv_done[(li - 1) & 3], ((li - 1) >> 2) & 1, abort, a.status));
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(&sm->pv_done[(li - 1) & 3], ((li - 1) >> 2) & 1, abort, a.status, lim));
         tc::fence_after_sync();
         if (ok) {
 #pragma unroll 1
@@ -668,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&sm->p_full[buf]);
     }
     // ---- epilogue: per-head sums, then O (partials, or the final output)
-    ok = __all_sync(0xffffffffu, ok && (ntiles == 0 || tc::mbar_wait(&sm->o_done, 0, abort, a.status)));
+    ok = __all_sync(0xffffffffu, ok && (ntiles == 0 || tc::mbar_wait(&sm->o_done, 0, abort, a.status, lim)));
     tc::fence_after_sync();
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1)

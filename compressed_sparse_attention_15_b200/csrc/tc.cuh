@@ -72,25 +72,42 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // waits in these kernels last microseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Bounded wait for the phase of parity `parity`. On timeout raises
-// CSA_STATUS_WAIT_TIMEOUT, sets *abort and returns false; returns false at
-// once if another role has set *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+// The limit of a kernel's bounded waits: bytes 8..15 of the caller's
+// workspace (the status page), in nanoseconds, or kWaitLimitNs when zero.
+// (A test shortens it to make a wait run out; callers leave it zero.)
+__device__ __forceinline__ uint64_t wait_limit_of(const uint32_t *status) {
+  if (!status) return kWaitLimitNs;
+  const uint64_t v = *reinterpret_cast<const volatile uint64_t *>(status + 2);
+  return v ? v : kWaitLimitNs;
+}
+
+// Bounded wait for the phase of parity `parity`. On timeout (after `limit`
+// ns) raises CSA_STATUS_WAIT_TIMEOUT, sets *abort and returns false; returns
+// false at once if another role has set *abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status,
+                                          uint64_t limit) {
+  // The clock is read every 64th try, or every try under a short limit.
+  const uint32_t every = limit < 1000000u ? 0u : 63u;
   uint64_t t0 = 0;
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if ((i & 63) == 63) {
+    if ((i & every) == every) {
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kWaitLimitNs) {
+      } else if (now - t0 > limit) {
         raise_status(status, CSA_STATUS_WAIT_TIMEOUT);
         *abort = 1;
         return false;
       }
     }
   }
+}
+
+// The same with the default limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+  return mbar_wait(bar, parity, abort, status, kWaitLimitNs);
 }
 
 // Bounded wait used while draining at teardown (no abort check).

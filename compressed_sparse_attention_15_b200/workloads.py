@@ -21,6 +21,9 @@ Recipe (tensor id: distribution):
  14 sq     [Q, Hi]        U(0,1)/64 + 1/256            their per-row scales (fp32)
  15 ki8    [B, N, Di]     E4M3 codes of 64 * N(0,1)   FP8 indexer keys
  16 sk     [B, N]         U(0,1)/64 + 1/256            their per-row scales (fp32)
+ 17 ikv_raw   [1, bulk_T, Di] N(0,1)   raw indexer KV of the bulk-compressed sequence
+ 18 igate_raw [1, bulk_T, Di] N(0,1)   its gate logits
+ 19 iape   [win, Di]      N(0,0.1)    the indexer compressor's position embedding (fp32)
     norm_w [D]            1.0         RMSNorm weight (fp32)
 bf16 tensors are drawn in fp32 and rounded once to bf16 (RNE); FP8 codes are
 fp32 draws rounded once to E4M3 (RNE, torch's float8_e4m3fn conversion).
@@ -35,7 +38,7 @@ import torch
 from . import synth
 
 TID = {"q": 1, "kv_cmp": 2, "kv_win": 3, "qi": 4, "wi": 5, "ki": 6, "sink": 7, "kv_raw": 8, "gate": 9, "ape": 10,
-       "gate_raw": 12, "qi8": 13, "sq": 14, "ki8": 15, "sk": 16}
+       "gate_raw": 12, "qi8": 13, "sq": 14, "ki8": 15, "sk": 16, "ikv_raw": 17, "igate_raw": 18, "iape": 19}
 FP8_CODE_STD = 64.0  # FP8 code draws are FP8_CODE_STD * N(0,1), inside the E4M3 range (448)
 
 
@@ -132,14 +135,14 @@ def tensor_shape(w: Workload, name: str):
         "qi": (w.Q, w.Hi, w.Di), "wi": (w.Q, w.Hi), "ki": (w.B, w.N, w.Di), "sink": (w.H,),
         "kv_raw": (1, w.bulk_T, w.D), "gate_raw": (1, w.bulk_T, w.D), "ape": (w.win, w.D),
         "gate": (w.B, w.T_c, w.D), "qi8": (w.Q, w.Hi, w.Di), "sq": (w.Q, w.Hi), "ki8": (w.B, w.N, w.Di),
-        "sk": (w.B, w.N),
+        "sk": (w.B, w.N), "ikv_raw": (1, w.bulk_T, w.Di), "igate_raw": (1, w.bulk_T, w.Di), "iape": (w.win, w.Di),
     }[name]
 
 
 def _dtype_of(w: Workload, name: str):
     if name in ("qi8", "ki8"):
         return torch.uint8
-    return torch.float32 if name in ("wi", "sink", "ape", "norm_w", "sq", "sk") else w.dtype
+    return torch.float32 if name in ("wi", "sink", "ape", "iape", "norm_w", "sq", "sk") else w.dtype
 
 
 def _codes(x: torch.Tensor) -> torch.Tensor:
@@ -156,7 +159,7 @@ def make(w: Workload, name: str, device="cpu") -> torch.Tensor:
         return synth.uniform(w.seed, TID[name], shape, device=device) / 64 + 1.0 / 256
     if name in ("qi8", "ki8"):
         return _codes(synth.normal(w.seed, TID[name], shape, device=device))
-    std = 0.1 if name == "ape" else 1.0
+    std = 0.1 if name in ("ape", "iape") else 1.0
     return synth.normal(w.seed, TID[name], shape, std=std, dtype=dt, device=device)
 
 
@@ -169,7 +172,7 @@ def rows(w: Workload, name: str, flat_rows) -> torch.Tensor:
     if name in ("sq", "sk"):
         flat = torch.as_tensor(flat_rows, dtype=torch.int64)
         return synth.uniform_at(w.seed, TID[name], flat) / 64 + 1.0 / 256
-    std = 0.1 if name == "ape" else 1.0
+    std = 0.1 if name in ("ape", "iape") else 1.0
     return synth.normal_rows(w.seed, TID[name], shape, flat_rows, std=std, dtype=_dtype_of(w, name))
 
 

@@ -34,6 +34,12 @@
  *    bytes hold the status word; the library writes the rest freely. The
  *    status word must be zero before the first call (cudaMemset once); calls
  *    only ever OR bits into it.
+ *  - Bounded waits: every wait of a tensor-core kernel on its own pipeline
+ *    gives up after a time limit, raises CSA_STATUS_WAIT_TIMEOUT, drops the
+ *    rest of its work (that output is invalid) and returns, so the context
+ *    stays usable. The limit is 2 s unless bytes 8..15 of the workspace hold a
+ *    non-zero uint64 number of nanoseconds (for tests of the timeout path;
+ *    leave them zero otherwise).
  */
 #ifndef CSA_H_
 #define CSA_H_

@@ -75,3 +75,17 @@ def test_roofline_names_the_dominant_kernel(name, kernel, bound):
     if w.mode == "csa":
         fused = {"compress": 0.01, "index_scores": 0.01, "topk_mqa": 0.01}
         assert bench.roofline_of(w, fused, 6452.8, None, 1676.0)["kernel"] == kernel
+
+
+def test_oracle_timing_on_a_query_subset():
+    # the CPU-baseline leg: a subset of queries, extrapolated to the batch
+    w = WL.WORKLOADS["tiny_csa_prefill_fp32"]
+    r = bench.time_oracle(w, 1, 5.0, queries=[0, 100, 255], rope=(8, 10000.0))
+    assert r["value"] > 0 and r["kind"] == "oracle"
+    assert r["sample"].startswith("3 queries (3 evenly spaced queries, 1 appends)")
+
+
+def test_secondary_lines_cover_the_other_workloads():
+    names = {n for _, n, _ in bench.SECONDARY}
+    assert names == set(WL.WORKLOADS) - {"tiny_csa_prefill_fp32"}
+    assert any(rope for _, _, rope in bench.SECONDARY)
