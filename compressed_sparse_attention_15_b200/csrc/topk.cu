@@ -14,7 +14,9 @@
 // block give each kept entry its output slot, so the output is ascending and
 // deterministic.
 //
-// Launch shapes. Few queries (a decode batch): the list of one query is cut
+// Launch shapes. Lists of up to 16K entries: one 1024-thread CTA per query
+// holding every key in registers (topk_block_kernel, few block barriers).
+// Longer lists with few queries (a decode batch): the list of one query is cut
 // into C contiguous slices, one CTA of a thread-block cluster each (C <= 8,
 // about SMs / Q); the slices' histograms are summed through distributed
 // shared memory at every radix pass, and each CTA emits its own slice at the
@@ -337,6 +339,328 @@ __global__ void __launch_bounds__(kThreads) topk_stage2_kernel(TopkArgs a, const
                         [out, idxs](uint32_t slot, int j, uint32_t) { out[slot] = idxs[j]; });
 }
 
+// ---------------------------------------------------------------- one CTA
+// One 1024-thread CTA per query with every key in registers: warp w holds the
+// 32 R positions [32 R w, 32 R (w + 1)), lane l those of them congruent to l
+// mod 32 (n <= 1024 R; coalesced loads). Selection on one SM is bound by
+// instruction issue, so most keys are dropped early: a sample of the keys
+// (one per thread) gives a lower threshold with enough keys above it (the
+// sample's rank is the expected count plus four standard deviations), those
+// keys go to shared memory in position order, and the exact radix select
+// runs over them only. When the candidates are too few or too many for the
+// buffer, the radix select runs over all keys instead. Either way the
+// selection is exact.
+
+struct BlockShared {
+  uint32_t hist[2][kBins];
+  uint32_t wtot[2][kWarps];
+  uint32_t wmin[kWarps], wmax[kWarps];
+  uint32_t wg[kWarps], we[kWarps];
+  uint32_t dec[2][3];  // per pass parity: boundary bin, keys above it, keys in it
+  uint32_t cand[kFew];
+  uint32_t ncand;
+  uint32_t sel_t, sel_ngt;  // the few-candidates finish, computed by warp 0
+};
+constexpr int kCandCap = 4096;  // candidate buffer (dynamic shared memory: keys, then positions)
+
+// Exclusive prefix over the warps of a per-warp value (every lane passes its
+// warp's value). One barrier; every thread gets its warp's offset and the
+// total.
+__device__ __forceinline__ void warp_offsets(uint32_t *slot, uint32_t v, int lane, int warp, uint32_t &off,
+                                             uint32_t &total) {
+  if (lane == 0) slot[warp] = v;
+  __syncthreads();
+  uint32_t inc = slot[lane];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  const uint32_t p = __shfl_sync(0xffffffffu, inc, warp > 0 ? warp - 1 : 0);
+  off = warp > 0 ? p : 0u;
+  total = __shfl_sync(0xffffffffu, inc, 31);
+}
+
+// One radix pass's histogram scan: the bins of `h` hold the matching keys;
+// finds the bin where the count from the top reaches `want` (computed by
+// want_of(total) once the total is known) and returns (bin, keys above it,
+// keys in it), `want` and `total` in every thread; the bin is meaningful
+// only for 1 <= want <= total. Three barriers (the caller's histogram is
+// complete at the first).
+template <class WantOf>
+__device__ __forceinline__ void boundary_bin(BlockShared &sh, const uint32_t *h, int pass, int lane, int warp,
+                                             WantOf want_of, uint32_t &bin, uint32_t &above_out, uint32_t &cb,
+                                             uint32_t &want, uint32_t &total) {
+  __syncthreads();
+  // warp w scans bins [kBins - 64 (w + 1), kBins - 64 w) from the top: lane
+  // l holds bins hb = kBins - 1 - 64 w - 2 l and hb - 1
+  const int hb = kBins - 1 - 64 * warp - 2 * lane;
+  const uint32_t c_hi = h[hb], c_lo = h[hb - 1], c = c_hi + c_lo;
+  uint32_t inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) sh.wtot[pass & 1][warp] = inc;
+  __syncthreads();
+  uint32_t winc = sh.wtot[pass & 1][lane];  // every warp combines the 32 warp totals itself
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, winc, o);
+    if (lane >= o) winc += y;
+  }
+  total = __shfl_sync(0xffffffffu, winc, 31);
+  want = want_of(total);
+  const uint32_t w_above = __shfl_sync(0xffffffffu, winc, warp > 0 ? warp - 1 : 0);
+  const uint32_t above = (warp > 0 ? w_above : 0u) + inc - c;  // matching keys in the bins above this lane's two
+  if (above < want && want <= above + c) {  // exactly one lane of the block (when 1 <= want <= total)
+    const bool in_hi = want <= above + c_hi;
+    uint32_t *d = sh.dec[pass & 1];
+    d[0] = in_hi ? (uint32_t)hb : (uint32_t)(hb - 1);
+    d[1] = in_hi ? above : above + c_hi;
+    d[2] = in_hi ? c_hi : c_lo;
+  }
+  __syncthreads();
+  bin = sh.dec[pass & 1][0];
+  above_out = sh.dec[pass & 1][1];
+  cb = sh.dec[pass & 1][2];
+}
+
+// Exact radix select over the keys kv[r] (r < nv) of every thread, in units u
+// = kv - base, `range` the largest u: returns in every thread the threshold
+// tau_u and kk, the number of keys equal to it that are kept (the other k -
+// kk kept keys exceed it). Both histograms are clear on entry and sh.ncand is
+// 0; MSD digits of 11 bits from the top set bit of the range.
+template <int RR>
+__device__ __forceinline__ void radix_select(BlockShared &sh, const uint32_t (&kv)[RR], int nv, uint32_t base,
+                                             uint32_t range, uint32_t k, int lane, int warp, uint32_t &tau_u,
+                                             uint32_t &kk_out) {
+  uint32_t prefix = 0u, mask = 0u, kk = k;
+  tau_u = 0u;  // range 0: every key equals base
+  int top = range == 0u ? 0 : 32 - __clz(range);
+  for (int pass = 0; top > 0; ++pass) {
+    const int width = top >= 11 ? 11 : top;
+    const int shift = top - width;
+    const uint32_t dmask = (1u << width) - 1u;
+    uint32_t *h = sh.hist[pass & 1];
+#pragma unroll
+    for (int r = 0; r < RR; ++r) {
+      const uint32_t u = kv[r] - base;
+      if (r < nv && (u & mask) == prefix) atomicAdd(&h[(u >> shift) & dmask], 1u);
+    }
+    uint32_t bin, above, cb, want, total;
+    boundary_bin(sh, h, pass, lane, warp, [kk](uint32_t) { return kk; }, bin, above, cb, want, total);
+    kk -= above;
+    prefix |= bin << shift;
+    mask |= dmask << shift;
+    top = shift;
+    // no thread reads this histogram any more: cleared for pass + 2
+    for (int i = threadIdx.x; i < kBins; i += kThreads) h[i] = 0u;
+    if (top == 0) {  // every bit fixed: the prefix is the threshold
+      tau_u = prefix;
+      break;
+    }
+    if (kk == cb && prefix != 0u) {  // every key of the boundary bin is kept: u >= prefix
+      tau_u = prefix - 1u;
+      kk = 0u;
+      break;
+    }
+    if (cb <= (uint32_t)kFew) {
+      // Few keys in the boundary bin: gather them; warp 0 finds the kk-th
+      // largest among them.
+#pragma unroll
+      for (int r = 0; r < RR; ++r) {
+        const uint32_t u = kv[r] - base;
+        if (r < nv && (u & mask) == prefix) sh.cand[atomicAdd(&sh.ncand, 1u)] = u;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int nc = (int)sh.ncand;
+        uint32_t t, ngt;
+        sel::warp_select(lane < nc ? sh.cand[lane] : 0u, nc, kk, t, ngt);
+        if (lane == 0) {
+          sh.sel_t = t;
+          sh.sel_ngt = ngt;
+        }
+      }
+      __syncthreads();
+      tau_u = sh.sel_t;
+      kk -= sh.sel_ngt;
+      break;
+    }
+  }
+  kk_out = kk;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads) topk_block_kernel(TopkArgs a) {
+  __shared__ alignas(16) BlockShared sh;
+  extern __shared__ uint32_t cbuf[];  // R >= 8: [kCandCap] candidate keys, then [kCandCap] positions
+  pdl_wait();
+  pdl_release();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int q = blockIdx.x;
+  const int n = clamp_count(a.n_cmp[q], a.N_max, threadIdx.x == 0 ? a.status : nullptr);
+  const int k = a.k;
+  int32_t *out = a.out_idx + (size_t)q * k;
+  if (n <= k) {
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const float *s = a.scores + (size_t)q * a.N_max;
+  // key r of this thread: position base + 32 r, valid for r < nvr
+  const int base = 32 * R * warp + lane;
+  const int nvr = base < n ? min(R, (n - base + 31) / 32) : 0;
+  uint32_t key[R];  // the raw bits first: every load in flight before the first is used
+#pragma unroll
+  for (int r = 0; r < R; ++r) key[r] = r < nvr ? __float_as_uint(__ldcg(s + base + 32 * r)) : 0u;
+  uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    key[r] = score_key(__uint_as_float(key[r]));
+    if (r < nvr) {
+      lo = min(lo, key[r]);
+      hi = max(hi, key[r]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    sh.wmin[warp] = lo;
+    sh.wmax[warp] = hi;
+  }
+  for (int i = threadIdx.x; i < 2 * kBins; i += kThreads) (&sh.hist[0][0])[i] = 0u;
+  if (threadIdx.x == 0) sh.ncand = 0u;
+  __syncthreads();
+  lo = sh.wmin[lane];
+  hi = sh.wmax[lane];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const uint32_t kmin = lo, range = hi - lo;
+
+  if constexpr (R >= 8) {
+    // The sample: key warp % R of every thread (1,024 keys, 32 runs of 32).
+    const int rs = warp % R;
+    uint32_t su = 0u;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (r == rs) su = key[r] - kmin;
+    const int top = range == 0u ? 0 : 32 - __clz(range);
+    const int shift1 = top > 11 ? top - 11 : 0;
+    if (rs < nvr) atomicAdd(&sh.hist[0][su >> shift1], 1u);
+    // rank m among the S samples: the expected number of samples in the
+    // top k, plus four standard deviations and 8
+    auto rank_of = [&](uint32_t S) {
+      const float mu = (float)k * (float)S / (float)n;
+      return (uint32_t)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
+    };
+    uint32_t bin, above, cb, m, S;
+    boundary_bin(sh, sh.hist[0], 0, lane, warp, rank_of, bin, above, cb, m, S);
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh.hist[0][i] = 0u;  // cleared for the selection
+    if (range != 0u && m < S) {
+      // candidates: keys at or above the lower edge of the sample's boundary bin
+      const uint32_t ulow = bin << shift1;
+      uint32_t c = 0u;
+#pragma unroll
+      for (int r = 0; r < R; ++r) c += __popc(__ballot_sync(0xffffffffu, r < nvr && key[r] - kmin >= ulow));
+      uint32_t off, C;
+      warp_offsets(sh.wg, c, lane, warp, off, C);
+      if (C >= (uint32_t)k && C <= (uint32_t)kCandCap) {
+        // in position order: warp by warp, key slot by key slot, lane by lane
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const bool sel = r < nvr && key[r] - kmin >= ulow;
+          const uint32_t mm = __ballot_sync(0xffffffffu, sel);
+          if (sel) {
+            const uint32_t slot = off + __popc(mm & lt);
+            cbuf[slot] = key[r] - kmin - ulow;
+            cbuf[kCandCap + slot] = (uint32_t)(base + 32 * r);
+          }
+          off += __popc(mm);
+        }
+        __syncthreads();
+        // thread t: candidates 4t .. 4t + 3
+        const int c0 = 4 * (int)threadIdx.x;
+        const int ncv = max(0, min(4, (int)C - c0));
+        uint32_t cv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cv[i] = i < ncv ? cbuf[c0 + i] : 0u;
+        uint32_t tau, kk;
+        radix_select<4>(sh, cv, ncv, 0u, range - ulow, (uint32_t)k, lane, warp, tau, kk);
+        // ordered compaction over the candidates
+        uint32_t g = 0u, e = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          g += (i < ncv && cv[i] > tau) ? 1u : 0u;
+          e += (i < ncv && cv[i] == tau) ? 1u : 0u;
+        }
+        uint32_t gi = g, ei = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t yg = __shfl_up_sync(0xffffffffu, gi, o), ye = __shfl_up_sync(0xffffffffu, ei, o);
+          if (lane >= o) {
+            gi += yg;
+            ei += ye;
+          }
+        }
+        uint32_t og, oe, tg, te;
+        warp_offsets(sh.wg, __shfl_sync(0xffffffffu, gi, 31), lane, warp, og, tg);
+        warp_offsets(sh.we, __shfl_sync(0xffffffffu, ei, 31), lane, warp, oe, te);
+        uint32_t G = og + gi - g, E = oe + ei - e;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i < ncv && cv[i] > tau) {
+            out[G + min(E, kk)] = (int32_t)cbuf[kCandCap + c0 + i];
+            ++G;
+          } else if (i < ncv && cv[i] == tau) {
+            if (E < kk) out[G + E] = (int32_t)cbuf[kCandCap + c0 + i];
+            ++E;
+          }
+        }
+        return;
+      }
+    }
+    __syncthreads();  // the sample's histogram is clear before the selection over every key
+  }
+
+  // Selection over every key, then the ordered compaction: warp w's kept
+  // keys go to the slots after those of warps 0 .. w - 1, in position order
+  // within the warp (ballots); ties take the first kk positions.
+  uint32_t tau_u, kk;
+  radix_select<R>(sh, key, nvr, kmin, range, (uint32_t)k, lane, warp, tau_u, kk);
+  const uint32_t tau = tau_u + kmin;
+  uint32_t g = 0u, e = 0u;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const bool v = r < nvr;
+    g += __popc(__ballot_sync(0xffffffffu, v && key[r] > tau));
+    e += __popc(__ballot_sync(0xffffffffu, v && key[r] == tau));
+  }
+  uint32_t G, E, tg, te;
+  warp_offsets(sh.wg, g, lane, warp, G, tg);
+  warp_offsets(sh.we, e, lane, warp, E, te);
+  if (g + e == 0u) return;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int j = base + 32 * r;
+    const bool is_gt = r < nvr && key[r] > tau, is_eq = r < nvr && key[r] == tau;
+    const uint32_t mg = __ballot_sync(0xffffffffu, is_gt), me = __ballot_sync(0xffffffffu, is_eq);
+    const uint32_t Gl = G + __popc(mg & lt), El = E + __popc(me & lt);
+    if (is_gt) out[Gl + min(El, kk)] = j;
+    else if (is_eq && El < kk) out[Gl + El] = j;
+    G += __popc(mg);
+    E += __popc(me);
+  }
+}
+
 }  // namespace
 
 // Cluster size for one query's list: about SMs / Q CTAs, at most 8, at
@@ -364,7 +688,15 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, s
     cudaFuncSetAttribute(topk_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 * 4);
     cudaFuncSetAttribute(topk_stage2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
+    for (auto kern : {topk_block_kernel<8>, topk_block_kernel<16>})
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * kCandCap * (int)sizeof(uint32_t));
   });
+  // Lists of up to 16 K entries: one CTA per query, keys in registers.
+  if (a.N_max <= 16 * kThreads) {
+    const int R = (a.N_max + kThreads - 1) / kThreads;
+    auto kern = R <= 4 ? topk_block_kernel<4> : R <= 8 ? topk_block_kernel<8> : topk_block_kernel<16>;
+    return launch_pdl(kern, dim3(a.Q), dim3(kThreads), R <= 4 ? 0 : 2 * kCandCap * sizeof(uint32_t), stream, a);
+  }
   if (const int C = plan_cluster(a.Q, a.N_max, a.k)) {
     const int S = ((a.N_max + C - 1) / C + 31) & ~31;
     return launch_pdl_cluster(topk_cluster_kernel, dim3(C, a.Q), dim3(kThreads), (size_t)S * 4, stream, (unsigned)C,

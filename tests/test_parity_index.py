@@ -63,10 +63,12 @@ def test_topk_exact_on_given_scores(cuda_device, N, k):
 
 
 @pytest.mark.parametrize("Q,N,k,shape", [
-    (32, 16383, 512, "cluster of 4 CTAs per query (64K-context decode batch)"),
+    (32, 16383, 512, "one CTA per query, 16 keys per thread in registers (64K-context decode batch)"),
+    (3, 2000, 64, "one CTA per query, 4 keys per thread in registers"),
+    (100, 5000, 512, "one CTA per query, 8 keys per thread in registers"),
     (8, 262143, 1024, "cluster of 8 CTAs per query, 32K entries each (1M-context decode batch)"),
-    (5, 4500, 512, "cluster of 3, a short last slice"),
-    (100, 5000, 512, "one CTA per query, keys cached"),
+    (5, 30000, 512, "cluster of 8, a short last slice"),
+    (100, 20000, 512, "one CTA per query, keys cached in shared memory"),
     (100, 60000, 64, "two stages: segment winners, then a merge"),
     (76, 1 << 20, 2048, "one CTA per query re-reading the scores (winners too many to merge)"),
 ])

@@ -33,6 +33,10 @@ def _dev(cuda_device, *ts):
     (3, 1, 50, 30, 8, 64, 7, 5, torch.bfloat16),         # small odd shapes (generic kernel)
     (4, 4, 300, 40, 64, 512, 200, 16, torch.float32),
     (4, 2, 2000, 200, 128, 512, 1024, 128, torch.bfloat16),  # V4-Pro: 128 heads (two 64-head groups), top-1024
+    # 16+ queries: one CTA per (query, 64 heads) walking all of the query's tiles
+    (16, 4, 2000, 200, 64, 512, 512, 128, torch.bfloat16),
+    (18, 6, 100, 64, 64, 512, 40, 128, torch.bfloat16),   # one selected tile, windows clipped
+    (16, 2, 2000, 200, 128, 512, 1024, 128, torch.bfloat16),  # 128 heads, 18 tiles per query
 ])
 def test_sparse_mqa_matches_oracle(cuda_device, Q, B, N, T_raw, H, D, k, W, dtype):
     q, kv_cmp, kv_win, sink = _mqa_inputs(1, Q, B, N, T_raw, H, D, dtype)
@@ -85,12 +89,12 @@ def test_sparse_with_all_entries_equals_hca(cuda_device):
     assert_close(b, ref, torch.bfloat16, "hca")
 
 
-@pytest.mark.parametrize("mode", ["sparse", "hca"])
-def test_mqa_growing_logits_force_running_max_updates(cuda_device, mode):
+@pytest.mark.parametrize("mode,Q", [("sparse", 3), ("hca", 3), ("sparse", 16)])
+def test_mqa_growing_logits_force_running_max_updates(cuda_device, mode, Q):
     # Row norms grow along the row list and the softmax scale is large, so
     # later 128-row tiles raise the per-head running maximum far past the
     # first tile's: exercises the deferred rescaling of the accumulator.
-    Q, B, N, T_raw, H, D, k, W = 3, 3, 900, 128, 64, 512, 768, 128
+    B, N, T_raw, H, D, k, W = Q, 900, 128, 64, 512, 768, 128
     q, kv_cmp, kv_win, sink = _mqa_inputs(6, Q, B, N, T_raw, H, D, torch.float32)
     grow = torch.linspace(0.2, 2.0, N).reshape(1, N, 1)
     kv_cmp = (kv_cmp * grow).to(torch.bfloat16)
@@ -102,7 +106,7 @@ def test_mqa_growing_logits_force_running_max_updates(cuda_device, mode):
         out = ops.sparse_mqa(*_dev(cuda_device, q, kv_cmp, idx, kv_win, we, sink), scale, W)
         ref = [O.sparse_mqa(q[i], kv_cmp[i], idx[i].numpy(), kv_win[i], T_raw - 1, W, sink, scale) for i in range(Q)]
     else:
-        n = torch.tensor([N, N // 2, 300], dtype=torch.int32)
+        n = torch.tensor([N, N // 2, 300][:Q], dtype=torch.int32)
         out = ops.hca_mqa(*_dev(cuda_device, q, kv_cmp, n, kv_win, we, sink), scale, W)
         ref = [O.hca_mqa(q[i], kv_cmp[i], int(n[i]), kv_win[i], T_raw - 1, W, sink, scale) for i in range(Q)]
     torch.cuda.synchronize()
