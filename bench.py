@@ -107,7 +107,7 @@ SECONDARY = (("hca_decode_1m", "hca_decode_1m", None), ("csa_decode_1m", "csa_de
 # A step part whose algorithmic bytes and FLOPs are another's: the attention
 # with the selection made inside it moves what the attention moves.
 PART_ALIAS = {"topk_mqa": "mqa"}
-# The fused decode-step kernel moves the whole step's bytes.
+# One csa_decode_step call moves the whole step's bytes.
 WHOLE_STEP = "decode_step"
 
 
@@ -320,14 +320,15 @@ def _time_steps(step, flush, stream, K):
 
 
 def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=False, rope=None):
-    """Times the step on both paths (the whole step as one fused kernel, and
-    the separate kernels), reports the faster; the other path's time and the
+    """Times the step on both paths (the whole step as one csa_decode_step
+    call, its kernels chained on one stream; and the separate calls, the
+    append on a forked stream), reports the faster; the other path's time and the
     separate kernels' per-kernel times are kept for the record."""
     flush = L2Flush(device)
     stream = torch.cuda.current_stream(device)
     steps, launches = {}, {}
     for fused in (True, False):
-        if args.path != "both" and (args.path == "fused") != fused:
+        if args.path != "both" and (args.path == "step_call") != fused:
             continue
         n0 = _lib.lib().csa_launch_count()
         caches = steps[True].caches if True in steps else None
@@ -338,7 +339,7 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     torch.cuda.synchronize()
     K0 = max(5, args.steps // 5)
     trial = {f: _time_steps(st, flush, stream, K0) for f, st in steps.items()}
-    # the fused kernel only when clearly faster (its per-kernel split is one part)
+    # the step call only when clearly faster (its per-kernel split is one part)
     fused = len(trial) == 1 and True in trial or (len(trial) == 2 and trial[True] < 0.97 * trial[False])
     step = steps[fused]
     launches_per_step = launches[fused]
@@ -386,10 +387,10 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
                 acc[n] += ev[i].elapsed_time(ev[i + 1]) / Kp
         per.update(acc)
     status = step.ds.status()
-    paths = {("fused" if f else "separate"): round(v, 4) for f, v in trial.items()}
+    paths = {("step_call" if f else "separate"): round(v, 4) for f, v in trial.items()}
     return {"ms": ms_max, "ms_local": ms, "per_kernel_ms": per, "launches_per_step": int(launches_per_step),
             "wall_s": wall, "clocks": clocks.summary(), "status": status, "K": K, "step": step,
-            "path": "fused" if fused else "separate", "paths_ms": paths}
+            "path": "step_call" if fused else "separate", "paths_ms": paths}
 
 
 def time_bulk_compress(args, w: WL.Workload, device, hbm_gbs):
@@ -465,7 +466,7 @@ def time_index_compress(args, w: WL.Workload, device, hbm_gbs):
 
 
 def path_parts(per_kernel_ms, path):
-    """The per-kernel times of the path that was timed: the fused kernel, or
+    """The per-kernel times of the path that was timed: the step call, or
     the separate kernels."""
     if path == "fused":
         return {k: v for k, v in per_kernel_ms.items() if k == WHOLE_STEP}
@@ -718,8 +719,9 @@ def main():
     ap.add_argument("--clock-log", default=None,
                     help="file for the nvidia-smi samples taken during the timed region (default: a temporary file)")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
-    ap.add_argument("--path", default="both", choices=["both", "fused", "separate"],
-                    help="the decode step as one fused kernel, as the separate kernels, or the faster of both")
+    ap.add_argument("--path", default="both", choices=["both", "step_call", "separate"],
+                    help="the decode step as one csa_decode_step call (its kernels chained on one stream), as "
+                         "separate calls, or the faster of both")
     ap.add_argument("--once", action="store_true",
                     help="profiling aid: build the step without a graph and launch each of its kernels once more")
     ap.add_argument("--once-bulk", default=None, choices=["compress", "index_compress"],
@@ -765,7 +767,7 @@ def main():
         print(json.dumps({"once_bulk": args.once_bulk, "tokens": wb.bulk_T}))
         return 0
     if args.once:
-        step = Step(w, torch.device("cuda", 0), graph=False, fused=args.path == "fused")  # runs the step once
+        step = Step(w, torch.device("cuda", 0), graph=False, fused=args.path == "step_call")  # runs the step once
         torch.cuda.synchronize()
         for _, f in step.parts():
             f()
@@ -783,7 +785,8 @@ def main():
     w = WL.shard(w, rank)  # this rank's own sequences (same shapes)
     r = time_ours(args, w, device, dist_on, rank, world)
     traffic = load_traffic(args.traffic_json, w.name)
-    roof = roofline_of(w, path_parts(r["per_kernel_ms"], r["path"]), hbm, traffic, tflops)
+    # the dominant kernel's own timing (the chained step runs the same kernels)
+    roof = roofline_of(w, path_parts(r["per_kernel_ms"], "separate"), hbm, traffic, tflops)
     roof["peak_kind"] = f"{peak_kind} HBM copy bandwidth"
     e2e = e2e_ours(args, w, r["step"], device)
     del r["step"]
@@ -798,7 +801,7 @@ def main():
             try:
                 s = time_ours(args, sw, device, False, 0, 1, secondary=True, rope=rope)
                 del s["step"]
-                rf = roofline_of(sw, path_parts(s["per_kernel_ms"], s["path"]), hbm,
+                rf = roofline_of(sw, path_parts(s["per_kernel_ms"], "separate"), hbm,
                                  load_traffic(args.traffic_json, label), tflops)
                 line = {"workload": name, "queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1),
                         "ms_per_step": round(s["ms"], 4), "path": s["path"], "paths_ms": s["paths_ms"],

@@ -16,6 +16,8 @@ CSA_DTYPE_F32 = 0
 CSA_DTYPE_BF16 = 1
 CSA_DTYPE_E4M3 = 2
 CSA_MAX_TOPK = 2048
+CSA_STEP_CHAINED = 0
+CSA_STEP_PERSISTENT = 1
 
 # Every function the header declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -68,6 +70,7 @@ class DecodeStepArgs(ctypes.Structure):
         ("app_win", _I), ("app_stride", _I), ("app_T", _I), ("rope_dims", _I),
         ("app_kv_seq_stride", _LL), ("app_gate_seq_stride", _LL), ("app_row0", _LL),
         ("rope_theta", ctypes.c_double),
+        ("variant", _I),
     ]
 
 

@@ -214,6 +214,34 @@ int csa::check_index_topk(const void *qi, const float *wi, const void *ki, const
   return CSA_OK;
 }
 
+// The launches of csa_index_topk / csa_index_topk_fp8 once their arguments
+// are checked: the scores into the workspace after the status page, then the
+// top-k with the rest of it as scratch. (Also the decode step's chain.)
+int csa::index_topk_launch(ScoreArgs sa, int k, int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  sa.scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kStatusBytes);
+  sa.status = status_of(ws);
+  cudaError_t e = launch_index_scores(sa, stream);
+  if (e != cudaSuccess) return cuda_rc(e);
+  TopkArgs ta{sa.scores, sa.n_cmp, out_idx, sa.Q, sa.N_max, k, status_of(ws)};
+  const size_t sbytes = align256((size_t)sa.Q * sa.N_max * sizeof(float));
+  return cuda_rc(launch_topk(ta, stream, static_cast<char *>(ws) + kStatusBytes + sbytes, ws_bytes - kStatusBytes - sbytes));
+}
+
+extern "C" {
+static int check_scores_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                            const int32_t *n_cmp, int Q, int B, int Hi, int Di, int N_max, int q_per_seq);
+}
+
+int csa::check_index_topk_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                              const int32_t *n_cmp, int k, const int32_t *out_idx, int Q, int B, int Hi, int Di,
+                              int N_max, int q_per_seq) {
+  int rc = check_scores_fp8(qi8, sq, wi, ki8, sk, n_cmp, Q, B, Hi, Di, N_max, q_per_seq);
+  if (rc) return rc;
+  if (!out_idx || (reinterpret_cast<uintptr_t>(out_idx) & 3) || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  return CSA_OK;
+}
+
 extern "C" {
 
 int csa_index_topk(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int k, int32_t *out_idx,
@@ -224,14 +252,8 @@ int csa_index_topk(const void *qi, const float *wi, const void *ki, const int32_
   if (!out_idx || (reinterpret_cast<uintptr_t>(out_idx) & 3) || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
   if (!ws || !ws_aligned(ws) || ws_bytes < csa_index_topk_workspace_bytes(Q, N_max, k)) return CSA_ERR_WORKSPACE;
   if (!device_ok()) return CSA_ERR_UNSUPPORTED;
-  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kStatusBytes);
-  ScoreArgs sa{qi, wi, ki, n_cmp, scores, Q, B, Hi, Di, N_max, q_per_seq, dtype, status_of(ws)};
-  cudaError_t e = launch_index_scores(sa, (cudaStream_t)stream);
-  if (e != cudaSuccess) return CSA_ERR_CUDA;
-  TopkArgs ta{scores, n_cmp, out_idx, Q, N_max, k, status_of(ws)};
-  const size_t sbytes = align256((size_t)Q * N_max * sizeof(float));
-  return cuda_rc(launch_topk(ta, (cudaStream_t)stream, static_cast<char *>(ws) + kStatusBytes + sbytes,
-                             ws_bytes - kStatusBytes - sbytes));
+  ScoreArgs sa{qi, wi, ki, n_cmp, nullptr, Q, B, Hi, Di, N_max, q_per_seq, dtype, status_of(ws)};
+  return index_topk_launch(sa, k, out_idx, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 static int check_scores_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
@@ -266,14 +288,8 @@ int csa_index_topk_fp8(const uint8_t *qi8, const float *sq, const float *wi, con
   if (!out_idx || (reinterpret_cast<uintptr_t>(out_idx) & 3) || k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID;
   if (!ws || !ws_aligned(ws) || ws_bytes < csa_index_topk_workspace_bytes(Q, N_max, k)) return CSA_ERR_WORKSPACE;
   if (!device_ok()) return CSA_ERR_UNSUPPORTED;
-  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kStatusBytes);
-  ScoreArgs sa{qi8, wi, ki8, n_cmp, scores, Q, B, Hi, Di, N_max, q_per_seq, CSA_DTYPE_E4M3, status_of(ws), sq, sk};
-  cudaError_t e = launch_index_scores(sa, (cudaStream_t)stream);
-  if (e != cudaSuccess) return CSA_ERR_CUDA;
-  TopkArgs ta{scores, n_cmp, out_idx, Q, N_max, k, status_of(ws)};
-  const size_t sbytes = align256((size_t)Q * N_max * sizeof(float));
-  return cuda_rc(launch_topk(ta, (cudaStream_t)stream, static_cast<char *>(ws) + kStatusBytes + sbytes,
-                             ws_bytes - kStatusBytes - sbytes));
+  ScoreArgs sa{qi8, wi, ki8, n_cmp, nullptr, Q, B, Hi, Di, N_max, q_per_seq, CSA_DTYPE_E4M3, status_of(ws), sq, sk};
+  return index_topk_launch(sa, k, out_idx, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 size_t csa_mqa_workspace_bytes(int Q, int H, int D, int rows_max) {

@@ -1897,12 +1897,13 @@ extern "C" {
 size_t csa_decode_step_workspace_bytes(const csa_decode_step_args *s) {
   if (!s || !nonneg_sizes(*s)) return 256;
   StepPlan p;
-  if (make_plan(*s, &p)) return layout_of(*s, p).total;
+  if (s->variant == CSA_STEP_PERSISTENT && make_plan(*s, &p)) return layout_of(*s, p).total;
   return fallback_bytes(*s);
 }
 
 int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, csa_stream_t stream) {
   if (!s || !nonneg_sizes(*s)) return CSA_ERR_INVALID;
+  if (s->variant != CSA_STEP_CHAINED && s->variant != CSA_STEP_PERSISTENT) return CSA_ERR_INVALID;
   if (!s->q || !s->kv_cmp || !s->kv_win || !s->win_end || !s->sink || !s->out || !s->n_cmp) return CSA_ERR_INVALID;
   const bool csa = s->qi != nullptr;
   if (csa && (!s->wi || !s->ki || !s->idx_out || s->k < 1 || s->k > CSA_MAX_TOPK ||
@@ -1919,7 +1920,7 @@ int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, cs
     return CSA_ERR_WORKSPACE;
   StepPlan p;
   cudaStream_t st = (cudaStream_t)stream;
-  if (make_plan(*s, &p)) {
+  if (s->variant == CSA_STEP_PERSISTENT && make_plan(*s, &p)) {
     const Layout L = layout_of(*s, p);
     cudaError_t e = p.fp8 ? launch_fused<true>(*s, p, L, static_cast<char *>(ws), st)
                           : launch_fused<false>(*s, p, L, static_cast<char *>(ws), st);
@@ -1930,7 +1931,8 @@ int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, cs
     }
     cudaGetLastError();  // a tensor map the encoder rejected: the separate kernels serve the call
   }
-  // The separate kernels, one after another on the stream.
+  // The chained kernels, one after another on the stream (each launch a
+  // programmatic dependent of the one before).
   int rc = CSA_OK;
   if (s->app_kv) {
     void *out = static_cast<char *>(const_cast<void *>(s->kv_cmp)) + (size_t)s->app_row0 * s->D * (s->dtype == CSA_DTYPE_F32 ? 4 : 2);
@@ -1945,12 +1947,20 @@ int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, cs
     if (rc) return rc;
   }
   if (csa) {
-    rc = s->index_dtype == CSA_DTYPE_E4M3
-             ? csa_index_topk_fp8(static_cast<const uint8_t *>(s->qi), s->sq, s->wi,
-                                  static_cast<const uint8_t *>(s->ki), s->sk, s->n_cmp, s->k, s->idx_out, s->Q, s->B,
-                                  s->Hi, s->Di, s->N_max, s->q_per_seq, ws, ws_bytes, stream)
-             : csa_index_topk(s->qi, s->wi, s->ki, s->n_cmp, s->k, s->idx_out, s->Q, s->B, s->Hi, s->Di, s->N_max,
-                              s->q_per_seq, s->index_dtype, ws, ws_bytes, stream);
+    const bool fp8 = s->index_dtype == CSA_DTYPE_E4M3;
+    rc = fp8 ? check_index_topk_fp8(static_cast<const uint8_t *>(s->qi), s->sq, s->wi,
+                                    static_cast<const uint8_t *>(s->ki), s->sk, s->n_cmp, s->k, s->idx_out, s->Q,
+                                    s->B, s->Hi, s->Di, s->N_max, s->q_per_seq)
+             : check_index_topk(s->qi, s->wi, s->ki, s->n_cmp, s->k, s->idx_out, s->Q, s->B, s->Hi, s->Di,
+                                s->N_max, s->q_per_seq, s->index_dtype);
+    if (rc) return rc;
+    if (ws_bytes < csa_index_topk_workspace_bytes(s->Q, s->N_max, s->k)) return CSA_ERR_WORKSPACE;
+    ScoreArgs sa{s->qi, s->wi, s->ki, s->n_cmp, nullptr, s->Q, s->B, s->Hi, s->Di, s->N_max, s->q_per_seq,
+                 s->index_dtype, nullptr, fp8 ? s->sq : nullptr, fp8 ? s->sk : nullptr};
+    // After the append (which writes only kv_cmp rows) the scorer starts at
+    // once and waits for the append only before it exits.
+    sa.late_wait = s->app_kv ? 1 : 0;
+    rc = index_topk_launch(sa, s->k, s->idx_out, ws, ws_bytes, st);
     if (rc) return rc;
     return csa_sparse_mqa(s->q, s->kv_cmp, s->idx_out, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H, s->D,
                           s->N_max, s->k, s->win_len, s->win_end, s->T_raw, s->q_per_seq, s->dtype, ws, ws_bytes,

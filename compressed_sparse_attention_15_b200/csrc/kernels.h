@@ -87,6 +87,12 @@ struct ScoreArgs {
   uint32_t *status;
   const float *sq = nullptr;  // CSA_DTYPE_E4M3: per (query, head) scale [Q, Hi]
   const float *sk = nullptr;  // CSA_DTYPE_E4M3: per entry scale [B, N_max]
+  // 1: the kernel before this one in the stream writes none of the inputs
+  // (the decode step's cache append), so the tensor-core kernel starts at
+  // once and waits for it only before exiting (the completion order, and
+  // with it the visibility of the append to the kernels after this one, is
+  // kept); 0: wait before reading anything.
+  int late_wait = 0;
 };
 cudaError_t launch_index_scores(const ScoreArgs &a, cudaStream_t stream);
 
@@ -106,6 +112,11 @@ size_t topk_scratch_bytes(int Q, int N_max, int k);
 // (CSA_OK or the code csa_index_topk would return).
 int check_index_topk(const void *qi, const float *wi, const void *ki, const int32_t *n_cmp, int k,
                      const int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max, int q_per_seq, int dtype);
+int check_index_topk_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
+                         const int32_t *n_cmp, int k, const int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max,
+                         int q_per_seq);
+// Scores, then top-k, on `stream` (sa.scores and sa.status are set from ws).
+int index_topk_launch(ScoreArgs sa, int k, int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream);
 
 // ---------------------------------------------------------------- per-device setup
 // Kernel attributes are set, and device facts cached, once per device (a

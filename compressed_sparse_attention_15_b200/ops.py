@@ -382,10 +382,12 @@ def hca_mqa(q, kv_cmp, n_cmp, kv_win, win_end, sink, scale: float, win_len: int,
 
 def decode_step(q, kv_cmp, kv_win, win_end, sink, scale: float, win_len: int, n_cmp, *, qi=None, wi=None, ki=None,
                 k: int | None = None, qi8=None, sq=None, ki8=None, sk=None, append=None, out=None, idx_out=None,
-                q_per_seq=None, ws: Workspace | None = None):
+                q_per_seq=None, ws: Workspace | None = None, persistent: bool = False):
     """One decode step in one call (csa_decode_step): the cache append, then
     for CSA (qi or qi8 given) the indexer top-k and the sparse attention, for
-    HCA the dense attention over the n_cmp visible entries.
+    HCA the dense attention over the n_cmp visible entries. persistent=True
+    asks for the one-persistent-kernel variant (CSA_STEP_PERSISTENT), else the
+    chained kernels (CSA_STEP_CHAINED).
 
     append = None or a dict with kv, gate ([B, T, D], rows contiguous, any
     sequence stride), ape, norm_w, win, stride, row0 (first cache row written)
@@ -404,6 +406,7 @@ def decode_step(q, kv_cmp, kv_win, win_end, sink, scale: float, win_len: int, n_
     a.scale = float(scale)
     a.Q, a.B, a.H, a.D, a.N_max, a.win_len, a.T_raw, a.q_per_seq = Q, B, H, D, N_max, int(win_len), T_raw, qps
     a.dtype = _dtype_code(q)
+    a.variant = _lib.CSA_STEP_PERSISTENT if persistent else _lib.CSA_STEP_CHAINED
     fp8 = qi8 is not None
     if qi is not None or fp8:
         if k is None:

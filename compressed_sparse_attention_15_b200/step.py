@@ -10,14 +10,17 @@ The step over device-resident caches is:
      (csa_index_topk, or csa_index_topk_fp8 with FP8 indexer inputs);
   3. attend over the selected (CSA) or all visible (HCA) entries + the
      sliding window + the per-head sink (csa_sparse_mqa / hca_mqa).
-With fused=True the whole step is one csa_decode_step call: one persistent
-kernel in which the selection and attention of some queries overlap the
-indexer key scan of others (the separate kernels serve shapes it does not
-take). With fused=False (the default; measured faster on the benchmark
-workloads) the parts are separate calls; there, fuse_select=True makes a CSA
-step only score in 2 (csa_index_scores(_fp8)) and run 3 as
-csa_topk_sparse_mqa, the selection inside the attention kernel where its
-launch plan allows.
+With fused=True the whole step is one csa_decode_step call: by default the
+same kernels chained by programmatic dependent launch on one stream, the
+indexer's scorer starting without waiting for the append (the append writes
+none of its inputs), so the append overlaps the key scan with no second
+stream; persistent=True asks instead for the one persistent kernel in which
+the selection and attention of some queries overlap the key scan of others
+(measured slower: its per-query chains are latency-bound). With fused=False
+(the default) the parts are separate calls, the append on a forked stream;
+there, fuse_select=True makes a CSA step only score in 2
+(csa_index_scores(_fp8)) and run 3 as csa_topk_sparse_mqa, the selection
+inside the attention kernel where its launch plan allows.
 The library never allocates or synchronises, so the launches are captured
 once into a CUDA graph and each step is one graph launch. Buffers are bound
 at construction; later steps see whatever the caller wrote into them.
@@ -34,7 +37,7 @@ class DecodeStep:
                  ape, norm_w, gate, append_src0: int, append_dst0: int, win: int, stride: int,
                  qi=None, wi=None, ki=None, k: int | None = None, out=None, graph: bool = True,
                  qi8=None, sq=None, ki8=None, sk=None, append_rope=None, fuse_select: bool = False,
-                 fused: bool = False):
+                 fused: bool = False, persistent: bool = False):
         self.fp8 = qi8 is not None
         self.csa = qi is not None or self.fp8
         self.q, self.kv_cmp, self.kv_win, self.sink = q, kv_cmp, kv_win, sink
@@ -52,6 +55,7 @@ class DecodeStep:
         self.out = out if out is not None else torch.empty_like(q)
         self.idx = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev) if self.csa else None
         self.fused = bool(fused)
+        self.persistent = bool(persistent)
         self.fuse_select = bool(fuse_select) and self.csa and not self.fused
         self.append_src0, self.append_dst0 = int(append_src0), int(append_dst0)
         self.scores = (torch.empty((q.shape[0], kv_cmp.shape[1]), dtype=torch.float32, device=dev)
@@ -104,14 +108,15 @@ class DecodeStep:
         if self.fp8:
             ops.decode_step(self.q, self.kv_cmp, self.kv_win, self.win_end, self.sink, self.scale, self.win_len,
                             self.n_cmp, qi8=self.qi8, sq=self.sq, wi=self.wi, ki8=self.ki8, sk=self.sk, k=self.k,
-                            append=append, out=self.out, idx_out=self.idx, ws=self.ws_index)
+                            append=append, out=self.out, idx_out=self.idx, ws=self.ws_index,
+                            persistent=self.persistent)
         elif self.csa:
             ops.decode_step(self.q, self.kv_cmp, self.kv_win, self.win_end, self.sink, self.scale, self.win_len,
                             self.n_cmp, qi=self.qi, wi=self.wi, ki=self.ki, k=self.k, append=append, out=self.out,
-                            idx_out=self.idx, ws=self.ws_index)
+                            idx_out=self.idx, ws=self.ws_index, persistent=self.persistent)
         else:
             ops.decode_step(self.q, self.kv_cmp, self.kv_win, self.win_end, self.sink, self.scale, self.win_len,
-                            self.n_cmp, append=append, out=self.out, ws=self.ws_index)
+                            self.n_cmp, append=append, out=self.out, ws=self.ws_index, persistent=self.persistent)
 
     def parts(self):
         if self.fused:

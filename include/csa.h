@@ -388,19 +388,25 @@ int csa_index_topk_noalloc(const void *qi, const float *wi, const void *ki, cons
  *      HCA (qi == NULL): hca_mqa over the entries j < n_cmp[q].
  * Every argument keeps the meaning, layout and limits it has in those calls.
  *
- * For bf16 attention with H = 64 or 128, D = 512, one query per sequence
- * (q_per_seq = 1) and the indexer shape 64 x 128, the step is ONE persistent
- * kernel: each SM pulls tasks (append, key-tile chunks, top-k, attention
- * splits, split merges) from device-side queues as their inputs complete,
- * so the selection and attention of some queries overlap the key scan of
- * others. Other shapes run the separate kernels. Split plans differ from the
- * separate calls', so outputs agree with them to rounding, not bit for bit.
+ * variant = CSA_STEP_CHAINED (0): the kernels of those calls, launched as
+ * one chain of programmatic dependent launches on `stream` with no host
+ * synchronisation; the indexer's tensor-core scorer does not wait for the
+ * append before it starts (it reads none of the rows the append writes: qi,
+ * wi, ki and n_cmp must not overlap kv_cmp), so the two overlap. Outputs are
+ * those of the separate calls, bit for bit.
+ * variant = CSA_STEP_PERSISTENT (1), for bf16 attention with H = 64 or 128,
+ * D = 512, one query per sequence (q_per_seq = 1) and the indexer shape
+ * 64 x 128: ONE persistent kernel in which each SM pulls tasks (append,
+ * key-tile chunks, top-k, attention splits, split merges) from device-side
+ * queues as their inputs complete. Its split plans differ from the separate
+ * calls', so its outputs agree with them to rounding, not bit for bit; other
+ * shapes take the chained kernels.
  *
  * Workspace: csa_decode_step_workspace_bytes(args) bytes, 256-byte aligned,
  * zero-filled before the first call (cudaMemset once); the step leaves its
  * counters at zero for the next call. Bytes 0..3 hold the status word (as for
- * every call); bytes 8..15 may hold a limit in nanoseconds for every bounded
- * wait of the fused kernel (0 = 2 s; for tests of the timeout path).
+ * every call); bytes 8..15 may hold a limit in nanoseconds for the bounded
+ * waits (0 = 2 s; for tests of the timeout path).
  * Calls sharing one workspace must not overlap on the GPU.
  * Returns CSA_ERR_INVALID / CSA_ERR_WORKSPACE before any launch.
  * ---------------------------------------------------------------------- */
@@ -432,7 +438,10 @@ typedef struct csa_decode_step_args {
   int app_win, app_stride, app_T, rope_dims;
   long long app_kv_seq_stride, app_gate_seq_stride, app_row0;
   double rope_theta;
+  int variant;             /* CSA_STEP_CHAINED or CSA_STEP_PERSISTENT */
 } csa_decode_step_args;
+
+enum { CSA_STEP_CHAINED = 0, CSA_STEP_PERSISTENT = 1 };
 
 size_t csa_decode_step_workspace_bytes(const csa_decode_step_args *args);
 int csa_decode_step(const csa_decode_step_args *args, void *ws, size_t ws_bytes, csa_stream_t stream);

@@ -1,7 +1,8 @@
-"""The whole decode step in one call (csa_decode_step, the persistent fused
-kernel): the cache append, the indexer top-k and the sparse attention (CSA),
-or the append and the dense attention (HCA), against the fp64 oracle's chain
-on the same seeded inputs, and against the separate kernels."""
+"""The whole decode step in one call (csa_decode_step, both variants: the
+chained kernels and the one persistent kernel): the cache append, the indexer
+top-k and the sparse attention (CSA), or the append and the dense attention
+(HCA), against the fp64 oracle's chain on the same seeded inputs, and against
+the separate kernels."""
 import numpy as np
 import pytest
 import torch
@@ -43,7 +44,7 @@ def appended_rows(raw, gate, ape, win, stride, rope=None):
 
 # ---------------------------------------------------------------- full size
 
-def _decode_step(w, dev, fused=True):
+def _decode_step(w, dev, fused=True, persistent=False):
     fp8 = w.index_fmt == "e4m3"
     names = ["q", "kv_cmp", "kv_win", "sink", "gate", "ape"]
     if w.mode == "csa":
@@ -54,7 +55,7 @@ def _decode_step(w, dev, fused=True):
                     ape=d["ape"], norm_w=WL.norm_w(w, dev), gate=d["gate"], append_src0=w.c_src0,
                     append_dst0=w.c_dst0, win=w.win, stride=w.stride, qi=d.get("qi"), wi=d.get("wi"),
                     ki=d.get("ki"), qi8=d.get("qi8"), sq=d.get("sq"), ki8=d.get("ki8"), sk=d.get("sk"),
-                    k=w.k if w.mode == "csa" else None, fused=fused)
+                    k=w.k if w.mode == "csa" else None, fused=fused, persistent=persistent)
     return ds, d
 
 
@@ -105,13 +106,14 @@ FULL = {
 }
 
 
+@pytest.mark.parametrize("persistent", [False, True])
 @pytest.mark.parametrize("name", sorted(FULL))
-def test_full_size_step_matches_oracle(cuda_device, name):
+def test_full_size_step_matches_oracle(cuda_device, name, persistent):
     # The benchmark's workloads in its launch configuration (the step replayed
     # from its CUDA graph, twice: the second replay starts from the counters
     # the first left), sampled queries against the oracle chain.
     w = WL.WORKLOADS[name]
-    ds, _ = _decode_step(w, cuda_device)
+    ds, _ = _decode_step(w, cuda_device, persistent=persistent)
     ds.run()
     first = ds.out.clone()
     ds.run()
@@ -122,18 +124,25 @@ def test_full_size_step_matches_oracle(cuda_device, name):
     assert _check_full(w, ds, queries) >= len(queries) - 1
 
 
+@pytest.mark.parametrize("persistent", [False, True])
 @pytest.mark.parametrize("name", ["csa_decode_64k", "hca_decode_1m", "csa_decode_64k_fp8"])
-def test_fused_step_matches_separate_kernels(cuda_device, name):
-    # The same step through the separate kernels: the selections are the same
-    # sets (the scores are computed by the same products in the same order),
-    # the outputs agree within the bf16 tolerance.
+def test_step_call_matches_separate_kernels(cuda_device, name, persistent):
+    # The same step through the separate kernels. The chained variant runs
+    # those kernels: the same selection and bit-identical outputs. The
+    # persistent kernel: the same selection sets (the scores are the same
+    # products in the same order), outputs within the bf16 tolerance.
     w = WL.WORKLOADS[name]
-    ds_f, d = _decode_step(w, cuda_device, fused=True)
+    ds_f, d = _decode_step(w, cuda_device, fused=True, persistent=persistent)
     out_f = ds_f.run().clone()
     idx_f = ds_f.idx.clone() if ds_f.idx is not None else None
     ds_s, _ = _decode_step(w, cuda_device, fused=False)
     out_s = ds_s.run()
     torch.cuda.synchronize()
+    if not persistent:
+        assert torch.equal(out_f, out_s)
+        if idx_f is not None:
+            assert torch.equal(idx_f, ds_s.idx)
+        return
     if idx_f is not None:
         assert torch.equal(torch.sort(idx_f, dim=1).values, torch.sort(ds_s.idx, dim=1).values)
     err = (out_f.float() - out_s.float()).abs()
@@ -143,8 +152,8 @@ def test_fused_step_matches_separate_kernels(cuda_device, name):
 # ---------------------------------------------------------------- small cases
 
 def _small_case(dev, *, Q, N, k, H=64, W=128, n=None, ends=None, T_raw=160, fp8=False, hca=False, seed=3,
-                append=True, rope=None, check=None):
-    """One fused step on seeded synthetic inputs; every (or check[]) query's
+                append=True, rope=None, check=None, persistent=False):
+    """One step call on seeded synthetic inputs; every (or check[]) query's
     output and selection against the oracle."""
     B, D, Hi, Di = Q, 512, 64, 128
     g = lambda tid, shape, **kw: synth.normal(seed, tid, shape, **kw)
@@ -161,7 +170,7 @@ def _small_case(dev, *, Q, N, k, H=64, W=128, n=None, ends=None, T_raw=160, fp8=
     nw = torch.ones(D)
     row0 = max(0, N - 1)
     src0 = T_raw - T_c
-    kw = {}
+    kw = {"persistent": persistent}
     if not hca:
         if fp8:
             qi8 = WL._codes(g(13, (Q, Hi, Di)))
@@ -169,12 +178,12 @@ def _small_case(dev, *, Q, N, k, H=64, W=128, n=None, ends=None, T_raw=160, fp8=
             sq = synth.uniform(seed, 14, (Q, Hi)) / 64 + 1.0 / 256
             sk = synth.uniform(seed, 16, (B, N)) / 64 + 1.0 / 256
             wi = synth.uniform(seed, 5, (Q, Hi))
-            kw = dict(qi8=qi8.to(dev), sq=sq.to(dev), wi=wi.to(dev), ki8=ki8.to(dev), sk=sk.to(dev), k=k)
+            kw.update(qi8=qi8.to(dev), sq=sq.to(dev), wi=wi.to(dev), ki8=ki8.to(dev), sk=sk.to(dev), k=k)
         else:
             qi = g(4, (Q, Hi, Di), dtype=torch.bfloat16)
             wi = synth.uniform(seed, 5, (Q, Hi))
             ki = g(6, (B, N, Di), dtype=torch.bfloat16)
-            kw = dict(qi=qi.to(dev), wi=wi.to(dev), ki=ki.to(dev), k=k)
+            kw.update(qi=qi.to(dev), wi=wi.to(dev), ki=ki.to(dev), k=k)
     kv_cmp_d, kv_win_d = kv_cmp.to(dev), kv_win.to(dev)
     app = None
     pos0 = None
@@ -226,56 +235,66 @@ def _small_case(dev, *, Q, N, k, H=64, W=128, n=None, ends=None, T_raw=160, fp8=
     return compared
 
 
-def test_ragged_counts_and_short_lists(cuda_device):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_ragged_counts_and_short_lists(cuda_device, persistent):
     # 3001 entries (a ragged last key tile); n above, at and below k, one and
     # zero visible entries (the attention then reads the window and the sink)
     n = [3001, 513, 512, 1, 0, 2000]
-    assert _small_case(cuda_device, Q=6, N=3001, k=512, n=n) >= 5
+    assert _small_case(cuda_device, persistent=persistent, Q=6, N=3001, k=512, n=n) >= 5
 
 
-def test_short_windows(cuda_device):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_short_windows(cuda_device, persistent):
     # windows of 1, 5, 64, 65 and 128 rows (queries near the start of their
     # raw buffer), the window split then partly or mostly masked
     ends = [0, 4, 63, 64, 159]
-    assert _small_case(cuda_device, Q=5, N=2500, k=256, ends=ends, W=128) >= 4
+    assert _small_case(cuda_device, persistent=persistent, Q=5, N=2500, k=256, ends=ends, W=128) >= 4
 
 
-def test_window_of_64(cuda_device):
-    assert _small_case(cuda_device, Q=4, N=1800, k=128, W=64, ends=[30, 63, 100, 159]) >= 3
+@pytest.mark.parametrize("persistent", [False, True])
+def test_window_of_64(cuda_device, persistent):
+    assert _small_case(cuda_device, persistent=persistent, Q=4, N=1800, k=128, W=64, ends=[30, 63, 100, 159]) >= 3
 
 
-def test_pro_heads_and_top_1024(cuda_device):
-    assert _small_case(cuda_device, Q=3, N=4000, k=1024, H=128) >= 2
+@pytest.mark.parametrize("persistent", [False, True])
+def test_pro_heads_and_top_1024(cuda_device, persistent):
+    assert _small_case(cuda_device, persistent=persistent, Q=3, N=4000, k=1024, H=128) >= 2
 
 
-def test_fp8_indexer(cuda_device):
-    assert _small_case(cuda_device, Q=5, N=3001, k=512, fp8=True, n=[3001, 600, 512, 9, 2999]) >= 4
+@pytest.mark.parametrize("persistent", [False, True])
+def test_fp8_indexer(cuda_device, persistent):
+    assert _small_case(cuda_device, persistent=persistent, Q=5, N=3001, k=512, fp8=True, n=[3001, 600, 512, 9, 2999]) >= 4
 
 
-def test_hca_dense_ragged(cuda_device):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_hca_dense_ragged(cuda_device, persistent):
     # dense lists of 700 entries (not a multiple of the 64-row tile), counts
     # down to zero; the appended entry is the last row
-    assert _small_case(cuda_device, Q=6, N=700, k=0, hca=True, n=[700, 699, 65, 64, 1, 0]) == 6
+    assert _small_case(cuda_device, persistent=persistent, Q=6, N=700, k=0, hca=True, n=[700, 699, 65, 64, 1, 0]) == 6
 
 
-def test_hca_without_append(cuda_device):
-    assert _small_case(cuda_device, Q=4, N=1500, k=0, hca=True, append=False) == 4
+@pytest.mark.parametrize("persistent", [False, True])
+def test_hca_without_append(cuda_device, persistent):
+    assert _small_case(cuda_device, persistent=persistent, Q=4, N=1500, k=0, hca=True, append=False) == 4
 
 
-def test_append_with_rope(cuda_device):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_append_with_rope(cuda_device, persistent):
     # the append rotates the new entry's last 64 dims (theta 160000)
-    assert _small_case(cuda_device, Q=4, N=2048, k=256, rope=(64, 160000.0), n=[2048] * 4) >= 3
+    assert _small_case(cuda_device, persistent=persistent, Q=4, N=2048, k=256, rope=(64, 160000.0), n=[2048] * 4) >= 3
 
 
-def test_many_queries(cuda_device):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_many_queries(cuda_device, persistent):
     # 200 queries: many tasks of every kind per CTA, the queues wrap many times
-    assert _small_case(cuda_device, Q=200, N=1500, k=64, check=range(0, 200, 23)) >= 8
+    assert _small_case(cuda_device, persistent=persistent, Q=200, N=1500, k=64, check=range(0, 200, 23)) >= 8
 
 
-def test_two_segment_selection(cuda_device):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_two_segment_selection(cuda_device, persistent):
     # lists longer than one block's key cache take the two-stage selection
     # (per-segment winners, then the winners' top-k)
-    assert _small_case(cuda_device, Q=2, N=60000, k=512, append=False) >= 1
+    assert _small_case(cuda_device, persistent=persistent, Q=2, N=60000, k=512, append=False) >= 1
 
 
 def test_rejects_bad_arguments(cuda_device):
