@@ -316,14 +316,8 @@ int csa_sparse_mqa(const void *q, const void *kv_cmp, const int32_t *idx, const 
                    float scale, void *out, int Q, int B, int H, int D, int N_max, int k, int win_len,
                    const int32_t *win_end, int T_raw, int q_per_seq, int dtype, void *ws, size_t ws_bytes,
                    csa_stream_t stream) {
-  int rc = check_mqa(q, kv_cmp, kv_win, sink, out, Q, B, H, D, N_max, win_len, win_end, T_raw, q_per_seq, dtype);
-  if (rc) return rc;
-  if (!idx || (reinterpret_cast<uintptr_t>(idx) & 3) || k < 1 || (long long)k + win_len > 65536) return CSA_ERR_INVALID;
-  if (!ws || !ws_aligned(ws) || ws_bytes < csa_mqa_workspace_bytes(Q, H, D, k + win_len)) return CSA_ERR_WORKSPACE;
-  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
-  MqaArgs a{q, kv_cmp, kv_win, idx, nullptr, win_end, sink, scale, out, Q, B, H, D, N_max, k, win_len, T_raw,
-            q_per_seq, dtype, static_cast<char *>(ws) + kStatusBytes, ws_bytes - kStatusBytes, status_of(ws)};
-  return cuda_rc(launch_mqa(a, (cudaStream_t)stream));
+  return attend_call(q, kv_cmp, idx, nullptr, kv_win, sink, scale, out, Q, B, H, D, N_max, k, win_len, win_end,
+                     T_raw, q_per_seq, dtype, false, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 size_t csa_topk_sparse_mqa_workspace_bytes(int Q, int H, int D, int N_max, int k, int win_len) {
@@ -366,14 +360,8 @@ int csa_topk_sparse_mqa(const float *scores, const int32_t *n_cmp, int k, int32_
 int hca_mqa(const void *q, const void *kv_cmp, const void *kv_win, const float *sink, float scale, void *out, int Q,
             int B, int H, int D, int N_max, const int32_t *n_cmp, int win_len, const int32_t *win_end, int T_raw,
             int q_per_seq, int dtype, void *ws, size_t ws_bytes, csa_stream_t stream) {
-  int rc = check_mqa(q, kv_cmp, kv_win, sink, out, Q, B, H, D, N_max, win_len, win_end, T_raw, q_per_seq, dtype);
-  if (rc) return rc;
-  if (!n_cmp || (reinterpret_cast<uintptr_t>(n_cmp) & 3)) return CSA_ERR_INVALID;
-  if (!ws || !ws_aligned(ws) || ws_bytes < csa_mqa_workspace_bytes(Q, H, D, N_max + win_len)) return CSA_ERR_WORKSPACE;
-  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
-  MqaArgs a{q, kv_cmp, kv_win, nullptr, n_cmp, win_end, sink, scale, out, Q, B, H, D, N_max, 0, win_len, T_raw,
-            q_per_seq, dtype, static_cast<char *>(ws) + kStatusBytes, ws_bytes - kStatusBytes, status_of(ws)};
-  return cuda_rc(launch_mqa(a, (cudaStream_t)stream));
+  return attend_call(q, kv_cmp, nullptr, n_cmp, kv_win, sink, scale, out, Q, B, H, D, N_max, 0, win_len, win_end,
+                     T_raw, q_per_seq, dtype, false, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 unsigned long long csa_launch_count(void) { return __atomic_load_n(&csa::g_launches, __ATOMIC_RELAXED); }
@@ -393,3 +381,27 @@ int csa_workspace_status(void *ws, csa_stream_t stream, uint32_t *status) {
 }
 
 }  // extern "C"
+
+// The checks and the launch of csa_sparse_mqa (idx given) / hca_mqa (n_cmp
+// given); early: see MqaArgs::early (the decode step's chain).
+int csa::attend_call(const void *q, const void *kv_cmp, const int32_t *idx, const int32_t *n_cmp, const void *kv_win,
+                     const float *sink, float scale, void *out, int Q, int B, int H, int D, int N_max, int k,
+                     int win_len, const int32_t *win_end, int T_raw, int q_per_seq, int dtype, bool early, void *ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_mqa(q, kv_cmp, kv_win, sink, out, Q, B, H, D, N_max, win_len, win_end, T_raw, q_per_seq, dtype);
+  if (rc) return rc;
+  if (idx) {
+    if ((reinterpret_cast<uintptr_t>(idx) & 3) || k < 1 || (long long)k + win_len > 65536) return CSA_ERR_INVALID;
+    if (!ws || !ws_aligned(ws) || ws_bytes < csa_mqa_workspace_bytes(Q, H, D, k + win_len)) return CSA_ERR_WORKSPACE;
+  } else {
+    if (!n_cmp || (reinterpret_cast<uintptr_t>(n_cmp) & 3)) return CSA_ERR_INVALID;
+    if (!ws || !ws_aligned(ws) || ws_bytes < csa_mqa_workspace_bytes(Q, H, D, N_max + win_len))
+      return CSA_ERR_WORKSPACE;
+    k = 0;
+  }
+  if (!device_ok()) return CSA_ERR_UNSUPPORTED;
+  MqaArgs a{q, kv_cmp, kv_win, idx, idx ? nullptr : n_cmp, win_end, sink, scale, out, Q, B, H, D, N_max, k, win_len,
+            T_raw, q_per_seq, dtype, static_cast<char *>(ws) + kStatusBytes, ws_bytes - kStatusBytes, status_of(ws)};
+  a.early = early ? 1 : 0;
+  return cuda_rc(launch_mqa(a, stream));
+}

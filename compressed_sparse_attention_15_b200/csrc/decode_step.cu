@@ -1962,12 +1962,17 @@ int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, cs
     sa.late_wait = s->app_kv ? 1 : 0;
     rc = index_topk_launch(sa, s->k, s->idx_out, ws, ws_bytes, st);
     if (rc) return rc;
-    return csa_sparse_mqa(s->q, s->kv_cmp, s->idx_out, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H, s->D,
-                          s->N_max, s->k, s->win_len, s->win_end, s->T_raw, s->q_per_seq, s->dtype, ws, ws_bytes,
-                          stream);
+    // The attention loads the queries and runs the window tiles before it
+    // waits for the top-k (which writes none of them).
+    return attend_call(s->q, s->kv_cmp, s->idx_out, nullptr, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H,
+                       s->D, s->N_max, s->k, s->win_len, s->win_end, s->T_raw, s->q_per_seq, s->dtype, true, ws,
+                       ws_bytes, st);
   }
-  return hca_mqa(s->q, s->kv_cmp, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H, s->D, s->N_max, s->n_cmp,
-                 s->win_len, s->win_end, s->T_raw, s->q_per_seq, s->dtype, ws, ws_bytes, stream);
+  // HCA: the window tiles before the wait for the append (which writes only
+  // kv_cmp rows); without an append, the caller's kernel may write anything.
+  return attend_call(s->q, s->kv_cmp, nullptr, s->n_cmp, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H, s->D,
+                     s->N_max, 0, s->win_len, s->win_end, s->T_raw, s->q_per_seq, s->dtype, s->app_kv != nullptr, ws,
+                     ws_bytes, st);
 }
 
 }  // extern "C"

@@ -171,8 +171,19 @@ struct MqaArgs {
   uint32_t *status;
   const float *scores;     // non-null: select the top-k of these indexer scores in the kernel (idx unused)
   int32_t *idx_out;        // ... and write the selection here
+  // 1: the kernel before this one in the stream writes none of q, kv_win,
+  // win_end, sink and n_cmp (the decode step's top-k, or its append for
+  // HCA): the tensor-core kernel loads the queries and runs the window tiles
+  // before waiting for it; 0: it waits before reading anything.
+  int early = 0;
 };
 cudaError_t launch_mqa(const MqaArgs &a, cudaStream_t stream);
+// csa_sparse_mqa (idx given) / hca_mqa (idx null, n_cmp given): checks, then
+// the launch; early sets MqaArgs::early.
+int attend_call(const void *q, const void *kv_cmp, const int32_t *idx, const int32_t *n_cmp, const void *kv_win,
+                const float *sink, float scale, void *out, int Q, int B, int H, int D, int N_max, int k, int win_len,
+                const int32_t *win_end, int T_raw, int q_per_seq, int dtype, bool early, void *ws, size_t ws_bytes,
+                cudaStream_t stream);
 // Top-k selection fused into the tensor-core MQA (a.scores set); *taken is
 // false when the shape or the launch plan does not allow it.
 cudaError_t launch_topk_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken);

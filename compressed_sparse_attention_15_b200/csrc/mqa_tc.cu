@@ -97,10 +97,13 @@ constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kQBytes + 2 * kPBytes + si
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per block");
 static_assert(2 * kPBytes == 2 * sel::kBins * 4, "the P buffers hold the two selection histograms");
 
-// Row list of one query: compressed rows [0, nsel) (padded with unused rows
-// up to nsel4, a multiple of 4), then the window rows [nsel4, R).
+// Row list of one query: the window rows [0, nwin) (kv_win rows wlo ..
+// wlo + nwin - 1, padded with unused rows to whole tiles: w64), then the
+// compressed rows [w64, w64 + nsel) in list order (selected entries, or the
+// visible entries of a dense list; nsel4 = nsel padded to a multiple of 4).
+// Window tiles are contiguous runs and need nothing the selection produces.
 struct RowList {
-  int nsel, nsel4, wlo, R;
+  int nsel, nsel4, wlo, nwin, w64, R;
 };
 
 __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *status) {
@@ -112,9 +115,27 @@ __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *
     e = e < 0 ? 0 : a.T_raw - 1;
   }
   L.wlo = max(0, e - a.win_len + 1);
+  L.nwin = e - L.wlo + 1;
+  L.w64 = (L.nwin + kRows - 1) / kRows * kRows;
   L.nsel4 = (L.nsel + 3) & ~3;
-  L.R = L.nsel4 + (e - L.wlo + 1);
+  L.R = L.w64 + L.nsel;
   return L;
+}
+
+// The tiles [t0, t1) of split `split`: runs of tiles_per_split tiles; with
+// early window tiles (the window computed before the kernel waits on its
+// predecessor) split 0 takes the window tiles on top of its run of
+// compressed tiles and the runs cover the compressed tiles only.
+__device__ __forceinline__ void split_tiles(const RowList &L, int split, int tiles_per_split, bool early, int &t0,
+                                            int &t1) {
+  const int tiles_all = (L.R + kRows - 1) / kRows, wt = L.w64 / kRows;
+  if (early) {
+    t0 = split == 0 ? 0 : wt + split * tiles_per_split;
+    t1 = min(tiles_all, wt + (split + 1) * tiles_per_split);
+  } else {
+    t0 = split * tiles_per_split;
+    t1 = min(tiles_all, t0 + tiles_per_split);
+  }
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
@@ -223,12 +244,13 @@ __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)
 
 // Top-k of query qq's indexer scores by the cluster of its splits, all
 // threads taking part (the selection csa_topk makes). List position r of the
-// selection lands in sel[r] of the split whose tiles hold it, and in idx_out
+// selection (row w64 + r of the row list) lands in sel[r] of the split whose
+// tiles hold it, and in idx_out
 // (written by head group 0); each selected row is prefetched into L2 as it is
 // found. The slice's keys use the tile buffers and the histograms the P
 // buffers, neither in use yet.
 __device__ void select_rows(const MqaArgs &a, Small *sm, uint8_t *kv, uint8_t *ps, int qq, int hg, int b,
-                            int tiles_per_split) {
+                            int tiles_per_split, int w64) {
   const uint32_t C = cluster_size(), c = cluster_rank();
   const int n = clamp_count(a.n_cmp[qq], a.N_max, (threadIdx.x == 0 && c == 0) ? a.status : nullptr);
   const int k = a.k;
@@ -249,7 +271,7 @@ __device__ void select_rows(const MqaArgs &a, Small *sm, uint8_t *kv, uint8_t *p
     const int rows_per_split = kRows * tiles_per_split;
     sel::cluster_select<kThreads, 8, kMaxSplits>(
         sm->cs, reinterpret_cast<uint32_t *>(ps), keys, len, j0, k, C, c, lo, hi, [&](uint32_t slot, int j) {
-          st_peer(&sm->sel[slot], slot / (uint32_t)rows_per_split, (uint32_t)j);
+          st_peer(&sm->sel[slot], (slot + (uint32_t)w64) / (uint32_t)rows_per_split, (uint32_t)j);
           if (out) out[slot] = j;
           bulk_prefetch_l2(rows + (size_t)j * kD, kD * 2);
         });
@@ -306,15 +328,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = sm->tmem_base;
   volatile int *abort = &sm->abort;
-  pdl_wait();  // inputs (indices, queries, caches) may come from the previous kernel
+  // early: the queries and the window tiles do not depend on the previous
+  // kernel; every role waits for it before its first compressed tile, and
+  // before any global write. Otherwise everything waits here.
+  const bool early = !kFused && a.early;
+  if (!early) pdl_wait();  // inputs (indices, queries, caches) may come from the previous kernel
   const uint64_t lim = tc::wait_limit_of(a.status);
   pdl_release();
 
   const RowList L = row_list(a, qq, threadIdx.x == 0 ? a.status : nullptr);
-  const int tiles_all = (L.R + kRows - 1) / kRows;
-  const int t0 = split * tiles_per_split;
-  const int t1 = min(tiles_all, t0 + tiles_per_split);
+  int t0, t1;
+  split_tiles(L, split, tiles_per_split, early, t0, t1);
   const int ntiles = max(0, t1 - t0);
+  const int wt = L.w64 / kRows;  // window tiles (list tiles [0, wt))
   constexpr bool fused = kFused;
   const bool sparse = fused || a.idx != nullptr;
   if (warp == kMmaWarp && lane == 0 && ntiles > 0) {
@@ -322,9 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
     for (int bx = 0; bx < kD / 64; ++bx) tc::tma_load_2d(qs + bx * kQBoxBytes, &tm_q, bx * 64, qv * kH, &sm->q_full);
   }
-  if constexpr (kFused) select_rows(a, sm, kv, ps, qq, hg, b, tiles_per_split);
-  // entry of the selection at list position r < nsel
-  auto sel_at = [&](int r) -> int { return fused ? sm->sel[r] : a.idx[(size_t)qq * a.k + r]; };
+  if constexpr (kFused) select_rows(a, sm, kv, ps, qq, hg, b, tiles_per_split, L.w64);
+  // entry of the selection at list position p < nsel
+  auto sel_at = [&](int p) -> int { return fused ? sm->sel[p] : a.idx[(size_t)qq * a.k + p]; };
 
   if (warp < kLoadWarps) {
     // ------------------------------------------------------------ loaders
@@ -338,29 +364,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     // its next kAhead tiles into L2 while the buffer is busy.
     const int g = warp / kWarpsPerBuf, part = warp % kWarpsPerBuf;
     const uint32_t buf_base = tc::smem_u32(kv) + g * kTileBytes;
+    bool waited = !early;
     if (warp == 0 && lane == 0) {
       tc::prefetch_tmap(&tm_cmp_t);
       tc::prefetch_tmap(&tm_win_t);
     }
-    // Source row of list position r (null: padding or an unused slot).
+    // Source row of row-list row r (null: padding or an unused slot).
     auto src_row = [&](int r) -> const bf16 * {
-      if (r < L.nsel) {
-        int j = sparse ? sel_at(r) : r;
+      if (r < L.w64)
+        return r < L.nwin ? static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + L.wlo + r) * kD : nullptr;
+      const int p = r - L.w64;
+      if (p < L.nsel) {
+        int j = sparse ? sel_at(p) : p;
         if (j < -1 || j >= a.N_max) {
           raise_status(a.status, CSA_STATUS_BAD_INDEX);
           j = -1;
         }
         return j >= 0 ? static_cast<const bf16 *>(a.kv_cmp) + ((size_t)b * a.N_max + j) * kD : nullptr;
       }
-      if (r >= L.nsel4 && r < L.R)
-        return static_cast<const bf16 *>(a.kv_win) + ((size_t)b * a.T_raw + L.wlo + (r - L.nsel4)) * kD;
       return nullptr;
     };
     // A tile is one contiguous run when it lies in the window part, or in the
     // compressed part of a dense (HCA) row list.
     auto is_run = [&](int r0, bool &win_run) {
-      win_run = r0 >= L.nsel4;
-      return win_run || (!sparse && r0 + kRows <= L.nsel4);
+      win_run = r0 < L.w64;
+      return win_run || (!sparse && r0 - L.w64 + kRows <= L.nsel4);
     };
     // Bring this warp's rows of tile li into L2 ahead of their load, which can
     // only start once the tile buffer is free: the load then waits on L2.
@@ -374,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (is_run(r0, win_run)) {
         if (lane == 0) {
           // first row of this warp's part, and how many rows of the sequence's buffer remain from it
-          const int first = win_run ? L.wlo + (r0 - L.nsel4) + kRowsPerWarp * part : r0 + kRowsPerWarp * part;
+          const int first = win_run ? L.wlo + r0 + kRowsPerWarp * part : r0 - L.w64 + kRowsPerWarp * part;
           const int avail = (win_run ? a.T_raw : a.N_max) - first;
           const int rows = avail < kRowsPerWarp ? avail : kRowsPerWarp;
           if (rows > 0) {
@@ -383,13 +411,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_prefetch_l2(base, (uint32_t)rows * kD * 2);
           }
         }
-      } else if (lane < kRowsPerWarp) {
+      } else if (lane < kRowsPerWarp && (!early || waited)) {  // (a gathered tile's rows need the selection)
         if (const bf16 *p = src_row(r0 + kRowsPerWarp * part + lane)) bulk_prefetch_l2(p, kD * 2);
       }
     };
     int last = -1;
     for (int li = g; li < ntiles; li += 2) {
       const int r0 = (t0 + li) * kRows;
+      if (t0 + li >= wt && !waited) {  // the first compressed tile: the previous kernel must be done
+        pdl_wait();
+        waited = true;
+      }
       bool win_run;
       const bool run = is_run(r0, win_run);
       __syncwarp();  // the previous tile's copies have read rowp[warp]
@@ -402,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (run) {
         if (part == 0 && lane == 0) {
           tc::mbar_arrive_expect_tx(&sm->kv_full[g], kTileBytes);
-          const int row = win_run ? b * a.T_raw + L.wlo + (r0 - L.nsel4) : b * a.N_max + r0;
+          const int row = win_run ? b * a.T_raw + L.wlo + r0 : b * a.N_max + (r0 - L.w64);
           for (int bx = 0; bx < 8; ++bx)
             tc::tma_load_2d(kv + g * kTileBytes + bx * kBoxBytes, win_run ? &tm_win_t : &tm_cmp_t, 64 * bx, row,
                             &sm->kv_full[g]);
@@ -518,24 +550,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l[16];  // running sums of heads 8c + 2cq + e at l[2c + e]
 #pragma unroll
     for (int i = 0; i < 16; ++i) l[i] = 0.f;
-    bool ok = true;
-    int idxA = 0, idxB = 0;
-    if (ntiles > 0 && sparse) {
-      const int r = t0 * kRows + rowA;
-      if (r < L.nsel) idxA = sel_at(r);
-      if (r + 8 < L.nsel) idxB = sel_at(r + 8);
-    }
+    bool ok = true, waited = !early;
+    // a row-list row holds a key: a window row below nwin, a compressed row
+    // with a valid entry
+    auto valid_row = [&](int r) -> bool {
+      if (r < L.w64) return r < L.nwin;
+      const int p = r - L.w64;
+      if (p >= L.nsel) return false;
+      if (!sparse) return true;
+      const int j = sel_at(p);
+      return j >= 0 && j < a.N_max;
+    };
     for (int li = 0; li < ntiles; ++li) {
       const int buf = li & 1;
+      if (!waited && t0 + li >= wt) {  // the first compressed tile: the previous kernel must be done
+        pdl_wait();
+        waited = true;
+      }
+      const int rA = (t0 + li) * kRows + rowA, rB = rA + 8;
+      const bool validA = valid_row(rA), validB = valid_row(rB);
       const bool got = __all_sync(0xffffffffu, tc::mbar_wait(&sm->s_full[buf], (li >> 1) & 1, abort, a.status, lim));
       tc::fence_after_sync();
-      const int rA = (t0 + li) * kRows + rowA, rB = rA + 8;
-      const bool validA = rA < L.nsel4 ? (rA < L.nsel && (!sparse || (idxA >= 0 && idxA < a.N_max))) : rA < L.R;
-      const bool validB = rB < L.nsel4 ? (rB < L.nsel && (!sparse || (idxB >= 0 && idxB < a.N_max))) : rB < L.R;
-      if (li + 1 < ntiles && sparse) {  // the next tile's indices, loaded while this tile is processed
-        idxA = rA + kRows < L.nsel ? sel_at(rA + kRows) : 0;
-        idxB = rB + kRows < L.nsel ? sel_at(rB + kRows) : 0;
-      }
       uint32_t v[32];
       tmem_ld_16x256b_x8(tmem + lane_off + kColS + 64 * buf, v);
       tc::tmem_ld_wait();
@@ -669,6 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&sm->p_full[buf]);
     }
     // ---- epilogue: per-head sums, then O (partials, or the final output)
+    if (!waited) pdl_wait();  // (no global write before the previous kernel is done)
     ok = __all_sync(0xffffffffu, ok && (ntiles == 0 || tc::mbar_wait(&sm->o_done, 0, abort, a.status, lim)));
     tc::fence_after_sync();
 #pragma unroll
@@ -943,7 +979,13 @@ bool tc_shape(const MqaArgs &a) {
          aligned16(a.kv_cmp) && aligned16(a.kv_win) && aligned16(a.out);
 }
 
-int rows_max_of(const MqaArgs &a) { return ((((a.idx || a.scores) ? a.k : a.N_max) + 3) & ~3) + a.win_len; }
+// Rows of the longest row list: the window padded to whole tiles, then the
+// compressed rows (early: the compressed rows alone, which the split plan
+// covers; split 0 takes the window tiles on top).
+int rows_max_of(const MqaArgs &a, bool early) {
+  const int nsel = (a.idx || a.scores) ? a.k : a.N_max;
+  return early ? nsel : (a.win_len + kRows - 1) / kRows * kRows + nsel;
+}
 
 }  // namespace
 
@@ -952,7 +994,7 @@ int rows_max_of(const MqaArgs &a) { return ((((a.idx || a.scores) ? a.k : a.N_ma
 size_t mqa_tc_partial_bytes(int Q, int H, int D, int rows_max) {
   if ((H != kH && H != 2 * kH) || D != kD || Q < 1) return 0;
   Q *= H / kH;  // one row list per group of 64 heads
-  const int tiles = (rows_max + 3 + kRows - 1) / kRows;
+  const int tiles = (rows_max + kRows + kRows - 1) / kRows;  // (+ the window's padding to whole tiles)
   int s = num_sms_cached() / Q;
   s = s > kMaxSplits ? kMaxSplits : s;
   s = s < 1 ? 1 : (s > tiles ? tiles : s);
@@ -968,7 +1010,8 @@ cudaError_t launch_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   int splits, tps;
   bool cluster_merge;
   const int G = a.H / kH, QV = a.Q * G;  // blocks per split: one per group of 64 heads of a query
-  plan_splits(QV, rows_max_of(a), &splits, &tps, &cluster_merge);
+  const bool early = a.early && !a.scores;
+  plan_splits(QV, rows_max_of(a, early), &splits, &tps, &cluster_merge);
   // In-kernel selection: the splits of a query must be one cluster, and each
   // block's slice of the scores must fit in its tile buffers.
   if (a.scores && (!cluster_merge || a.k > kSelMax || (((a.N_max + splits - 1) / splits + 31) & ~31) > kSelKeys ||

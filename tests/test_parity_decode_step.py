@@ -128,9 +128,11 @@ def test_full_size_step_matches_oracle(cuda_device, name, persistent):
 @pytest.mark.parametrize("name", ["csa_decode_64k", "hca_decode_1m", "csa_decode_64k_fp8"])
 def test_step_call_matches_separate_kernels(cuda_device, name, persistent):
     # The same step through the separate kernels. The chained variant runs
-    # those kernels: the same selection and bit-identical outputs. The
-    # persistent kernel: the same selection sets (the scores are the same
-    # products in the same order), outputs within the bf16 tolerance.
+    # the same scorer and top-k (the same selection, element for element);
+    # its attention takes the window tiles first, so the outputs agree to
+    # rounding. The persistent kernel: the same selection sets (the scores
+    # are the same products in the same order), outputs within the bf16
+    # tolerance.
     w = WL.WORKLOADS[name]
     ds_f, d = _decode_step(w, cuda_device, fused=True, persistent=persistent)
     out_f = ds_f.run().clone()
@@ -138,11 +140,8 @@ def test_step_call_matches_separate_kernels(cuda_device, name, persistent):
     ds_s, _ = _decode_step(w, cuda_device, fused=False)
     out_s = ds_s.run()
     torch.cuda.synchronize()
-    if not persistent:
-        assert torch.equal(out_f, out_s)
-        if idx_f is not None:
-            assert torch.equal(idx_f, ds_s.idx)
-        return
+    if not persistent and idx_f is not None:
+        assert torch.equal(idx_f, ds_s.idx)
     if idx_f is not None:
         assert torch.equal(torch.sort(idx_f, dim=1).values, torch.sort(ds_s.idx, dim=1).values)
     err = (out_f.float() - out_s.float()).abs()
