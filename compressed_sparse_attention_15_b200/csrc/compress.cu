@@ -150,8 +150,12 @@ __device__ __forceinline__ uint4 pack8(const float f[8]) {
 template <bool kRope>
 __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, int G) {
   extern __shared__ float ws[];  // [G][3][8][nvec] partial states, then [32] sums, then [3][8][nvec] block state
-  pdl_wait();
+  if (!a.late_wait) pdl_wait();
   pdl_release();
+  // late_wait: complete only after the kernel this one follows
+  auto finish = [&] {
+    if (a.late_wait && threadIdx.x == 0) pdl_wait();
+  };
   const int nvec = a.D / 8;
   const int v = threadIdx.x % nvec, g = threadIdx.x / nvec;
   const uint32_t C = cluster_size(), crank = cluster_rank();
@@ -303,6 +307,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
       o[d] = __float2bfloat16_rn(x);
     }
     cluster_sync();  // no block leaves while a peer may still read its share
+    finish();
     return;
   }
   const float ss = warp_sum(ssl);
@@ -322,6 +327,7 @@ __global__ void __launch_bounds__(512) compress_window_kernel(CompressArgs a, in
     if constexpr (kRope) rope8(a, b, j, 8 * t, c);
     reinterpret_cast<uint4 *>(o)[t] = pack8(c);
   }
+  finish();
 }
 
 // ------------------------------------------------------------------ streaming (CSA)

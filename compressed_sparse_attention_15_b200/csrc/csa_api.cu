@@ -71,7 +71,7 @@ const char *csa_strerror(int code) {
 static int compress_common(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio,
                            int win, int stride, void *out, int B, int T, int D, long long kv_seq_stride,
                            long long gate_seq_stride, long long out_seq_stride, int dtype, int rope_dims,
-                           double rope_theta, const int64_t *pos0, csa_stream_t stream) {
+                           double rope_theta, const int64_t *pos0, csa_stream_t stream, bool late_wait = false) {
   if (!kv || !gate || !ape || !norm_w || !out) return CSA_ERR_INVALID;
   if (!dtype_ok(dtype) || B < 1 || D < 1 || D > 4096 || win < 1 || win > 128 || stride < 1) return CSA_ERR_INVALID;
   if (ratio != stride || T < win) return CSA_ERR_INVALID;
@@ -91,6 +91,7 @@ static int compress_common(const void *kv, const void *gate, const float *ape, c
   a.rope_dims = rope_dims;
   a.rope_theta = rope_theta;
   a.pos0 = pos0;
+  a.late_wait = late_wait ? 1 : 0;
   return cuda_rc(launch_compress(a, (cudaStream_t)stream));
 }
 
@@ -217,14 +218,30 @@ int csa::check_index_topk(const void *qi, const float *wi, const void *ki, const
 // The launches of csa_index_topk / csa_index_topk_fp8 once their arguments
 // are checked: the scores into the workspace after the status page, then the
 // top-k with the rest of it as scratch. (Also the decode step's chain.)
-int csa::index_topk_launch(ScoreArgs sa, int k, int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream) {
+int csa::index_scores_into_ws(ScoreArgs sa, void *ws, cudaStream_t stream) {
   sa.scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kStatusBytes);
   sa.status = status_of(ws);
-  cudaError_t e = launch_index_scores(sa, stream);
-  if (e != cudaSuccess) return cuda_rc(e);
-  TopkArgs ta{sa.scores, sa.n_cmp, out_idx, sa.Q, sa.N_max, k, status_of(ws)};
+  return cuda_rc(launch_index_scores(sa, stream));
+}
+
+int csa::topk_from_ws(const ScoreArgs &sa, int k, int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kStatusBytes);
+  TopkArgs ta{scores, sa.n_cmp, out_idx, sa.Q, sa.N_max, k, status_of(ws)};
   const size_t sbytes = align256((size_t)sa.Q * sa.N_max * sizeof(float));
   return cuda_rc(launch_topk(ta, stream, static_cast<char *>(ws) + kStatusBytes + sbytes, ws_bytes - kStatusBytes - sbytes));
+}
+
+int csa::index_topk_launch(ScoreArgs sa, int k, int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  const int rc = index_scores_into_ws(sa, ws, stream);
+  return rc ? rc : topk_from_ws(sa, k, out_idx, ws, ws_bytes, stream);
+}
+
+int csa::compress_call(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
+                       int stride, void *out, int B, int T, int D, long long kv_seq_stride, long long gate_seq_stride,
+                       long long out_seq_stride, int dtype, int rope_dims, double rope_theta, const int64_t *pos0,
+                       bool late_wait, cudaStream_t stream) {
+  return compress_common(kv, gate, ape, norm_w, ratio, win, stride, out, B, T, D, kv_seq_stride, gate_seq_stride,
+                         out_seq_stride, dtype, rope_dims, rope_theta, pos0, (csa_stream_t)stream, late_wait);
 }
 
 extern "C" {

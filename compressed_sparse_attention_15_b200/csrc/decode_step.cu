@@ -1932,20 +1932,21 @@ int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, cs
     cudaGetLastError();  // a tensor map the encoder rejected: the separate kernels serve the call
   }
   // The chained kernels, one after another on the stream (each launch a
-  // programmatic dependent of the one before).
+  // programmatic dependent of the one before). CSA: scorer, append, top-k,
+  // attention -- the append needs nothing the scorer writes, so it starts
+  // at once, on the SMs the scorer's CTAs leave, and waits for the scorer
+  // only before it exits (the top-k then follows both); HCA: append,
+  // attention.
   int rc = CSA_OK;
-  if (s->app_kv) {
-    void *out = static_cast<char *>(const_cast<void *>(s->kv_cmp)) + (size_t)s->app_row0 * s->D * (s->dtype == CSA_DTYPE_F32 ? 4 : 2);
+  auto append = [&](bool late_wait) -> int {
+    if (!s->app_kv) return CSA_OK;
+    void *out = static_cast<char *>(const_cast<void *>(s->kv_cmp)) +
+                (size_t)s->app_row0 * s->D * (s->dtype == CSA_DTYPE_F32 ? 4 : 2);
     const long long oss = (long long)s->N_max * s->D;
-    rc = s->rope_dims ? csa_compress_rope(s->app_kv, s->app_gate, s->ape, s->norm_w, s->app_stride, s->app_win,
-                                          s->app_stride, out, s->B, s->app_T, s->D, s->app_kv_seq_stride,
-                                          s->app_gate_seq_stride, oss, s->rope_dims, s->rope_theta, s->pos0, s->dtype,
-                                          stream)
-                      : csa_compress(s->app_kv, s->app_gate, s->ape, s->norm_w, s->app_stride, s->app_win,
-                                     s->app_stride, out, s->B, s->app_T, s->D, s->app_kv_seq_stride,
-                                     s->app_gate_seq_stride, oss, s->dtype, stream);
-    if (rc) return rc;
-  }
+    return compress_call(s->app_kv, s->app_gate, s->ape, s->norm_w, s->app_stride, s->app_win, s->app_stride, out,
+                         s->B, s->app_T, s->D, s->app_kv_seq_stride, s->app_gate_seq_stride, oss, s->dtype,
+                         s->rope_dims, s->rope_theta, s->pos0, late_wait, st);
+  };
   if (csa) {
     const bool fp8 = s->index_dtype == CSA_DTYPE_E4M3;
     rc = fp8 ? check_index_topk_fp8(static_cast<const uint8_t *>(s->qi), s->sq, s->wi,
@@ -1957,17 +1958,16 @@ int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, cs
     if (ws_bytes < csa_index_topk_workspace_bytes(s->Q, s->N_max, s->k)) return CSA_ERR_WORKSPACE;
     ScoreArgs sa{s->qi, s->wi, s->ki, s->n_cmp, nullptr, s->Q, s->B, s->Hi, s->Di, s->N_max, s->q_per_seq,
                  s->index_dtype, nullptr, fp8 ? s->sq : nullptr, fp8 ? s->sk : nullptr};
-    // After the append (which writes only kv_cmp rows) the scorer starts at
-    // once and waits for the append only before it exits.
-    sa.late_wait = s->app_kv ? 1 : 0;
-    rc = index_topk_launch(sa, s->k, s->idx_out, ws, ws_bytes, st);
-    if (rc) return rc;
+    if ((rc = index_scores_into_ws(sa, ws, st))) return rc;
+    if ((rc = append(true))) return rc;
+    if ((rc = topk_from_ws(sa, s->k, s->idx_out, ws, ws_bytes, st))) return rc;
     // The attention loads the queries and runs the window tiles before it
     // waits for the top-k (which writes none of them).
     return attend_call(s->q, s->kv_cmp, s->idx_out, nullptr, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H,
                        s->D, s->N_max, s->k, s->win_len, s->win_end, s->T_raw, s->q_per_seq, s->dtype, true, ws,
                        ws_bytes, st);
   }
+  if ((rc = append(false))) return rc;
   // HCA: the window tiles before the wait for the append (which writes only
   // kv_cmp rows); without an append, the caller's kernel may write anything.
   return attend_call(s->q, s->kv_cmp, nullptr, s->n_cmp, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H, s->D,

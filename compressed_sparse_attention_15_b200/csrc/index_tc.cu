@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
-  if (!a.late_wait) pdl_wait();  // inputs may come from the previous kernel in the stream
+  pdl_wait();  // inputs may come from the previous kernel in the stream
   pdl_release();
   const uint64_t lim = tc::wait_limit_of(a.status);
 
@@ -364,7 +364,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (a.late_wait && threadIdx.x == 0) pdl_wait();  // complete only after the kernel this one follows
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, F::kTmemCols);

@@ -65,6 +65,11 @@ struct CompressArgs {
   int rope_dims = 0;
   double rope_theta = 0.0;
   const int64_t *pos0 = nullptr;
+  // 1: the kernel before this one in the stream reads and writes none of
+  // kv, gate, ape, norm_w and out (the decode step's scorer): the per-entry
+  // window kernel starts at once and waits for it only before exiting (so
+  // the kernels after it still follow both); 0: wait before reading anything.
+  int late_wait = 0;
 };
 cudaError_t launch_compress(const CompressArgs &a, cudaStream_t stream);
 // The indexer's compressor (pool + RMSNorm + Hadamard rotation; D in 64..512,
@@ -87,12 +92,6 @@ struct ScoreArgs {
   uint32_t *status;
   const float *sq = nullptr;  // CSA_DTYPE_E4M3: per (query, head) scale [Q, Hi]
   const float *sk = nullptr;  // CSA_DTYPE_E4M3: per entry scale [B, N_max]
-  // 1: the kernel before this one in the stream writes none of the inputs
-  // (the decode step's cache append), so the tensor-core kernel starts at
-  // once and waits for it only before exiting (the completion order, and
-  // with it the visibility of the append to the kernels after this one, is
-  // kept); 0: wait before reading anything.
-  int late_wait = 0;
 };
 cudaError_t launch_index_scores(const ScoreArgs &a, cudaStream_t stream);
 
@@ -115,8 +114,17 @@ int check_index_topk(const void *qi, const float *wi, const void *ki, const int3
 int check_index_topk_fp8(const uint8_t *qi8, const float *sq, const float *wi, const uint8_t *ki8, const float *sk,
                          const int32_t *n_cmp, int k, const int32_t *out_idx, int Q, int B, int Hi, int Di, int N_max,
                          int q_per_seq);
-// Scores, then top-k, on `stream` (sa.scores and sa.status are set from ws).
+// Scores, then top-k, on `stream` (sa.scores and sa.status are set from ws),
+// as one call or as its two launches (other work may go between them).
 int index_topk_launch(ScoreArgs sa, int k, int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream);
+int index_scores_into_ws(ScoreArgs sa, void *ws, cudaStream_t stream);
+int topk_from_ws(const ScoreArgs &sa, int k, int32_t *out_idx, void *ws, size_t ws_bytes, cudaStream_t stream);
+// csa_compress / csa_compress_rope: checks, then the launch; late_wait sets
+// CompressArgs::late_wait.
+int compress_call(const void *kv, const void *gate, const float *ape, const float *norm_w, int ratio, int win,
+                  int stride, void *out, int B, int T, int D, long long kv_seq_stride, long long gate_seq_stride,
+                  long long out_seq_stride, int dtype, int rope_dims, double rope_theta, const int64_t *pos0,
+                  bool late_wait, cudaStream_t stream);
 
 // ---------------------------------------------------------------- per-device setup
 // Kernel attributes are set, and device facts cached, once per device (a

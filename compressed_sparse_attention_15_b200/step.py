@@ -11,10 +11,10 @@ The step over device-resident caches is:
   3. attend over the selected (CSA) or all visible (HCA) entries + the
      sliding window + the per-head sink (csa_sparse_mqa / hca_mqa).
 With fused=True the whole step is one csa_decode_step call: by default the
-same kernels chained by programmatic dependent launch on one stream, the
-indexer's scorer starting without waiting for the append (the append writes
-none of its inputs), so the append overlaps the key scan with no second
-stream; persistent=True asks instead for the one persistent kernel in which
+same kernels chained by programmatic dependent launch on one stream (CSA:
+the scorer first, the append running in its tail, then the top-k, then the
+attention, which computes its window tiles before the top-k is done), with
+no second stream; persistent=True asks instead for the one persistent kernel in which
 the selection and attention of some queries overlap the key scan of others
 (measured slower: its per-query chains are latency-bound). With fused=False
 (the default) the parts are separate calls, the append on a forked stream;

@@ -390,10 +390,15 @@ int csa_index_topk_noalloc(const void *qi, const float *wi, const void *ki, cons
  *
  * variant = CSA_STEP_CHAINED (0): the kernels of those calls, launched as
  * one chain of programmatic dependent launches on `stream` with no host
- * synchronisation; the indexer's tensor-core scorer does not wait for the
- * append before it starts (it reads none of the rows the append writes: qi,
- * wi, ki and n_cmp must not overlap kv_cmp), so the two overlap. Outputs are
- * those of the separate calls, bit for bit.
+ * synchronisation. CSA runs the scorer first and the append after it, the
+ * append starting at once (the scorer reads none of what it reads or
+ * writes: qi, wi, ki and n_cmp must not overlap kv_cmp, app_kv, app_gate)
+ * on the SMs the scorer leaves; the top-k follows both; the attention loads
+ * the queries and computes the window tiles before the top-k is done (q,
+ * kv_win, win_end and sink must not be written by the caller's kernel
+ * launched just before this call with programmatic dependent launch). The
+ * selection is that of the separate calls; the attention outputs agree with
+ * them to rounding (the window tiles are summed first).
  * variant = CSA_STEP_PERSISTENT (1), for bf16 attention with H = 64 or 128,
  * D = 512, one query per sequence (q_per_seq = 1) and the indexer shape
  * 64 x 128: ONE persistent kernel in which each SM pulls tasks (append,
