@@ -14,12 +14,14 @@
 // accumulator, so each epilogue thread owns one entry's 64 head products and
 // the weighted ReLU sum over heads is thread-local.
 //
-// Pipeline (persistent, one CTA per SM, 192 threads):
+// Pipeline (persistent, one CTA per SM; 192 threads, 320 for E4M3):
 //   warp 0      TMA producer: 32 KB key tiles (128 bf16 / 256 FP8 entries)
 //               into a 5-stage ring, and the query's head block (16 / 8 KB)
 //               into one of two query slots;
 //   warp 1      MMA issuer (one thread) and TMEM owner (2 accumulators);
-//   warps 2..5  epilogue: tcgen05.ld, ReLU, weighted sum, coalesced store.
+//   warps 2..   epilogue, one per TMEM lane quarter and 128-entry row block
+//               (4 warps; 8 for the two blocks of an E4M3 tile): tcgen05.ld,
+//               ReLU, weighted sum, coalesced store.
 // Each CTA walks a contiguous range of the flat (query, tile) space. Every
 // wait is bounded; a timeout raises CSA_STATUS_WAIT_TIMEOUT, all roles stop,
 // in-flight copies and MMAs are drained (bounded) and TMEM is freed.
@@ -40,7 +42,7 @@ namespace csa {
 namespace {
 
 constexpr int kHi = 64, kDi = 128;
-constexpr int kThreads = 192;
+
 
 // Per element format: a stage is 32 KB of keys in two TMA boxes of 128 rows x
 // 128 bytes (the swizzle span): bf16 tiles are 128 entries split along the
@@ -66,6 +68,10 @@ struct Fmt {
   static constexpr uint32_t kIdesc = kFp8 ? tc::idesc_e4m3(128, 64) : tc::idesc_bf16(128, 64 * kG, 0, 0);
   // per epilogue warp: its group's head weights and visible counts
   static constexpr uint32_t kWBytes = kG == 1 ? 0 : 4 * (kG * kHi * 4 + kG * 4);
+  // Epilogue warps: one per TMEM lane quarter and row block, so that each
+  // warp reduces one 128-entry block of a tile (E4M3 tiles hold two).
+  static constexpr int kEpiWarps = 4 * kSub;
+  static constexpr int kThreads = 32 * (2 + kEpiWarps);
 };
 
 template <int kStages>
@@ -100,7 +106,7 @@ __device__ __forceinline__ Tile tile_of(long long t, int tiles_per_q, int tile_r
 }
 
 template <bool kFp8, int kG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Fmt<kFp8, kG>::kThreads, 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
                            ScoreArgs a, int tiles_per_q, long long total, long long per_cta) {
   using F = Fmt<kFp8, kG>;
@@ -125,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->qfull[s], 1);
       tc::mbar_init(&bars->qempty[s], 1);
       tc::mbar_init(&bars->accfull[s], 1);
-      tc::mbar_init(&bars->accempty[s], 4 * 32);
+      tc::mbar_init(&bars->accempty[s], F::kEpiWarps * 32);
     }
     tc::mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -280,21 +286,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int sub = (warp - 2) >> 2;  // the tile's 128-entry block this warp reduces
     const int row = quarter * 32 + lane;
     int acc = 0, cur_q = -1, cur_n = 0;
     uint32_t accph = 0;
     float w[kHi];
-    float sk_next[F::kSub];
-    auto load_sk = [&](long long tt) {  // key scales of tile tt's rows of this thread (1 past the cache)
+    float sk_next = 1.f;
+    auto load_sk = [&](long long tt) {  // key scale of tile tt's row of this thread (1 past the cache)
       const Tile tn = tile_of(tt, tiles_per_q, F::kTileRows);
-#pragma unroll
-      for (int sub = 0; sub < F::kSub; ++sub) {
-        const int j = tn.j0 + 128 * sub + row;
-        sk_next[sub] = j < a.N_max ? __ldg(a.sk + (size_t)(tn.q / a.q_per_seq) * a.N_max + j) : 1.f;
-      }
+      const int j = tn.j0 + 128 * sub + row;
+      sk_next = j < a.N_max ? __ldg(a.sk + (size_t)(tn.q / a.q_per_seq) * a.N_max + j) : 1.f;
     };
-#pragma unroll
-    for (int sub = 0; sub < F::kSub; ++sub) sk_next[sub] = 1.f;
     if constexpr (kFp8) {
       if (t_begin < t_end) load_sk(t_begin);
     }
@@ -323,18 +325,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // E4M3: the key scales of this tile were loaded one tile ahead; start
       // the next tile's now, so their latency hides behind this tile's work.
-      float skv[F::kSub];
-#pragma unroll
-      for (int sub = 0; sub < F::kSub; ++sub) skv[sub] = sk_next[sub];
+      const float skv = sk_next;
       if constexpr (kFp8) {
         if (t + 1 < t_end) load_sk(t + 1);
       }
       const bool ok = tc::mbar_wait(&bars->accfull[acc], accph, abort, a.status, lim);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc::fence_after_sync();
-      float sc[F::kSub];
-#pragma unroll
-      for (int sub = 0; sub < F::kSub; ++sub) {
+      float sc;
+      {
         uint32_t v0[32], v1[32];
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * F::kAccCols + 64 * sub;
         tc::tmem_ld32(taddr, v0);
@@ -345,16 +344,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < 32; ++h) s = fmaf(w[h], fmaxf(__uint_as_float(v0[h]), 0.f), s);
 #pragma unroll
         for (int h = 0; h < 32; ++h) s = fmaf(w[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s);
-        sc[sub] = s;
+        sc = s;
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->accempty[acc]);
-#pragma unroll
-      for (int sub = 0; sub < F::kSub; ++sub) {
+      {
         const int j = tl.j0 + 128 * sub + row;
-        if (j < cur_n) {
-          a.scores[(size_t)tl.q * a.N_max + j] = kFp8 ? sc[sub] * skv[sub] : sc[sub];
-        }
+        if (j < cur_n) a.scores[(size_t)tl.q * a.N_max + j] = kFp8 ? sc * skv : sc;
       }
       if (++acc == 2) {
         acc = 0;
@@ -400,7 +396,7 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t stream, bool *taken) {
                          (int)smem_bytes<kFp8, kG>());
   });
   *taken = true;
-  return launch_pdl(index_scores_tc_kernel<kFp8, kG>, dim3((unsigned)grid), dim3(kThreads), smem_bytes<kFp8, kG>(),
+  return launch_pdl(index_scores_tc_kernel<kFp8, kG>, dim3((unsigned)grid), dim3(F::kThreads), smem_bytes<kFp8, kG>(),
                     stream, tm_ki, tm_qi, a, tiles_per_q, total, per_cta);
 }
 
