@@ -404,7 +404,7 @@ int csa_workspace_status(void *ws, csa_stream_t stream, uint32_t *status) {
 int csa::attend_call(const void *q, const void *kv_cmp, const int32_t *idx, const int32_t *n_cmp, const void *kv_win,
                      const float *sink, float scale, void *out, int Q, int B, int H, int D, int N_max, int k,
                      int win_len, const int32_t *win_end, int T_raw, int q_per_seq, int dtype, bool early, void *ws,
-                     size_t ws_bytes, cudaStream_t stream) {
+                     size_t ws_bytes, cudaStream_t stream, int dep_row0, int dep_rows) {
   int rc = check_mqa(q, kv_cmp, kv_win, sink, out, Q, B, H, D, N_max, win_len, win_end, T_raw, q_per_seq, dtype);
   if (rc) return rc;
   if (idx) {
@@ -420,5 +420,7 @@ int csa::attend_call(const void *q, const void *kv_cmp, const int32_t *idx, cons
   MqaArgs a{q, kv_cmp, kv_win, idx, idx ? nullptr : n_cmp, win_end, sink, scale, out, Q, B, H, D, N_max, k, win_len,
             T_raw, q_per_seq, dtype, static_cast<char *>(ws) + kStatusBytes, ws_bytes - kStatusBytes, status_of(ws)};
   a.early = early ? 1 : 0;
+  a.dep_row0 = dep_row0;
+  a.dep_rows = dep_rows;
   return cuda_rc(launch_mqa(a, stream));
 }

@@ -1968,11 +1968,13 @@ int csa_decode_step(const csa_decode_step_args *s, void *ws, size_t ws_bytes, cs
                        ws_bytes, st);
   }
   if ((rc = append(false))) return rc;
-  // HCA: the window tiles before the wait for the append (which writes only
-  // kv_cmp rows); without an append, the caller's kernel may write anything.
+  // HCA: only the tiles holding the appended rows wait for the append (which
+  // writes nothing else the attention reads); without an append, the
+  // caller's kernel may write anything.
+  const int n_new = s->app_kv ? (s->app_T - s->app_win) / s->app_stride + 1 : 0;
   return attend_call(s->q, s->kv_cmp, nullptr, s->n_cmp, s->kv_win, s->sink, s->scale, s->out, s->Q, s->B, s->H, s->D,
                      s->N_max, 0, s->win_len, s->win_end, s->T_raw, s->q_per_seq, s->dtype, s->app_kv != nullptr, ws,
-                     ws_bytes, st);
+                     ws_bytes, st, s->app_kv ? (int)s->app_row0 : -1, n_new);
 }
 
 }  // extern "C"

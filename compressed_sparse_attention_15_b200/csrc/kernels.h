@@ -182,8 +182,12 @@ struct MqaArgs {
   // 1: the kernel before this one in the stream writes none of q, kv_win,
   // win_end, sink and n_cmp (the decode step's top-k, or its append for
   // HCA): the tensor-core kernel loads the queries and runs the window tiles
-  // before waiting for it; 0: it waits before reading anything.
+  // before waiting for it; 0: it waits before reading anything. With early
+  // set and a dense list (idx null), dep_row0 >= 0 names the only cache rows
+  // that kernel writes, [dep_row0, dep_row0 + dep_rows) of every sequence:
+  // only tiles holding them wait.
   int early = 0;
+  int dep_row0 = -1, dep_rows = 0;
 };
 cudaError_t launch_mqa(const MqaArgs &a, cudaStream_t stream);
 // csa_sparse_mqa (idx given) / hca_mqa (idx null, n_cmp given): checks, then
@@ -191,7 +195,7 @@ cudaError_t launch_mqa(const MqaArgs &a, cudaStream_t stream);
 int attend_call(const void *q, const void *kv_cmp, const int32_t *idx, const int32_t *n_cmp, const void *kv_win,
                 const float *sink, float scale, void *out, int Q, int B, int H, int D, int N_max, int k, int win_len,
                 const int32_t *win_end, int T_raw, int q_per_seq, int dtype, bool early, void *ws, size_t ws_bytes,
-                cudaStream_t stream);
+                cudaStream_t stream, int dep_row0 = -1, int dep_rows = 0);
 // Top-k selection fused into the tensor-core MQA (a.scores set); *taken is
 // false when the shape or the launch plan does not allow it.
 cudaError_t launch_topk_mqa_tc(const MqaArgs &a, cudaStream_t stream, bool *taken);

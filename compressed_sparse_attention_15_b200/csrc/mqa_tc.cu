@@ -123,13 +123,13 @@ __device__ __forceinline__ RowList row_list(const MqaArgs &a, int qq, uint32_t *
 }
 
 // The tiles [t0, t1) of split `split`: runs of tiles_per_split tiles; with
-// early window tiles (the window computed before the kernel waits on its
-// predecessor) split 0 takes the window tiles on top of its run of
-// compressed tiles and the runs cover the compressed tiles only.
-__device__ __forceinline__ void split_tiles(const RowList &L, int split, int tiles_per_split, bool early, int &t0,
-                                            int &t1) {
+// the window on top (a selection's window tiles computed before the kernel
+// waits on its predecessor, its compressed tiles after) split 0 takes the
+// window tiles on top of its run and the runs cover the compressed tiles.
+__device__ __forceinline__ void split_tiles(const RowList &L, int split, int tiles_per_split, bool window_on_top,
+                                            int &t0, int &t1) {
   const int tiles_all = (L.R + kRows - 1) / kRows, wt = L.w64 / kRows;
-  if (early) {
+  if (window_on_top) {
     t0 = split == 0 ? 0 : wt + split * tiles_per_split;
     t1 = min(tiles_all, wt + (split + 1) * tiles_per_split);
   } else {
@@ -337,12 +337,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_release();
 
   const RowList L = row_list(a, qq, threadIdx.x == 0 ? a.status : nullptr);
-  int t0, t1;
-  split_tiles(L, split, tiles_per_split, early, t0, t1);
-  const int ntiles = max(0, t1 - t0);
-  const int wt = L.w64 / kRows;  // window tiles (list tiles [0, wt))
   constexpr bool fused = kFused;
   const bool sparse = fused || a.idx != nullptr;
+  // (a selection's compressed tiles all wait: split 0 takes the window tiles
+  // on top of its run; a dense list's tiles are split evenly)
+  int t0, t1;
+  split_tiles(L, split, tiles_per_split, early && sparse, t0, t1);
+  const int ntiles = max(0, t1 - t0);
+  // Whether this CTA's tile li needs the previous kernel done (early mode):
+  // a compressed tile of a selection, or of a dense list holding a row that
+  // kernel writes.
+  auto tile_dep = [&](int li) -> bool {
+    const int r0 = (t0 + li) * kRows;
+    if (r0 < L.w64) return false;
+    if (sparse || a.dep_row0 < 0) return true;
+    const int p0 = r0 - L.w64, p1 = min(p0 + kRows, L.nsel);
+    return p0 < p1 && p0 < a.dep_row0 + a.dep_rows && a.dep_row0 < p1;
+  };
   if (warp == kMmaWarp && lane == 0 && ntiles > 0) {
     tc::prefetch_tmap(&tm_q);
     tc::mbar_arrive_expect_tx(&sm->q_full, kQBytes);
@@ -418,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int last = -1;
     for (int li = g; li < ntiles; li += 2) {
       const int r0 = (t0 + li) * kRows;
-      if (t0 + li >= wt && !waited) {  // the first compressed tile: the previous kernel must be done
+      if (!waited && tile_dep(li)) {  // the first tile that needs the previous kernel done
         pdl_wait();
         waited = true;
       }
@@ -563,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int li = 0; li < ntiles; ++li) {
       const int buf = li & 1;
-      if (!waited && t0 + li >= wt) {  // the first compressed tile: the previous kernel must be done
+      if (!waited && tile_dep(li)) {  // the first tile that needs the previous kernel done
         pdl_wait();
         waited = true;
       }
@@ -980,11 +991,11 @@ bool tc_shape(const MqaArgs &a) {
 }
 
 // Rows of the longest row list: the window padded to whole tiles, then the
-// compressed rows (early: the compressed rows alone, which the split plan
-// covers; split 0 takes the window tiles on top).
-int rows_max_of(const MqaArgs &a, bool early) {
+// compressed rows (window_on_top: the compressed rows alone, which the split
+// plan covers; split 0 takes the window tiles on top).
+int rows_max_of(const MqaArgs &a, bool window_on_top) {
   const int nsel = (a.idx || a.scores) ? a.k : a.N_max;
-  return early ? nsel : (a.win_len + kRows - 1) / kRows * kRows + nsel;
+  return window_on_top ? nsel : (a.win_len + kRows - 1) / kRows * kRows + nsel;
 }
 
 }  // namespace
@@ -1010,8 +1021,8 @@ cudaError_t launch_tc(const MqaArgs &a, cudaStream_t stream, bool *taken) {
   int splits, tps;
   bool cluster_merge;
   const int G = a.H / kH, QV = a.Q * G;  // blocks per split: one per group of 64 heads of a query
-  const bool early = a.early && !a.scores;
-  plan_splits(QV, rows_max_of(a, early), &splits, &tps, &cluster_merge);
+  const bool window_on_top = a.early && !a.scores && a.idx;  // see split_tiles
+  plan_splits(QV, rows_max_of(a, window_on_top), &splits, &tps, &cluster_merge);
   // In-kernel selection: the splits of a query must be one cluster, and each
   // block's slice of the scores must fit in its tile buffers.
   if (a.scores && (!cluster_merge || a.k > kSelMax || (((a.N_max + splits - 1) / splits + 31) & ~31) > kSelKeys ||
