@@ -339,8 +339,8 @@ def time_ours(args, w: WL.Workload, device, dist_on, rank, world, secondary=Fals
     torch.cuda.synchronize()
     K0 = max(5, args.steps // 5)
     trial = {f: _time_steps(st, flush, stream, K0) for f, st in steps.items()}
-    # the step call only when clearly faster (its per-kernel split is one part)
-    fused = len(trial) == 1 and True in trial or (len(trial) == 2 and trial[True] < 0.97 * trial[False])
+    # the faster path (the per-kernel times come from the separate calls either way)
+    fused = len(trial) == 1 and True in trial or (len(trial) == 2 and trial[True] <= trial[False])
     step = steps[fused]
     launches_per_step = launches[fused]
 
@@ -466,9 +466,9 @@ def time_index_compress(args, w: WL.Workload, device, hbm_gbs):
 
 
 def path_parts(per_kernel_ms, path):
-    """The per-kernel times of the path that was timed: the step call, or
+    """The per-kernel times of one path (empty if it was not built): the step call, or
     the separate kernels."""
-    if path == "fused":
+    if path == "step_call":
         return {k: v for k, v in per_kernel_ms.items() if k == WHOLE_STEP}
     return {k: v for k, v in per_kernel_ms.items() if k != WHOLE_STEP}
 
@@ -786,7 +786,8 @@ def main():
     r = time_ours(args, w, device, dist_on, rank, world)
     traffic = load_traffic(args.traffic_json, w.name)
     # the dominant kernel's own timing (the chained step runs the same kernels)
-    roof = roofline_of(w, path_parts(r["per_kernel_ms"], "separate"), hbm, traffic, tflops)
+    roof = roofline_of(w, path_parts(r["per_kernel_ms"], "separate") or path_parts(r["per_kernel_ms"], r["path"]),
+                       hbm, traffic, tflops)
     roof["peak_kind"] = f"{peak_kind} HBM copy bandwidth"
     e2e = e2e_ours(args, w, r["step"], device)
     del r["step"]
@@ -801,7 +802,8 @@ def main():
             try:
                 s = time_ours(args, sw, device, False, 0, 1, secondary=True, rope=rope)
                 del s["step"]
-                rf = roofline_of(sw, path_parts(s["per_kernel_ms"], "separate"), hbm,
+                rf = roofline_of(sw, path_parts(s["per_kernel_ms"], "separate") or
+                                 path_parts(s["per_kernel_ms"], s["path"]), hbm,
                                  load_traffic(args.traffic_json, label), tflops)
                 line = {"workload": name, "queries_per_s": round(sw.Q / (s["ms"] * 1e-3), 1),
                         "ms_per_step": round(s["ms"], 4), "path": s["path"], "paths_ms": s["paths_ms"],
