@@ -129,7 +129,9 @@ def test_index_topk_full_size(cuda_device, name, nq):
     qi, wi, ki = (WL.make(w, t, cuda_device) for t in ("qi", "wi", "ki"))
     p = w.positions()
     n = ops.visible_entries(p, w.win, w.stride)
-    idx = ops.index_topk(qi, wi, ki, n.to(cuda_device), w.k, q_per_seq=w.q_per_seq).cpu().numpy()
+    ws = ops.Workspace(cuda_device)
+    idx = ops.index_topk(qi, wi, ki, n.to(cuda_device), w.k, q_per_seq=w.q_per_seq, ws=ws).cpu().numpy()
+    assert ws.status() == 0
     del ki
     qs = np.unique(np.linspace(0, w.Q - 1, nq).round().astype(int))
     seqs = sorted({int(q) // w.q_per_seq for q in qs})
@@ -141,3 +143,29 @@ def test_index_topk_full_size(cuda_device, name, nq):
         ref_idx, ref_s = O.index_topk(qi_h[q], wi_h[q], ki_h[b], int(p[q]), w.k, w.win, w.stride)
         swaps += check_topk_set(idx[q], ref_idx, ref_s, w.k, int(n[q]))
     assert swaps <= max(2, len(qs) // 4)
+
+
+@pytest.mark.parametrize("Q,N", [(32, 16383), (4, 300), (3, 129)])
+def test_scores_repeat_exactly_on_one_workspace(cuda_device, Q, N):
+    # Three calls on one workspace give bit-identical scores equal to the
+    # oracle's, a clean status, and leave the workspace header (status word,
+    # wait limit, reserved bytes) at zero for the next call.
+    qi = synth.normal(11, 1, (Q, 64, 128), dtype=torch.bfloat16)
+    wi = synth.uniform(11, 2, (Q, 64))
+    ki = synth.normal(11, 3, (Q, N, 128), dtype=torch.bfloat16)
+    n = torch.tensor([N - (q % 3) * 7 for q in range(Q)], dtype=torch.int32)
+    d = [t.to(cuda_device) for t in (qi, wi, ki, n)]
+    ws = ops.Workspace(cuda_device)
+    runs = []
+    for _ in range(3):
+        out = torch.zeros((Q, N), dtype=torch.float32, device=cuda_device)
+        ops.index_scores(*d, out=out, ws=ws)
+        torch.cuda.synchronize()
+        assert int(ws.buf[:256].count_nonzero()) == 0
+        runs.append(out.cpu().numpy())
+    assert np.array_equal(runs[0], runs[1]) and np.array_equal(runs[0], runs[2])
+    for q in range(Q):
+        nv = int(n[q])
+        ref = O.index_scores(qi[q], wi[q], ki[q], nv)
+        scale = max(np.abs(ref).max(initial=0.0), 1.0)
+        assert np.max(np.abs(f64(runs[0][q, :nv]) - ref), initial=0.0) <= 1e-4 * scale
