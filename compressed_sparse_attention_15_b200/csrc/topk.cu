@@ -20,9 +20,10 @@
 // into C contiguous slices, one CTA of a thread-block cluster each (C <= 8,
 // about SMs / Q); the slices' histograms are summed through distributed
 // shared memory at every radix pass, and each CTA emits its own slice at the
-// offset given by the counts of the slices before it. Many queries: one
-// 1024-thread CTA per query with the keys cached in shared memory (up to
-// 48K entries). Longer lists with many queries take two stages: the exact
+// offset given by the counts of the slices before it. Many queries with
+// lists of up to 40K entries: one 1024-thread CTA per query, keys cached in
+// shared memory, the same sample-and-filter scheme (topk_filter_kernel); up
+// to 48K entries: the exact passes over the cached keys. Longer lists with many queries take two stages: the exact
 // top-k of 4K-32K-entry segments in parallel, then the same selection over
 // the concatenated segment winners. Without scratch space a single CTA per
 // query does it all (re-reading the scores per pass beyond 48K entries).
@@ -362,6 +363,7 @@ struct BlockShared {
   uint32_t sel_t, sel_ngt;  // the few-candidates finish, computed by warp 0
 };
 constexpr int kCandCap = 4096;  // candidate buffer (dynamic shared memory: keys, then positions)
+constexpr int kFilterKeys = 40 * 1024;  // longest list of topk_filter_kernel (keys + candidates in shared memory)
 
 // Exclusive prefix over the warps of a per-warp value (every lane passes its
 // warp's value). One barrier; every thread gets its warp's offset and the
@@ -493,6 +495,53 @@ __device__ __forceinline__ void radix_select(BlockShared &sh, const uint32_t (&k
   kk_out = kk;
 }
 
+// The exact top k of C candidates (k <= C <= kCandCap) gathered in shared
+// memory in position order: cbuf[i] the key in units above the floor (the
+// largest unit is urange), cbuf[kCandCap + i] the position. Writes the k
+// positions to out in ascending order (ties: the first positions). Every
+// thread of the block takes part; both histograms are clear and sh.ncand is 0.
+__device__ __forceinline__ void select_candidates(BlockShared &sh, const uint32_t *cbuf, int C, uint32_t urange,
+                                                  uint32_t k, int32_t *out, int lane, int warp) {
+  // thread t: candidates 4t .. 4t + 3
+  const int c0 = 4 * (int)threadIdx.x;
+  const int ncv = max(0, min(4, C - c0));
+  uint32_t cv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) cv[i] = i < ncv ? cbuf[c0 + i] : 0u;
+  uint32_t tau, kk;
+  radix_select<4>(sh, cv, ncv, 0u, urange, k, lane, warp, tau, kk);
+  // ordered compaction over the candidates
+  uint32_t g = 0u, e = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    g += (i < ncv && cv[i] > tau) ? 1u : 0u;
+    e += (i < ncv && cv[i] == tau) ? 1u : 0u;
+  }
+  uint32_t gi = g, ei = e;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t yg = __shfl_up_sync(0xffffffffu, gi, o), ye = __shfl_up_sync(0xffffffffu, ei, o);
+    if (lane >= o) {
+      gi += yg;
+      ei += ye;
+    }
+  }
+  uint32_t og, oe, tg, te;
+  warp_offsets(sh.wg, __shfl_sync(0xffffffffu, gi, 31), lane, warp, og, tg);
+  warp_offsets(sh.we, __shfl_sync(0xffffffffu, ei, 31), lane, warp, oe, te);
+  uint32_t G = og + gi - g, E = oe + ei - e;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (i < ncv && cv[i] > tau) {
+      out[G + min(E, kk)] = (int32_t)cbuf[kCandCap + c0 + i];
+      ++G;
+    } else if (i < ncv && cv[i] == tau) {
+      if (E < kk) out[G + E] = (int32_t)cbuf[kCandCap + c0 + i];
+      ++E;
+    }
+  }
+}
+
 template <int R>
 __global__ void __launch_bounds__(kThreads) topk_block_kernel(TopkArgs a) {
   __shared__ alignas(16) BlockShared sh;
@@ -587,44 +636,7 @@ __global__ void __launch_bounds__(kThreads) topk_block_kernel(TopkArgs a) {
           off += __popc(mm);
         }
         __syncthreads();
-        // thread t: candidates 4t .. 4t + 3
-        const int c0 = 4 * (int)threadIdx.x;
-        const int ncv = max(0, min(4, (int)C - c0));
-        uint32_t cv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) cv[i] = i < ncv ? cbuf[c0 + i] : 0u;
-        uint32_t tau, kk;
-        radix_select<4>(sh, cv, ncv, 0u, range - ulow, (uint32_t)k, lane, warp, tau, kk);
-        // ordered compaction over the candidates
-        uint32_t g = 0u, e = 0u;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          g += (i < ncv && cv[i] > tau) ? 1u : 0u;
-          e += (i < ncv && cv[i] == tau) ? 1u : 0u;
-        }
-        uint32_t gi = g, ei = e;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t yg = __shfl_up_sync(0xffffffffu, gi, o), ye = __shfl_up_sync(0xffffffffu, ei, o);
-          if (lane >= o) {
-            gi += yg;
-            ei += ye;
-          }
-        }
-        uint32_t og, oe, tg, te;
-        warp_offsets(sh.wg, __shfl_sync(0xffffffffu, gi, 31), lane, warp, og, tg);
-        warp_offsets(sh.we, __shfl_sync(0xffffffffu, ei, 31), lane, warp, oe, te);
-        uint32_t G = og + gi - g, E = oe + ei - e;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (i < ncv && cv[i] > tau) {
-            out[G + min(E, kk)] = (int32_t)cbuf[kCandCap + c0 + i];
-            ++G;
-          } else if (i < ncv && cv[i] == tau) {
-            if (E < kk) out[G + E] = (int32_t)cbuf[kCandCap + c0 + i];
-            ++E;
-          }
-        }
+        select_candidates(sh, cbuf, (int)C, range - ulow, (uint32_t)k, out, lane, warp);
         return;
       }
     }
@@ -661,6 +673,96 @@ __global__ void __launch_bounds__(kThreads) topk_block_kernel(TopkArgs a) {
   }
 }
 
+// Lists of 16K to 40K entries when every query has its own CTA (many
+// queries: a prefill chunk): the block kernel's sample-and-filter scheme over
+// keys cached in shared memory instead of registers (R = ceil(n / 1024) per
+// thread, positions base + 32 r, so each warp owns a contiguous run). If the
+// sample's floor admits fewer than k or more than kCandCap keys, the exact
+// multi-pass select runs over the cached keys instead.
+__global__ void __launch_bounds__(kThreads) topk_filter_kernel(TopkArgs a) {
+  extern __shared__ uint32_t kc[];  // [N_max rounded to 4] keys, then [kCandCap] keys, [kCandCap] positions
+  __shared__ alignas(16) BlockShared sh;
+  __shared__ TopkShared ts;
+  pdl_wait();
+  pdl_release();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int q = blockIdx.x;
+  const int n = clamp_count(a.n_cmp[q], a.N_max, threadIdx.x == 0 ? a.status : nullptr);
+  const int k = a.k;
+  int32_t *out = a.out_idx + (size_t)q * k;
+  if (n <= k) {
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const float *s = a.scores + (size_t)q * a.N_max;
+  uint32_t *cbuf = kc + ((a.N_max + 3) & ~3);
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  sel::cache_keys<kThreads>(kc, s, n, lo, hi);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    sh.wmin[warp] = lo;
+    sh.wmax[warp] = hi;
+  }
+  for (int i = threadIdx.x; i < 2 * kBins; i += kThreads) (&sh.hist[0][0])[i] = 0u;
+  if (threadIdx.x == 0) sh.ncand = 0u;
+  __syncthreads();  // (also: every key is cached)
+  lo = sh.wmin[lane];
+  hi = sh.wmax[lane];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const uint32_t kmin = lo, range = hi - lo;
+  const int R = (n + kThreads - 1) / kThreads;
+  const int base = 32 * R * warp + lane;
+  const int nvr = base < n ? min(R, (n - base + 31) / 32) : 0;
+  {
+    // The sample: key warp % R of every thread (up to 1,024 keys).
+    const int rs = warp % R;
+    const int top = range == 0u ? 0 : 32 - __clz(range);
+    const int shift1 = top > 11 ? top - 11 : 0;
+    if (rs < nvr) atomicAdd(&sh.hist[0][(kc[base + 32 * rs] - kmin) >> shift1], 1u);
+    auto rank_of = [&](uint32_t S) {  // as in the block kernel
+      const float mu = (float)k * (float)S / (float)n;
+      return (uint32_t)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
+    };
+    uint32_t bin, above, cb, m, S;
+    boundary_bin(sh, sh.hist[0], 0, lane, warp, rank_of, bin, above, cb, m, S);
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh.hist[0][i] = 0u;  // cleared for the selection
+    if (range != 0u && m < S) {
+      const uint32_t ulow = bin << shift1;
+      uint32_t c = 0u;
+      for (int r = 0; r < R; ++r) c += __popc(__ballot_sync(0xffffffffu, r < nvr && kc[base + 32 * r] - kmin >= ulow));
+      uint32_t off, C;
+      warp_offsets(sh.wg, c, lane, warp, off, C);
+      if (C >= (uint32_t)k && C <= (uint32_t)kCandCap) {
+        for (int r = 0; r < R; ++r) {  // in position order, as in the block kernel
+          const uint32_t u = r < nvr ? kc[base + 32 * r] - kmin : 0u;
+          const bool sel = r < nvr && u >= ulow;
+          const uint32_t mm = __ballot_sync(0xffffffffu, sel);
+          if (sel) {
+            const uint32_t slot = off + __popc(mm & lt);
+            cbuf[slot] = u - ulow;
+            cbuf[kCandCap + slot] = (uint32_t)(base + 32 * r);
+          }
+          off += __popc(mm);
+        }
+        __syncthreads();
+        select_candidates(sh, cbuf, (int)C, range - ulow, (uint32_t)k, out, lane, warp);
+        return;
+      }
+    }
+  }
+  __syncthreads();
+  select_and_emit<true>(ts, kc, s, n, k, [out](uint32_t slot, int j, uint32_t) { out[slot] = j; });
+}
+
 }  // namespace
 
 // Cluster size for one query's list: about SMs / Q CTAs, at most 8, at
@@ -690,6 +792,8 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, s
     cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemKeys * 4);
     for (auto kern : {topk_block_kernel<8>, topk_block_kernel<16>})
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * kCandCap * (int)sizeof(uint32_t));
+    cudaFuncSetAttribute(topk_filter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (kFilterKeys + 2 * kCandCap) * (int)sizeof(uint32_t));
   });
   // Lists of up to 16 K entries: one CTA per query, keys in registers.
   if (a.N_max <= 16 * kThreads) {
@@ -701,6 +805,12 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, s
     const int S = ((a.N_max + C - 1) / C + 31) & ~31;
     return launch_pdl_cluster(topk_cluster_kernel, dim3(C, a.Q), dim3(kThreads), (size_t)S * 4, stream, (unsigned)C,
                               a);
+  }
+  // Up to 40 K entries with a CTA per query: sample, filter, select over
+  // the keys cached in shared memory.
+  if (a.N_max <= kFilterKeys) {
+    const size_t smem = (((size_t)a.N_max + 3) & ~(size_t)3) * 4 + 2 * kCandCap * sizeof(uint32_t);
+    return launch_pdl(topk_filter_kernel, dim3(a.Q), dim3(kThreads), smem, stream, a);
   }
   int seg = 0, nseg = 0;
   const size_t need = topk_scratch_bytes(a.Q, a.N_max, a.k);
