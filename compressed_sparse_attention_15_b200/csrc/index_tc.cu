@@ -262,20 +262,39 @@ __global__ void __launch_bounds__(Fmt<kFp8, kG>::kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc::fence_after_sync();
       const int j = tl.j0 + row;
-#pragma unroll 1
+      // The group's 64 head products of query g are loaded while those of
+      // query g - 1 are reduced (two register buffers); the reduction runs
+      // as 8 independent chains.
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * F::kAccCols;
+      uint32_t v[2][2][32];
+      tc::tmem_ld32(tbase, v[0][0]);
+      tc::tmem_ld32(tbase + 32, v[0][1]);
+      tc::tmem_ld_wait();
+      tc::tmem_regs_ready(v[0][0]);
+      tc::tmem_regs_ready(v[0][1]);
+#pragma unroll
       for (int g = 0; g < kG; ++g) {
-        uint32_t v0[32], v1[32];
-        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + acc * F::kAccCols + 64 * g;
-        tc::tmem_ld32(taddr, v0);
-        tc::tmem_ld32(taddr + 32, v1);
-        tc::tmem_ld_wait();
+        const int b = g & 1;
+        if (g + 1 < kG) {
+          tc::tmem_ld32(tbase + 64 * (g + 1), v[b ^ 1][0]);
+          tc::tmem_ld32(tbase + 64 * (g + 1) + 32, v[b ^ 1][1]);
+        }
         const float *wg = wq + g * kHi;
-        float s = 0.f;
+        float p[8];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) s = fmaf(wg[h], fmaxf(__uint_as_float(v0[h]), 0.f), s);
+        for (int c = 0; c < 8; ++c) p[c] = 0.f;
 #pragma unroll
-        for (int h = 0; h < 32; ++h) s = fmaf(wg[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s);
+        for (int h = 0; h < 32; ++h) p[h & 7] = fmaf(wg[h], fmaxf(__uint_as_float(v[b][0][h]), 0.f), p[h & 7]);
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+          p[h & 7] = fmaf(wg[32 + h], fmaxf(__uint_as_float(v[b][1][h]), 0.f), p[h & 7]);
+        const float s = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         if (j < nq[g]) a.scores[(size_t)(tl.q * kG + g) * a.N_max + j] = s;
+        if (g + 1 < kG) {
+          tc::tmem_ld_wait();
+          tc::tmem_regs_ready(v[b ^ 1][0]);
+          tc::tmem_regs_ready(v[b ^ 1][1]);
+        }
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->accempty[acc]);
