@@ -14,14 +14,16 @@
 // accumulator, so each epilogue thread owns one entry's 64 head products and
 // the weighted ReLU sum over heads is thread-local.
 //
-// Pipeline (persistent, one CTA per SM; 192 threads, 320 for E4M3):
+// Pipeline (persistent, one CTA per SM; 192 threads, 320 for E4M3 and for
+// query groups):
 //   warp 0      TMA producer: 32 KB key tiles (128 bf16 / 256 FP8 entries)
 //               into a 5-stage ring, and the query's head block (16 / 8 KB)
 //               into one of two query slots;
 //   warp 1      MMA issuer (one thread) and TMEM owner (2 accumulators);
 //   warps 2..   epilogue, one per TMEM lane quarter and 128-entry row block
-//               (4 warps; 8 for the two blocks of an E4M3 tile): tcgen05.ld,
-//               ReLU, weighted sum, coalesced store.
+//               (4 warps; 8 for the two blocks of an E4M3 tile, or for the
+//               two halves of a query group): tcgen05.ld, ReLU, weighted
+//               sum, coalesced store.
 // Each CTA walks a contiguous range of the flat (query, tile) space. Every
 // wait is bounded; a timeout raises CSA_STATUS_WAIT_TIMEOUT, all roles stop,
 // in-flight copies and MMAs are drained (bounded) and TMEM is freed.
@@ -66,12 +68,14 @@ struct Fmt {
   static constexpr uint32_t kAccCols = 64 * kSub * kG;     // TMEM columns of one accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static constexpr uint32_t kIdesc = kFp8 ? tc::idesc_e4m3(128, 64) : tc::idesc_bf16(128, 64 * kG, 0, 0);
-  // per epilogue warp: its group's head weights and visible counts
-  static constexpr uint32_t kWBytes = kG == 1 ? 0 : 4 * (kG * kHi * 4 + kG * 4);
   // Epilogue warps: one per TMEM lane quarter and row block, so that each
-  // warp reduces one 128-entry block of a tile (E4M3 tiles hold two).
-  static constexpr int kEpiWarps = 4 * kSub;
+  // warp reduces one 128-entry block of a tile (E4M3 tiles hold two); for
+  // query groups two per lane quarter, each reducing half of the group's
+  // queries.
+  static constexpr int kEpiWarps = 4 * kSub * (kG > 1 ? 2 : 1);
   static constexpr int kThreads = 32 * (2 + kEpiWarps);
+  // per epilogue warp: its group's head weights and visible counts
+  static constexpr uint32_t kWBytes = kG == 1 ? 0 : kEpiWarps * (kG * kHi * 4 + kG * 4);
 };
 
 template <int kStages>
@@ -116,7 +120,7 @@ __global__ void __launch_bounds__(Fmt<kFp8, kG>::kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stage_buf = smem;
   uint8_t *q_buf = smem + kStages * kTileBytes;
-  float *w_buf = reinterpret_cast<float *>(q_buf + F::kQSlots * kQBytes);  // kG > 1: [4 warps][kG x 64 + kG]
+  float *w_buf = reinterpret_cast<float *>(q_buf + F::kQSlots * kQBytes);  // kG > 1: [epilogue warp][kG x 64 + kG]
   Bars<kStages> *bars = reinterpret_cast<Bars<kStages> *>(q_buf + F::kQSlots * kQBytes + F::kWBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long t_begin = (long long)blockIdx.x * per_cta;
@@ -241,6 +245,8 @@ __global__ void __launch_bounds__(Fmt<kFp8, kG>::kThreads, 1)
     // memory (no warp waits on another when the group changes).
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
+    constexpr int kGW = kG / (F::kEpiWarps / 4);  // queries of the group this warp reduces
+    const int g0 = kGW * ((warp - 2) >> 2);
     float *wq = w_buf + (warp - 2) * (kG * kHi + kG);
     int *nq = reinterpret_cast<int *>(wq + kG * kHi);  // the group's visible counts
     int acc = 0, cur_g = -1;
@@ -265,7 +271,7 @@ __global__ void __launch_bounds__(Fmt<kFp8, kG>::kThreads, 1)
       // The group's 64 head products of query g are loaded while those of
       // query g - 1 are reduced (two register buffers); the reduction runs
       // as 8 independent chains.
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * F::kAccCols;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * F::kAccCols + 64 * g0;
       uint32_t v[2][2][32];
       tc::tmem_ld32(tbase, v[0][0]);
       tc::tmem_ld32(tbase + 32, v[0][1]);
@@ -273,11 +279,11 @@ __global__ void __launch_bounds__(Fmt<kFp8, kG>::kThreads, 1)
       tc::tmem_regs_ready(v[0][0]);
       tc::tmem_regs_ready(v[0][1]);
 #pragma unroll
-      for (int g = 0; g < kG; ++g) {
-        const int b = g & 1;
-        if (g + 1 < kG) {
-          tc::tmem_ld32(tbase + 64 * (g + 1), v[b ^ 1][0]);
-          tc::tmem_ld32(tbase + 64 * (g + 1) + 32, v[b ^ 1][1]);
+      for (int gi = 0; gi < kGW; ++gi) {
+        const int b = gi & 1, g = g0 + gi;
+        if (gi + 1 < kGW) {
+          tc::tmem_ld32(tbase + 64 * (gi + 1), v[b ^ 1][0]);
+          tc::tmem_ld32(tbase + 64 * (gi + 1) + 32, v[b ^ 1][1]);
         }
         const float *wg = wq + g * kHi;
         float p[8];
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(Fmt<kFp8, kG>::kThreads, 1)
           p[h & 7] = fmaf(wg[32 + h], fmaxf(__uint_as_float(v[b][1][h]), 0.f), p[h & 7]);
         const float s = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         if (j < nq[g]) a.scores[(size_t)(tl.q * kG + g) * a.N_max + j] = s;
-        if (g + 1 < kG) {
+        if (gi + 1 < kGW) {
           tc::tmem_ld_wait();
           tc::tmem_regs_ready(v[b ^ 1][0]);
           tc::tmem_regs_ready(v[b ^ 1][1]);
