@@ -14,16 +14,16 @@
 // accumulator, so each epilogue thread owns one entry's 64 head products and
 // the weighted ReLU sum over heads is thread-local.
 //
-// Pipeline (persistent, one CTA per SM; 192 threads, 320 for E4M3 and for
+// Pipeline (persistent, one CTA per SM; 192 threads, 320 for E4M3, 576 for
 // query groups):
 //   warp 0      TMA producer: 32 KB key tiles (128 bf16 / 256 FP8 entries)
 //               into a 5-stage ring, and the query's head block (16 / 8 KB)
 //               into one of two query slots;
 //   warp 1      MMA issuer (one thread) and TMEM owner (2 accumulators);
 //   warps 2..   epilogue, one per TMEM lane quarter and 128-entry row block
-//               (4 warps; 8 for the two blocks of an E4M3 tile, or for the
-//               two halves of a query group): tcgen05.ld, ReLU, weighted
-//               sum, coalesced store.
+//               (4 warps; 8 for the two blocks of an E4M3 tile, 16 for the
+//               4 queries of a group): tcgen05.ld, ReLU, weighted sum,
+//               coalesced store.
 // Each CTA walks a contiguous range of the flat (query, tile) space. Every
 // wait is bounded; a timeout raises CSA_STATUS_WAIT_TIMEOUT, all roles stop,
 // in-flight copies and MMAs are drained (bounded) and TMEM is freed.
@@ -70,9 +70,8 @@ struct Fmt {
   static constexpr uint32_t kIdesc = kFp8 ? tc::idesc_e4m3(128, 64) : tc::idesc_bf16(128, 64 * kG, 0, 0);
   // Epilogue warps: one per TMEM lane quarter and row block, so that each
   // warp reduces one 128-entry block of a tile (E4M3 tiles hold two); for
-  // query groups two per lane quarter, each reducing half of the group's
-  // queries.
-  static constexpr int kEpiWarps = 4 * kSub * (kG > 1 ? 2 : 1);
+  // query groups one per lane quarter and query of the group.
+  static constexpr int kEpiWarps = 4 * kSub * (kG > 1 ? kG : 1);
   static constexpr int kThreads = 32 * (2 + kEpiWarps);
   // per epilogue warp: its group's head weights and visible counts
   static constexpr uint32_t kWBytes = kG == 1 ? 0 : kEpiWarps * (kG * kHi * 4 + kG * 4);
