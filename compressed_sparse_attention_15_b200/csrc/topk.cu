@@ -18,7 +18,10 @@
 // holding every key in registers (topk_block_kernel, few block barriers).
 // Longer lists with few queries (a decode batch): the list of one query is cut
 // into C contiguous slices, one CTA of a thread-block cluster each (C <= 8,
-// about SMs / Q); the slices' histograms are summed through distributed
+// about SMs / Q). Slices of up to 40K keys first try the sample-and-filter
+// scheme over the cluster (four cluster barriers: key range, summed sample
+// histograms, candidate counts, candidates gathered into CTA 0, which selects
+// among them); otherwise the slices' histograms are summed through distributed
 // shared memory at every radix pass, and each CTA emits its own slice at the
 // offset given by the counts of the slices before it. Many queries with
 // lists of up to 40K entries: one 1024-thread CTA per query, keys cached in
@@ -220,33 +223,6 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int use_cach
   }
 }
 
-// One query per cluster; CTA c of C selects over the slice
-// [c * S, c * S + S) of the list, S = ceil(n / C) rounded up to 32.
-__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkArgs a) {
-  extern __shared__ uint32_t keys[];
-  __shared__ alignas(16) uint32_t hist[2 * kBins];
-  __shared__ sel::Shared cs;
-  pdl_wait();
-  pdl_release();
-  const uint32_t C = cluster_size(), c = cluster_rank();
-  const int q = blockIdx.y;
-  const int n = clamp_count(a.n_cmp[q], a.N_max, (threadIdx.x == 0 && c == 0) ? a.status : nullptr);
-  const int k = a.k;
-  int32_t *out = a.out_idx + (size_t)q * k;
-  if (n <= k) {  // the same for every CTA of the cluster: no CTA touches a peer
-    if (c == 0)
-      for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
-    return;
-  }
-  const int S = ((n + (int)C - 1) / (int)C + 31) & ~31;
-  const int j0 = (int)c * S;
-  const int len = max(0, min(S, n - j0));
-  uint32_t lo = 0xffffffffu, hi = 0u;
-  sel::cache_keys<kThreads>(keys, a.scores + (size_t)q * a.N_max + j0, len, lo, hi);
-  sel::cluster_select<kThreads, 4, 8>(cs, hist, keys, len, j0, k, C, c, lo, hi,
-                                      [&](uint32_t slot, int j) { out[slot] = j; });
-  cluster_wait();  // no peer reads this CTA's shared memory any more
-}
 
 // Two-stage selection for long lists. Stage 1: segment g of query q (`seg`
 // entries) keeps its own top-k (an entry of the global top-k set is always in
@@ -763,6 +739,170 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(TopkArgs a) {
   select_and_emit<true>(ts, kc, s, n, k, [out](uint32_t slot, int j, uint32_t) { out[slot] = j; });
 }
 
+// One query per cluster; CTA c of C selects over the slice
+// [c * S, c * S + S) of the list, S = ceil(n / C) rounded up to 32, cached
+// in shared memory. With `filt` (the slice and a candidate buffer fit in
+// shared memory) the block kernel's sample-and-filter scheme runs over the
+// cluster first (cluster_filter); when the sampled floor admits fewer than
+// k or more than kCandCap keys, every CTA takes the exact cluster radix
+// select instead.
+__device__ bool cluster_filter(BlockShared &sh, sel::Shared &cs, uint32_t *hist, const uint32_t *keys, uint32_t *cbuf,
+                               int len, int j0, int S, int n, int k, uint32_t C, uint32_t c, uint32_t lo, uint32_t hi,
+                               int32_t *out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  // (1) the cluster's key range
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    sh.wmin[warp] = lo;
+    sh.wmax[warp] = hi;
+  }
+  for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0u;  // this slice's sample histogram
+  for (int i = threadIdx.x; i < 2 * kBins; i += kThreads) (&sh.hist[0][0])[i] = 0u;
+  if (threadIdx.x == 0) sh.ncand = 0u;
+  __syncthreads();
+  if (warp == 0) {
+    lo = sh.wmin[lane];
+    hi = sh.wmax[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+      cs.lmin = lo;
+      cs.lmax = hi;
+    }
+  }
+  cluster_sync();  // every slice's range is published
+  if (warp == 0) {
+    lo = (uint32_t)lane < C ? ld_peer(&cs.lmin, lane) : 0xffffffffu;
+    hi = (uint32_t)lane < C ? ld_peer(&cs.lmax, lane) : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+      cs.kmin = lo;
+      cs.krange = hi - lo;
+    }
+  }
+  __syncthreads();
+  const uint32_t kmin = cs.kmin, range = cs.krange;
+  // (2) the sample: one key per thread, spread over the slice; the slices'
+  // histograms are summed into sh.hist[0]
+  const int top = range == 0u ? 0 : 32 - __clz(range);
+  const int shift1 = top > 11 ? top - 11 : 0;
+  {
+    const int js = (int)(((long long)threadIdx.x * S) / kThreads);
+    if (js < len) atomicAdd(&hist[(keys[js] - kmin) >> shift1], 1u);
+  }
+  cluster_sync();  // every slice's sample histogram is complete
+  for (int b = 4 * (int)threadIdx.x; b < kBins; b += 4 * kThreads) {
+    uint4 t = make_uint4(0u, 0u, 0u, 0u);
+    for (uint32_t r = 0; r < C; ++r) {
+      const uint4 v = ld_peer_u4(&hist[b], r);
+      t.x += v.x;
+      t.y += v.y;
+      t.z += v.z;
+      t.w += v.w;
+    }
+    *reinterpret_cast<uint4 *>(&sh.hist[0][b]) = t;
+  }
+  auto rank_of = [&](uint32_t Sn) {  // as in the block kernel
+    const float mu = (float)k * (float)Sn / (float)n;
+    return (uint32_t)ceilf(mu + 4.f * sqrtf(mu) + 8.f);
+  };
+  uint32_t bin, above, cb, m, Sn;
+  boundary_bin(sh, sh.hist[0], 0, lane, warp, rank_of, bin, above, cb, m, Sn);
+  for (int i = threadIdx.x; i < kBins; i += kThreads) sh.hist[0][i] = 0u;  // cleared for the selection
+  const bool floor_ok = range != 0u && m < Sn;
+  const uint32_t ulow = bin << shift1;
+  // (3) this slice's candidates (keys at or above the floor), counted in
+  // position order: warp w scans a contiguous run of the slice
+  const int per_warp = (((len + kWarps - 1) / kWarps) + 31) & ~31;
+  const int wlo = min(len, warp * per_warp), whi = min(len, wlo + per_warp);
+  uint32_t cnt = 0u;
+  for (int base = wlo; base < whi; base += 32) {
+    const int j = base + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, floor_ok && j < whi && keys[j] - kmin >= ulow));
+  }
+  uint32_t off, Cl;
+  warp_offsets(sh.wg, cnt, lane, warp, off, Cl);
+  if (threadIdx.x == 0) cs.cnt_gt = Cl;
+  cluster_sync();  // every slice's count is published; no peer reads a sample histogram any more
+  if (warp == 0) {
+    const uint32_t x = (uint32_t)lane < C ? ld_peer(&cs.cnt_gt, lane) : 0u;
+    uint32_t inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const uint32_t excl = __shfl_sync(0xffffffffu, inc - x, (int)c), total = __shfl_sync(0xffffffffu, inc, 31);
+    if (lane == 0) {
+      cs.base_gt = excl;
+      cs.bcnt = total;
+    }
+  }
+  __syncthreads();
+  const uint32_t Ctot = cs.bcnt, cbase = cs.base_gt;
+  if (!(floor_ok && Ctot >= (uint32_t)k && Ctot <= (uint32_t)kCandCap)) return false;  // the same in every CTA
+  // (4) the candidates go to CTA 0 in position order; it selects among them
+  uint32_t slot0 = cbase + off;
+  for (int base = wlo; base < whi; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = j < whi ? keys[j] - kmin : 0u;
+    const bool selb = j < whi && u >= ulow;
+    const uint32_t mm = __ballot_sync(0xffffffffu, selb);
+    if (selb) {
+      const uint32_t slot = slot0 + __popc(mm & lt);
+      st_peer(&cbuf[slot], 0u, u - ulow);
+      st_peer(&cbuf[kCandCap + slot], 0u, (uint32_t)(j0 + j));
+    }
+    slot0 += __popc(mm);
+  }
+  cluster_sync();  // every candidate is in CTA 0; no CTA touches a peer after this
+  if (c == 0) select_candidates(sh, cbuf, (int)Ctot, range - ulow, (uint32_t)k, out, lane, warp);
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkArgs a, int filt) {
+  extern __shared__ uint32_t keys[];  // [S] slice keys (then, with filt, [2 kCandCap] candidates)
+  __shared__ alignas(16) uint32_t hist[2 * kBins];
+  __shared__ sel::Shared cs;
+  __shared__ alignas(16) BlockShared sh;
+  pdl_wait();
+  pdl_release();
+  const uint32_t C = cluster_size(), c = cluster_rank();
+  const int q = blockIdx.y;
+  const int n = clamp_count(a.n_cmp[q], a.N_max, (threadIdx.x == 0 && c == 0) ? a.status : nullptr);
+  const int k = a.k;
+  int32_t *out = a.out_idx + (size_t)q * k;
+  if (n <= k) {  // the same for every CTA of the cluster: no CTA touches a peer
+    if (c == 0)
+      for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const int S = ((n + (int)C - 1) / (int)C + 31) & ~31;
+  const int j0 = (int)c * S;
+  const int len = max(0, min(S, n - j0));
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  sel::cache_keys<kThreads>(keys, a.scores + (size_t)q * a.N_max + j0, len, lo, hi);
+  if (filt) {
+    uint32_t *cbuf = keys + (((a.N_max + (int)C - 1) / (int)C + 31) & ~31);  // past the largest slice
+    if (cluster_filter(sh, cs, hist, keys, cbuf, len, j0, S, n, k, C, c, lo, hi, out)) return;
+  }
+  sel::cluster_select<kThreads, 4, 8>(cs, hist, keys, len, j0, k, C, c, lo, hi,
+                                      [&](uint32_t slot, int j) { out[slot] = j; });
+  cluster_wait();  // no peer reads this CTA's shared memory any more
+}
+
 }  // namespace
 
 // Cluster size for one query's list: about SMs / Q CTAs, at most 8, at
@@ -803,8 +943,10 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream, void *scratch, s
   }
   if (const int C = plan_cluster(a.Q, a.N_max, a.k)) {
     const int S = ((a.N_max + C - 1) / C + 31) & ~31;
-    return launch_pdl_cluster(topk_cluster_kernel, dim3(C, a.Q), dim3(kThreads), (size_t)S * 4, stream, (unsigned)C,
-                              a);
+    // the sample-and-filter front when the slice and the candidate buffer fit
+    const int filt = S <= kFilterKeys ? 1 : 0;
+    const size_t smem = (size_t)S * 4 + (filt ? 2 * kCandCap * sizeof(uint32_t) : 0);
+    return launch_pdl_cluster(topk_cluster_kernel, dim3(C, a.Q), dim3(kThreads), smem, stream, (unsigned)C, a, filt);
   }
   // Up to 40 K entries with a CTA per query: sample, filter, select over
   // the keys cached in shared memory.

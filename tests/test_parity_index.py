@@ -68,6 +68,7 @@ def test_topk_exact_on_given_scores(cuda_device, N, k):
     (100, 5000, 512, "one CTA per query, 8 keys per thread in registers"),
     (8, 262143, 1024, "cluster of 8 CTAs per query, 32K entries each (1M-context decode batch)"),
     (5, 30000, 512, "cluster of 8, a short last slice"),
+    (8, 262143, 64, "cluster of 8 sampling and filtering, a small k"),
     (100, 20000, 512, "one CTA per query, sample and filter over keys cached in shared memory"),
     (200, 33791, 512, "sample and filter over cached keys, the prefill chunk's list length"),
     (150, 40960, 2048, "sample and filter over cached keys, the longest such list"),
@@ -92,13 +93,15 @@ def test_topk_every_launch_shape(cuda_device, Q, N, k, shape):
         assert np.all(got[q, m:] == -1)
 
 
+@pytest.mark.parametrize("Q,N", [(160, 30000), (8, 100000)])
 @pytest.mark.parametrize("levels", [1, 4])
-def test_topk_filter_falls_back_when_the_floor_admits_too_many(cuda_device, levels):
-    # 30,000 scores over 1 or 4 distinct values: the sampled floor admits far
-    # more than the 4,096 candidates the filter holds (or the range is empty),
-    # so the exact select over every cached key decides; ties take the
+def test_topk_filter_falls_back_when_the_floor_admits_too_many(cuda_device, Q, N, levels):
+    # Scores over 1 or 4 distinct values: the sampled floor admits far more
+    # than the 4,096 candidates the filter holds (or the range is empty), so
+    # the exact select decides, over the cached keys of one CTA per query
+    # (160 queries) or of a cluster of 8 per query (8 queries); ties take the
     # smallest positions.
-    Q, N, k = 160, 30000, 512
+    k = 512
     u = synth.uniform(6, 14, (Q, N))
     s = torch.floor(u * levels) if levels > 1 else torch.zeros((Q, N))
     n = torch.tensor([N - (q % 4) for q in range(Q)], dtype=torch.int32)
