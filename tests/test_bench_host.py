@@ -89,3 +89,28 @@ def test_secondary_lines_cover_the_other_workloads():
     names = {n for _, n, _ in bench.SECONDARY}
     assert names == set(WL.WORKLOADS) - {"tiny_csa_prefill_fp32"}
     assert any(rope for _, _, rope in bench.SECONDARY)
+
+
+def test_committed_traffic_records_are_consistent():
+    # profiles/traffic.json (the `traffic` of each bench line) holds, per
+    # workload and bench part, positive DRAM bytes per launch whose source is
+    # a committed summary that names the kernel; and bench.load_traffic reads
+    # every bench workload's record.
+    import json
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    bench_names = {n for _, n, _ in bench.SECONDARY} | {"csa_decode_64k"}
+    for name, parts in rec.items():
+        assert name in bench_names, name
+        for part, v in parts.items():
+            assert part in ("compress", "index_scores", "topk", "mqa"), (name, part)
+            assert v["dram_bytes_per_launch"] > 0, (name, part)
+            src = os.path.join(ROOT, v["source"])
+            assert os.path.isfile(src), (name, part, v["source"])
+            with open(src) as f:
+                text = f.read()
+            for kernel in v["kernel"].split(" + "):
+                assert kernel in text, (name, part, kernel)
+        assert bench.load_traffic(os.path.join(ROOT, "profiles", "traffic.json"), name) == {
+            p: v["dram_bytes_per_launch"] for p, v in parts.items()}
+    assert {"csa_decode_64k", "hca_decode_1m", "csa_decode_1m"} <= set(rec)
